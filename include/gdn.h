@@ -1,0 +1,178 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet token mixer.
+ *
+ * The layer is the linear-attention mixer that fills 69 of the 92 layers of
+ * Qwen3.8-2.4T-A95B ("Qwen3.8-2.4T-A95B vs Inkling", component table, Gated
+ * DeltaNet row; "Qwen3.8 2.4T A95B", key facts, layer stack "Linear x69").
+ * Per token it
+ *   1. runs a depthwise causal convolution of kernel 4 (no bias) + SiLU over
+ *      the q, k and v channels (Gated DeltaNet row; raw config field
+ *      linear_conv_kernel_dim = 4),
+ *   2. L2-normalises q and k per q/k head,
+ *   3. forms per value head the decay g = -exp(A_log) * softplus(a + dt_bias)
+ *      and the write strength beta = sigmoid(b) (Gated DeltaNet row),
+ *   4. applies the gated delta rule to an FP32 d_v x d_k state per value head
+ *      (raw config field mamba_ssm_dtype = float32),
+ *         S_t = exp(g_t) S_{t-1} (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *         o_t = S_t q_t,
+ *      where value head h reads q/k head h / (H_v / H_k) (Gated DeltaNet row:
+ *      16 q/k heads serve 128 value heads, 8 each),
+ *   5. normalises o per value head by RMS (eps = rms_norm_eps = 1e-6, raw
+ *      config fields) and multiplies by a weight and by SiLU(z) ("Qwen3.8-
+ *      2.4T-A95B vs Inkling", component table, output-gate row:
+ *      output_gate_type swish after a per-head RMSNorm).
+ * The in- and out-projections that produce qkv, a, b, z and consume y are
+ * not part of this library.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers (cudaMalloc'd or equivalent) on
+ *     the current device, except the gdn_config / gdn_params structs and the
+ *     `bytes` out-parameter, which are host memory.  The caller owns every
+ *     buffer; the library allocates nothing.
+ *   - Tensors are row-major and contiguous; every tensor pointer must be
+ *     16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued on it; no entry point synchronises the host.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED or
+ *     GDN_ERR_WORKSPACE; launch failures return GDN_ERR_CUDA.  Nothing traps
+ *     and no C++ exception crosses the ABI.  Entry points are stateless and
+ *     may be called from several host threads at once.
+ *   - Channel layout of a pre-conv qkv row (conv_dim = (2 H_k + H_v) d):
+ *     q of q/k head j at [j d, (j+1) d), k of head j at [H_k d + j d, ...),
+ *     v of value head h at [2 H_k d + h d, ...).
+ *   - The state of one value head is stored [d_v][d_k] (row = value channel).
+ */
+#ifndef GDN_H
+#define GDN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GDN_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define GDN_API __attribute__((visibility("default")))
+#else
+#define GDN_API
+#endif
+
+typedef enum gdn_status {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1, /* NULL/misaligned pointer, bad size or inconsistent shape */
+    GDN_ERR_UNSUPPORTED = 2, /* well-formed, but no kernel for this shape (head_dim, kernel) */
+    GDN_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than the size query says */
+    GDN_ERR_CUDA = 4         /* a CUDA launch or runtime call failed */
+} gdn_status;
+
+typedef enum gdn_dtype {
+    GDN_F32 = 0, /* float32 activations */
+    GDN_BF16 = 1 /* bfloat16 activations */
+} gdn_dtype;
+
+/* Head layout and scalar settings of one layer. */
+typedef struct gdn_config {
+    int32_t num_qk_heads; /* H_k >= 1 */
+    int32_t num_v_heads;  /* H_v, a multiple of H_k (G = H_v / H_k value heads per q/k head) */
+    int32_t head_dim;     /* d = d_k = d_v; this build supports 32 and 128 */
+    int32_t conv_kernel;  /* causal conv width; this build supports 4 */
+    float rms_eps;        /* epsilon of the gated RMSNorm (1e-6 for Qwen3.8) */
+    float l2_eps;         /* epsilon inside the q/k L2 norm: x / sqrt(sum x^2 + l2_eps) */
+    float q_scale;        /* extra factor on normalised q (1.0 = none) */
+    int32_t act_dtype;    /* gdn_dtype of qkv, a, b, z, y and the conv caches */
+} gdn_config;
+
+/* Layer parameters, all float32 device arrays. */
+typedef struct gdn_params {
+    const float *conv_w;  /* [conv_dim, conv_kernel]; tap conv_kernel-1 multiplies the current token */
+    const float *A_log;   /* [H_v] */
+    const float *dt_bias; /* [H_v] */
+    const float *norm_w;  /* [d], shared by all value heads */
+} gdn_params;
+
+/*
+ * Bytes of device workspace gdn_prefill needs for `total_tokens` packed
+ * tokens in `batch` sequences.  Writes *bytes; returns GDN_ERR_INVALID_ARG for
+ * a bad config or negative sizes, GDN_ERR_UNSUPPORTED for an unsupported one.
+ */
+GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
+                                      size_t *bytes);
+
+/*
+ * Prefill over a packed varlen batch: sequence n owns token rows
+ * cu_seqlens[n] .. cu_seqlens[n+1]-1 of every [N, ...] tensor, N = total_tokens.
+ *
+ *   qkv           [N, conv_dim]      act_dtype   pre-conv q|k|v rows
+ *   a, b          [N, H_v]           act_dtype   gate inputs
+ *   z             [N, H_v, d]        act_dtype   output-gate input
+ *   cu_seqlens    [batch+1]          int32, DEVICE; cu_seqlens[0] = 0,
+ *                                    non-decreasing, cu_seqlens[batch] = N
+ *                                    (zero-length sequences are allowed: their
+ *                                    state and conv window pass through)
+ *   initial_state [batch, H_v, d, d] float32, or NULL for zero states
+ *   initial_conv  [batch, K-1, conv_dim] act_dtype: the K-1 pre-conv rows
+ *                                    before each sequence, oldest first; NULL = zeros
+ *   y             [N, H_v, d]        act_dtype   output (gated RMSNorm of o)
+ *   final_state   [batch, H_v, d, d] float32, or NULL to skip; may equal
+ *                                    initial_state (in-place update)
+ *   final_conv    [batch, K-1, conv_dim] act_dtype, or NULL to skip: the last
+ *                                    K-1 pre-conv rows of [initial_conv; sequence];
+ *                                    may equal initial_conv
+ *   o_raw         [N, H_v, d]        float32 pre-norm recurrence output, or NULL
+ *   workspace     device scratch of at least gdn_prefill_workspace_size bytes,
+ *                 256-byte aligned; its contents on entry do not matter.
+ * The values of cu_seqlens are read on the device only; a cu_seqlens array
+ * that breaks the rules above gives unspecified output (never an
+ * out-of-bounds access outside [0, N) rows).
+ */
+GDN_API gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                       const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                       int32_t batch, int64_t total_tokens, const float *initial_state,
+                       const void *initial_conv, void *y, float *final_state, void *final_conv,
+                       float *o_raw, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Decode: one new token for each of `batch` sequences against their resident
+ * states, updated in place.
+ *
+ *   qkv        [batch, conv_dim]      act_dtype   the new tokens' pre-conv rows
+ *   a, b       [batch, H_v]           act_dtype
+ *   z          [batch, H_v, d]        act_dtype
+ *   state      [batch, H_v, d, d]     float32, in/out
+ *   conv_cache [batch, K-1, conv_dim] act_dtype, in/out: the last K-1 pre-conv
+ *                                     rows, oldest first; on return the oldest
+ *                                     row is dropped and the new row appended
+ *   y          [batch, H_v, d]        act_dtype   output
+ * Needs no workspace.
+ */
+GDN_API gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                      const void *a, const void *b, const void *z, float *state,
+                      void *conv_cache, int32_t batch, void *y, void *stream);
+
+/*
+ * Timing hook for benchmarks.  Arms a one-shot on the calling host thread:
+ * the next gdn_prefill or gdn_decode call made by this thread records
+ * `begin_event` on its stream immediately before launching its main kernel
+ * (the recurrence) and `end_event` immediately after it, so that
+ * cudaEventElapsedTime gives that kernel's device time alone.  Both are
+ * cudaEvent_t handles created by the caller; pass NULL, NULL to disarm.  A
+ * call that fails argument checks leaves the hook armed.  Returns
+ * GDN_ERR_INVALID_ARG if exactly one event is NULL.
+ */
+GDN_API gdn_status gdn_profile_next_call(void *begin_event, void *end_event);
+
+/* Static English text for a status code (never NULL). */
+GDN_API const char *gdn_status_string(gdn_status status);
+
+/* GDN_ABI_VERSION of the loaded library. */
+GDN_API int32_t gdn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_H */

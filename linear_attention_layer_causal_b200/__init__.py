@@ -1,1 +1,220 @@
-"""B200 (sm_100a) Gated DeltaNet token mixer: placeholder until the binding lands."""
+"""B200 (sm_100a) Gated DeltaNet token mixer.
+
+Thin ctypes binding over ``libgdn.so`` (C ABI in ``include/gdn.h``).  This
+module only marshals arguments: it turns torch tensors into device pointers
+and the current CUDA stream into a ``cudaStream_t``, allocates outputs and
+workspace with torch, and raises on a non-zero status.  Every step of the
+layer runs in the library's CUDA kernels; there is no CPU path, and calling
+into the library without the built extension raises.
+
+    import linear_attention_layer_causal_b200 as gdn
+    cfg = gdn.Config(num_qk_heads=16, num_v_heads=128, head_dim=128)
+    out = gdn.prefill(cfg, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_w,
+                      initial_state=S0, return_final_state=True)
+    y = gdn.decode(cfg, qkv1, a1, b1, z1, state, conv_cache, conv_w, A_log, dt_bias, norm_w)
+
+The layer: kernel-4 causal conv + SiLU over q|k|v, q/k L2 norm, gates
+g = -exp(A_log) softplus(a + dt_bias) and beta = sigmoid(b), the gated delta
+rule on an FP32 state per value head, and the per-head RMSNorm gated by
+SiLU(z) (Gated DeltaNet and output-gate rows of the component table on
+"Qwen3.8-2.4T-A95B vs Inkling").
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn.so")
+
+GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA = range(5)
+GDN_F32, GDN_BF16 = 0, 1
+
+EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_status_string",
+            "gdn_abi_version", "gdn_profile_next_call")
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+class _Config(ctypes.Structure):
+    _fields_ = [("num_qk_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("conv_kernel", ctypes.c_int32),
+                ("rms_eps", ctypes.c_float), ("l2_eps", ctypes.c_float),
+                ("q_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32)]
+
+
+class _Params(ctypes.Structure):
+    _fields_ = [("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
+                ("dt_bias", ctypes.c_void_p), ("norm_w", ctypes.c_void_p)]
+
+
+@dataclass(frozen=True)
+class Config:
+    """Head layout of one layer (H_k q/k heads, H_v value heads, head dim d)."""
+    num_qk_heads: int
+    num_v_heads: int
+    head_dim: int
+    conv_kernel: int = 4
+    rms_eps: float = 1e-6
+    l2_eps: float = 1e-6
+    q_scale: float = 1.0
+    act_dtype: str = "bf16"  # "bf16" or "f32"
+
+    @property
+    def conv_dim(self) -> int:
+        return (2 * self.num_qk_heads + self.num_v_heads) * self.head_dim
+
+    def _c(self) -> _Config:
+        return _Config(self.num_qk_heads, self.num_v_heads, self.head_dim, self.conv_kernel,
+                       self.rms_eps, self.l2_eps, self.q_scale,
+                       GDN_BF16 if self.act_dtype == "bf16" else GDN_F32)
+
+    @staticmethod
+    def of(wl) -> "Config":
+        """The Config of a workloads.Workload."""
+        return Config(wl.num_qk_heads, wl.num_v_heads, wl.head_dim, wl.conv_kernel,
+                      act_dtype=wl.dtype)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m linear_attention_layer_causal_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        cfgp, parp = ctypes.POINTER(_Config), ctypes.POINTER(_Params)
+        L.gdn_prefill_workspace_size.argtypes = [cfgp, i32, i64, ctypes.POINTER(sz)]
+        L.gdn_prefill_workspace_size.restype = ctypes.c_int
+        L.gdn_prefill.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, vp,
+                                  vp, vp, sz, vp]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_profile_next_call.argtypes = [vp, vp]
+        L.gdn_profile_next_call.restype = ctypes.c_int
+        L.gdn_abi_version.argtypes = []
+        L.gdn_abi_version.restype = ctypes.c_int32
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdn_status_string(status).decode()
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors passed to the library must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _act(cfg: Config):
+    import torch
+    return torch.bfloat16 if cfg.act_dtype == "bf16" else torch.float32
+
+
+def _params(conv_w, A_log, dt_bias, norm_w) -> _Params:
+    return _Params(_ptr(conv_w), _ptr(A_log), _ptr(dt_bias), _ptr(norm_w))
+
+
+def profile_next_call(begin_event, end_event) -> None:
+    """Time the main kernel of this thread's next prefill/decode call between two
+    torch.cuda.Event(enable_timing=True) events (see gdn_profile_next_call)."""
+    b = None if begin_event is None else begin_event.cuda_event
+    e = None if end_event is None else end_event.cuda_event
+    st = lib().gdn_profile_next_call(b, e)
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_profile_next_call")
+
+
+def prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().gdn_prefill_workspace_size(ctypes.byref(cfg._c()), batch, total_tokens,
+                                          ctypes.byref(n))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill_workspace_size")
+    return n.value
+
+
+def prefill(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_w, *,
+            initial_state=None, initial_conv=None, return_final_state=False,
+            return_final_conv=False, return_o_raw=False, y=None, final_state=None,
+            final_conv=None, workspace=None, stream=None) -> dict:
+    """Packed varlen prefill (see gdn_prefill in include/gdn.h).
+
+    Returns a dict with "y" and, when requested, "final_state", "final_conv"
+    and "o_raw".  Output buffers and the workspace may be passed in to avoid
+    allocation; ``final_state`` may be ``initial_state`` for an in-place update.
+    """
+    import torch
+    N = qkv.shape[0]
+    B = cu_seqlens.shape[0] - 1
+    dev = qkv.device
+    if y is None:
+        y = torch.empty((N, cfg.num_v_heads, cfg.head_dim), dtype=_act(cfg), device=dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, cfg.num_v_heads, cfg.head_dim, cfg.head_dim),
+                                  dtype=torch.float32, device=dev)
+    if final_conv is None and return_final_conv:
+        final_conv = torch.empty((B, cfg.conv_kernel - 1, cfg.conv_dim), dtype=_act(cfg),
+                                 device=dev)
+    o_raw = torch.empty((N, cfg.num_v_heads, cfg.head_dim), dtype=torch.float32,
+                        device=dev) if return_o_raw else None
+    need = prefill_workspace_size(cfg, B, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    st = lib().gdn_prefill(ctypes.byref(cfg._c()),
+                           ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                           _ptr(qkv), _ptr(a), _ptr(b), _ptr(z), _ptr(cu_seqlens), B, N,
+                           _ptr(initial_state), _ptr(initial_conv), _ptr(y), _ptr(final_state),
+                           _ptr(final_conv), _ptr(o_raw), _ptr(workspace), workspace.numel(),
+                           _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill")
+    out = {"y": y}
+    if final_state is not None:
+        out["final_state"] = final_state
+    if final_conv is not None:
+        out["final_conv"] = final_conv
+    if o_raw is not None:
+        out["o_raw"] = o_raw
+    return out
+
+
+def decode(cfg: Config, qkv, a, b, z, state, conv_cache, conv_w, A_log, dt_bias, norm_w, *,
+           y=None, stream=None):
+    """One token per sequence; `state` and `conv_cache` are updated in place.  Returns y."""
+    import torch
+    B = qkv.shape[0]
+    if y is None:
+        y = torch.empty((B, cfg.num_v_heads, cfg.head_dim), dtype=_act(cfg), device=qkv.device)
+    st = lib().gdn_decode(ctypes.byref(cfg._c()),
+                          ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                          _ptr(qkv), _ptr(a), _ptr(b), _ptr(z), _ptr(state), _ptr(conv_cache), B,
+                          _ptr(y), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode")
+    return y

@@ -1,0 +1,239 @@
+// gdn_api.cu -- the C ABI declared in include/gdn.h: host-side argument
+// checks, workspace carve-up and kernel launches.  Every check runs before the
+// first CUDA call, so a rejected call launches nothing and touches no device.
+#include <math.h>
+
+#include "gdn_common.cuh"
+#include "gdn_internal.h"
+
+namespace gdn {
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t round_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gdn_status check_config(const gdn_config *c) {
+    if (c == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (c->num_qk_heads < 1 || c->num_v_heads < 1 || c->head_dim < 1 || c->conv_kernel < 1)
+        return GDN_ERR_INVALID_ARG;
+    if (c->num_v_heads % c->num_qk_heads != 0)
+        return GDN_ERR_INVALID_ARG;
+    if (c->act_dtype != GDN_F32 && c->act_dtype != GDN_BF16)
+        return GDN_ERR_INVALID_ARG;
+    if (!(c->rms_eps >= 0.f) || !(c->l2_eps >= 0.f) || !isfinite(c->rms_eps) ||
+        !isfinite(c->l2_eps) || !isfinite(c->q_scale))
+        return GDN_ERR_INVALID_ARG;
+    if (c->head_dim != 32 && c->head_dim != 128)
+        return GDN_ERR_UNSUPPORTED;
+    if (c->conv_kernel != 4)
+        return GDN_ERR_UNSUPPORTED;
+    if (c->num_v_heads / c->num_qk_heads > 64)
+        return GDN_ERR_UNSUPPORTED;
+    // conv_dim * 16-byte channel groups must index in int
+    const int64_t conv_dim = (int64_t)(2 * (int64_t)c->num_qk_heads + c->num_v_heads) * c->head_dim;
+    if (conv_dim > (int64_t)1 << 26)
+        return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+gdn_status check_params(const gdn_params *p) {
+    if (p == nullptr || p->conv_w == nullptr || p->A_log == nullptr || p->dt_bias == nullptr ||
+        p->norm_w == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(p->conv_w) || !aligned16(p->norm_w))
+        return GDN_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(p->A_log) & 3u) || (reinterpret_cast<uintptr_t>(p->dt_bias) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+bool elem_aligned(const void *p, bool bf16) {
+    return p == nullptr || (reinterpret_cast<uintptr_t>(p) & (bf16 ? 1u : 3u)) == 0;
+}
+
+gdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
+
+thread_local ProfileHook tl_hook;
+
+} // namespace
+
+ProfileHook take_profile_hook() {
+    ProfileHook h = tl_hook;
+    tl_hook = ProfileHook{};
+    return h;
+}
+
+size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N) {
+    const size_t es = bf16 ? 2 : 4;
+    return round_up((size_t)N * 2 * Hk * D * es) + round_up((size_t)N * Hv * D * es);
+}
+
+} // namespace gdn
+
+using namespace gdn;
+
+extern "C" {
+
+int32_t gdn_abi_version(void) { return GDN_ABI_VERSION; }
+
+gdn_status gdn_profile_next_call(void *begin_event, void *end_event) {
+    if ((begin_event == nullptr) != (end_event == nullptr))
+        return GDN_ERR_INVALID_ARG;
+    tl_hook.begin = (cudaEvent_t)begin_event;
+    tl_hook.end = (cudaEvent_t)end_event;
+    return GDN_OK;
+}
+
+const char *gdn_status_string(gdn_status s) {
+    switch (s) {
+    case GDN_OK: return "success";
+    case GDN_ERR_INVALID_ARG: return "invalid argument (pointer, alignment, size or shape)";
+    case GDN_ERR_UNSUPPORTED: return "unsupported shape for this build";
+    case GDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case GDN_ERR_CUDA: return "CUDA launch or runtime error";
+    }
+    return "unknown status";
+}
+
+gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
+                                      size_t *bytes) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if (bytes == nullptr || batch < 0 || total_tokens < 0)
+        return GDN_ERR_INVALID_ARG;
+    *bytes = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads, cfg->head_dim,
+                                     cfg->act_dtype == GDN_BF16, total_tokens);
+    return GDN_OK;
+}
+
+gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                       const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                       int32_t batch, int64_t total_tokens, const float *initial_state,
+                       const void *initial_conv, void *y, float *final_state, void *final_conv,
+                       float *o_raw, void *workspace, size_t workspace_bytes, void *stream) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if ((st = check_params(params)) != GDN_OK)
+        return st;
+    if (batch < 0 || total_tokens < 0 || batch > 65535)
+        return batch > 65535 ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID_ARG;
+    if (batch == 0 && total_tokens > 0)
+        return GDN_ERR_INVALID_ARG;
+    if (batch > 0 && cu_seqlens == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    const bool bf16 = cfg->act_dtype == GDN_BF16;
+    if (total_tokens > 0 && (qkv == nullptr || a == nullptr || b == nullptr || z == nullptr ||
+                             y == nullptr))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(z) || !aligned16(y) || !aligned16(initial_state) ||
+        !aligned16(initial_conv) || !aligned16(final_state) || !aligned16(final_conv) ||
+        !aligned16(o_raw) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    const size_t need = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads,
+                                                cfg->head_dim, bf16, total_tokens);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return GDN_ERR_WORKSPACE;
+
+    PrefillArgs p{};
+    p.Hk = cfg->num_qk_heads;
+    p.Hv = cfg->num_v_heads;
+    p.D = cfg->head_dim;
+    p.G = p.Hv / p.Hk;
+    p.bf16 = bf16;
+    p.rms_eps = cfg->rms_eps;
+    p.l2_eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale;
+    p.qkv = qkv; p.a = a; p.b = b; p.z = z;
+    p.cu = cu_seqlens;
+    p.batch = batch;
+    p.N = total_tokens;
+    p.init_state = initial_state;
+    p.init_conv = initial_conv;
+    p.y = y;
+    p.final_state = final_state;
+    p.final_conv = final_conv;
+    p.o_raw = o_raw;
+    p.conv_w = params->conv_w;
+    p.A_log = params->A_log;
+    p.dt_bias = params->dt_bias;
+    p.norm_w = params->norm_w;
+    const size_t es = bf16 ? 2 : 4;
+    p.ws_qk = workspace;
+    p.ws_v = (char *)workspace + round_up((size_t)total_tokens * 2 * p.Hk * p.D * es);
+
+    cudaStream_t s = (cudaStream_t)stream;
+    const ProfileHook hook = take_profile_hook();
+    if (batch == 0)
+        return GDN_OK;
+    cudaError_t e = launch_conv_prep(p, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.begin, s);
+    if (e == cudaSuccess)
+        e = launch_recurrent_prefill(p, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.end, s);
+    if (e == cudaSuccess)
+        e = launch_final_conv(p, s);
+    return cuda_status(e);
+}
+
+gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                      const void *a, const void *b, const void *z, float *state,
+                      void *conv_cache, int32_t batch, void *y, void *stream) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if ((st = check_params(params)) != GDN_OK)
+        return st;
+    if (batch < 0)
+        return GDN_ERR_INVALID_ARG;
+    if (batch > 65535)
+        return GDN_ERR_UNSUPPORTED;
+    if (batch == 0) {
+        take_profile_hook();
+        return GDN_OK;
+    }
+    const bool bf16 = cfg->act_dtype == GDN_BF16;
+    if (qkv == nullptr || a == nullptr || b == nullptr || z == nullptr || state == nullptr ||
+        conv_cache == nullptr || y == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(z) || !aligned16(y) || !aligned16(state) ||
+        !aligned16(conv_cache) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16))
+        return GDN_ERR_INVALID_ARG;
+    DecodeArgs p{};
+    p.Hk = cfg->num_qk_heads;
+    p.Hv = cfg->num_v_heads;
+    p.D = cfg->head_dim;
+    p.G = p.Hv / p.Hk;
+    p.bf16 = bf16;
+    p.rms_eps = cfg->rms_eps;
+    p.l2_eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale;
+    p.qkv = qkv; p.a = a; p.b = b; p.z = z;
+    p.state = state;
+    p.conv_cache = conv_cache;
+    p.batch = batch;
+    p.y = y;
+    p.conv_w = params->conv_w;
+    p.A_log = params->A_log;
+    p.dt_bias = params->dt_bias;
+    p.norm_w = params->norm_w;
+    cudaStream_t s = (cudaStream_t)stream;
+    const ProfileHook hook = take_profile_hook();
+    cudaError_t e = record_if(hook.begin, s);
+    if (e == cudaSuccess)
+        e = launch_decode(p, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.end, s);
+    return cuda_status(e);
+}
+
+} // extern "C"

@@ -1,0 +1,134 @@
+"""The C-ABI library: it loads, exports every symbol include/gdn.h declares,
+and rejects bad arguments on the host before launching anything.
+
+The argument-error cases pass fake device pointers; they only run where no
+CUDA device is present, so that a validation bug can never hand a kernel a
+bogus address.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_attention_layer_causal_b200 as gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"GDN_API\s+[\w\s\*]*?\b(gdn_\w+)\s*\(", txt)
+    return names
+
+
+def test_library_exports_every_declared_symbol():
+    L = gdn.lib()
+    declared = _declared()
+    assert set(gdn.EXPORTED) <= set(declared)
+    for name in declared:
+        assert hasattr(L, name), f"{name} declared in include/ but not exported"
+    assert L.gdn_abi_version() == 1
+
+
+def test_status_strings():
+    for s in range(5):
+        assert gdn.status_string(s)
+    assert gdn.status_string(99) == "unknown status"
+
+
+QWEN38 = gdn.Config(16, 128, 128)
+
+
+def test_workspace_size_arithmetic():
+    n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
+    # normalised q|k and convolved v, bf16, each region rounded to 256 bytes
+    assert n == 4096 * 2 * 16 * 128 * 2 + 4096 * 128 * 128 * 2
+    assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
+    tiny = gdn.Config(2, 4, 32, act_dtype="f32")
+    assert gdn.prefill_workspace_size(tiny, 1, 3) == 1536 + 1536
+    assert gdn.prefill_workspace_size(tiny, 1, 1) == 512 + 512
+
+
+@pytest.mark.parametrize("cfg,code", [
+    (gdn.Config(0, 4, 32), gdn.GDN_ERR_INVALID_ARG),
+    (gdn.Config(3, 4, 32), gdn.GDN_ERR_INVALID_ARG),        # H_v not a multiple of H_k
+    (gdn.Config(2, 4, 64), gdn.GDN_ERR_UNSUPPORTED),        # head dim without a kernel
+    (gdn.Config(2, 4, 32, conv_kernel=3), gdn.GDN_ERR_UNSUPPORTED),
+    (gdn.Config(2, 4, 32, rms_eps=-1.0), gdn.GDN_ERR_INVALID_ARG),
+    (gdn.Config(2, 4, 32, l2_eps=float("nan")), gdn.GDN_ERR_INVALID_ARG),
+])
+def test_bad_config_rejected(cfg, code):
+    n = ctypes.c_size_t(0)
+    assert gdn.lib().gdn_prefill_workspace_size(ctypes.byref(cfg._c()), 1, 10, ctypes.byref(n)) == code
+
+
+def _fake_call(**over):
+    """gdn_prefill with fake 256-aligned device pointers; `over` replaces arguments."""
+    cfg = over.pop("cfg", gdn.Config(2, 4, 32))
+    P = 1 << 20
+    par = gdn._Params(P, P + 256, P + 512, P + 768)
+    args = dict(qkv=P * 2, a=P * 3, b=P * 4, z=P * 5, cu=P * 6, batch=1, N=10, S0=None,
+                C0=None, y=P * 7, S1=None, C1=None, o=None, ws=P * 8, wsb=1 << 20)
+    args.update(over)
+    params = over.get("params", par)
+    return gdn.lib().gdn_prefill(ctypes.byref(cfg._c()), ctypes.byref(params), args["qkv"],
+                                 args["a"], args["b"], args["z"], args["cu"], args["batch"],
+                                 args["N"], args["S0"], args["C0"], args["y"], args["S1"],
+                                 args["C1"], args["o"], args["ws"], args["wsb"], None)
+
+
+no_gpu = pytest.mark.skipif(
+    __import__("torch").cuda.is_available(), reason="argument-error cases run only without a GPU")
+
+
+@no_gpu
+@pytest.mark.parametrize("over,code", [
+    (dict(qkv=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(y=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cu=None), gdn.GDN_ERR_INVALID_ARG),
+    (dict(qkv=(1 << 21) + 8), gdn.GDN_ERR_INVALID_ARG),     # 8-byte aligned only
+    (dict(S0=(1 << 22) + 4), gdn.GDN_ERR_INVALID_ARG),
+    (dict(a=(1 << 22) + 1), gdn.GDN_ERR_INVALID_ARG),       # odd address for bf16
+    (dict(batch=-1), gdn.GDN_ERR_INVALID_ARG),
+    (dict(N=-5), gdn.GDN_ERR_INVALID_ARG),
+    (dict(batch=0, N=10), gdn.GDN_ERR_INVALID_ARG),
+    (dict(batch=70000), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(ws=None), gdn.GDN_ERR_WORKSPACE),
+    (dict(wsb=100), gdn.GDN_ERR_WORKSPACE),
+    (dict(ws=(1 << 23) + 16), gdn.GDN_ERR_WORKSPACE),       # not 256-byte aligned
+    (dict(params=gdn._Params(None, 256, 512, 768)), gdn.GDN_ERR_INVALID_ARG),
+    (dict(params=gdn._Params(8, 256, 512, 768)), gdn.GDN_ERR_INVALID_ARG),
+    (dict(cfg=gdn.Config(2, 4, 48)), gdn.GDN_ERR_UNSUPPORTED),
+])
+def test_prefill_argument_errors(over, code):
+    assert _fake_call(**over) == code
+
+
+@no_gpu
+def test_decode_argument_errors():
+    L = gdn.lib()
+    cfg = gdn.Config(2, 4, 32)
+    par = gdn._Params(1 << 20, (1 << 20) + 256, (1 << 20) + 512, (1 << 20) + 768)
+    P = 1 << 24
+    ok = [P, P * 2, P * 3, P * 4, P * 5, P * 6, 3, P * 7, None]
+    def call(i, v):
+        a = list(ok)
+        a[i] = v
+        return L.gdn_decode(ctypes.byref(cfg._c()), ctypes.byref(par), *a)
+    assert call(4, None) == gdn.GDN_ERR_INVALID_ARG          # state
+    assert call(5, None) == gdn.GDN_ERR_INVALID_ARG          # conv cache
+    assert call(4, P + 8) == gdn.GDN_ERR_INVALID_ARG         # misaligned state
+    assert call(6, -1) == gdn.GDN_ERR_INVALID_ARG
+    assert call(6, 0) == gdn.GDN_OK                          # empty batch: nothing to do
+    assert L.gdn_decode(None, ctypes.byref(par), *ok) == gdn.GDN_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(gdn, "_lib", None)
+    monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "libgdn.so"))
+    with pytest.raises(RuntimeError, match="missing"):
+        gdn.lib()
