@@ -246,6 +246,8 @@ def run_ours(args, rank, world, dev, dist):
         kern = [kb[i].elapsed_time(ke[i]) for i in range(K)]
         return total, sum(kern) / K
 
+    if args.only == "decode":
+        return run_decode(args, rank, world, dev, pk, timed, max_over_ranks)
     clocks = ClockSampler(dev.index)
     for _ in range(args.warmup):
         step()
@@ -269,33 +271,10 @@ def run_ours(args, rank, world, dev, dist):
             "hbm_view": {"achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": round(gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": byts}}
 
-    # ---- decode: 256 sequences x 1 token, resident states
-    dwl = W.QWEN38_DECODE
-    dcfg = gdn.Config.of(dwl)
-    d = W.make_decode(dwl, dev, seed=dwl.seed + 7919 * rank)
-    DP = [d[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
-    dy = torch.empty((dwl.decode_batch, dcfg.num_v_heads, dcfg.head_dim), dtype=torch.bfloat16,
-                     device=dev)
-
-    def dstep():
-        gdn.decode(dcfg, d["qkv"], d["a"], d["b"], d["z"], d["state"], d["conv_cache"], *DP, y=dy)
-
-    for _ in range(args.warmup):
-        dstep()
-    dtot, dkern = timed(dstep, args.steps)
-    dtot, dkern = max_over_ranks(dtot), max_over_ranks(dkern)
-    dB = dwl.decode_batch
-    dbytes = decode_bytes(dcfg.num_qk_heads, dcfg.num_v_heads, dcfg.head_dim, dB)
-    dgbs = dbytes / (dkern / 1e3) / 1e9
-    decode = {"metric": "GDN decode tokens/s at Qwen3.8 layer shape", "unit": "tokens/s",
-              "value": dB * world * args.steps / (dtot / 1e3), "ms_per_step": dtot / args.steps,
-              "config": {"workload": dwl.name, "batch": dB, "state_gib": dbytes / 2 / 2**30},
-              "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(dgbs, 1),
-                           "peak": pk["hbm_gbs"], "unit": "GB/s",
-                           "frac": round(dgbs / pk["hbm_gbs"], 4),
-                           "traffic": traffic_of("decode_kernel"), "algorithmic_bytes": dbytes,
-                           "kernel_ms": round(dkern, 4), "peak_source": pk["source"] + " copy"}}
-    del d
+    if args.only == "prefill":
+        return {"metric": METRIC, "value": value, "unit": UNIT, "ms_per_step": ms_per_step,
+                "roofline": roof, "clocks": clk}
+    decode = run_decode(args, rank, world, dev, pk, timed, max_over_ranks)
 
     # ---- end to end through the public API from pinned host buffers
     host = {k: inp[k].cpu().pin_memory() for k in ("qkv", "a", "b", "z")}
@@ -332,6 +311,38 @@ def run_ours(args, rank, world, dev, dist):
     return line
 
 
+def run_decode(args, rank, world, dev, pk, timed, max_over_ranks):
+    """Decode: B sequences x 1 token against resident FP32 states (in place)."""
+    import torch
+
+    import linear_attention_layer_causal_b200 as gdn
+    from linear_attention_layer_causal_b200 import workloads as W
+    dwl = W.QWEN38_DECODE
+    dcfg = gdn.Config.of(dwl)
+    dB = args.decode_batch
+    d = W.make_decode(dwl, dev, batch=dB, seed=dwl.seed + 7919 * rank)
+    DP = [d[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
+    dy = torch.empty((dB, dcfg.num_v_heads, dcfg.head_dim), dtype=torch.bfloat16, device=dev)
+
+    def dstep():
+        gdn.decode(dcfg, d["qkv"], d["a"], d["b"], d["z"], d["state"], d["conv_cache"], *DP, y=dy)
+
+    for _ in range(args.warmup):
+        dstep()
+    dtot, dkern = timed(dstep, args.steps)
+    dtot, dkern = max_over_ranks(dtot), max_over_ranks(dkern)
+    dbytes = decode_bytes(dcfg.num_qk_heads, dcfg.num_v_heads, dcfg.head_dim, dB)
+    dgbs = dbytes / (dkern / 1e3) / 1e9
+    return {"metric": "GDN decode tokens/s at Qwen3.8 layer shape", "unit": "tokens/s",
+            "value": dB * world * args.steps / (dtot / 1e3), "ms_per_step": dtot / args.steps,
+            "config": {"workload": dwl.name, "batch": dB, "state_gib": 4 * dB * 128 ** 3 / 2 ** 30},
+            "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(dgbs, 1),
+                         "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": round(dgbs / pk["hbm_gbs"], 4),
+                         "traffic": traffic_of("decode_kernel"), "algorithmic_bytes": dbytes,
+                         "kernel_ms": round(dkern, 4), "peak_source": pk["source"] + " copy"}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -339,6 +350,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+                    help="run only one part (for profiling small cases)")
+    ap.add_argument("--decode-batch", type=int, default=256)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -361,7 +375,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=dev)
     line = run_ours(args, rank, world, dev, dist)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.only == "all":
         from linear_attention_layer_causal_b200 import workloads as W
         inp = W.make_prefill(W.QWEN38_PREFILL, "cpu")
         v, info = oracle_throughput(W.QWEN38_PREFILL, inp)

@@ -143,6 +143,9 @@ def _params(conv_w, A_log, dt_bias, norm_w) -> _Params:
 def profile_next_call(begin_event, end_event) -> None:
     """Time the main kernel of this thread's next prefill/decode call between two
     torch.cuda.Event(enable_timing=True) events (see gdn_profile_next_call)."""
+    for ev in (begin_event, end_event):
+        if ev is not None and not ev.cuda_event:
+            ev.record()  # torch creates the underlying cudaEvent_t on first record
     b = None if begin_event is None else begin_event.cuda_event
     e = None if end_event is None else end_event.cuda_event
     st = lib().gdn_profile_next_call(b, e)

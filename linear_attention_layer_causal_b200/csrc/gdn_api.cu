@@ -67,9 +67,9 @@ ProfileHook take_profile_hook() {
     return h;
 }
 
-size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N) {
-    const size_t es = bf16 ? 2 : 4;
-    return round_up((size_t)N * 2 * Hk * D * es) + round_up((size_t)N * Hv * D * es);
+size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N) {
+    // float32 normalised q|k and convolved v
+    return round_up((size_t)N * 2 * Hk * D * 4) + round_up((size_t)N * Hv * D * 4);
 }
 
 } // namespace gdn
@@ -165,9 +165,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     p.A_log = params->A_log;
     p.dt_bias = params->dt_bias;
     p.norm_w = params->norm_w;
-    const size_t es = bf16 ? 2 : 4;
     p.ws_qk = workspace;
-    p.ws_v = (char *)workspace + round_up((size_t)total_tokens * 2 * p.Hk * p.D * es);
+    p.ws_v = (char *)workspace + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
 
     cudaStream_t s = (cudaStream_t)stream;
     const ProfileHook hook = take_profile_hook();

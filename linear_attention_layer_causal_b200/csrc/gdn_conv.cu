@@ -24,8 +24,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(kConvThreads)
 conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int batch,
                  int64_t N, const T *__restrict__ init_conv, const float *__restrict__ conv_w,
-                 int Hk, int Hv, float l2_eps, float q_scale, T *__restrict__ qk_out,
-                 T *__restrict__ v_out) {
+                 int Hk, int Hv, float l2_eps, float q_scale, float *__restrict__ qk_out,
+                 float *__restrict__ v_out) {
     constexpr int V = Vec16<T>::N;
     constexpr int LANES = D / V; // lanes per head
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "head must tile a warp");
@@ -75,19 +75,15 @@ conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int 
         ss = group_sum<LANES>(ss);
         if (!active)
             continue;
-        Vec16<T> o;
-        if (region < 2) {
-            const float f = rsqrtf(ss + l2_eps) * (region == 0 ? q_scale : 1.0f);
+        // q and k leave L2-normalised, v as is; all in float32 so that no
+        // rounding is added before the recurrence
+        const float f = region == 2 ? 1.0f : rsqrtf(ss + l2_eps) * (region == 0 ? q_scale : 1.0f);
+        float *dst = region < 2 ? qk_out + t * (2 * Hk * D) + cc
+                                : v_out + t * ((int64_t)Hv * D) + (cc - 2 * Hk * D);
 #pragma unroll
-            for (int i = 0; i < V; ++i)
-                o.set(i, acc[i] * f);
-            st16(qk_out + t * (2 * Hk * D) + cc, o);
-        } else {
-#pragma unroll
-            for (int i = 0; i < V; ++i)
-                o.set(i, acc[i]);
-            st16(v_out + t * ((int64_t)Hv * D) + (cc - 2 * Hk * D), o);
-        }
+        for (int i = 0; i < V; i += 4)
+            *reinterpret_cast<float4 *>(dst + i) =
+                make_float4(acc[i] * f, acc[i + 1] * f, acc[i + 2] * f, acc[i + 3] * f);
     }
 }
 
@@ -128,7 +124,7 @@ cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
               (C / V + kConvThreads - 1) / kConvThreads);
     conv_prep_kernel<T, D><<<grid, kConvThreads, 0, s>>>(
         (const T *)p.qkv, p.cu, p.batch, p.N, (const T *)p.init_conv, p.conv_w, p.Hk, p.Hv,
-        p.l2_eps, p.q_scale, (T *)p.ws_qk, (T *)p.ws_v);
+        p.l2_eps, p.q_scale, (float *)p.ws_qk, (float *)p.ws_v);
     return cudaGetLastError();
 }
 

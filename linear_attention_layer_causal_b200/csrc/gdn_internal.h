@@ -23,8 +23,8 @@ struct PrefillArgs {
     float *o_raw;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
     // workspace carve-up
-    void *ws_qk; // [N, 2*Hk*D] activation dtype: normalised q | k
-    void *ws_v;  // [N, Hv*D]   activation dtype: convolved v
+    void *ws_qk; // [N, 2*Hk*D] float32: normalised q | k
+    void *ws_v;  // [N, Hv*D]   float32: convolved v
 };
 
 struct DecodeArgs {

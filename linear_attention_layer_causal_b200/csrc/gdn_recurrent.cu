@@ -49,8 +49,8 @@ recurrent_prefill_kernel(PrefillArgs p) {
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
 
-    const T *qk = (const T *)p.ws_qk;
-    const T *vv = (const T *)p.ws_v;
+    const float *qk = (const float *)p.ws_qk;
+    const float *vv = (const float *)p.ws_v;
     const T *za = (const T *)p.z;
     const T *ga = (const T *)p.a;
     const T *gb = (const T *)p.b;
@@ -74,21 +74,17 @@ recurrent_prefill_kernel(PrefillArgs p) {
     for (int64_t b0 = 0; b0 < len; b0 += kTB) {
         const int nb = (len - b0) < kTB ? (int)(len - b0) : kTB;
         // ---- stage k, q, v of this batch as float, and the gates
-        constexpr int V = Vec16<T>::N;
-        for (int e = tid; e < kTB * (D / V); e += NT) {
-            const int tk = e / (D / V);
-            const int c = (e % (D / V)) * V;
+        for (int e = tid; e < kTB * (D / 4); e += NT) {
+            const int tk = e / (D / 4);
+            const int c = (e % (D / 4)) * 4;
             if (tk < nb) {
                 const int64_t t = start + b0 + tk;
-                Vec16<T> qx = ld16_nc(qk + t * QK + j * D + c);
-                Vec16<T> kx = ld16_nc(qk + t * QK + p.Hk * D + j * D + c);
-                Vec16<T> vx = ld16_nc(vv + t * HD + (int64_t)h * D + c);
-#pragma unroll
-                for (int i = 0; i < V; ++i) {
-                    sm.q[tk][c + i] = qx.get(i);
-                    sm.k[tk][c + i] = kx.get(i);
-                    sm.v[tk][c + i] = vx.get(i);
-                }
+                *reinterpret_cast<float4 *>(&sm.q[tk][c]) =
+                    __ldg(reinterpret_cast<const float4 *>(qk + t * QK + j * D + c));
+                *reinterpret_cast<float4 *>(&sm.k[tk][c]) =
+                    __ldg(reinterpret_cast<const float4 *>(qk + t * QK + p.Hk * D + j * D + c));
+                *reinterpret_cast<float4 *>(&sm.v[tk][c]) =
+                    __ldg(reinterpret_cast<const float4 *>(vv + t * HD + (int64_t)h * D + c));
             }
         }
         if (tid < nb) {

@@ -45,12 +45,13 @@ QWEN38 = gdn.Config(16, 128, 128)
 
 def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
-    # normalised q|k and convolved v, bf16, each region rounded to 256 bytes
-    assert n == 4096 * 2 * 16 * 128 * 2 + 4096 * 128 * 128 * 2
+    # normalised q|k and convolved v, float32, each region rounded to 256 bytes
+    assert n == 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
     tiny = gdn.Config(2, 4, 32, act_dtype="f32")
     assert gdn.prefill_workspace_size(tiny, 1, 3) == 1536 + 1536
     assert gdn.prefill_workspace_size(tiny, 1, 1) == 512 + 512
+    assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 1, 3) == 1536 + 1536
 
 
 @pytest.mark.parametrize("cfg,code", [

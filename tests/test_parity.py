@@ -63,10 +63,12 @@ def test_qwen38_prefill_all_heads(cuda_device):
     wl = W.QWEN38_PREFILL
     cfg = gdn.Config.of(wl)
     inp = W.make_prefill(wl, cuda_device)
-    out = _gpu_prefill(cfg, inp, return_final_state=True, return_final_conv=True)
+    out = _gpu_prefill(cfg, inp, return_final_state=True, return_final_conv=True,
+                       return_o_raw=True)
     torch.cuda.synchronize()
     ref = _oracle_seq(wl, inp, 0)
     assert_output_close(out["y"], ref["y"])
+    assert_output_close(out["o_raw"], ref["o"], "o_raw")
     assert_state_close(out["final_state"][0], ref["state"])
     np.testing.assert_array_equal(to64(out["final_conv"][0]), ref["conv_window"])
 
