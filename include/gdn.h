@@ -154,6 +154,44 @@ GDN_API gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, c
                       void *conv_cache, int32_t batch, void *y, void *stream);
 
 /*
+ * Size of the fixed device scratch array used by gdn_prefill_noalloc:
+ * 64 MiB, held on every GPU that loads the library until the process exits.
+ */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * gdn_prefill for callers that cannot allocate device memory.  (The pages
+ * have no counterpart of this entry point; it exists for integration.)
+ *
+ * Some callers cannot obtain device scratch at call time: a plugin hosted by
+ * a framework that owns all of the GPU's memory and hands it only the input
+ * and output buffers, or a latency-critical loop that must never call
+ * cudaMalloc/cudaFree, which can synchronise the whole device.  This entry
+ * point takes the same arguments as gdn_prefill minus the workspace; its
+ * scratch is one fixed array of GDN_NOALLOC_SCRATCH_BYTES inside the library,
+ * and it allocates nothing.
+ *
+ *   - Limit: a call whose gdn_prefill_workspace_size exceeds
+ *     GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_WORKSPACE before any CUDA
+ *     call (at the Qwen3.8 layer shape, 80 KiB per token: up to 819 tokens).
+ *   - Set-up: the first call on a device, with that device current, looks up
+ *     the array's device address (cudaGetSymbolAddress) and caches it; make
+ *     that first call before any stream capture.
+ *   - Sharing: every call on a device uses the same array, which keeps the
+ *     last call's contents.  Nothing in it needs to start at zero.  Calls
+ *     whose work overlaps on the GPU (different streams or host threads on
+ *     the same device) race on the array and give wrong results: order them.
+ * Returns what gdn_prefill returns, or GDN_ERR_CUDA if the address look-up
+ * fails.
+ */
+GDN_API gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_params *params,
+                                       const void *qkv, const void *a, const void *b,
+                                       const void *z, const int32_t *cu_seqlens, int32_t batch,
+                                       int64_t total_tokens, const float *initial_state,
+                                       const void *initial_conv, void *y, float *final_state,
+                                       void *final_conv, float *o_raw, void *stream);
+
+/*
  * Timing hook for benchmarks.  Arms a one-shot on the calling host thread:
  * the next gdn_prefill or gdn_decode call made by this thread records
  * `begin_event` on its stream immediately before launching its main kernel

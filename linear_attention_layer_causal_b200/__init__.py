@@ -32,7 +32,10 @@ GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUD
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_status_string",
-            "gdn_abi_version", "gdn_profile_next_call")
+            "gdn_abi_version", "gdn_profile_next_call", "gdn_prefill_noalloc")
+
+# Fixed scratch of gdn_prefill_noalloc (GDN_NOALLOC_SCRATCH_BYTES in include/gdn.h).
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class GdnError(RuntimeError):
@@ -99,6 +102,9 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, vp,
                                   vp, vp, sz, vp]
         L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_prefill_noalloc.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp,
+                                          vp, vp, vp, vp]
+        L.gdn_prefill_noalloc.restype = ctypes.c_int
         L.gdn_decode.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -205,6 +211,33 @@ def prefill(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_
     if o_raw is not None:
         out["o_raw"] = o_raw
     return out
+
+
+def prefill_noalloc(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_w, *,
+                    y, initial_state=None, initial_conv=None, final_state=None, final_conv=None,
+                    o_raw=None, stream=None) -> None:
+    """gdn_prefill_noalloc: prefill into caller-provided outputs with the library's
+    fixed internal scratch, for callers that cannot allocate device memory (a
+    plugin whose host framework owns the GPU's memory, a loop that must never
+    call cudaMalloc/cudaFree).  Nothing is allocated here or in the library.
+
+    Calls on one device share the scratch: calls that overlap on the GPU race.
+    The first call on a device looks up the scratch's address; make it before
+    any stream capture.  Raises GdnError if the call needs more than
+    NOALLOC_SCRATCH_BYTES of scratch (see prefill_workspace_size)."""
+    N = qkv.shape[0]
+    B = cu_seqlens.shape[0] - 1
+    st = lib().gdn_prefill_noalloc(ctypes.byref(cfg._c()),
+                                   ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                                   _ptr(qkv), _ptr(a), _ptr(b), _ptr(z), _ptr(cu_seqlens), B, N,
+                                   _ptr(initial_state), _ptr(initial_conv), _ptr(y),
+                                   _ptr(final_state), _ptr(final_conv), _ptr(o_raw),
+                                   _stream(stream))
+    if st == GDN_ERR_WORKSPACE:
+        raise GdnError(st, f"gdn_prefill_noalloc: needs {prefill_workspace_size(cfg, B, N)} bytes "
+                           f"of scratch, more than the fixed {NOALLOC_SCRATCH_BYTES}")
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill_noalloc")
 
 
 def decode(cfg: Config, qkv, a, b, z, state, conv_cache, conv_w, A_log, dt_bias, norm_w, *,

@@ -128,6 +128,22 @@ def test_decode_argument_errors():
     assert L.gdn_decode(None, ctypes.byref(par), *ok) == gdn.GDN_ERR_INVALID_ARG
 
 
+@no_gpu
+def test_noalloc_rejects_oversized_calls_on_the_host():
+    """The fixed-scratch prefill refuses, before any CUDA call, a call that needs
+    more than GDN_NOALLOC_SCRATCH_BYTES of scratch."""
+    L = gdn.lib()
+    cfg = gdn.Config(16, 128, 128)
+    P = 1 << 20
+    par = gdn._Params(P, P + 256, P + 512, P + 768)
+    args = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, 820, None, None, P * 7, None, None, None, None]
+    assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *args) == \
+        gdn.GDN_ERR_WORKSPACE
+    bad = gdn.Config(3, 4, 32)
+    assert L.gdn_prefill_noalloc(ctypes.byref(bad._c()), ctypes.byref(par), *args) == \
+        gdn.GDN_ERR_INVALID_ARG
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(gdn, "_lib", None)
     monkeypatch.setattr(gdn, "LIB_PATH", str(tmp_path / "libgdn.so"))
