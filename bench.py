@@ -202,7 +202,7 @@ def run_ours(args, rank, world, dev, dist):
 
     pk = peaks()
     wl = W.QWEN38_PREFILL
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, args.algo)
     inp = W.make_prefill(wl, dev, seed=wl.seed + 7919 * rank)
     P = [inp[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
     N, B = sum(inp["seqlens"]), len(inp["seqlens"])
@@ -263,9 +263,11 @@ def run_ours(args, rank, world, dev, dist):
     byts = prefill_bytes(cfg.num_qk_heads, cfg.num_v_heads, cfg.head_dim, N, B)
     tf = flops / (kern_ms_max / 1e3) / 1e12
     gbs = byts / (kern_ms_max / 1e3) / 1e9
-    roof = {"kernel": "recurrent_prefill_kernel", "bound": "tensor", "achieved": round(tf, 2),
+    kname = "chunk_prefill_kernel" if cfg.head_dim == 128 and cfg.algo != "serial" \
+        else "recurrent_prefill_kernel"
+    roof = {"kernel": kname, "bound": "tensor", "achieved": round(tf, 2),
             "peak": pk["bf16_tflops"], "unit": "TFLOP/s", "frac": round(tf / pk["bf16_tflops"], 4),
-            "traffic": traffic_of("recurrent_prefill_kernel"),
+            "traffic": traffic_of(kname),
             "algorithmic_flops": flops, "kernel_ms": round(kern_ms_max, 4),
             "peak_source": pk["source"] + " burst bf16",
             "hbm_view": {"achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -307,7 +309,8 @@ def run_ours(args, rank, world, dev, dist):
                        "global_batch": world, "seq_len": N, "parallelism": f"replicas x{world}",
                        "l2": "no flush: inputs of one step (~447 MB) exceed the 126 MB L2"},
             "roofline": roof, "decode": decode, "e2e": e2e,
-            "gpu_launches": 2 * args.steps, "clocks": clk}
+            "gpu_launches": (3 if kname == "chunk_prefill_kernel" else 2) * args.steps,
+            "clocks": clk}
     return line
 
 
@@ -353,6 +356,8 @@ def main():
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="run only one part (for profiling small cases)")
     ap.add_argument("--decode-batch", type=int, default=256)
+    ap.add_argument("--algo", default="auto", choices=["auto", "chunked", "serial"],
+                    help="prefill algorithm (auto = tensor-core chunks at head dim 128)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

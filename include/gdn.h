@@ -84,7 +84,15 @@ typedef struct gdn_config {
     float l2_eps;         /* epsilon inside the q/k L2 norm: x / sqrt(sum x^2 + l2_eps) */
     float q_scale;        /* extra factor on normalised q (1.0 = none) */
     int32_t act_dtype;    /* gdn_dtype of qkv, a, b, z, y and the conv caches */
+    int32_t algo;         /* gdn_algo: prefill algorithm (GDN_ALGO_AUTO = 0 is right for most callers) */
 } gdn_config;
+
+/* Prefill algorithm.  Both compute the same recurrence; decode ignores it. */
+typedef enum gdn_algo {
+    GDN_ALGO_AUTO = 0,    /* chunked for head_dim 128, token-serial otherwise */
+    GDN_ALGO_SERIAL = 1,  /* token-serial FP32 recurrence on CUDA cores (any head_dim) */
+    GDN_ALGO_CHUNKED = 2  /* 64-token chunks on the tensor cores (head_dim 128 only) */
+} gdn_algo;
 
 /* Layer parameters, all float32 device arrays. */
 typedef struct gdn_params {
@@ -124,7 +132,11 @@ GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t bat
  *                                    may equal initial_conv
  *   o_raw         [N, H_v, d]        float32 pre-norm recurrence output, or NULL
  *   workspace     device scratch of at least gdn_prefill_workspace_size bytes,
- *                 256-byte aligned; its contents on entry do not matter.
+ *                 256-byte aligned; its contents on entry do not matter.  Its
+ *                 first 4 bytes become a status word: 0 after a successful
+ *                 call; nonzero if a wait inside a kernel gave up (the call's
+ *                 outputs are then invalid).  Read it after the stream work
+ *                 has completed.
  * The values of cu_seqlens are read on the device only; a cu_seqlens array
  * that breaks the rules above gives unspecified output (never an
  * out-of-bounds access outside [0, N) rows).
@@ -173,7 +185,7 @@ GDN_API gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, c
  *
  *   - Limit: a call whose gdn_prefill_workspace_size exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_WORKSPACE before any CUDA
- *     call (at the Qwen3.8 layer shape, 80 KiB per token: up to 819 tokens).
+ *     call (at the Qwen3.8 layer shape, 88 KiB per token: up to 744 tokens).
  *   - Set-up: the first call on a device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
  *     that first call before any stream capture.

@@ -48,7 +48,8 @@ class _Config(ctypes.Structure):
     _fields_ = [("num_qk_heads", ctypes.c_int32), ("num_v_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("conv_kernel", ctypes.c_int32),
                 ("rms_eps", ctypes.c_float), ("l2_eps", ctypes.c_float),
-                ("q_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32)]
+                ("q_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32),
+                ("algo", ctypes.c_int32)]
 
 
 class _Params(ctypes.Structure):
@@ -67,6 +68,7 @@ class Config:
     l2_eps: float = 1e-6
     q_scale: float = 1.0
     act_dtype: str = "bf16"  # "bf16" or "f32"
+    algo: str = "auto"       # prefill algorithm: "auto", "serial" or "chunked"
 
     @property
     def conv_dim(self) -> int:
@@ -75,13 +77,14 @@ class Config:
     def _c(self) -> _Config:
         return _Config(self.num_qk_heads, self.num_v_heads, self.head_dim, self.conv_kernel,
                        self.rms_eps, self.l2_eps, self.q_scale,
-                       GDN_BF16 if self.act_dtype == "bf16" else GDN_F32)
+                       GDN_BF16 if self.act_dtype == "bf16" else GDN_F32,
+                       {"auto": 0, "serial": 1, "chunked": 2}[self.algo])
 
     @staticmethod
-    def of(wl) -> "Config":
+    def of(wl, algo: str = "auto") -> "Config":
         """The Config of a workloads.Workload."""
         return Config(wl.num_qk_heads, wl.num_v_heads, wl.head_dim, wl.conv_kernel,
-                      act_dtype=wl.dtype)
+                      act_dtype=wl.dtype, algo=algo)
 
 
 _lib = None
@@ -159,6 +162,14 @@ def profile_next_call(begin_event, end_event) -> None:
         raise GdnError(st, "gdn_profile_next_call")
 
 
+def workspace_status(workspace) -> int:
+    """The status word a prefill call left in its workspace (0 = ok); synchronises."""
+    import torch
+    if workspace is None or workspace.numel() < 4:
+        return 0
+    return int(workspace[:4].view(torch.int32).item())
+
+
 def prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
     n = ctypes.c_size_t(0)
     st = lib().gdn_prefill_workspace_size(ctypes.byref(cfg._c()), batch, total_tokens,
@@ -171,12 +182,14 @@ def prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
 def prefill(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_w, *,
             initial_state=None, initial_conv=None, return_final_state=False,
             return_final_conv=False, return_o_raw=False, y=None, final_state=None,
-            final_conv=None, workspace=None, stream=None) -> dict:
+            final_conv=None, workspace=None, stream=None, check_status=False) -> dict:
     """Packed varlen prefill (see gdn_prefill in include/gdn.h).
 
     Returns a dict with "y" and, when requested, "final_state", "final_conv"
     and "o_raw".  Output buffers and the workspace may be passed in to avoid
     allocation; ``final_state`` may be ``initial_state`` for an in-place update.
+    With ``check_status`` the call synchronises and raises if a kernel reported
+    a failure in the workspace status word.
     """
     import torch
     N = qkv.shape[0]
@@ -203,6 +216,8 @@ def prefill(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_
                            _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill")
+    if check_status and workspace_status(workspace) != 0:
+        raise GdnError(GDN_ERR_CUDA, f"gdn_prefill: device status {workspace_status(workspace)}")
     out = {"y": y}
     if final_state is not None:
         out["final_state"] = final_state

@@ -33,6 +33,10 @@ gdn_status check_config(const gdn_config *c) {
         return GDN_ERR_UNSUPPORTED;
     if (c->num_v_heads / c->num_qk_heads > 64)
         return GDN_ERR_UNSUPPORTED;
+    if (c->algo < GDN_ALGO_AUTO || c->algo > GDN_ALGO_CHUNKED)
+        return GDN_ERR_INVALID_ARG;
+    if (c->algo == GDN_ALGO_CHUNKED && c->head_dim != 128)
+        return GDN_ERR_UNSUPPORTED;
     // conv_dim * 16-byte channel groups must index in int
     const int64_t conv_dim = (int64_t)(2 * (int64_t)c->num_qk_heads + c->num_v_heads) * c->head_dim;
     if (conv_dim > (int64_t)1 << 26)
@@ -67,9 +71,13 @@ ProfileHook take_profile_hook() {
     return h;
 }
 
+// Header (status word), float32 normalised q|k, float32 convolved v and, for
+// head_dim 128, the chunk Gram rows of the chunked path.
 size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N) {
-    // float32 normalised q|k and convolved v
-    return round_up((size_t)N * 2 * Hk * D * 4) + round_up((size_t)N * Hv * D * 4);
+    if (N == 0)
+        return 0;
+    return kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4) +
+           round_up((size_t)N * Hv * D * 4) + (D == 128 ? round_up(kq_workspace_bytes(Hk, N)) : 0);
 }
 
 } // namespace gdn
@@ -165,18 +173,26 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     p.A_log = params->A_log;
     p.dt_bias = params->dt_bias;
     p.norm_w = params->norm_w;
-    p.ws_qk = workspace;
-    p.ws_v = (char *)workspace + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
+    p.chunked = p.D == 128 && cfg->algo != GDN_ALGO_SERIAL;
+    if (need > 0) {
+        char *w = (char *)workspace;
+        p.ws_err = (unsigned int *)w;
+        p.ws_qk = w + kWorkspaceHeader;
+        p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
+        p.ws_kq = (char *)p.ws_v + round_up((size_t)total_tokens * p.Hv * p.D * 4);
+    }
 
     cudaStream_t s = (cudaStream_t)stream;
     const ProfileHook hook = take_profile_hook();
     if (batch == 0)
         return GDN_OK;
     cudaError_t e = launch_conv_prep(p, s);
+    if (e == cudaSuccess && p.chunked)
+        e = launch_kq_prep(p, s);
     if (e == cudaSuccess)
         e = record_if(hook.begin, s);
     if (e == cudaSuccess)
-        e = launch_recurrent_prefill(p, s);
+        e = p.chunked ? launch_chunk_prefill(p, s) : launch_recurrent_prefill(p, s);
     if (e == cudaSuccess)
         e = record_if(hook.end, s);
     if (e == cudaSuccess)

@@ -25,11 +25,13 @@ __global__ void __launch_bounds__(kConvThreads)
 conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int batch,
                  int64_t N, const T *__restrict__ init_conv, const float *__restrict__ conv_w,
                  int Hk, int Hv, float l2_eps, float q_scale, float *__restrict__ qk_out,
-                 float *__restrict__ v_out) {
+                 float *__restrict__ v_out, unsigned int *__restrict__ err) {
     constexpr int V = Vec16<T>::N;
     constexpr int LANES = D / V; // lanes per head
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "head must tile a warp");
     const int C = (2 * Hk + Hv) * D;
+    if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        *err = 0u; // status word of this call; later kernels only set bits
     const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * V;
     const bool active = c0 < C;
     const int cc = active ? c0 : 0; // inactive lanes still join the shuffles
@@ -124,7 +126,7 @@ cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
               (C / V + kConvThreads - 1) / kConvThreads);
     conv_prep_kernel<T, D><<<grid, kConvThreads, 0, s>>>(
         (const T *)p.qkv, p.cu, p.batch, p.N, (const T *)p.init_conv, p.conv_w, p.Hk, p.Hv,
-        p.l2_eps, p.q_scale, (float *)p.ws_qk, (float *)p.ws_v);
+        p.l2_eps, p.q_scale, (float *)p.ws_qk, (float *)p.ws_v, p.ws_err);
     return cudaGetLastError();
 }
 

@@ -22,9 +22,12 @@ struct PrefillArgs {
     void *final_conv;
     float *o_raw;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
+    bool chunked;            // tensor-core chunked path (head_dim 128) or token-serial
     // workspace carve-up
-    void *ws_qk; // [N, 2*Hk*D] float32: normalised q | k
-    void *ws_v;  // [N, Hv*D]   float32: convolved v
+    unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)
+    void *ws_qk;             // [N, 2*Hk*D] float32: normalised q | k
+    void *ws_v;              // [N, Hv*D]   float32: convolved v
+    void *ws_kq;             // [N, Hk, 2, 64] float32: chunk Gram rows (chunked path)
 };
 
 struct DecodeArgs {
@@ -52,10 +55,14 @@ inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
 
 // Workspace bytes for the prefill path (each region 256-byte aligned).
 size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N);
+constexpr size_t kWorkspaceHeader = 256; // holds the device status word
 
 cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_final_conv(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_recurrent_prefill(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_chunk_prefill(const PrefillArgs &p, cudaStream_t s);
+size_t kq_workspace_bytes(int Hk, int64_t N);
 cudaError_t launch_decode(const DecodeArgs &p, cudaStream_t s);
 
 } // namespace gdn

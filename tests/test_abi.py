@@ -45,13 +45,14 @@ QWEN38 = gdn.Config(16, 128, 128)
 
 def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
-    # normalised q|k and convolved v, float32, each region rounded to 256 bytes
-    assert n == 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4
+    # 256-byte header (status word), float32 normalised q|k and convolved v, and
+    # for head_dim 128 the chunk Gram rows [N, H_k, 2, 64]; regions rounded to 256 B
+    assert n == 256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 2 * 64 * 4
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
     tiny = gdn.Config(2, 4, 32, act_dtype="f32")
-    assert gdn.prefill_workspace_size(tiny, 1, 3) == 1536 + 1536
-    assert gdn.prefill_workspace_size(tiny, 1, 1) == 512 + 512
-    assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 1, 3) == 1536 + 1536
+    assert gdn.prefill_workspace_size(tiny, 1, 3) == 256 + 1536 + 1536
+    assert gdn.prefill_workspace_size(tiny, 1, 1) == 256 + 512 + 512
+    assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 1, 3) == 256 + 1536 + 1536
 
 
 @pytest.mark.parametrize("cfg,code", [
@@ -61,10 +62,19 @@ def test_workspace_size_arithmetic():
     (gdn.Config(2, 4, 32, conv_kernel=3), gdn.GDN_ERR_UNSUPPORTED),
     (gdn.Config(2, 4, 32, rms_eps=-1.0), gdn.GDN_ERR_INVALID_ARG),
     (gdn.Config(2, 4, 32, l2_eps=float("nan")), gdn.GDN_ERR_INVALID_ARG),
+    (gdn.Config(2, 4, 32, algo="chunked"), gdn.GDN_ERR_UNSUPPORTED),  # chunked needs d = 128
 ])
 def test_bad_config_rejected(cfg, code):
     n = ctypes.c_size_t(0)
     assert gdn.lib().gdn_prefill_workspace_size(ctypes.byref(cfg._c()), 1, 10, ctypes.byref(n)) == code
+
+
+def test_unknown_algo_rejected():
+    c = gdn.Config(2, 4, 32)._c()
+    c.algo = 3
+    n = ctypes.c_size_t(0)
+    assert gdn.lib().gdn_prefill_workspace_size(ctypes.byref(c), 1, 10, ctypes.byref(n)) == \
+        gdn.GDN_ERR_INVALID_ARG
 
 
 def _fake_call(**over):
@@ -136,7 +146,7 @@ def test_noalloc_rejects_oversized_calls_on_the_host():
     cfg = gdn.Config(16, 128, 128)
     P = 1 << 20
     par = gdn._Params(P, P + 256, P + 512, P + 768)
-    args = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, 820, None, None, P * 7, None, None, None, None]
+    args = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, 745, None, None, P * 7, None, None, None, None]
     assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *args) == \
         gdn.GDN_ERR_WORKSPACE
     bad = gdn.Config(3, 4, 32)

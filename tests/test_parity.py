@@ -26,8 +26,13 @@ def _shape(wl):
 
 
 def _gpu_prefill(cfg, inp, **kw):
+    kw.setdefault("check_status", True)
     return gdn.prefill(cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["cu_seqlens"],
                        *[inp[k] for k in PARAMS], initial_state=inp.get("initial_state"), **kw)
+
+
+# the two prefill algorithms for head_dim 128: tensor-core chunks and token-serial
+ALGOS = pytest.mark.parametrize("algo", ["chunked", "serial"])
 
 
 def _oracle_seq(wl, inp, n, group=None, heads=None, conv=None):
@@ -58,10 +63,11 @@ def test_tiny_layer_full(cuda_device):
     assert_state_close(out["final_state"][0], ref["state"], rel=1e-4)
 
 
-def test_qwen38_prefill_all_heads(cuda_device):
+@ALGOS
+def test_qwen38_prefill_all_heads(cuda_device, algo):
     """Qwen3.8 layer, B = 1, T = 4096, bf16: every value head against the oracle."""
     wl = W.QWEN38_PREFILL
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     out = _gpu_prefill(cfg, inp, return_final_state=True, return_final_conv=True,
                        return_o_raw=True)
@@ -73,10 +79,11 @@ def test_qwen38_prefill_all_heads(cuda_device):
     np.testing.assert_array_equal(to64(out["final_conv"][0]), ref["conv_window"])
 
 
-def test_qwen38_long_prefill_sampled(cuda_device):
+@ALGOS
+def test_qwen38_long_prefill_sampled(cuda_device, algo):
     """Qwen3.8 layer, B = 4 x T = 16384 with N(0, 0.02) initial states: sampled heads."""
     wl = W.QWEN38_LONG
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     out = _gpu_prefill(cfg, inp, return_final_state=True, return_final_conv=True)
     torch.cuda.synchronize()
@@ -112,10 +119,11 @@ def test_qwen38_decode_sampled(cuda_device):
     np.testing.assert_array_equal(to64(inp["conv_cache"][seqs]), ref["conv_window"])
 
 
-def test_qwen36_varlen_sampled(cuda_device):
+@ALGOS
+def test_qwen36_varlen_sampled(cuda_device, algo):
     """64 packed sequences with lengths U[256, 8192], 16 q/k / 32 value heads: sampled units."""
     wl = W.QWEN36_VARLEN
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     lens = inp["seqlens"]
     out = _gpu_prefill(cfg, inp, return_final_state=True)
@@ -136,11 +144,12 @@ EDGE = W.Workload("edge", 2, 4, 128, seqlens=(0, 1, 2, 3, 5, 33, 64, 0, 100, 31)
                   seed=77)
 
 
+@ALGOS
 @pytest.mark.parametrize("with_conv", [False, True])
-def test_edge_lengths_full(cuda_device, with_conv):
+def test_edge_lengths_full(cuda_device, with_conv, algo):
     """Empty, shorter-than-window and ragged sequences, with and without incoming conv windows."""
     wl = EDGE
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     B = len(wl.seqlens)
     conv = None
@@ -164,10 +173,11 @@ def test_edge_lengths_full(cuda_device, with_conv):
         assert torch.equal(out["final_state"][n], inp["initial_state"][n])
 
 
-def test_in_place_state_and_conv(cuda_device):
+@ALGOS
+def test_in_place_state_and_conv(cuda_device, algo):
     """final_state = initial_state and final_conv = initial_conv give the out-of-place result."""
     wl = EDGE
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     B = len(wl.seqlens)
     g = torch.Generator(device=cuda_device).manual_seed(6)
@@ -184,11 +194,12 @@ def test_in_place_state_and_conv(cuda_device):
     assert torch.equal(C, ref["final_conv"])
 
 
-def test_split_prefill_and_decode_continue_the_sequence(cuda_device):
+@ALGOS
+def test_split_prefill_and_decode_continue_the_sequence(cuda_device, algo):
     """prefill [0, T1) + prefill [T1, T) with carried state and conv window, then decode one
     token, equals prefill [0, T + 1) -- all on the device."""
     wl = W.Workload("cont", 4, 16, 128, seqlens=(301,), state_std=0.02, seed=91)
-    cfg = gdn.Config.of(wl)
+    cfg = gdn.Config.of(wl, algo)
     inp = W.make_prefill(wl, cuda_device)
     T1, T = 130, 300
     P = [inp[k] for k in PARAMS]
@@ -210,6 +221,10 @@ def test_split_prefill_and_decode_continue_the_sequence(cuda_device):
                     cache, *P)
     torch.cuda.synchronize()
     ys = torch.cat([p1["y"], p2["y"], y1])
-    assert_output_close(ys, whole["y"], "continued y", rel=2e-3, mx=1e-2)
-    assert_state_close(state, whole["final_state"], "continued state", rel=1e-4)
+    # the two runs split the sequence at different chunk boundaries, so with
+    # tf32 products they agree to rounding level only
+    tight = algo == "serial"
+    assert_output_close(ys, whole["y"], "continued y", rel=2e-3 if tight else 5e-3,
+                        mx=1e-2 if tight else 2e-2)
+    assert_state_close(state, whole["final_state"], "continued state", rel=1e-4 if tight else 2e-3)
     assert torch.equal(cache[0], inp["qkv"][T - 2:T + 1])

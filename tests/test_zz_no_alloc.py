@@ -55,16 +55,16 @@ def test_noalloc_matches_prefill_on_consecutive_calls(cuda_device):
 
 
 def test_noalloc_largest_call_and_limit(cuda_device):
-    """At the Qwen3.8 layer shape the fixed scratch holds 819 tokens: 819 runs and
-    matches gdn_prefill, 820 is rejected before anything is launched."""
-    wl = W.Workload("noalloc_max", 16, 128, 128, seqlens=(819,), state_std=0.02, seed=3)
+    """At the Qwen3.8 layer shape the fixed scratch holds 744 tokens: 744 runs and
+    matches gdn_prefill, 745 is rejected before anything is launched."""
+    wl = W.Workload("noalloc_max", 16, 128, 128, seqlens=(744,), state_std=0.02, seed=3)
     cfg = gdn.Config.of(wl)
-    assert gdn.prefill_workspace_size(cfg, 1, 819) <= gdn.NOALLOC_SCRATCH_BYTES
-    assert gdn.prefill_workspace_size(cfg, 1, 820) > gdn.NOALLOC_SCRATCH_BYTES
+    assert gdn.prefill_workspace_size(cfg, 1, 744) <= gdn.NOALLOC_SCRATCH_BYTES
+    assert gdn.prefill_workspace_size(cfg, 1, 745) > gdn.NOALLOC_SCRATCH_BYTES
     inp = W.make_prefill(wl, cuda_device)
     _check(*_both(cfg, inp))
-    big = W.make_prefill(wl, cuda_device, seqlens=(820,), seed=4)
-    y = torch.empty((820, 128, 128), dtype=torch.bfloat16, device=cuda_device)
+    big = W.make_prefill(wl, cuda_device, seqlens=(745,), seed=4)
+    y = torch.empty((745, 128, 128), dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(gdn.GdnError) as e:
         gdn.prefill_noalloc(cfg, big["qkv"], big["a"], big["b"], big["z"], big["cu_seqlens"],
                             *[big[k] for k in P], y=y)
