@@ -33,6 +33,8 @@
 //
 // The gated RMSNorm y = o / rms(o) * w * SiLU(z) ("Qwen3.8-2.4T-A95B vs
 // Inkling", output-gate row) is fused into the output store.
+#include <cuda.h>
+
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
@@ -142,11 +144,12 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
 constexpr int kThreads = 128; // 4 warps: thread i owns TMEM lane i (= value channel i)
 
 // TMEM columns
-constexpr uint32_t kColS = 0;    // state S, 128 columns
+constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns
 constexpr uint32_t kColU = 128;  // U^T (starts as U~^T), 64 columns
 constexpr uint32_t kColO = 192;  // O^T, 64 columns
 constexpr uint32_t kColW = 256;  // W^T, 64 columns
-constexpr uint32_t kColSr = 320; // S rounded to tf32 (the A operand), 128 columns
+constexpr uint32_t kColSr = 320; // S rounded to tf32 (A operand of the state products), 128
+constexpr uint32_t kColUk = 448; // U^T diag(gamma_C / gamma) rounded to tf32, 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 // Both operand layouts below split a tile of R rows along its contiguous
@@ -163,52 +166,82 @@ __device__ __forceinline__ int swz_mn(int k, int c, int R) {
     return (c >> 5) * (R * 32) + k * 32 + ((((c & 31) >> 3) ^ (k & 3)) << 3) + (c & 7);
 }
 
-struct __align__(1024) ChunkSmem {
-    float V[kC * kD];  // A, MN-major: V^T
-    float K[kC * kD];  // A, MN-major: K^T; then B, K-major: -W (same bytes, rewritten)
-    float Q[kC * kD];  // B, K-major: diag(gamma) Q
-    float Kp[kC * kD]; // B, MN-major: diag(gamma_C / gamma) K
-    float Tb[kC * kC]; // B, K-major: T diag(beta)
-    float Tg[kC * kC]; // B, K-major: T diag(beta gamma)
-    float P[kC * kC];  // B, K-major: P
-    float A[kC][kC + 1];
-    float g[kC], beta[kC], G[kC];
+template <typename T> struct __align__(1024) ChunkSmem {
+    float V[kC * kD];     // A, MN-major: V^T of this chunk; after MMA 1, B K-major: -W
+    float Q[kC * kD];     // B, K-major: Q
+    float K[2][kC * kD];  // A / B, MN-major: K of this chunk and the next (ping-pong)
+    float Tb[kC * kC];    // B, K-major: T diag(beta)
+    float Tg[kC * kC];    // B, K-major: T diag(beta gamma)
+    float P[kC * kC];     // B, K-major: P (lands as raw Q K^T rows)
+    float A[kC * kC];     // the next chunk's A (lands as raw K K^T rows), then T; K-major swizzle
+    T Z[sizeof(T) == 2 ? kC * kD : 1]; // z rows of this chunk (16-bit activations only)
+    float G[2][kC], beta[2][kC]; // cumulative log-decay and beta, this chunk / next
+    float gam[2][kC], kd[2][kC];  // gamma_r = e^{G_r} and gamma_C / gamma_r
+    float scan[2];
     float red[4][kC];
     float rstd[kC];
-    unsigned long long bar;
+    unsigned long long bar_mma;
+    unsigned long long bar_v, bar_q, bar_k[2], bar_p, bar_a, bar_z;
     uint32_t tmem;
-    int abort;
 };
 
 constexpr long long kWaitLimit = 2000000000LL; // ~1 s of SM cycles
 
+// Rounds a float32 tile of `n` floats to tf32 in place (elementwise, any layout).
+template <int NF> __device__ __forceinline__ void round_tile(float *t, int tid) {
+#pragma unroll 4
+    for (int e = tid; e < NF / 4; e += kThreads) {
+        float4 *p4 = reinterpret_cast<float4 *>(t) + e;
+        *p4 = sm100::tf32_rna(*p4);
+    }
+}
+
+// The tensor maps of one call: 64-row boxes of the workspace and of z.
+struct ChunkMaps {
+    CUtensorMap v;  // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle
+    CUtensorMap k;  // normalised k, [N, Hk*128] of the q|k rows, 32-column boxes, MN-major swizzle
+    CUtensorMap q;  // normalised q, [N, Hk*128], 32-column boxes, 128-byte swizzle (K-major)
+    CUtensorMap kq; // Gram rows, [N, Hk*128] fp32, 32-column boxes, 128-byte swizzle
+    CUtensorMap z;  // z, [N, Hv*128] 16-bit, 128-column boxes, no swizzle
+};
+
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs p) {
+__global__ void __launch_bounds__(kThreads, 1)
+chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     using namespace sm100;
     extern __shared__ unsigned char chunk_smem_raw[];
-    ChunkSmem &sm = *reinterpret_cast<ChunkSmem *>(
+    ChunkSmem<T> &sm = *reinterpret_cast<ChunkSmem<T> *>(
         (reinterpret_cast<uintptr_t>(chunk_smem_raw) + 1023) & ~uintptr_t(1023));
 
     const int h = blockIdx.x;
     const int n = blockIdx.y;
     const int j = h / p.G;
     const int tid = threadIdx.x;
-    const int warp = tid >> 5;
+    const int warp = tid >> 5, lane = tid & 31;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
+    const int nchunks = (int)((len + kC - 1) / kC);
 
-    const float *qkw = (const float *)p.ws_qk;
-    const float *vw = (const float *)p.ws_v;
-    const float *kqw = (const float *)p.ws_kq;
-    const int QKW = 2 * p.Hk * kD;
     const int64_t HD = (int64_t)p.Hv * kD;
 
-    const uint32_t bar = smem_u32(&sm.bar);
+    const uint32_t bar_mma = smem_u32(&sm.bar_mma);
+    const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
+    const uint32_t bar_p = smem_u32(&sm.bar_p), bar_a = smem_u32(&sm.bar_a);
+    const uint32_t bar_z = smem_u32(&sm.bar_z);
+    const uint32_t bar_k0 = smem_u32(&sm.bar_k[0]), bar_k1 = smem_u32(&sm.bar_k[1]);
     if (tid == 0) {
-        mbar_init(bar, 1);
-        sm.abort = 0;
+        mbar_init(bar_mma, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_k0, 1);
+        mbar_init(bar_k1, 1);
+        mbar_init(bar_p, 1);
+        mbar_init(bar_a, 1);
+        mbar_init(bar_z, 1);
     }
+    if (tid == 0)
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     if (warp == 0) {
         tmem_alloc(smem_u32(&sm.tmem), kTmemCols);
         tmem_relinquish();
@@ -217,12 +250,11 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16; // this warp's TMEM lanes
-    const uint32_t tS = tmem + lane_base + kColS, tO = tmem + lane_base + kColO;
-    const uint32_t tW = tmem + lane_base + kColW, tU = tmem + lane_base + kColU;
-    const uint32_t tSr = tmem + lane_base + kColSr;
+    const uint32_t lb = (uint32_t)(warp * 32) << 16; // this warp's TMEM lanes
+    uint32_t ph_mma = 0, ph_v = 0, ph_q = 0, ph_k0 = 0, ph_k1 = 0, ph_p = 0, ph_a = 0, ph_z = 0;
+    bool ok = true;
 
-    // ---- initial state: row tid of S0 into TMEM lane tid
+    // ---- initial state into TMEM (row tid = lane tid), with its tf32 copy
     {
         const float *src = p.init_state ? p.init_state + (((size_t)n * p.Hv + h) * kD + tid) * kD
                                         : nullptr;
@@ -235,107 +267,283 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
                                : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
             }
-            tmem_st32(tS + cb * 32, v);
+            tmem_st32(tmem + lb + kColS + cb * 32, v);
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 v[i] = tf32_rna(v[i]);
-            tmem_st32(tSr + cb * 32, v);
+            tmem_st32(tmem + lb + kColSr + cb * 32, v);
         }
         tmem_wait_st();
     }
     const float negA = -expf(__ldg(p.A_log + h));
     const float dtb = __ldg(p.dt_bias + h);
     const float wn = __ldg(p.norm_w + tid);
-    uint32_t phase = 0;
-    bool ok = true;
 
-    const uint32_t aV = smem_u32(sm.V), aK = smem_u32(sm.K), aQ = smem_u32(sm.Q);
-    const uint32_t aKp = smem_u32(sm.Kp), aTb = smem_u32(sm.Tb), aTg = smem_u32(sm.Tg);
-    const uint32_t aP = smem_u32(sm.P);
-    constexpr uint32_t kBlk = kC * 128; // bytes per 32-column block of a 64-row tile
-
-    for (int64_t c0 = 0; c0 < len && ok; c0 += kC) {
-        const int nr = (len - c0) < kC ? (int)(len - c0) : kC;
-        const int64_t t0 = start + c0;
-        // ---- gates and the cumulative log-decay of the chunk
+    auto rows_of = [&](int c) { return (int)((len - (int64_t)c * kC) < kC ? (len - (int64_t)c * kC) : kC); };
+    // gate inputs of chunk c, row tid (threads < 64); zero beyond the sequence
+    auto load_ab = [&](int c, float &av, float &bv) {
+        av = 0.f;
+        bv = 0.f;
+        if (tid < kC && c < nchunks && tid < rows_of(c)) {
+            const int64_t t = start + (int64_t)c * kC + tid;
+            av = to_f(((const T *)p.a)[t * p.Hv + h]);
+            bv = to_f(((const T *)p.b)[t * p.Hv + h]);
+        }
+    };
+    // g, beta and the inclusive prefix G of a chunk into slot `sl` (threads < 64)
+    auto gates = [&](int c, float av, float bv, int sl) {
         if (tid < kC) {
-            float g = 0.f, be = 0.f;
-            if (tid < nr) {
-                const int64_t t = t0 + tid;
-                g = negA * softplusf_(to_f(((const T *)p.a)[t * p.Hv + h]) + dtb);
-                be = sigmoidf_(to_f(((const T *)p.b)[t * p.Hv + h]));
-            }
-            sm.g[tid] = g;
-            sm.beta[tid] = be;
-        }
-        __syncthreads();
-        if (tid < kC) {
-            float acc = 0.f;
-            for (int i = 0; i <= tid; ++i)
-                acc += sm.g[i];
-            sm.G[tid] = acc;
-        }
-        __syncthreads();
-        const float Glast = sm.G[kC - 1]; // padded rows carry g = 0
-        // ---- operand tiles
-        for (int e = tid; e < kC * (kD / 4); e += kThreads) {
-            const int r = e / (kD / 4), c = (e % (kD / 4)) * 4;
-            float4 vv = make_float4(0.f, 0.f, 0.f, 0.f), kk = vv, qq = vv;
-            if (r < nr) {
-                const int64_t t = t0 + r;
-                vv = __ldg(reinterpret_cast<const float4 *>(vw + t * HD + (int64_t)h * kD + c));
-                kk = __ldg(reinterpret_cast<const float4 *>(qkw + t * QKW + p.Hk * kD + j * kD + c));
-                qq = __ldg(reinterpret_cast<const float4 *>(qkw + t * QKW + j * kD + c));
-            }
-            const float gam = expf(sm.G[r]);
-            const float kpf = expf(Glast - sm.G[r]);
-            const int o = swz(r, c, kC), om = swz_mn(r, c, kC); // 4 floats stay contiguous
-            *reinterpret_cast<float4 *>(sm.V + om) = tf32_rna(vv);
-            *reinterpret_cast<float4 *>(sm.K + om) = tf32_rna(kk);
-            *reinterpret_cast<float4 *>(sm.Q + o) =
-                tf32_rna(make_float4(qq.x * gam, qq.y * gam, qq.z * gam, qq.w * gam));
-            *reinterpret_cast<float4 *>(sm.Kp + om) =
-                tf32_rna(make_float4(kk.x * kpf, kk.y * kpf, kk.z * kpf, kk.w * kpf));
-        }
-        for (int e = tid; e < kC * kC; e += kThreads) {
-            const int r = e / kC, s = e % kC;
-            float a = 0.f, pv = 0.f;
-            if (r < nr && s <= r) {
-                const float *row = kqw + ((t0 + r) * p.Hk + j) * (2 * kC);
-                const float dec = expf(sm.G[r] - sm.G[s]);
-                pv = dec * __ldg(row + kC + s);
-                if (s < r)
-                    a = sm.beta[r] * dec * __ldg(row + s);
-            }
-            sm.A[r][s] = a;
-            sm.P[swz(r, s, kC)] = tf32_rna(pv);
-        }
-        __syncthreads();
-        // ---- T = (I + A)^-1 by forward substitution, one column per thread
-        if (tid < kC) {
-            const int c = tid;
-            float Tc[kC];
+            const bool in = c < nchunks && tid < rows_of(c);
+            float g = in ? negA * softplusf_(av + dtb) : 0.f;
+            const float be = in ? sigmoidf_(bv) : 0.f;
 #pragma unroll
-            for (int r = 0; r < kC; ++r) {
+            for (int o = 1; o < 32; o <<= 1) {
+                const float x = __shfl_up_sync(0xffffffffu, g, o);
+                if (lane >= o)
+                    g += x;
+            }
+            if (tid == 31)
+                sm.scan[0] = g;
+            sm.beta[sl][tid] = be;
+            sm.G[sl][tid] = g; // warp 1 adds warp 0's total below
+        }
+        __syncthreads();
+        if (tid >= 32 && tid < kC)
+            sm.G[sl][tid] += sm.scan[0];
+        __syncthreads();
+        if (tid < kC) {
+            const float Gr = sm.G[sl][tid];
+            sm.gam[sl][tid] = expf(Gr);
+            sm.kd[sl][tid] = expf(sm.G[sl][kC - 1] - Gr);
+        }
+    };
+    // K K^T rows of the slot's chunk -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
+    auto build_A = [&](int sl) {
+#pragma unroll
+        for (int e = tid; e < kC * kC / 4; e += kThreads) {
+            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+            float4 *p4 = reinterpret_cast<float4 *>(sm.A + swz(r, c, kC));
+            float4 x = *p4;
+            const float br = sm.beta[sl][r], Gr = sm.G[sl][r];
+            // the kq rows are 0 for s >= r and for padded rows; the clamp keeps
+            // the unused upper triangle finite (G_r - G_s > 0 there)
+            x.x *= br * __expf(fminf(Gr - sm.G[sl][c], 0.f));
+            x.y *= br * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f));
+            x.z *= br * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f));
+            x.w *= br * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f));
+            *p4 = x;
+        }
+    };
+    // Q K^T rows -> P in place (K-major swizzled): P[r][s] = e^{G_r - G_s} QK[r][s], tf32
+    auto build_P = [&](int sl) {
+#pragma unroll
+        for (int e = tid; e < kC * kC / 4; e += kThreads) {
+            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+            float4 *p4 = reinterpret_cast<float4 *>(sm.P + swz(r, c, kC));
+            float4 x = *p4;
+            const float Gr = sm.G[sl][r];
+            x.x = tf32_rna(x.x * __expf(fminf(Gr - sm.G[sl][c], 0.f)));
+            x.y = tf32_rna(x.y * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f)));
+            x.z = tf32_rna(x.z * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f)));
+            x.w = tf32_rna(x.w * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f)));
+            *p4 = x;
+        }
+    };
+    // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A,
+    // by block doubling: invert the four 16 x 16 diagonal blocks by forward
+    // substitution, then join pairs of blocks with [T1 0; X T2], X = -T2 A21 T1,
+    // at 32 and at 64 rows.  Finally T diag(beta) and T diag(beta gamma) are
+    // written as tf32 B operands.  All 128 threads take part; sm.Tg serves as
+    // scratch for the products A21 T1.
+    auto solve = [&](int sl) {
+        float *At = sm.A;
+        float *Y = sm.Tg; // scratch
+        {   // 16 x 16 diagonal blocks: warp w, lane l < 16 owns column 16 w + l
+            const int c = 16 * warp + (lane & 15);
+            float t[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
                 float acc = 0.f;
 #pragma unroll
                 for (int i = 0; i < r; ++i)
-                    acc = fmaf(sm.A[r][i], Tc[i], acc);
-                Tc[r] = r == c ? 1.f : (r < c ? 0.f : -acc);
+                    acc = fmaf(At[swz(16 * warp + r, 16 * warp + i, kC)], t[i], acc);
+                const int rr = 16 * warp + r;
+                t[r] = rr == c ? 1.f : (rr < c ? 0.f : -acc);
             }
-            const float bc = sm.beta[c];
-            const float bgc = bc * expf(sm.G[c]);
+            __syncwarp();
+            if (lane < 16) {
 #pragma unroll
-            for (int r = 0; r < kC; ++r) {
-                sm.Tb[swz(r, c, kC)] = tf32_rna(Tc[r] * bc);
-                sm.Tg[swz(r, c, kC)] = tf32_rna(Tc[r] * bgc);
+                for (int r = 0; r < 16; ++r)
+                    At[swz(16 * warp + r, c, kC)] = t[r];
             }
         }
+        __syncthreads();
+        // join at 32 rows: blocks b = 0 (rows 0..31) and b = 1 (rows 32..63);
+        // thread: block b = tid / 64, output rows 2 (tid % 64 / 8) .. +1, columns 2 (tid % 8) .. +1
+        {
+            const int b = tid >> 6, q = tid & 63;
+            const int o = 32 * b;                 // block origin
+            const int r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
+            // Y = A21 T1 (16 x 16): A21 rows o+16.., columns o..; T1 at (o, o)
+            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a0 = At[swz(o + 16 + r0, o + i, kC)];
+                const float a1 = At[swz(o + 16 + r0 + 1, o + i, kC)];
+                const float t0 = At[swz(o + i, o + c0, kC)];
+                const float t1 = At[swz(o + i, o + c0 + 1, kC)];
+                y00 = fmaf(a0, t0, y00); y01 = fmaf(a0, t1, y01);
+                y10 = fmaf(a1, t0, y10); y11 = fmaf(a1, t1, y11);
+            }
+            Y[b * 256 + r0 * 16 + c0] = y00;
+            Y[b * 256 + r0 * 16 + c0 + 1] = y01;
+            Y[b * 256 + (r0 + 1) * 16 + c0] = y10;
+            Y[b * 256 + (r0 + 1) * 16 + c0 + 1] = y11;
+            __syncthreads();
+            // X = -T2 Y, T2 at (o + 16, o + 16), written over A21
+            float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const float a0 = At[swz(o + 16 + r0, o + 16 + i, kC)];
+                const float a1 = At[swz(o + 16 + r0 + 1, o + 16 + i, kC)];
+                const float t0 = Y[b * 256 + i * 16 + c0];
+                const float t1 = Y[b * 256 + i * 16 + c0 + 1];
+                x00 = fmaf(a0, t0, x00); x01 = fmaf(a0, t1, x01);
+                x10 = fmaf(a1, t0, x10); x11 = fmaf(a1, t1, x11);
+            }
+            __syncthreads(); // A21 is read by others above (it lies in the same rows)
+            At[swz(o + 16 + r0, o + c0, kC)] = -x00;
+            At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x01;
+            At[swz(o + 16 + r0 + 1, o + c0, kC)] = -x10;
+            At[swz(o + 16 + r0 + 1, o + c0 + 1, kC)] = -x11;
+        }
+        __syncthreads();
+        // join at 64 rows: Y = A21 T1 (32 x 32), then X = -T2 Y over A21
+        // thread: rows 2 (tid / 8) .. +1 of the 32, columns 4 (tid % 8) .. +3
+        {
+            const int r0 = 2 * (tid >> 3), c0 = 4 * (tid & 7);
+            float y[2][4] = {};
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                const float a0 = At[swz(32 + r0, i, kC)];
+                const float a1 = At[swz(32 + r0 + 1, i, kC)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(i, c0, kC));
+                y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
+                y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
+                y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
+                y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
+            }
+            *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) = make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
+            *reinterpret_cast<float4 *>(Y + (r0 + 1) * 36 + c0) = make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
+            __syncthreads();
+            float x[2][4] = {};
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                const float a0 = At[swz(32 + r0, 32 + i, kC)];
+                const float a1 = At[swz(32 + r0 + 1, 32 + i, kC)];
+                const float4 t4 = *reinterpret_cast<const float4 *>(Y + i * 36 + c0);
+                x[0][0] = fmaf(a0, t4.x, x[0][0]); x[0][1] = fmaf(a0, t4.y, x[0][1]);
+                x[0][2] = fmaf(a0, t4.z, x[0][2]); x[0][3] = fmaf(a0, t4.w, x[0][3]);
+                x[1][0] = fmaf(a1, t4.x, x[1][0]); x[1][1] = fmaf(a1, t4.y, x[1][1]);
+                x[1][2] = fmaf(a1, t4.z, x[1][2]); x[1][3] = fmaf(a1, t4.w, x[1][3]);
+            }
+            __syncthreads();
+            *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
+                make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
+            *reinterpret_cast<float4 *>(At + swz(32 + r0 + 1, c0, kC)) =
+                make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
+        }
+        __syncthreads();
+        // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
+#pragma unroll
+        for (int e = tid; e < kC * kC / 4; e += kThreads) {
+            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+            const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(r, c, kC));
+            const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][c]);
+            const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][c]);
+            const float4 tb = make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+            *reinterpret_cast<float4 *>(sm.Tb + swz(r, c, kC)) = tf32_rna(tb);
+            *reinterpret_cast<float4 *>(sm.Tg + swz(r, c, kC)) =
+                tf32_rna(make_float4(tb.x * g4.x, tb.y * g4.y, tb.z * g4.z, tb.w * g4.w));
+        }
+    };
+    // TMA issue (thread 0): nb 32-column boxes of 64 rows at x0 + 32 b, row t0
+    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar) {
+        if (tid == 0) {
+            mbar_arrive_expect_tx(bar, (uint32_t)(nb * kC * 32 * sizeof(float)));
+            for (int b = 0; b < nb; ++b)
+                tma_load_2d(smem_u32(dst + b * kC * 32), m, x0 + 32 * b, (int)t0, bar);
+        }
+    };
+    auto issue_z = [&](int c) {
+        if constexpr (sizeof(T) == 2) {
+            if (tid == 0) {
+                mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
+                tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)(start + (int64_t)c * kC), bar_z);
+            }
+        } else if (tid == 0) {
+            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_z) : "memory");
+        }
+    };
+    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
+    auto wait = [&](uint32_t bar, uint32_t &ph) {
+        const bool w = mbar_wait_bounded(bar, ph, kWaitLimit);
+        ph ^= 1u;
+        return w;
+    };
+
+    float av = 0.f, bv = 0.f; // gate inputs of the chunk after the next one to be gated
+    if (nchunks > 0) {
+        // ---- prologue: everything of chunk 0, and the K, K K^T rows of chunk 1
+        tma_tile(sm.V, &maps.v, xv, start, 4, bar_v);
+        tma_tile(sm.Q, &maps.q, xq, start, 4, bar_q);
+        tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0);
+        tma_tile(sm.P, &maps.kq, xkk + kC, start, 2, bar_p);
+        tma_tile(sm.A, &maps.kq, xkk, start, 2, bar_a);
+        issue_z(0);
+        load_ab(0, av, bv);
+        gates(0, av, bv, 0);
+        ok = wait(bar_a, ph_a) && ok;
+        __syncthreads();
+        build_A(0);
+        __syncthreads();
+        solve(0);
+        __syncthreads(); // A is free again
+        if (nchunks > 1) {
+            tma_tile(sm.K[1], &maps.k, xq, start + kC, 4, bar_k1);
+            tma_tile(sm.A, &maps.kq, xkk, start + kC, 2, bar_a);
+        }
+        ok = wait(bar_v, ph_v) && ok;
+        ok = wait(bar_q, ph_q) && ok;
+        ok = wait(bar_k0, ph_k0) && ok;
+        ok = wait(bar_p, ph_p) && ok;
+        round_tile<kC * kD>(sm.Q, tid);
+        round_tile<kC * kD>(sm.K[0], tid);
+        build_P(0);
+        load_ab(1, av, bv);
+        if (__syncthreads_or(!ok))
+            ok = false;
+    }
+
+    const uint32_t aV = smem_u32(sm.V), aQ = smem_u32(sm.Q);
+    const uint32_t aTb = smem_u32(sm.Tb), aTg = smem_u32(sm.Tg), aP = smem_u32(sm.P);
+    constexpr uint32_t kBlk = kC * 128; // bytes per 32-column block of a 64-row tile
+
+    for (int c = 0; c < nchunks; ++c) {
+        const int cur = c & 1, nxt = cur ^ 1;
+        const int nr = rows_of(c);
+        const int64_t t0 = start + (int64_t)c * kC;
+        const bool has_next = c + 1 < nchunks;
+        const uint32_t aK = smem_u32(sm.K[cur]);
+
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) { // leave together
+            ok = false;
+            break;
+        }
         tc_fence_after();
-        // ---- MMA 1: U~^T and W^T
+        // ---- MMA 1: U~^T = V^T (T diag b)^T and W^T = K^T (T diag b gamma)^T
         if (tid == 0) {
             const uint32_t id = idesc_tf32(128, kC, true, false);
 #pragma unroll
@@ -345,35 +553,34 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
                 mma_tf32_ss(tmem + kColU, sdesc_sw128_b32(aV + s * 1024, kBlk, 512), b1, id, s > 0);
                 mma_tf32_ss(tmem + kColW, sdesc_sw128_b32(aK + s * 1024, kBlk, 512), b2, id, s > 0);
             }
-            mma_commit(bar);
+            mma_commit(bar_mma);
         }
-        ok = mbar_wait_bounded(bar, phase, kWaitLimit);
-        phase ^= 1;
+        // the next chunk's gates while the tensor core works
+        gates(c + 1, av, bv, nxt);
+        ok = wait(bar_mma, ph_mma) && ok;
         if (__syncthreads_or(!ok))
             break;
         tc_fence_after();
-        // ---- -W into the (now free) K tile, K-major: rows r, columns k = tid
-        {
+        // ---- -W into the V tile (K-major: rows r, columns k = tid), tf32
 #pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                float w[32];
-                tmem_ld32(tW + cb * 32, w);
-                tmem_wait_ld();
+        for (int cb = 0; cb < 2; ++cb) {
+            float w[32];
+            tmem_ld32(tmem + lb + kColW + cb * 32, w);
+            tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    sm.K[swz(cb * 32 + i, tid, kC)] = tf32_rna(-w[i]);
-            }
+            for (int i = 0; i < 32; ++i)
+                sm.V[swz(cb * 32 + i, tid, kC)] = tf32_rna(-w[i]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- MMA 2: U^T = U~^T - S0 W^T and O^T = S0 (gamma Q)^T
+        // ---- MMA 2: U^T = U~^T - S0 W^T and O^T = S0 Q^T
         if (tid == 0) {
             const uint32_t id = idesc_tf32(128, kC, false, false);
 #pragma unroll
             for (int s = 0; s < kD / 8; ++s) {
-                const uint64_t bw = sdesc_sw128(aK + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
+                const uint64_t bw = sdesc_sw128(aV + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
                 mma_tf32_ts(tmem + kColU, tmem + kColSr + 8 * s, bw, id, 1);
             }
 #pragma unroll
@@ -381,42 +588,63 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
                 const uint64_t bq = sdesc_sw128(aQ + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
                 mma_tf32_ts(tmem + kColO, tmem + kColSr + 8 * s, bq, id, s > 0);
             }
-            mma_commit(bar);
+            mma_commit(bar_mma);
         }
-        ok = mbar_wait_bounded(bar, phase, kWaitLimit);
-        phase ^= 1;
+        // the next chunk's T while the tensor core works
+        if (has_next) {
+            ok = wait(bar_a, ph_a) && ok;
+            __syncthreads();
+            build_A(nxt);
+            __syncthreads();
+            solve(nxt);
+        }
+        ok = wait(bar_mma, ph_mma) && ok;
         if (__syncthreads_or(!ok))
             break;
         tc_fence_after();
-        // ---- S <- gamma_C S, and U rounded to tf32 in place (A operand of MMA 3)
+        // V (now -W) and Q are free: fetch the next chunk's
+        if (has_next) {
+            tma_tile(sm.V, &maps.v, xv, t0 + kC, 4, bar_v);
+            tma_tile(sm.Q, &maps.q, xq, t0 + kC, 4, bar_q);
+        }
+        // ---- TMEM pass: U -> tf32; U diag(gamma_C/gamma) -> tf32 copy;
+        //      O columns r scaled by gamma_r; S scaled by gamma_C
         {
-            const float gC = expf(Glast);
+#pragma unroll
+            for (int cb = 0; cb < 2; ++cb) {
+                float u[32], o[32];
+                tmem_ld32(tmem + lb + kColU + cb * 32, u);
+                tmem_ld32(tmem + lb + kColO + cb * 32, o);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    o[i] *= sm.gam[cur][cb * 32 + i];
+                tmem_st32(tmem + lb + kColO + cb * 32, o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    o[i] = tf32_rna(u[i] * sm.kd[cur][cb * 32 + i]);
+                    u[i] = tf32_rna(u[i]);
+                }
+                tmem_st32(tmem + lb + kColU + cb * 32, u);
+                tmem_st32(tmem + lb + kColUk + cb * 32, o);
+            }
+            const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) {
                 float v[32];
-                tmem_ld32(tS + cb * 32, v);
+                tmem_ld32(tmem + lb + kColS + cb * 32, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     v[i] *= gC;
-                tmem_st32(tS + cb * 32, v);
-            }
-#pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                float v[32];
-                tmem_ld32(tU + cb * 32, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    v[i] = tf32_rna(v[i]);
-                tmem_st32(tU + cb * 32, v);
+                tmem_st32(tmem + lb + kColS + cb * 32, v);
             }
             tmem_wait_st();
         }
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- MMA 3: O^T += U^T P^T and S += U^T K'
+        // ---- MMA 3: O^T += U^T P^T and S += (U diag(gamma_C/gamma))^T K
         if (tid == 0) {
             const uint32_t idp = idesc_tf32(128, kC, false, false);
             const uint32_t ids = idesc_tf32(128, kD, false, true);
@@ -424,33 +652,42 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
             for (int s = 0; s < kC / 8; ++s) {
                 const uint64_t bp = sdesc_sw128(aP + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
                 mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, bp, idp, 1);
-                const uint64_t bk = sdesc_sw128_b32(aKp + s * 1024, kBlk, 512);
-                mma_tf32_ts(tmem + kColS, tmem + kColU + 8 * s, bk, ids, 1);
+                const uint64_t bk = sdesc_sw128_b32(aK + s * 1024, kBlk, 512);
+                mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, bk, ids, 1);
             }
-            mma_commit(bar);
+            mma_commit(bar_mma);
         }
-        ok = mbar_wait_bounded(bar, phase, kWaitLimit);
-        phase ^= 1;
+        ok = wait(bar_z, ph_z) && ok; // z rows of this chunk
+        ok = wait(bar_mma, ph_mma) && ok;
         if (__syncthreads_or(!ok))
             break;
         tc_fence_after();
+        // P and K[cur] are free: fetch the next chunk's Q K^T rows, and K and
+        // K K^T rows of the chunk after it
+        if (has_next)
+            tma_tile(sm.P, &maps.kq, xkk + kC, t0 + kC, 2, bar_p);
+        if (c + 2 < nchunks) {
+            tma_tile(sm.K[cur], &maps.k, xq, t0 + 2 * kC, 4, cur ? bar_k1 : bar_k0);
+            tma_tile(sm.A, &maps.kq, xkk, t0 + 2 * kC, 2, bar_a);
+        }
+        load_ab(c + 2, av, bv);
         // ---- the next chunk's A operand: S rounded to tf32
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             float v[32];
-            tmem_ld32(tS + cb * 32, v);
+            tmem_ld32(tmem + lb + kColS + cb * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 v[i] = tf32_rna(v[i]);
-            tmem_st32(tSr + cb * 32, v);
+            tmem_st32(tmem + lb + kColSr + cb * 32, v);
         }
-        tmem_wait_st();
         // ---- epilogue: o[v = tid][r], gated RMSNorm over v, store
         float oa[32], ob[32];
-        tmem_ld32(tO, oa);
-        tmem_ld32(tO + 32, ob);
+        tmem_ld32(tmem + lb + kColO, oa);
+        tmem_ld32(tmem + lb + kColO + 32, ob);
         tmem_wait_ld();
+        tmem_wait_st();
         {
             float sq[kC];
 #pragma unroll
@@ -459,7 +696,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
                 sq[r + 32] = ob[r] * ob[r];
             }
             // reduce-scatter over the 32 lanes: lane l ends with two sums
-            const int lane = tid & 31;
 #pragma unroll
             for (int w = 32; w >= 2; w >>= 1) {
                 const int off = w >> 1;
@@ -483,25 +719,38 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
                                    sm.red[3][tid]) / (float)kD + p.rms_eps);
         __syncthreads();
         {
-            const T *zz = (const T *)p.z;
             T *yy = (T *)p.y;
 #pragma unroll
             for (int r = 0; r < kC; ++r) {
                 if (r < nr) {
                     const float ov = r < 32 ? oa[r] : ob[r - 32];
                     const int64_t idx = (t0 + r) * HD + (int64_t)h * kD + tid;
-                    const float zv = to_f(zz[idx]);
+                    float zv;
+                    if constexpr (sizeof(T) == 2)
+                        zv = to_f(sm.Z[r * kD + tid]);
+                    else
+                        zv = to_f(((const T *)p.z)[idx]);
                     yy[idx] = from_f<T>(ov * sm.rstd[r] * wn * siluf_(zv));
                     if (p.o_raw != nullptr)
                         p.o_raw[idx] = ov;
                 }
             }
         }
-        tc_fence_before();
-        __syncthreads(); // tiles and TMEM regions are reused by the next chunk
-        tc_fence_after();
+        __syncthreads(); // Z is read; red/rstd are reused
+        if (has_next) {
+            issue_z(c + 1);
+            // the next chunk's tiles
+            ok = wait(bar_v, ph_v) && ok;
+            ok = wait(bar_q, ph_q) && ok;
+            ok = wait(nxt ? bar_k1 : bar_k0, nxt ? ph_k1 : ph_k0) && ok;
+            ok = wait(bar_p, ph_p) && ok;
+            round_tile<kC * kD>(sm.Q, tid);
+            round_tile<kC * kD>(sm.K[nxt], tid);
+            build_P(nxt);
+        }
     }
 
+    ok = !__syncthreads_or(!ok); // one verdict for the whole CTA
     if (!ok) {
         if (tid == 0 && p.ws_err != nullptr)
             atomicOr(p.ws_err, 1u);
@@ -510,7 +759,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
 #pragma unroll
         for (int cb = 0; cb < 4; ++cb) {
             float v[32];
-            tmem_ld32(tS + cb * 32, v);
+            tmem_ld32(tmem + lb + kColS + cb * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
@@ -524,14 +773,70 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_prefill_kernel(PrefillArgs 
         tmem_dealloc(tmem, kTmemCols);
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The driver's tensor-map encoder, looked up once through the runtime.
+EncodeTiledFn encoder() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(f);
+    }();
+    return fn;
+}
+
+// Row-major 2-D map over `rows` rows of `cols` elements (row pitch `pitch`
+// bytes), boxes of `box_cols` x 64 rows.
+bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t cols,
+               uint64_t rows, uint64_t pitch, uint32_t box_cols, CUtensorMapSwizzle sw) {
+    EncodeTiledFn enc = encoder();
+    if (enc == nullptr)
+        return false;
+    const cuuint64_t dims[2] = {cols, rows};
+    const cuuint64_t strides[1] = {pitch};
+    const cuuint32_t box[2] = {box_cols, (cuuint32_t)kC};
+    const cuuint32_t es[2] = {1, 1};
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStream_t s) {
-    const size_t smem = sizeof(ChunkSmem) + 1024;
+    const size_t smem = sizeof(ChunkSmem<T>) + 1024;
     cudaError_t e = cudaFuncSetAttribute(chunk_prefill_kernel<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
+    ChunkMaps maps;
+    memset(&maps, 0, sizeof(maps));
+    if (p.N > 0) {
+        const uint64_t N = (uint64_t)p.N, F = sizeof(float);
+        const uint64_t qkw = 2ull * p.Hk * kD;
+        const bool okm =
+            encode_2d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_v, (uint64_t)p.Hv * kD, N,
+                      (uint64_t)p.Hv * kD * F, 32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
+            encode_2d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                      (const float *)p.ws_qk + (size_t)p.Hk * kD, (uint64_t)p.Hk * kD, N, qkw * F,
+                      32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
+            encode_2d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_qk, (uint64_t)p.Hk * kD, N,
+                      qkw * F, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.kq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_kq, (uint64_t)p.Hk * 2 * kC,
+                      N, (uint64_t)p.Hk * 2 * kC * F, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            (sizeof(T) != 2 ||
+             encode_2d(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.z, (uint64_t)p.Hv * kD, N,
+                       (uint64_t)p.Hv * kD * sizeof(T), kD, CU_TENSOR_MAP_SWIZZLE_NONE));
+        if (!okm)
+            return cudaErrorInvalidValue;
+    }
     dim3 grid(p.Hv, p.batch);
-    chunk_prefill_kernel<T><<<grid, kThreads, smem, s>>>(p);
+    chunk_prefill_kernel<T><<<grid, kThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 

@@ -25,7 +25,7 @@ __global__ void __launch_bounds__(kConvThreads)
 conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int batch,
                  int64_t N, const T *__restrict__ init_conv, const float *__restrict__ conv_w,
                  int Hk, int Hv, float l2_eps, float q_scale, float *__restrict__ qk_out,
-                 float *__restrict__ v_out, unsigned int *__restrict__ err) {
+                 float *__restrict__ v_out, unsigned int *__restrict__ err, bool round_v) {
     constexpr int V = Vec16<T>::N;
     constexpr int LANES = D / V; // lanes per head
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "head must tile a warp");
@@ -78,8 +78,17 @@ conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int 
         if (!active)
             continue;
         // q and k leave L2-normalised, v as is; all in float32 so that no
-        // rounding is added before the recurrence
+        // rounding is added before the recurrence, except that v, when only
+        // the tensor-core path reads it, is rounded to its tf32 operand here
         const float f = region == 2 ? 1.0f : rsqrtf(ss + l2_eps) * (region == 0 ? q_scale : 1.0f);
+        if (region == 2 && round_v) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                uint32_t r;
+                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(acc[i]));
+                acc[i] = __uint_as_float(r);
+            }
+        }
         float *dst = region < 2 ? qk_out + t * (2 * Hk * D) + cc
                                 : v_out + t * ((int64_t)Hv * D) + (cc - 2 * Hk * D);
 #pragma unroll
@@ -126,7 +135,7 @@ cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
               (C / V + kConvThreads - 1) / kConvThreads);
     conv_prep_kernel<T, D><<<grid, kConvThreads, 0, s>>>(
         (const T *)p.qkv, p.cu, p.batch, p.N, (const T *)p.init_conv, p.conv_w, p.Hk, p.Hv,
-        p.l2_eps, p.q_scale, (float *)p.ws_qk, (float *)p.ws_v, p.ws_err);
+        p.l2_eps, p.q_scale, (float *)p.ws_qk, (float *)p.ws_v, p.ws_err, p.chunked);
     return cudaGetLastError();
 }
 

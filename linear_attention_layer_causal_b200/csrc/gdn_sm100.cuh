@@ -40,6 +40,36 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
     return true;
 }
 
+// Arrive on `bar` expecting `bytes` more bytes of asynchronous (TMA) traffic.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+// 2-D tiled TMA load of the box at (x, y) of `tmap` into shared memory at
+// `dst`, completing `bar`'s transaction count.  x times the element size must
+// be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int x, int y,
+                                            uint32_t bar) {
+    asm volatile("cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes "
+                 "[%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+                 "l"(tmap), "r"(x), "r"(y), "r"(bar)
+                 : "memory");
+}
+
+// Asynchronous 16-byte global -> shared copy; with zfill the destination is
+// zero-filled and nothing is read.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool zfill) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
+                 "r"(zfill ? 0 : 16)
+                 : "memory");
+}
+// Arrive on `bar` once all of this thread's earlier cp.async copies have landed
+// (the arrival is not counted in advance: the barrier expects one per thread).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
 // ------------------------------------------------------------ tensor memory
 
 // Allocate `ncols` TMEM columns (power of two >= 32); one full warp executes
