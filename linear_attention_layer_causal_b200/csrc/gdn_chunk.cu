@@ -19,15 +19,17 @@
 // Mapping onto the tensor core (M = 128 = d_v is the TMEM lane dimension):
 //   U~^T = V^T (T diag b)^T          A = V  (smem, MN-major)   B = T diag b (smem)
 //   W^T  = K^T (T diag b gamma)^T    A = K  (smem, MN-major)   B = T diag b gamma
-//   U^T  = U~^T + S0 (-W)^T          A = S0 (TMEM, tf32 copy)  B = -W (smem)
-//   O^T  = S0 (diag(gamma) Q)^T      A = S0 (TMEM, tf32 copy)  B = gamma Q (smem)
+//   U^T  = U~^T + S0 (-W)^T          A = S0 (TMEM)             B = -W (smem)
+//   O^T  = S0 Q^T, then column r * gamma_r     A = S0 (TMEM)   B = Q (smem)
 //   O^T += U^T P^T                   A = U^T (TMEM)            B = P (smem)
-//   S   <- gamma_C S + U^T K'        A = U^T (TMEM)            B = K' (smem, MN-major)
-// The FP32 state lives in TMEM for the whole sequence; a copy rounded to tf32
-// (also in TMEM) is the A operand of the state products.  All products run as
-// kind::tf32 with every operand rounded to nearest beforehand (the tensor
-// core's own conversion truncates, a bias that accumulates over the 128-term
-// sums); the intra-chunk Gram matrices K K^T and Q K^T, to which
+//   S   <- gamma_C S + (U diag(gamma_C/gamma))^T K    A = TMEM  B = K (smem, MN-major)
+// The FP32 state lives in TMEM for the whole sequence and is itself the A
+// operand of the state products.  All products run as kind::tf32.  The
+// operands computed here (T diag b, -W, P and both forms of U) are rounded to
+// nearest before the tensor core reads them, since its own conversion
+// truncates and the resulting bias in U accumulates through the state; v is
+// rounded where it is produced; for S, q and k the truncation costs nothing
+// measurable.  The intra-chunk Gram matrices K K^T and Q K^T, to which
 // near-cancelling outputs are most sensitive, come exact in FP32 from
 // kq_prep_kernel.
 //
@@ -141,15 +143,16 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
 
 // ------------------------------------------------------------ chunk kernel
 
-constexpr int kThreads = 128; // 4 warps: thread i owns TMEM lane i (= value channel i)
+// 8 warps.  TMEM lane i is value channel i; warps w and w + 4 both reach lanes
+// 32 (w % 4) .. + 31 and split the columns of every TMEM pass between them.
+constexpr int kThreads = 256;
 
 // TMEM columns
-constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns
+constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns; also the A operand of S Q^T, S W^T
 constexpr uint32_t kColU = 128;  // U^T (starts as U~^T), 64 columns
 constexpr uint32_t kColO = 192;  // O^T, 64 columns
 constexpr uint32_t kColW = 256;  // W^T, 64 columns
-constexpr uint32_t kColSr = 320; // S rounded to tf32 (A operand of the state products), 128
-constexpr uint32_t kColUk = 448; // U^T diag(gamma_C / gamma) rounded to tf32, 64 columns
+constexpr uint32_t kColUk = 320; // U^T diag(gamma_C / gamma) rounded to tf32, 64 columns
 constexpr uint32_t kTmemCols = 512;
 
 // Both operand layouts below split a tile of R rows along its contiguous
@@ -175,8 +178,8 @@ template <typename T> struct __align__(1024) ChunkSmem {
     float P[kC * kC];     // B, K-major: P (lands as raw Q K^T rows)
     float A[kC * kC];     // the next chunk's A (lands as raw K K^T rows), then T; K-major swizzle
     T Z[sizeof(T) == 2 ? kC * kD : 1]; // z rows of this chunk (16-bit activations only)
-    float G[2][kC], beta[2][kC]; // cumulative log-decay and beta, this chunk / next
-    float gam[2][kC], kd[2][kC];  // gamma_r = e^{G_r} and gamma_C / gamma_r
+    float G[2][kC], beta[2][kC];      // cumulative log-decay and beta, this chunk / next
+    float gam[2][kC], kd[2][kC];      // gamma_r = e^{G_r} and gamma_C / gamma_r
     float scan[2];
     float red[4][kC];
     float rstd[kC];
@@ -186,15 +189,6 @@ template <typename T> struct __align__(1024) ChunkSmem {
 };
 
 constexpr long long kWaitLimit = 2000000000LL; // ~1 s of SM cycles
-
-// Rounds a float32 tile of `n` floats to tf32 in place (elementwise, any layout).
-template <int NF> __device__ __forceinline__ void round_tile(float *t, int tid) {
-#pragma unroll 4
-    for (int e = tid; e < NF / 4; e += kThreads) {
-        float4 *p4 = reinterpret_cast<float4 *>(t) + e;
-        *p4 = sm100::tf32_rna(*p4);
-    }
-}
 
 // The tensor maps of one call: 64-row boxes of the workspace and of z.
 struct ChunkMaps {
@@ -218,11 +212,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     const int j = h / p.G;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
+    const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
     const int nchunks = (int)((len + kC - 1) / kC);
-
     const int64_t HD = (int64_t)p.Hv * kD;
 
     const uint32_t bar_mma = smem_u32(&sm.bar_mma);
@@ -239,9 +234,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         mbar_init(bar_p, 1);
         mbar_init(bar_a, 1);
         mbar_init(bar_z, 1);
-    }
-    if (tid == 0)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     if (warp == 0) {
         tmem_alloc(smem_u32(&sm.tmem), kTmemCols);
         tmem_relinquish();
@@ -250,16 +244,17 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const uint32_t lb = (uint32_t)(warp * 32) << 16; // this warp's TMEM lanes
+    const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16); // this warp's TMEM lanes
     uint32_t ph_mma = 0, ph_v = 0, ph_q = 0, ph_k0 = 0, ph_k1 = 0, ph_p = 0, ph_a = 0, ph_z = 0;
     bool ok = true;
 
-    // ---- initial state into TMEM (row tid = lane tid), with its tf32 copy
+    // ---- initial state into TMEM: row vch, this half's 64 columns
     {
-        const float *src = p.init_state ? p.init_state + (((size_t)n * p.Hv + h) * kD + tid) * kD
-                                        : nullptr;
+        const float *src = p.init_state
+                               ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
+                               : nullptr;
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 0; cb < 2; ++cb) {
             float v[32];
 #pragma unroll
             for (int i = 0; i < 32; i += 4) {
@@ -267,19 +262,18 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                                : make_float4(0.f, 0.f, 0.f, 0.f);
                 v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
             }
-            tmem_st32(tmem + lb + kColS + cb * 32, v);
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                v[i] = tf32_rna(v[i]);
-            tmem_st32(tmem + lb + kColSr + cb * 32, v);
+            tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
         }
         tmem_wait_st();
     }
     const float negA = -expf(__ldg(p.A_log + h));
     const float dtb = __ldg(p.dt_bias + h);
-    const float wn = __ldg(p.norm_w + tid);
+    const float wn = __ldg(p.norm_w + vch);
 
-    auto rows_of = [&](int c) { return (int)((len - (int64_t)c * kC) < kC ? (len - (int64_t)c * kC) : kC); };
+    auto rows_of = [&](int c) {
+        const int64_t left = len - (int64_t)c * kC;
+        return (int)(left < kC ? left : kC);
+    };
     // gate inputs of chunk c, row tid (threads < 64); zero beyond the sequence
     auto load_ab = [&](int c, float &av, float &bv) {
         av = 0.f;
@@ -290,7 +284,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             bv = to_f(((const T *)p.b)[t * p.Hv + h]);
         }
     };
-    // g, beta and the inclusive prefix G of a chunk into slot `sl` (threads < 64)
+    // g, beta, the inclusive prefix G, gamma = e^G and gamma_C / gamma of a
+    // chunk into slot `sl` (rows = threads < 64)
     auto gates = [&](int c, float av, float bv, int sl) {
         if (tid < kC) {
             const bool in = c < nchunks && tid < rows_of(c);
@@ -317,7 +312,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             sm.kd[sl][tid] = expf(sm.G[sl][kC - 1] - Gr);
         }
     };
-    // K K^T rows of the slot's chunk -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
+    // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
     auto build_A = [&](int sl) {
 #pragma unroll
         for (int e = tid; e < kC * kC / 4; e += kThreads) {
@@ -325,8 +320,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             float4 *p4 = reinterpret_cast<float4 *>(sm.A + swz(r, c, kC));
             float4 x = *p4;
             const float br = sm.beta[sl][r], Gr = sm.G[sl][r];
-            // the kq rows are 0 for s >= r and for padded rows; the clamp keeps
-            // the unused upper triangle finite (G_r - G_s > 0 there)
+            // the kq rows are 0 for s >= r and beta is 0 on padded rows; the
+            // clamp keeps the unused upper triangle finite (G_r - G_s > 0 there)
             x.x *= br * __expf(fminf(Gr - sm.G[sl][c], 0.f));
             x.y *= br * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f));
             x.z *= br * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f));
@@ -349,16 +344,15 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             *p4 = x;
         }
     };
-    // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A,
-    // by block doubling: invert the four 16 x 16 diagonal blocks by forward
+    // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A, by
+    // block doubling: invert the four 16 x 16 diagonal blocks by forward
     // substitution, then join pairs of blocks with [T1 0; X T2], X = -T2 A21 T1,
     // at 32 and at 64 rows.  Finally T diag(beta) and T diag(beta gamma) are
-    // written as tf32 B operands.  All 128 threads take part; sm.Tg serves as
-    // scratch for the products A21 T1.
+    // written as tf32 B operands.  sm.Tg serves as scratch for A21 T1.
     auto solve = [&](int sl) {
         float *At = sm.A;
-        float *Y = sm.Tg; // scratch
-        {   // 16 x 16 diagonal blocks: warp w, lane l < 16 owns column 16 w + l
+        float *Y = sm.Tg;
+        if (warp < 4) { // 16 x 16 diagonal block `warp`; lane l < 16 owns column 16 warp + l
             const int c = 16 * warp + (lane & 15);
             float t[16];
 #pragma unroll
@@ -378,80 +372,55 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
         }
         __syncthreads();
-        // join at 32 rows: blocks b = 0 (rows 0..31) and b = 1 (rows 32..63);
-        // thread: block b = tid / 64, output rows 2 (tid % 64 / 8) .. +1, columns 2 (tid % 8) .. +1
-        {
-            const int b = tid >> 6, q = tid & 63;
-            const int o = 32 * b;                 // block origin
-            const int r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
-            // Y = A21 T1 (16 x 16): A21 rows o+16.., columns o..; T1 at (o, o)
-            float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+        { // join at 32 rows, blocks b = 0 (rows 0..31) and 1 (rows 32..63); thread:
+          // row r0 of the 16 x 16 product, columns c0, c0 + 1
+            const int b = tid >> 7, q = tid & 127;
+            const int o = 32 * b, r0 = q >> 3, c0 = 2 * (q & 7);
+            float y0 = 0.f, y1 = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float a0 = At[swz(o + 16 + r0, o + i, kC)];
-                const float a1 = At[swz(o + 16 + r0 + 1, o + i, kC)];
-                const float t0 = At[swz(o + i, o + c0, kC)];
-                const float t1 = At[swz(o + i, o + c0 + 1, kC)];
-                y00 = fmaf(a0, t0, y00); y01 = fmaf(a0, t1, y01);
-                y10 = fmaf(a1, t0, y10); y11 = fmaf(a1, t1, y11);
+                const float a = At[swz(o + 16 + r0, o + i, kC)];
+                y0 = fmaf(a, At[swz(o + i, o + c0, kC)], y0);
+                y1 = fmaf(a, At[swz(o + i, o + c0 + 1, kC)], y1);
             }
-            Y[b * 256 + r0 * 16 + c0] = y00;
-            Y[b * 256 + r0 * 16 + c0 + 1] = y01;
-            Y[b * 256 + (r0 + 1) * 16 + c0] = y10;
-            Y[b * 256 + (r0 + 1) * 16 + c0 + 1] = y11;
+            Y[b * 256 + r0 * 16 + c0] = y0;
+            Y[b * 256 + r0 * 16 + c0 + 1] = y1;
             __syncthreads();
-            // X = -T2 Y, T2 at (o + 16, o + 16), written over A21
-            float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+            float x0 = 0.f, x1 = 0.f;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const float a0 = At[swz(o + 16 + r0, o + 16 + i, kC)];
-                const float a1 = At[swz(o + 16 + r0 + 1, o + 16 + i, kC)];
-                const float t0 = Y[b * 256 + i * 16 + c0];
-                const float t1 = Y[b * 256 + i * 16 + c0 + 1];
-                x00 = fmaf(a0, t0, x00); x01 = fmaf(a0, t1, x01);
-                x10 = fmaf(a1, t0, x10); x11 = fmaf(a1, t1, x11);
+                const float a = At[swz(o + 16 + r0, o + 16 + i, kC)];
+                x0 = fmaf(a, Y[b * 256 + i * 16 + c0], x0);
+                x1 = fmaf(a, Y[b * 256 + i * 16 + c0 + 1], x1);
             }
-            __syncthreads(); // A21 is read by others above (it lies in the same rows)
-            At[swz(o + 16 + r0, o + c0, kC)] = -x00;
-            At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x01;
-            At[swz(o + 16 + r0 + 1, o + c0, kC)] = -x10;
-            At[swz(o + 16 + r0 + 1, o + c0 + 1, kC)] = -x11;
+            __syncthreads();
+            At[swz(o + 16 + r0, o + c0, kC)] = -x0;
+            At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x1;
         }
         __syncthreads();
-        // join at 64 rows: Y = A21 T1 (32 x 32), then X = -T2 Y over A21
-        // thread: rows 2 (tid / 8) .. +1 of the 32, columns 4 (tid % 8) .. +3
-        {
-            const int r0 = 2 * (tid >> 3), c0 = 4 * (tid & 7);
-            float y[2][4] = {};
+        { // join at 64 rows: thread: row r0 of the 32 x 32 product, columns c0 .. c0 + 3
+            const int r0 = tid >> 3, c0 = 4 * (tid & 7);
+            float y[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
             for (int i = 0; i < 32; ++i) {
-                const float a0 = At[swz(32 + r0, i, kC)];
-                const float a1 = At[swz(32 + r0 + 1, i, kC)];
+                const float a = At[swz(32 + r0, i, kC)];
                 const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(i, c0, kC));
-                y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
-                y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
-                y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
-                y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
+                y[0] = fmaf(a, t4.x, y[0]); y[1] = fmaf(a, t4.y, y[1]);
+                y[2] = fmaf(a, t4.z, y[2]); y[3] = fmaf(a, t4.w, y[3]);
             }
-            *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) = make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
-            *reinterpret_cast<float4 *>(Y + (r0 + 1) * 36 + c0) = make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
+            *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) = make_float4(y[0], y[1], y[2], y[3]);
             __syncthreads();
-            float x[2][4] = {};
+            float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 8
             for (int i = 0; i < 32; ++i) {
-                const float a0 = At[swz(32 + r0, 32 + i, kC)];
-                const float a1 = At[swz(32 + r0 + 1, 32 + i, kC)];
+                const float a = At[swz(32 + r0, 32 + i, kC)];
                 const float4 t4 = *reinterpret_cast<const float4 *>(Y + i * 36 + c0);
-                x[0][0] = fmaf(a0, t4.x, x[0][0]); x[0][1] = fmaf(a0, t4.y, x[0][1]);
-                x[0][2] = fmaf(a0, t4.z, x[0][2]); x[0][3] = fmaf(a0, t4.w, x[0][3]);
-                x[1][0] = fmaf(a1, t4.x, x[1][0]); x[1][1] = fmaf(a1, t4.y, x[1][1]);
-                x[1][2] = fmaf(a1, t4.z, x[1][2]); x[1][3] = fmaf(a1, t4.w, x[1][3]);
+                x[0] = fmaf(a, t4.x, x[0]); x[1] = fmaf(a, t4.y, x[1]);
+                x[2] = fmaf(a, t4.z, x[2]); x[3] = fmaf(a, t4.w, x[3]);
             }
             __syncthreads();
             *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
-                make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
-            *reinterpret_cast<float4 *>(At + swz(32 + r0 + 1, c0, kC)) =
-                make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
+                make_float4(-x[0], -x[1], -x[2], -x[3]);
         }
         __syncthreads();
         // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
@@ -481,20 +450,20 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
                 tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)(start + (int64_t)c * kC), bar_z);
             }
-        } else if (tid == 0) {
+        } else if (tid == 0) { // float32 z is read straight from global memory
             asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_z) : "memory");
         }
     };
-    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
     auto wait = [&](uint32_t bar, uint32_t &ph) {
         const bool w = mbar_wait_bounded(bar, ph, kWaitLimit);
         ph ^= 1u;
         return w;
     };
+    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
 
-    float av = 0.f, bv = 0.f; // gate inputs of the chunk after the next one to be gated
+    float av = 0.f, bv = 0.f; // gate inputs of the next chunk to be gated
     if (nchunks > 0) {
-        // ---- prologue: everything of chunk 0, and the K, K K^T rows of chunk 1
+        // ---- prologue: everything of chunk 0, and the K and K K^T rows of chunk 1
         tma_tile(sm.V, &maps.v, xv, start, 4, bar_v);
         tma_tile(sm.Q, &maps.q, xq, start, 4, bar_q);
         tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0);
@@ -517,8 +486,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         ok = wait(bar_q, ph_q) && ok;
         ok = wait(bar_k0, ph_k0) && ok;
         ok = wait(bar_p, ph_p) && ok;
-        round_tile<kC * kD>(sm.Q, tid);
-        round_tile<kC * kD>(sm.K[0], tid);
         build_P(0);
         load_ab(1, av, bv);
         if (__syncthreads_or(!ok))
@@ -561,32 +528,32 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         if (__syncthreads_or(!ok))
             break;
         tc_fence_after();
-        // ---- -W into the V tile (K-major: rows r, columns k = tid), tf32
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
+        // ---- -W into the V tile (K-major: rows r, columns k = vch), tf32;
+        //      this half takes rows 32 hf .. 32 hf + 31
+        {
             float w[32];
-            tmem_ld32(tmem + lb + kColW + cb * 32, w);
+            tmem_ld32(tl + kColW + 32 * hf, w);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                sm.V[swz(cb * 32 + i, tid, kC)] = tf32_rna(-w[i]);
+                sm.V[swz(32 * hf + i, vch, kC)] = tf32_rna(-w[i]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- MMA 2: U^T = U~^T - S0 W^T and O^T = S0 Q^T
+        // ---- MMA 2: U^T = U~^T - S0 W^T and O^T = S0 Q^T (A = the FP32 state in TMEM)
         if (tid == 0) {
             const uint32_t id = idesc_tf32(128, kC, false, false);
 #pragma unroll
             for (int s = 0; s < kD / 8; ++s) {
                 const uint64_t bw = sdesc_sw128(aV + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + kColU, tmem + kColSr + 8 * s, bw, id, 1);
+                mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, bw, id, 1);
             }
 #pragma unroll
             for (int s = 0; s < kD / 8; ++s) {
                 const uint64_t bq = sdesc_sw128(aQ + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + kColO, tmem + kColSr + 8 * s, bq, id, s > 0);
+                mma_tf32_ts(tmem + kColO, tmem + kColS + 8 * s, bq, id, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -607,37 +574,34 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             tma_tile(sm.V, &maps.v, xv, t0 + kC, 4, bar_v);
             tma_tile(sm.Q, &maps.q, xq, t0 + kC, 4, bar_q);
         }
-        // ---- TMEM pass: U -> tf32; U diag(gamma_C/gamma) -> tf32 copy;
-        //      O columns r scaled by gamma_r; S scaled by gamma_C
+        // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
+        //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
         {
+            float u[32], o[32];
+            tmem_ld32(tl + kColU + 32 * hf, u);
+            tmem_ld32(tl + kColO + 32 * hf, o);
+            tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
-                float u[32], o[32];
-                tmem_ld32(tmem + lb + kColU + cb * 32, u);
-                tmem_ld32(tmem + lb + kColO + cb * 32, o);
-                tmem_wait_ld();
+            for (int i = 0; i < 32; ++i)
+                o[i] *= sm.gam[cur][32 * hf + i];
+            tmem_st32(tl + kColO + 32 * hf, o);
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    o[i] *= sm.gam[cur][cb * 32 + i];
-                tmem_st32(tmem + lb + kColO + cb * 32, o);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    o[i] = tf32_rna(u[i] * sm.kd[cur][cb * 32 + i]);
-                    u[i] = tf32_rna(u[i]);
-                }
-                tmem_st32(tmem + lb + kColU + cb * 32, u);
-                tmem_st32(tmem + lb + kColUk + cb * 32, o);
+            for (int i = 0; i < 32; ++i) {
+                o[i] = tf32_rna(u[i] * sm.kd[cur][32 * hf + i]);
+                u[i] = tf32_rna(u[i]);
             }
+            tmem_st32(tl + kColU + 32 * hf, u);
+            tmem_st32(tl + kColUk + 32 * hf, o);
             const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
+            for (int cb = 0; cb < 2; ++cb) {
                 float v[32];
-                tmem_ld32(tmem + lb + kColS + cb * 32, v);
+                tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     v[i] *= gC;
-                tmem_st32(tmem + lb + kColS + cb * 32, v);
+                tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
             }
             tmem_wait_st();
         }
@@ -662,8 +626,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         if (__syncthreads_or(!ok))
             break;
         tc_fence_after();
-        // P and K[cur] are free: fetch the next chunk's Q K^T rows, and K and
-        // K K^T rows of the chunk after it
+        // P and K[cur] are free: fetch the next chunk's Q K^T rows, and the K
+        // and K K^T rows of the chunk after it
         if (has_next)
             tma_tile(sm.P, &maps.kq, xkk + kC, t0 + kC, 2, bar_p);
         if (c + 2 < nchunks) {
@@ -671,72 +635,51 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             tma_tile(sm.A, &maps.kq, xkk, t0 + 2 * kC, 2, bar_a);
         }
         load_ab(c + 2, av, bv);
-        // ---- the next chunk's A operand: S rounded to tf32
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float v[32];
-            tmem_ld32(tmem + lb + kColS + cb * 32, v);
+        // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
+        //      RMSNorm over v, times w[v] SiLU(z), stored
+        {
+            float o[32], sq[32];
+            tmem_ld32(tl + kColO + 32 * hf, o);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                v[i] = tf32_rna(v[i]);
-            tmem_st32(tmem + lb + kColSr + cb * 32, v);
-        }
-        // ---- epilogue: o[v = tid][r], gated RMSNorm over v, store
-        float oa[32], ob[32];
-        tmem_ld32(tmem + lb + kColO, oa);
-        tmem_ld32(tmem + lb + kColO + 32, ob);
-        tmem_wait_ld();
-        tmem_wait_st();
-        {
-            float sq[kC];
+                sq[i] = o[i] * o[i];
+            // reduce-scatter over the 32 lanes: lane l ends with row 32 hf + l
 #pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                sq[r] = oa[r] * oa[r];
-                sq[r + 32] = ob[r] * ob[r];
-            }
-            // reduce-scatter over the 32 lanes: lane l ends with two sums
-#pragma unroll
-            for (int w = 32; w >= 2; w >>= 1) {
-                const int off = w >> 1;
-                const bool upper = (lane & off) != 0;
+            for (int w = 16; w >= 1; w >>= 1) {
+                const bool upper = (lane & w) != 0;
 #pragma unroll
                 for (int i = 0; i < w; ++i) {
                     const float send = upper ? sq[i] : sq[i + w];
                     const float keep = upper ? sq[i + w] : sq[i];
-                    sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+                    sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
                 }
             }
-            // lane bits (4..0) select, from the top, which half was kept at each step
-            const int rb = ((lane >> 4) & 1) * 32 + ((lane >> 3) & 1) * 16 + ((lane >> 2) & 1) * 8 +
-                           ((lane >> 1) & 1) * 4 + (lane & 1) * 2;
-            sm.red[warp][rb] = sq[0];
-            sm.red[warp][rb + 1] = sq[1];
-        }
-        __syncthreads();
-        if (tid < kC)
-            sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
-                                   sm.red[3][tid]) / (float)kD + p.rms_eps);
-        __syncthreads();
-        {
+            sm.red[lq][32 * hf + lane] = sq[0];
+            __syncthreads();
+            if (tid < kC)
+                sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
+                                       sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
+            __syncthreads();
             T *yy = (T *)p.y;
 #pragma unroll
-            for (int r = 0; r < kC; ++r) {
+            for (int i = 0; i < 32; ++i) {
+                const int r = 32 * hf + i;
                 if (r < nr) {
-                    const float ov = r < 32 ? oa[r] : ob[r - 32];
-                    const int64_t idx = (t0 + r) * HD + (int64_t)h * kD + tid;
+                    const int64_t idx = (t0 + r) * HD + (int64_t)h * kD + vch;
                     float zv;
                     if constexpr (sizeof(T) == 2)
-                        zv = to_f(sm.Z[r * kD + tid]);
+                        zv = to_f(sm.Z[r * kD + vch]);
                     else
                         zv = to_f(((const T *)p.z)[idx]);
-                    yy[idx] = from_f<T>(ov * sm.rstd[r] * wn * siluf_(zv));
+                    const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
+                    yy[idx] = from_f<T>(o[i] * sm.rstd[r] * wn * gate);
                     if (p.o_raw != nullptr)
-                        p.o_raw[idx] = ov;
+                        p.o_raw[idx] = o[i];
                 }
             }
         }
-        __syncthreads(); // Z is read; red/rstd are reused
+        __syncthreads(); // Z is read; red / rstd are reused
         if (has_next) {
             issue_z(c + 1);
             // the next chunk's tiles
@@ -744,8 +687,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             ok = wait(bar_q, ph_q) && ok;
             ok = wait(nxt ? bar_k1 : bar_k0, nxt ? ph_k1 : ph_k0) && ok;
             ok = wait(bar_p, ph_p) && ok;
-            round_tile<kC * kD>(sm.Q, tid);
-            round_tile<kC * kD>(sm.K[nxt], tid);
             build_P(nxt);
         }
     }
@@ -755,11 +696,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         if (tid == 0 && p.ws_err != nullptr)
             atomicOr(p.ws_err, 1u);
     } else if (p.final_state != nullptr) {
-        float *dst = p.final_state + (((size_t)n * p.Hv + h) * kD + tid) * kD;
+        float *dst = p.final_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf;
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
+        for (int cb = 0; cb < 2; ++cb) {
             float v[32];
-            tmem_ld32(tmem + lb + kColS + cb * 32, v);
+            tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
