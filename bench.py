@@ -309,7 +309,7 @@ def run_ours(args, rank, world, dev, dist):
                        "global_batch": world, "seq_len": N, "parallelism": f"replicas x{world}",
                        "l2": "no flush: inputs of one step (~447 MB) exceed the 126 MB L2"},
             "roofline": roof, "decode": decode, "e2e": e2e,
-            "gpu_launches": (3 if kname == "chunk_prefill_kernel" else 2) * args.steps,
+            "gpu_launches": (4 if kname == "chunk_prefill_kernel" else 2) * args.steps,
             "clocks": clk}
     return line
 

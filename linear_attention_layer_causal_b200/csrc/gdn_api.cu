@@ -72,12 +72,16 @@ ProfileHook take_profile_hook() {
 }
 
 // Header (status word), float32 normalised q|k, float32 convolved v and, for
-// head_dim 128, the chunk Gram rows of the chunked path.
-size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N) {
+// head_dim 128, the chunk Gram rows and the per-sequence chunk offsets of the
+// chunked path.
+size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N, int batch) {
     if (N == 0)
         return 0;
-    return kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4) +
-           round_up((size_t)N * Hv * D * 4) + (D == 128 ? round_up(kq_workspace_bytes(Hk, N)) : 0);
+    size_t b = kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4) +
+               round_up((size_t)N * Hv * D * 4);
+    if (D == 128)
+        b += round_up(kq_workspace_bytes(Hk, N)) + round_up(((size_t)batch + 1) * sizeof(int32_t));
+    return b;
 }
 
 } // namespace gdn
@@ -115,7 +119,7 @@ gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int6
     if (bytes == nullptr || batch < 0 || total_tokens < 0)
         return GDN_ERR_INVALID_ARG;
     *bytes = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads, cfg->head_dim,
-                                     cfg->act_dtype == GDN_BF16, total_tokens);
+                                     cfg->act_dtype == GDN_BF16, total_tokens, batch);
     return GDN_OK;
 }
 
@@ -145,7 +149,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
         (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
         return GDN_ERR_INVALID_ARG;
     const size_t need = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads,
-                                                cfg->head_dim, bf16, total_tokens);
+                                                cfg->head_dim, bf16, total_tokens, batch);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
                      (reinterpret_cast<uintptr_t>(workspace) & 255u)))
         return GDN_ERR_WORKSPACE;
@@ -180,6 +184,8 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
         p.ws_qk = w + kWorkspaceHeader;
         p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
         p.ws_kq = (char *)p.ws_v + round_up((size_t)total_tokens * p.Hv * p.D * 4);
+        if (p.D == 128)
+            p.ws_offs = (int32_t *)((char *)p.ws_kq + round_up(kq_workspace_bytes(p.Hk, total_tokens)));
     }
 
     cudaStream_t s = (cudaStream_t)stream;

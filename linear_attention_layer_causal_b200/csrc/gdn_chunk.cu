@@ -51,93 +51,119 @@ constexpr int kD = 128; // head dim (d_k = d_v)
 // -------------------------------------------------------------- K K^T, Q K^T
 
 constexpr int kKqThreads = 256;
-constexpr int kKqRows = 64;      // packed tokens per CTA
-constexpr int kPad = kD + 1;     // padded smem row (conflict-free column access)
+constexpr int kTp = kC + 4; // row stride of the transposed tiles (16-byte aligned, banks staggered)
 
-// For q/k head j and packed token t at position r = t - cs of its chunk
-// (cs = sequence start + 64 * floor((t - start) / 64)):
-//   kq[t][j][0][s] = k_t . k_{cs+s} for s < r, else 0
-//   kq[t][j][1][s] = q_t . k_{cs+s} for s <= r, else 0
-// from the normalised float32 q|k rows of the workspace.
+// Chunk offsets: offs[n] = number of 64-token chunks in sequences 0 .. n-1
+// (offs[batch] = total).  One CTA of 1024 threads; each thread scans a run of
+// consecutive sequences, then the run totals are scanned across the block.
+__global__ void __launch_bounds__(1024)
+chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32_t *__restrict__ offs) {
+    __shared__ int32_t part[1024];
+    const int tid = threadIdx.x;
+    const int per = (batch + 1023) / 1024;
+    const int b0 = tid * per, b1 = b0 + per < batch ? b0 + per : batch;
+    int32_t sum = 0;
+    for (int n = b0; n < b1; ++n) {
+        int64_t s, e;
+        seq_bounds(cu, n, N, s, e);
+        sum += (int32_t)((e - s + kC - 1) / kC);
+    }
+    part[tid] = sum;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) { // inclusive scan of the run totals
+        const int32_t x = tid >= o ? part[tid - o] : 0;
+        __syncthreads();
+        part[tid] += x;
+        __syncthreads();
+    }
+    int32_t run = tid > 0 ? part[tid - 1] : 0;
+    for (int n = b0; n < b1; ++n) {
+        offs[n] = run;
+        int64_t s, e;
+        seq_bounds(cu, n, N, s, e);
+        run += (int32_t)((e - s + kC - 1) / kC);
+    }
+    if (tid == 1023)
+        offs[batch] = part[1023];
+}
+
+// One CTA per (chunk, q/k head j): with the chunk's rows t = t0 + r, r < nr,
+//   kq[t][j][0][s] = k_t . k_{t0+s} for s < r, else 0
+//   kq[t][j][1][s] = q_t . k_{t0+s} for s <= r, else 0
+// from the normalised float32 q|k rows of the workspace.  Thread (tr, ts) of
+// a 16 x 16 grid owns rows 4 tr .. + 3 and columns 4 ts .. + 3 of both
+// products (blocks above the diagonal are zero); the chunk's q and k sit
+// transposed in shared memory so that every step reads three float4s.
 __global__ void __launch_bounds__(kKqThreads)
 kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int batch, int64_t N,
-               int Hk, float *__restrict__ kq) {
-    extern __shared__ float ksm[];
-    float *Ks = ksm;                  // [2 kC][kPad] keys of packed rows [lo, lo + 2 kC)
-    float *Qs = Ks + 2 * kC * kPad;   // [kKqRows][kPad] queries of the tile's rows
-    __shared__ int64_t cs_row[kKqRows];
-    const int j = blockIdx.y;
-    const int64_t T0 = (int64_t)blockIdx.x * kKqRows;
-    const int64_t T1 = T0 + kKqRows < N ? T0 + kKqRows : N;
-    const int tid = threadIdx.x;
-    if (tid < kKqRows) {
-        const int64_t t = T0 + tid;
-        int64_t cs = t;
-        if (t < N) {
-            const int n = seq_of_token(cu, batch, t);
-            int64_t s0 = __ldg(cu + n);
-            s0 = s0 > t ? t : (s0 < 0 ? 0 : s0);
-            cs = s0 + ((t - s0) / kC) * kC;
+               int Hk, const int32_t *__restrict__ offs, float *__restrict__ kq) {
+    extern __shared__ __align__(16) float kq_smem[];
+    float *Kt = kq_smem;        // Kt[d][r] = k_{t0+r}[d]
+    float *Qt = Kt + kD * kTp;  // Qt[d][r] = q_{t0+r}[d]
+    const int ci = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+    if (ci >= __ldg(offs + batch))
+        return;
+    int lo = 0, hi = batch - 1; // the sequence n with offs[n] <= ci < offs[n+1]
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (__ldg(offs + mid) <= ci)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    int64_t s0, e0;
+    seq_bounds(cu, lo, N, s0, e0);
+    const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
+    const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
+    const int64_t QKW = 2 * (int64_t)Hk * kD;
+    for (int e = tid; e < kC * (kD / 4); e += kKqThreads) {
+        const int r = e % kC, d = (e / kC) * 4; // consecutive threads: consecutive rows
+        float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
+        if (r < nr) {
+            const float *row = qk + (t0 + r) * QKW + j * kD + d;
+            q4 = __ldg(reinterpret_cast<const float4 *>(row));
+            k4 = __ldg(reinterpret_cast<const float4 *>(row + Hk * kD));
         }
-        cs_row[tid] = cs;
+        Qt[(d + 0) * kTp + r] = q4.x; Qt[(d + 1) * kTp + r] = q4.y;
+        Qt[(d + 2) * kTp + r] = q4.z; Qt[(d + 3) * kTp + r] = q4.w;
+        Kt[(d + 0) * kTp + r] = k4.x; Kt[(d + 1) * kTp + r] = k4.y;
+        Kt[(d + 2) * kTp + r] = k4.z; Kt[(d + 3) * kTp + r] = k4.w;
     }
     __syncthreads();
-    const int64_t lo = cs_row[0]; // chunk starts are non-decreasing in t
-    const int QKW = 2 * Hk * kD;
-    // keys of rows [lo, T1) and queries of rows [T0, T1)
-    for (int e = tid; e < 2 * kC * (kD / 4); e += kKqThreads) {
-        const int rr = e / (kD / 4), c = (e % (kD / 4)) * 4;
-        const int64_t t = lo + rr;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < T1)
-            x = __ldg(reinterpret_cast<const float4 *>(qk + t * QKW + Hk * kD + j * kD + c));
-        float *dst = Ks + rr * kPad + c;
-        dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
+    const int tr = tid >> 4, ts = tid & 15;
+    float kk[4][4] = {}, qq[4][4] = {};
+    if (ts <= tr) {
+#pragma unroll 4
+        for (int d = 0; d < kD; ++d) {
+            const float4 kr = *reinterpret_cast<const float4 *>(Kt + d * kTp + 4 * tr);
+            const float4 qr = *reinterpret_cast<const float4 *>(Qt + d * kTp + 4 * tr);
+            const float4 ks = *reinterpret_cast<const float4 *>(Kt + d * kTp + 4 * ts);
+            const float a[4] = {kr.x, kr.y, kr.z, kr.w}, b[4] = {qr.x, qr.y, qr.z, qr.w};
+            const float c[4] = {ks.x, ks.y, ks.z, ks.w};
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    kk[x][y] = fmaf(a[x], c[y], kk[x][y]);
+                    qq[x][y] = fmaf(b[x], c[y], qq[x][y]);
+                }
+        }
     }
-    for (int e = tid; e < kKqRows * (kD / 4); e += kKqThreads) {
-        const int rr = e / (kD / 4), c = (e % (kD / 4)) * 4;
-        const int64_t t = T0 + rr;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < T1)
-            x = __ldg(reinterpret_cast<const float4 *>(qk + t * QKW + j * kD + c));
-        float *dst = Qs + rr * kPad + c;
-        dst[0] = x.x; dst[1] = x.y; dst[2] = x.z; dst[3] = x.w;
-    }
-    __syncthreads();
-    // warp w: tile rows 8w..8w+7; lane l: columns s = l and l + 32
-    const int warp = tid >> 5, lane = tid & 31;
-    for (int i = 0; i < 8; ++i) {
-        const int rl = warp * 8 + i;
-        const int64_t t = T0 + rl;
-        if (t >= T1)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const int r = 4 * tr + x;
+        if (r >= nr)
             break;
-        const int64_t cs = cs_row[rl];
-        const int r = (int)(t - cs);
-        const float *kt = Ks + (int)(t - lo) * kPad;
-        const float *qt = Qs + rl * kPad;
-        const int s0 = lane, s1 = lane + 32;
-        const float *k0 = Ks + (int)(cs - lo + s0) * kPad;
-        const float *k1 = Ks + (int)(cs - lo + (s1 < 2 * kC ? s1 : 0)) * kPad;
-        float kk0 = 0.f, kk1 = 0.f, qk0 = 0.f, qk1 = 0.f;
-        if (s0 <= r) {
-#pragma unroll 8
-            for (int d = 0; d < kD; ++d) {
-                kk0 = fmaf(kt[d], k0[d], kk0);
-                qk0 = fmaf(qt[d], k0[d], qk0);
-            }
+        float o1[4], o2[4];
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+            const int s = 4 * ts + y;
+            o1[y] = s < r ? kk[x][y] : 0.f;
+            o2[y] = s <= r ? qq[x][y] : 0.f;
         }
-        if (s1 <= r) {
-#pragma unroll 8
-            for (int d = 0; d < kD; ++d) {
-                kk1 = fmaf(kt[d], k1[d], kk1);
-                qk1 = fmaf(qt[d], k1[d], qk1);
-            }
-        }
-        float *o = kq + (t * Hk + j) * (2 * kC);
-        o[s0] = s0 < r ? kk0 : 0.f;
-        o[s1] = s1 < r ? kk1 : 0.f;
-        o[kC + s0] = s0 <= r ? qk0 : 0.f;
-        o[kC + s1] = s1 <= r ? qk1 : 0.f;
+        float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
+        *reinterpret_cast<float4 *>(o + 4 * ts) = make_float4(o1[0], o1[1], o1[2], o1[3]);
+        *reinterpret_cast<float4 *>(o + kC + 4 * ts) = make_float4(o2[0], o2[1], o2[2], o2[3]);
     }
 }
 
@@ -786,16 +812,20 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * 2 * kC * sizeof(float); }
 
 cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s) {
-    if (p.N == 0)
+    if (p.N == 0 || p.batch == 0)
         return cudaSuccess;
-    const size_t smem = sizeof(float) * (2 * kC + kKqRows) * kPad;
-    cudaError_t e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    chunk_offsets_kernel<<<1, 1024, 0, s>>>(p.cu, p.batch, p.N, p.ws_offs);
+    cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess)
         return e;
-    dim3 grid((unsigned)((p.N + kKqRows - 1) / kKqRows), p.Hk);
+    const size_t smem = sizeof(float) * 2 * kD * kTp;
+    e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess)
+        return e;
+    // upper bound on the chunk count: every sequence adds at most one partial chunk
+    dim3 grid((unsigned)((p.N + kC - 1) / kC + p.batch), p.Hk);
     kq_prep_kernel<<<grid, kKqThreads, smem, s>>>((const float *)p.ws_qk, p.cu, p.batch, p.N, p.Hk,
-                                                  (float *)p.ws_kq);
+                                                  p.ws_offs, (float *)p.ws_kq);
     return cudaGetLastError();
 }
 

@@ -28,6 +28,7 @@ struct PrefillArgs {
     void *ws_qk;             // [N, 2*Hk*D] float32: normalised q | k
     void *ws_v;              // [N, Hv*D]   float32: convolved v
     void *ws_kq;             // [N, Hk, 2, 64] float32: chunk Gram rows (chunked path)
+    int32_t *ws_offs;        // [batch + 1] chunk offsets per sequence (chunked path)
 };
 
 struct DecodeArgs {
@@ -54,7 +55,7 @@ inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
 }
 
 // Workspace bytes for the prefill path (each region 256-byte aligned).
-size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N);
+size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N, int batch);
 constexpr size_t kWorkspaceHeader = 256; // holds the device status word
 
 cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s);

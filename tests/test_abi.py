@@ -46,8 +46,10 @@ QWEN38 = gdn.Config(16, 128, 128)
 def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
     # 256-byte header (status word), float32 normalised q|k and convolved v, and
-    # for head_dim 128 the chunk Gram rows [N, H_k, 2, 64]; regions rounded to 256 B
-    assert n == 256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 2 * 64 * 4
+    # for head_dim 128 the chunk Gram rows [N, H_k, 2, 64] and the chunk offsets
+    # [batch + 1]; regions rounded to 256 B
+    assert n == 256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 2 * 64 * 4 + 256
+    assert gdn.prefill_workspace_size(QWEN38, 100, 4096) == n + 256  # 101 offsets: 512 bytes
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
     tiny = gdn.Config(2, 4, 32, act_dtype="f32")
     assert gdn.prefill_workspace_size(tiny, 1, 3) == 256 + 1536 + 1536
