@@ -196,8 +196,10 @@ __device__ __forceinline__ int swz_mn(int k, int c, int R) {
 }
 
 template <typename T> struct __align__(1024) ChunkSmem {
-    float V[kC * kD];     // A, MN-major: V^T of this chunk; after MMA 1, B K-major: -W
-    float Q[kC * kD];     // B, K-major: Q
+    // V and Q share 32-column blocks of 128 rows: rows 0..63 hold V (A,
+    // MN-major, for MMA 1), then -W; rows 64..127 hold Q; so that [-W; Q] is
+    // one K-major N = 128 operand of MMA 2
+    float VQ[2 * kC * kD];
     float K[2][kC * kD];  // A / B, MN-major: K of this chunk and the next (ping-pong)
     float Tb[kC * kC];    // B, K-major: T diag(beta)
     float Tg[kC * kC];    // B, K-major: T diag(beta gamma)
@@ -211,6 +213,7 @@ template <typename T> struct __align__(1024) ChunkSmem {
     float rstd[kC];
     unsigned long long bar_mma;
     unsigned long long bar_v, bar_q, bar_k[2], bar_p, bar_a, bar_z;
+    static constexpr int kVQBlk = 2 * kC * 32; // floats per 32-column block of VQ
     uint32_t tmem;
 };
 
@@ -290,6 +293,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
         }
+        float zero[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            zero[i] = 0.f;
+        tmem_st32(tl + kColO + 32 * hf, zero); // MMA 2 accumulates onto O
         tmem_wait_st();
     }
     const float negA = -expf(__ldg(p.A_log + h));
@@ -300,42 +308,54 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         const int64_t left = len - (int64_t)c * kC;
         return (int)(left < kC ? left : kC);
     };
-    // gate inputs of chunk c, row tid (threads < 64); zero beyond the sequence
-    auto load_ab = [&](int c, float &av, float &bv) {
-        av = 0.f;
-        bv = 0.f;
-        if (tid < kC && c < nchunks && tid < rows_of(c)) {
-            const int64_t t = start + (int64_t)c * kC + tid;
-            av = to_f(((const T *)p.a)[t * p.Hv + h]);
-            bv = to_f(((const T *)p.b)[t * p.Hv + h]);
+    // raw gate inputs of chunk c, rows lane and lane + 32 (warp 0); the
+    // conversion waits until gates() so the loads overlap other work
+    auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
+        if (warp == 0) {
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int r = lane + 32 * q;
+                ra[q] = from_f<T>(0.f);
+                rb[q] = from_f<T>(0.f);
+                if (c < nchunks && r < rows_of(c)) {
+                    const int64_t t = start + (int64_t)c * kC + r;
+                    ra[q] = ((const T *)p.a)[t * p.Hv + h];
+                    rb[q] = ((const T *)p.b)[t * p.Hv + h];
+                }
+            }
         }
     };
     // g, beta, the inclusive prefix G, gamma = e^G and gamma_C / gamma of a
-    // chunk into slot `sl` (rows = threads < 64)
-    auto gates = [&](int c, float av, float bv, int sl) {
-        if (tid < kC) {
-            const bool in = c < nchunks && tid < rows_of(c);
-            float g = in ? negA * softplusf_(av + dtb) : 0.f;
-            const float be = in ? sigmoidf_(bv) : 0.f;
+    // chunk into slot `sl`; warp 0 alone (rows lane, lane + 32), no block
+    // barrier: readers come after the next __syncthreads
+    auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
+        if (warp == 0) {
+            float g[2], be[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const bool in = c < nchunks && lane + 32 * q < rows_of(c);
+                g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
+                be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
+            }
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
-                const float x = __shfl_up_sync(0xffffffffu, g, o);
-                if (lane >= o)
-                    g += x;
+                const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
+                const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
+                if (lane >= o) {
+                    g[0] += x0;
+                    g[1] += x1;
+                }
             }
-            if (tid == 31)
-                sm.scan[0] = g;
-            sm.beta[sl][tid] = be;
-            sm.G[sl][tid] = g; // warp 1 adds warp 0's total below
-        }
-        __syncthreads();
-        if (tid >= 32 && tid < kC)
-            sm.G[sl][tid] += sm.scan[0];
-        __syncthreads();
-        if (tid < kC) {
-            const float Gr = sm.G[sl][tid];
-            sm.gam[sl][tid] = expf(Gr);
-            sm.kd[sl][tid] = expf(sm.G[sl][kC - 1] - Gr);
+            g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+            const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {
+                const int r = lane + 32 * q;
+                sm.G[sl][r] = g[q];
+                sm.beta[sl][r] = be[q];
+                sm.gam[sl][r] = expf(g[q]);
+                sm.kd[sl][r] = expf(Glast - g[q]);
+            }
         }
     };
     // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
@@ -419,7 +439,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 x0 = fmaf(a, Y[b * 256 + i * 16 + c0], x0);
                 x1 = fmaf(a, Y[b * 256 + i * 16 + c0 + 1], x1);
             }
-            __syncthreads();
+            // A21 was read only before the barrier above: overwrite it in place
             At[swz(o + 16 + r0, o + c0, kC)] = -x0;
             At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x1;
         }
@@ -444,7 +464,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 x[0] = fmaf(a, t4.x, x[0]); x[1] = fmaf(a, t4.y, x[1]);
                 x[2] = fmaf(a, t4.z, x[2]); x[3] = fmaf(a, t4.w, x[3]);
             }
-            __syncthreads();
             *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
                 make_float4(-x[0], -x[1], -x[2], -x[3]);
         }
@@ -463,11 +482,13 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         }
     };
     // TMA issue (thread 0): nb 32-column boxes of 64 rows at x0 + 32 b, row t0
-    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar) {
+    // (column block b lands at dst + b * bstride floats)
+    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar,
+                        int bstride = kC * 32) {
         if (tid == 0) {
             mbar_arrive_expect_tx(bar, (uint32_t)(nb * kC * 32 * sizeof(float)));
             for (int b = 0; b < nb; ++b)
-                tma_load_2d(smem_u32(dst + b * kC * 32), m, x0 + 32 * b, (int)t0, bar);
+                tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, bar);
         }
     };
     auto issue_z = [&](int c) {
@@ -487,11 +508,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     };
     const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
 
-    float av = 0.f, bv = 0.f; // gate inputs of the next chunk to be gated
+    T av[2], bv[2]; // raw gate inputs of the next chunk to be gated
     if (nchunks > 0) {
         // ---- prologue: everything of chunk 0, and the K and K K^T rows of chunk 1
-        tma_tile(sm.V, &maps.v, xv, start, 4, bar_v);
-        tma_tile(sm.Q, &maps.q, xq, start, 4, bar_q);
+        tma_tile(sm.VQ, &maps.v, xv, start, 4, bar_v, ChunkSmem<T>::kVQBlk);
+        tma_tile(sm.VQ + kC * 32, &maps.q, xq, start, 4, bar_q, ChunkSmem<T>::kVQBlk);
         tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0);
         tma_tile(sm.P, &maps.kq, xkk + kC, start, 2, bar_p);
         tma_tile(sm.A, &maps.kq, xkk, start, 2, bar_a);
@@ -518,16 +539,26 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             ok = false;
     }
 
-    const uint32_t aV = smem_u32(sm.V), aQ = smem_u32(sm.Q);
-    const uint32_t aTb = smem_u32(sm.Tb), aTg = smem_u32(sm.Tg), aP = smem_u32(sm.P);
-    constexpr uint32_t kBlk = kC * 128; // bytes per 32-column block of a 64-row tile
+    // shared-memory descriptors at k-step 0; a k-step adds its byte offset / 16
+    constexpr uint32_t kBlk = kC * 128;       // bytes per 32-column block of a 64-row tile
+    constexpr uint32_t kVQb = 2 * kC * 128;   // bytes per 32-column block of VQ
+    const uint32_t aVQ = smem_u32(sm.VQ);
+    const uint64_t dV = sdesc_sw128_b32(aVQ, kVQb, 512);              // A of MMA 1 (MN-major)
+    const uint64_t dWQ = sdesc_sw128(aVQ, 16, 1024);                  // B of MMA 2 (K-major, N 128)
+    const uint64_t dTb = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
+    const uint64_t dTg = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
+    const uint64_t dP = sdesc_sw128(smem_u32(sm.P), 16, 1024);
+    const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kBlk, 512); // MN-major K tiles
+    const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kBlk, 512);
+    // k-step s of a K-major operand: column block s / 4, 32 bytes per step within it
+    auto kstep = [](int s, uint32_t blk) { return (uint64_t)((((s >> 2) * blk) + (s & 3) * 32) >> 4); };
 
     for (int c = 0; c < nchunks; ++c) {
         const int cur = c & 1, nxt = cur ^ 1;
         const int nr = rows_of(c);
         const int64_t t0 = start + (int64_t)c * kC;
         const bool has_next = c + 1 < nchunks;
-        const uint32_t aK = smem_u32(sm.K[cur]);
+        const uint64_t dK = cur ? dK1 : dK0;
 
         fence_proxy_async_smem();
         tc_fence_before();
@@ -538,13 +569,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         tc_fence_after();
         // ---- MMA 1: U~^T = V^T (T diag b)^T and W^T = K^T (T diag b gamma)^T
         if (tid == 0) {
-            const uint32_t id = idesc_tf32(128, kC, true, false);
+            constexpr uint32_t id = idesc_tf32(128, kC, true, false);
 #pragma unroll
             for (int s = 0; s < kC / 8; ++s) {
-                const uint64_t b1 = sdesc_sw128(aTb + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                const uint64_t b2 = sdesc_sw128(aTg + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ss(tmem + kColU, sdesc_sw128_b32(aV + s * 1024, kBlk, 512), b1, id, s > 0);
-                mma_tf32_ss(tmem + kColW, sdesc_sw128_b32(aK + s * 1024, kBlk, 512), b2, id, s > 0);
+                mma_tf32_ss(tmem + kColU, dV + s * 64, dTb + kstep(s, kBlk), id, s > 0);
+                mma_tf32_ss(tmem + kColW, dK + s * 64, dTg + kstep(s, kBlk), id, s > 0);
             }
             mma_commit(bar_mma);
         }
@@ -562,25 +591,19 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; ++i)
-                sm.V[swz(32 * hf + i, vch, kC)] = tf32_rna(-w[i]);
+                sm.VQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(-w[i]);
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
         tc_fence_after();
-        // ---- MMA 2: U^T = U~^T - S0 W^T and O^T = S0 Q^T (A = the FP32 state in TMEM)
+        // ---- MMA 2: [U^T | O^T] += S0 [-W; Q]^T, one N = 128 product (A = the
+        //      FP32 state in TMEM); U^T starts as U~^T, O^T as zero
         if (tid == 0) {
-            const uint32_t id = idesc_tf32(128, kC, false, false);
+            constexpr uint32_t id = idesc_tf32(128, 2 * kC, false, false);
 #pragma unroll
-            for (int s = 0; s < kD / 8; ++s) {
-                const uint64_t bw = sdesc_sw128(aV + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, bw, id, 1);
-            }
-#pragma unroll
-            for (int s = 0; s < kD / 8; ++s) {
-                const uint64_t bq = sdesc_sw128(aQ + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + kColO, tmem + kColS + 8 * s, bq, id, s > 0);
-            }
+            for (int s = 0; s < kD / 8; ++s)
+                mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, dWQ + kstep(s, kVQb), id, 1);
             mma_commit(bar_mma);
         }
         // the next chunk's T while the tensor core works
@@ -597,8 +620,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         tc_fence_after();
         // V (now -W) and Q are free: fetch the next chunk's
         if (has_next) {
-            tma_tile(sm.V, &maps.v, xv, t0 + kC, 4, bar_v);
-            tma_tile(sm.Q, &maps.q, xq, t0 + kC, 4, bar_q);
+            tma_tile(sm.VQ, &maps.v, xv, t0 + kC, 4, bar_v, ChunkSmem<T>::kVQBlk);
+            tma_tile(sm.VQ + kC * 32, &maps.q, xq, t0 + kC, 4, bar_q, ChunkSmem<T>::kVQBlk);
         }
         // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
         //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
@@ -636,14 +659,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         tc_fence_after();
         // ---- MMA 3: O^T += U^T P^T and S += (U diag(gamma_C/gamma))^T K
         if (tid == 0) {
-            const uint32_t idp = idesc_tf32(128, kC, false, false);
-            const uint32_t ids = idesc_tf32(128, kD, false, true);
+            constexpr uint32_t idp = idesc_tf32(128, kC, false, false);
+            constexpr uint32_t ids = idesc_tf32(128, kD, false, true);
 #pragma unroll
             for (int s = 0; s < kC / 8; ++s) {
-                const uint64_t bp = sdesc_sw128(aP + (s >> 2) * kBlk + (s & 3) * 32, 16, 1024);
-                mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, bp, idp, 1);
-                const uint64_t bk = sdesc_sw128_b32(aK + s * 1024, kBlk, 512);
-                mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, bk, ids, 1);
+                mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, dP + kstep(s, kBlk), idp, 1);
+                mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, ids, 1);
             }
             mma_commit(bar_mma);
         }
@@ -687,23 +708,41 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
                                        sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
             __syncthreads();
-            T *yy = (T *)p.y;
+            // y[t0 + r][h][vch] for this half's rows r = 32 hf + i
+            T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
+            float *op = p.o_raw ? p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch : nullptr;
+            const int rows = nr - 32 * hf; // valid rows of this half (may be <= 0)
+            auto emit = [&](int i) {
+                float zv;
+                if constexpr (sizeof(T) == 2)
+                    zv = to_f(sm.Z[(32 * hf + i) * kD + vch]);
+                else
+                    zv = to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD + (int64_t)h * kD + vch]);
+                const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
+                yp[i * HD] = from_f<T>(o[i] * (sm.rstd[32 * hf + i] * wn) * gate);
+            };
+            if (rows >= 32) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const int r = 32 * hf + i;
-                if (r < nr) {
-                    const int64_t idx = (t0 + r) * HD + (int64_t)h * kD + vch;
-                    float zv;
-                    if constexpr (sizeof(T) == 2)
-                        zv = to_f(sm.Z[r * kD + vch]);
-                    else
-                        zv = to_f(((const T *)p.z)[idx]);
-                    const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
-                    yy[idx] = from_f<T>(o[i] * sm.rstd[r] * wn * gate);
-                    if (p.o_raw != nullptr)
-                        p.o_raw[idx] = o[i];
-                }
+                for (int i = 0; i < 32; ++i)
+                    emit(i);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < rows)
+                        emit(i);
             }
+            if (op != nullptr) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (i < rows)
+                        op[i * HD] = o[i];
+            }
+            // O is consumed: zero it, since MMA 2 accumulates onto it
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                o[i] = 0.f;
+            tmem_st32(tl + kColO + 32 * hf, o);
+            tmem_wait_st();
         }
         __syncthreads(); // Z is read; red / rstd are reused
         if (has_next) {
