@@ -168,15 +168,27 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
 }
 
 // ------------------------------------------------------------ chunk kernel
+//
+// Two warp groups work on consecutive chunks at once:
+//   state group (warps 0..7): reads and rewrites TMEM (the W pass, the pass
+//     that rounds U and scales O and S, the gated-RMSNorm epilogue) and issues
+//     MMA 2 and MMA 3 of the current chunk; warps w and w + 4 share TMEM lanes
+//     32 (w % 4) .. + 31 (lane i = value channel i) and split the columns;
+//   prep group (warps 8..11): builds the next chunk's gates, A, T = (I+A)^-1,
+//     T diag(beta), T diag(beta gamma) and P on the CUDA cores, issues every
+//     TMA load and MMA 1.
+// They hand over through mbarriers: MMA 1/2/3 completion (tcgen05.commit), a
+// "prep ready" arrival, and the TMA transaction barriers of each tile.
 
-// 8 warps.  TMEM lane i is value channel i; warps w and w + 4 both reach lanes
-// 32 (w % 4) .. + 31 and split the columns of every TMEM pass between them.
-constexpr int kThreads = 256;
+constexpr int kStateThreads = 256;
+constexpr int kPrepThreads = 128;
+constexpr int kThreads = kStateThreads + kPrepThreads;
+constexpr int kBarState = 1, kBarPrep = 2; // named barriers of the two groups
 
 // TMEM columns
-constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns; also the A operand of S Q^T, S W^T
+constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns; also the A operand of S [-W; Q]^T
 constexpr uint32_t kColU = 128;  // U^T (starts as U~^T), 64 columns
-constexpr uint32_t kColO = 192;  // O^T, 64 columns
+constexpr uint32_t kColO = 192;  // O^T, 64 columns (directly after U^T: MMA 2 writes both)
 constexpr uint32_t kColW = 256;  // W^T, 64 columns
 constexpr uint32_t kColUk = 320; // U^T diag(gamma_C / gamma) rounded to tf32, 64 columns
 constexpr uint32_t kTmemCols = 512;
@@ -206,15 +218,15 @@ template <typename T> struct __align__(1024) ChunkSmem {
     float P[kC * kC];     // B, K-major: P (lands as raw Q K^T rows)
     float A[kC * kC];     // the next chunk's A (lands as raw K K^T rows), then T; K-major swizzle
     T Z[sizeof(T) == 2 ? kC * kD : 1]; // z rows of this chunk (16-bit activations only)
-    float G[2][kC], beta[2][kC];      // cumulative log-decay and beta, this chunk / next
+    float G[2][kC], beta[2][kC];      // cumulative log-decay and beta, by chunk parity
     float gam[2][kC], kd[2][kC];      // gamma_r = e^{G_r} and gamma_C / gamma_r
-    float scan[2];
     float red[4][kC];
     float rstd[kC];
-    unsigned long long bar_mma;
+    unsigned long long bar_mma1, bar_mma2, bar_mma3, bar_prep;
     unsigned long long bar_v, bar_q, bar_k[2], bar_p, bar_a, bar_z;
-    static constexpr int kVQBlk = 2 * kC * 32; // floats per 32-column block of VQ
     uint32_t tmem;
+    int abort;
+    static constexpr int kVQBlk = 2 * kC * 32; // floats per 32-column block of VQ
 };
 
 constexpr long long kWaitLimit = 2000000000LL; // ~1 s of SM cycles
@@ -227,6 +239,28 @@ struct ChunkMaps {
     CUtensorMap kq; // Gram rows, [N, Hk*128] fp32, 32-column boxes, 128-byte swizzle
     CUtensorMap z;  // z, [N, Hv*128] 16-bit, 128-column boxes, no swizzle
 };
+
+// Barrier over the `n` threads of one warp group (named barrier `id`).
+__device__ __forceinline__ void group_sync(int id, int n) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+// The same, returning whether `pred` held on any of the group's threads.
+__device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
+    uint32_t r;
+    // operands: %0 = r (output), %1 = id, %2 = n, %3 = pred
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.u32 p, %3, 0;\n\t"
+                 "bar.red.or.pred q, %1, %2, p;\n\t"
+                 "selp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(id), "r"(n), "r"((uint32_t)pred)
+                 : "memory");
+    return r != 0;
+}
+// Plain arrival on an mbarrier (release); the waiter's try_wait acquires.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -241,28 +275,25 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     const int j = h / p.G;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
-    const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
+    const bool is_state = tid < kStateThreads;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
     const int nchunks = (int)((len + kC - 1) / kC);
     const int64_t HD = (int64_t)p.Hv * kD;
 
-    const uint32_t bar_mma = smem_u32(&sm.bar_mma);
+    const uint32_t bar_mma1 = smem_u32(&sm.bar_mma1), bar_mma2 = smem_u32(&sm.bar_mma2);
+    const uint32_t bar_mma3 = smem_u32(&sm.bar_mma3), bar_prep = smem_u32(&sm.bar_prep);
     const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
     const uint32_t bar_p = smem_u32(&sm.bar_p), bar_a = smem_u32(&sm.bar_a);
     const uint32_t bar_z = smem_u32(&sm.bar_z);
     const uint32_t bar_k0 = smem_u32(&sm.bar_k[0]), bar_k1 = smem_u32(&sm.bar_k[1]);
     if (tid == 0) {
-        mbar_init(bar_mma, 1);
-        mbar_init(bar_v, 1);
-        mbar_init(bar_q, 1);
-        mbar_init(bar_k0, 1);
-        mbar_init(bar_k1, 1);
-        mbar_init(bar_p, 1);
-        mbar_init(bar_a, 1);
-        mbar_init(bar_z, 1);
+        const uint32_t all[11] = {bar_mma1, bar_mma2, bar_mma3, bar_prep, bar_v, bar_q,
+                                  bar_k0, bar_k1, bar_p, bar_a, bar_z};
+        for (int b = 0; b < 11; ++b)
+            mbar_init(all[b], 1);
+        sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -273,494 +304,541 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16); // this warp's TMEM lanes
-    uint32_t ph_mma = 0, ph_v = 0, ph_q = 0, ph_k0 = 0, ph_k1 = 0, ph_p = 0, ph_a = 0, ph_z = 0;
-    bool ok = true;
-
-    // ---- initial state into TMEM: row vch, this half's 64 columns
-    {
-        const float *src = p.init_state
-                               ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
-                               : nullptr;
-#pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
-            float v[32];
-#pragma unroll
-            for (int i = 0; i < 32; i += 4) {
-                float4 x = src ? *reinterpret_cast<const float4 *>(src + cb * 32 + i)
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-                v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
-            }
-            tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
-        }
-        float zero[32];
-#pragma unroll
-        for (int i = 0; i < 32; ++i)
-            zero[i] = 0.f;
-        tmem_st32(tl + kColO + 32 * hf, zero); // MMA 2 accumulates onto O
-        tmem_wait_st();
-    }
     const float negA = -expf(__ldg(p.A_log + h));
     const float dtb = __ldg(p.dt_bias + h);
-    const float wn = __ldg(p.norm_w + vch);
-
+    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
     auto rows_of = [&](int c) {
         const int64_t left = len - (int64_t)c * kC;
         return (int)(left < kC ? left : kC);
-    };
-    // raw gate inputs of chunk c, rows lane and lane + 32 (warp 0); the
-    // conversion waits until gates() so the loads overlap other work
-    auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
-        if (warp == 0) {
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int r = lane + 32 * q;
-                ra[q] = from_f<T>(0.f);
-                rb[q] = from_f<T>(0.f);
-                if (c < nchunks && r < rows_of(c)) {
-                    const int64_t t = start + (int64_t)c * kC + r;
-                    ra[q] = ((const T *)p.a)[t * p.Hv + h];
-                    rb[q] = ((const T *)p.b)[t * p.Hv + h];
-                }
-            }
-        }
-    };
-    // g, beta, the inclusive prefix G, gamma = e^G and gamma_C / gamma of a
-    // chunk into slot `sl`; warp 0 alone (rows lane, lane + 32), no block
-    // barrier: readers come after the next __syncthreads
-    auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
-        if (warp == 0) {
-            float g[2], be[2];
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const bool in = c < nchunks && lane + 32 * q < rows_of(c);
-                g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
-                be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
-            }
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
-                const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
-                if (lane >= o) {
-                    g[0] += x0;
-                    g[1] += x1;
-                }
-            }
-            g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-            const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
-#pragma unroll
-            for (int q = 0; q < 2; ++q) {
-                const int r = lane + 32 * q;
-                sm.G[sl][r] = g[q];
-                sm.beta[sl][r] = be[q];
-                sm.gam[sl][r] = expf(g[q]);
-                sm.kd[sl][r] = expf(Glast - g[q]);
-            }
-        }
-    };
-    // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
-    auto build_A = [&](int sl) {
-#pragma unroll
-        for (int e = tid; e < kC * kC / 4; e += kThreads) {
-            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-            float4 *p4 = reinterpret_cast<float4 *>(sm.A + swz(r, c, kC));
-            float4 x = *p4;
-            const float br = sm.beta[sl][r], Gr = sm.G[sl][r];
-            // the kq rows are 0 for s >= r and beta is 0 on padded rows; the
-            // clamp keeps the unused upper triangle finite (G_r - G_s > 0 there)
-            x.x *= br * __expf(fminf(Gr - sm.G[sl][c], 0.f));
-            x.y *= br * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f));
-            x.z *= br * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f));
-            x.w *= br * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f));
-            *p4 = x;
-        }
-    };
-    // Q K^T rows -> P in place (K-major swizzled): P[r][s] = e^{G_r - G_s} QK[r][s], tf32
-    auto build_P = [&](int sl) {
-#pragma unroll
-        for (int e = tid; e < kC * kC / 4; e += kThreads) {
-            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-            float4 *p4 = reinterpret_cast<float4 *>(sm.P + swz(r, c, kC));
-            float4 x = *p4;
-            const float Gr = sm.G[sl][r];
-            x.x = tf32_rna(x.x * __expf(fminf(Gr - sm.G[sl][c], 0.f)));
-            x.y = tf32_rna(x.y * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f)));
-            x.z = tf32_rna(x.z * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f)));
-            x.w = tf32_rna(x.w * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f)));
-            *p4 = x;
-        }
-    };
-    // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A, by
-    // block doubling: invert the four 16 x 16 diagonal blocks by forward
-    // substitution, then join pairs of blocks with [T1 0; X T2], X = -T2 A21 T1,
-    // at 32 and at 64 rows.  Finally T diag(beta) and T diag(beta gamma) are
-    // written as tf32 B operands.  sm.Tg serves as scratch for A21 T1.
-    auto solve = [&](int sl) {
-        float *At = sm.A;
-        float *Y = sm.Tg;
-        if (warp < 4) { // 16 x 16 diagonal block `warp`; lane l < 16 owns column 16 warp + l
-            const int c = 16 * warp + (lane & 15);
-            float t[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
-#pragma unroll
-                for (int i = 0; i < r; ++i)
-                    acc = fmaf(At[swz(16 * warp + r, 16 * warp + i, kC)], t[i], acc);
-                const int rr = 16 * warp + r;
-                t[r] = rr == c ? 1.f : (rr < c ? 0.f : -acc);
-            }
-            __syncwarp();
-            if (lane < 16) {
-#pragma unroll
-                for (int r = 0; r < 16; ++r)
-                    At[swz(16 * warp + r, c, kC)] = t[r];
-            }
-        }
-        __syncthreads();
-        { // join at 32 rows, blocks b = 0 (rows 0..31) and 1 (rows 32..63); thread:
-          // row r0 of the 16 x 16 product, columns c0, c0 + 1
-            const int b = tid >> 7, q = tid & 127;
-            const int o = 32 * b, r0 = q >> 3, c0 = 2 * (q & 7);
-            float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float a = At[swz(o + 16 + r0, o + i, kC)];
-                y0 = fmaf(a, At[swz(o + i, o + c0, kC)], y0);
-                y1 = fmaf(a, At[swz(o + i, o + c0 + 1, kC)], y1);
-            }
-            Y[b * 256 + r0 * 16 + c0] = y0;
-            Y[b * 256 + r0 * 16 + c0 + 1] = y1;
-            __syncthreads();
-            float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                const float a = At[swz(o + 16 + r0, o + 16 + i, kC)];
-                x0 = fmaf(a, Y[b * 256 + i * 16 + c0], x0);
-                x1 = fmaf(a, Y[b * 256 + i * 16 + c0 + 1], x1);
-            }
-            // A21 was read only before the barrier above: overwrite it in place
-            At[swz(o + 16 + r0, o + c0, kC)] = -x0;
-            At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x1;
-        }
-        __syncthreads();
-        { // join at 64 rows: thread: row r0 of the 32 x 32 product, columns c0 .. c0 + 3
-            const int r0 = tid >> 3, c0 = 4 * (tid & 7);
-            float y[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                const float a = At[swz(32 + r0, i, kC)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(i, c0, kC));
-                y[0] = fmaf(a, t4.x, y[0]); y[1] = fmaf(a, t4.y, y[1]);
-                y[2] = fmaf(a, t4.z, y[2]); y[3] = fmaf(a, t4.w, y[3]);
-            }
-            *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) = make_float4(y[0], y[1], y[2], y[3]);
-            __syncthreads();
-            float x[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-            for (int i = 0; i < 32; ++i) {
-                const float a = At[swz(32 + r0, 32 + i, kC)];
-                const float4 t4 = *reinterpret_cast<const float4 *>(Y + i * 36 + c0);
-                x[0] = fmaf(a, t4.x, x[0]); x[1] = fmaf(a, t4.y, x[1]);
-                x[2] = fmaf(a, t4.z, x[2]); x[3] = fmaf(a, t4.w, x[3]);
-            }
-            *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
-                make_float4(-x[0], -x[1], -x[2], -x[3]);
-        }
-        __syncthreads();
-        // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
-#pragma unroll
-        for (int e = tid; e < kC * kC / 4; e += kThreads) {
-            const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-            const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(r, c, kC));
-            const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][c]);
-            const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][c]);
-            const float4 tb = make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
-            *reinterpret_cast<float4 *>(sm.Tb + swz(r, c, kC)) = tf32_rna(tb);
-            *reinterpret_cast<float4 *>(sm.Tg + swz(r, c, kC)) =
-                tf32_rna(make_float4(tb.x * g4.x, tb.y * g4.y, tb.z * g4.z, tb.w * g4.w));
-        }
-    };
-    // TMA issue (thread 0): nb 32-column boxes of 64 rows at x0 + 32 b, row t0
-    // (column block b lands at dst + b * bstride floats)
-    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar,
-                        int bstride = kC * 32) {
-        if (tid == 0) {
-            mbar_arrive_expect_tx(bar, (uint32_t)(nb * kC * 32 * sizeof(float)));
-            for (int b = 0; b < nb; ++b)
-                tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, bar);
-        }
-    };
-    auto issue_z = [&](int c) {
-        if constexpr (sizeof(T) == 2) {
-            if (tid == 0) {
-                mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
-                tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)(start + (int64_t)c * kC), bar_z);
-            }
-        } else if (tid == 0) { // float32 z is read straight from global memory
-            asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar_z) : "memory");
-        }
     };
     auto wait = [&](uint32_t bar, uint32_t &ph) {
         const bool w = mbar_wait_bounded(bar, ph, kWaitLimit);
         ph ^= 1u;
         return w;
     };
-    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
-
-    T av[2], bv[2]; // raw gate inputs of the next chunk to be gated
-    if (nchunks > 0) {
-        // ---- prologue: everything of chunk 0, and the K and K K^T rows of chunk 1
-        tma_tile(sm.VQ, &maps.v, xv, start, 4, bar_v, ChunkSmem<T>::kVQBlk);
-        tma_tile(sm.VQ + kC * 32, &maps.q, xq, start, 4, bar_q, ChunkSmem<T>::kVQBlk);
-        tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0);
-        tma_tile(sm.P, &maps.kq, xkk + kC, start, 2, bar_p);
-        tma_tile(sm.A, &maps.kq, xkk, start, 2, bar_a);
-        issue_z(0);
-        load_ab(0, av, bv);
-        gates(0, av, bv, 0);
-        ok = wait(bar_a, ph_a) && ok;
-        __syncthreads();
-        build_A(0);
-        __syncthreads();
-        solve(0);
-        __syncthreads(); // A is free again
-        if (nchunks > 1) {
-            tma_tile(sm.K[1], &maps.k, xq, start + kC, 4, bar_k1);
-            tma_tile(sm.A, &maps.kq, xkk, start + kC, 2, bar_a);
+    // TMA issue by the calling thread: nb 32-column boxes of 64 rows at
+    // x0 + 32 b, row t0, column block b landing at dst + b * bstride floats
+    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar,
+                        int bstride) {
+        mbar_arrive_expect_tx(bar, (uint32_t)(nb * kC * 32 * sizeof(float)));
+        for (int b = 0; b < nb; ++b)
+            tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, bar);
+    };
+    auto issue_z = [&](int c) { // by one thread
+        if constexpr (sizeof(T) == 2) {
+            mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
+            tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)(start + (int64_t)c * kC), bar_z);
+        } else { // float32 z is read straight from global memory
+            mbar_arrive(bar_z);
         }
-        ok = wait(bar_v, ph_v) && ok;
-        ok = wait(bar_q, ph_q) && ok;
-        ok = wait(bar_k0, ph_k0) && ok;
-        ok = wait(bar_p, ph_p) && ok;
-        build_P(0);
-        load_ab(1, av, bv);
-        if (__syncthreads_or(!ok))
-            ok = false;
-    }
+    };
 
-    // shared-memory descriptors at k-step 0; a k-step adds its byte offset / 16
-    constexpr uint32_t kBlk = kC * 128;       // bytes per 32-column block of a 64-row tile
-    constexpr uint32_t kVQb = 2 * kC * 128;   // bytes per 32-column block of VQ
-    const uint32_t aVQ = smem_u32(sm.VQ);
-    const uint64_t dV = sdesc_sw128_b32(aVQ, kVQb, 512);              // A of MMA 1 (MN-major)
-    const uint64_t dWQ = sdesc_sw128(aVQ, 16, 1024);                  // B of MMA 2 (K-major, N 128)
-    const uint64_t dTb = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
-    const uint64_t dTg = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
-    const uint64_t dP = sdesc_sw128(smem_u32(sm.P), 16, 1024);
-    const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kBlk, 512); // MN-major K tiles
-    const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kBlk, 512);
-    // k-step s of a K-major operand: column block s / 4, 32 bytes per step within it
-    auto kstep = [](int s, uint32_t blk) { return (uint64_t)((((s >> 2) * blk) + (s & 3) * 32) >> 4); };
-
-    for (int c = 0; c < nchunks; ++c) {
-        const int cur = c & 1, nxt = cur ^ 1;
-        const int nr = rows_of(c);
-        const int64_t t0 = start + (int64_t)c * kC;
-        const bool has_next = c + 1 < nchunks;
-        const uint64_t dK = cur ? dK1 : dK0;
-
-        fence_proxy_async_smem();
-        tc_fence_before();
-        if (__syncthreads_or(!ok)) { // leave together
-            ok = false;
-            break;
-        }
-        tc_fence_after();
-        // ---- MMA 1: U~^T = V^T (T diag b)^T and W^T = K^T (T diag b gamma)^T
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_tf32(128, kC, true, false);
+    bool ok = true;
+    if (!is_state) {
+        // ================================================================ prep group
+        const int ptid = tid - kStateThreads, pw = ptid >> 5;
+        const bool leader = ptid == 0;
+        auto psync = [&]() { group_sync(kBarPrep, kPrepThreads); };
+        // raw gate inputs of chunk c, rows lane and lane + 32 (first prep warp);
+        // converted only in gates() so that the loads overlap other work
+        auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
+            if (pw == 0) {
 #pragma unroll
-            for (int s = 0; s < kC / 8; ++s) {
-                mma_tf32_ss(tmem + kColU, dV + s * 64, dTb + kstep(s, kBlk), id, s > 0);
-                mma_tf32_ss(tmem + kColW, dK + s * 64, dTg + kstep(s, kBlk), id, s > 0);
+                for (int q = 0; q < 2; ++q) {
+                    const int r = lane + 32 * q;
+                    ra[q] = from_f<T>(0.f);
+                    rb[q] = from_f<T>(0.f);
+                    if (c < nchunks && r < rows_of(c)) {
+                        const int64_t t = start + (int64_t)c * kC + r;
+                        ra[q] = ((const T *)p.a)[t * p.Hv + h];
+                        rb[q] = ((const T *)p.b)[t * p.Hv + h];
+                    }
+                }
             }
-            mma_commit(bar_mma);
-        }
-        // the next chunk's gates while the tensor core works
-        gates(c + 1, av, bv, nxt);
-        ok = wait(bar_mma, ph_mma) && ok;
-        if (__syncthreads_or(!ok))
-            break;
-        tc_fence_after();
-        // ---- -W into the V tile (K-major: rows r, columns k = vch), tf32;
-        //      this half takes rows 32 hf .. 32 hf + 31
-        {
-            float w[32];
-            tmem_ld32(tl + kColW + 32 * hf, w);
-            tmem_wait_ld();
+        };
+        // g, beta, the inclusive prefix G, gamma = e^G and gamma_C / gamma of a
+        // chunk into slot `sl` (first prep warp; rows lane and lane + 32)
+        auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
+            if (pw == 0) {
+                float g[2], be[2];
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                sm.VQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(-w[i]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- MMA 2: [U^T | O^T] += S0 [-W; Q]^T, one N = 128 product (A = the
-        //      FP32 state in TMEM); U^T starts as U~^T, O^T as zero
-        if (tid == 0) {
-            constexpr uint32_t id = idesc_tf32(128, 2 * kC, false, false);
+                for (int q = 0; q < 2; ++q) {
+                    const bool in = c < nchunks && lane + 32 * q < rows_of(c);
+                    g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
+                    be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
+                }
 #pragma unroll
-            for (int s = 0; s < kD / 8; ++s)
-                mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, dWQ + kstep(s, kVQb), id, 1);
-            mma_commit(bar_mma);
-        }
-        // the next chunk's T while the tensor core works
-        if (has_next) {
-            ok = wait(bar_a, ph_a) && ok;
-            __syncthreads();
-            build_A(nxt);
-            __syncthreads();
-            solve(nxt);
-        }
-        ok = wait(bar_mma, ph_mma) && ok;
-        if (__syncthreads_or(!ok))
-            break;
-        tc_fence_after();
-        // V (now -W) and Q are free: fetch the next chunk's
-        if (has_next) {
-            tma_tile(sm.VQ, &maps.v, xv, t0 + kC, 4, bar_v, ChunkSmem<T>::kVQBlk);
-            tma_tile(sm.VQ + kC * 32, &maps.q, xq, t0 + kC, 4, bar_q, ChunkSmem<T>::kVQBlk);
-        }
-        // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
-        //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
-        {
-            float u[32], o[32];
-            tmem_ld32(tl + kColU + 32 * hf, u);
-            tmem_ld32(tl + kColO + 32 * hf, o);
-            tmem_wait_ld();
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
+                    const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
+                    if (lane >= o) {
+                        g[0] += x0;
+                        g[1] += x1;
+                    }
+                }
+                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+                const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
 #pragma unroll
-            for (int i = 0; i < 32; ++i)
-                o[i] *= sm.gam[cur][32 * hf + i];
-            tmem_st32(tl + kColO + 32 * hf, o);
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                o[i] = tf32_rna(u[i] * sm.kd[cur][32 * hf + i]);
-                u[i] = tf32_rna(u[i]);
+                for (int q = 0; q < 2; ++q) {
+                    const int r = lane + 32 * q;
+                    sm.G[sl][r] = g[q];
+                    sm.beta[sl][r] = be[q];
+                    sm.gam[sl][r] = expf(g[q]);
+                    sm.kd[sl][r] = expf(Glast - g[q]);
+                }
             }
-            tmem_st32(tl + kColU + 32 * hf, u);
-            tmem_st32(tl + kColUk + 32 * hf, o);
-            const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
+        };
+        // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
+        auto build_A = [&](int sl) {
+#pragma unroll 2
+            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
+                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+                float4 *p4 = reinterpret_cast<float4 *>(sm.A + swz(r, c, kC));
+                float4 x = *p4;
+                const float br = sm.beta[sl][r], Gr = sm.G[sl][r];
+                // the kq rows are 0 for s >= r and beta is 0 on padded rows; the
+                // clamp keeps the unused upper triangle finite (G_r - G_s > 0 there)
+                x.x *= br * __expf(fminf(Gr - sm.G[sl][c], 0.f));
+                x.y *= br * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f));
+                x.z *= br * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f));
+                x.w *= br * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f));
+                *p4 = x;
+            }
+        };
+        // Q K^T rows -> P in place (K-major swizzled): P[r][s] = e^{G_r - G_s} QK[r][s], tf32
+        auto build_P = [&](int sl) {
+#pragma unroll 2
+            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
+                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+                float4 *p4 = reinterpret_cast<float4 *>(sm.P + swz(r, c, kC));
+                float4 x = *p4;
+                const float Gr = sm.G[sl][r];
+                x.x = tf32_rna(x.x * __expf(fminf(Gr - sm.G[sl][c], 0.f)));
+                x.y = tf32_rna(x.y * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f)));
+                x.z = tf32_rna(x.z * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f)));
+                x.w = tf32_rna(x.w * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f)));
+                *p4 = x;
+            }
+        };
+        // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A,
+        // by block doubling: invert the four 16 x 16 diagonal blocks by forward
+        // substitution, then join pairs of blocks with [T1 0; X T2],
+        // X = -T2 A21 T1, at 32 and at 64 rows.  Finally T diag(beta) and
+        // T diag(beta gamma) are written as tf32 B operands.  sm.Tg serves as
+        // scratch for A21 T1 (MMA 1 has finished reading it).
+        auto solve = [&](int sl) {
+            float *At = sm.A;
+            float *Y = sm.Tg;
+            { // 16 x 16 diagonal block pw; lane l < 16 owns column 16 pw + l
+                const int c = 16 * pw + (lane & 15);
+                float t[16];
+#pragma unroll
+                for (int r = 0; r < 16; ++r) {
+                    float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                    for (int i = 0; i < r; ++i) {
+                        const float a = At[swz(16 * pw + r, 16 * pw + i, kC)];
+                        if (i & 1)
+                            acc1 = fmaf(a, t[i], acc1);
+                        else
+                            acc0 = fmaf(a, t[i], acc0);
+                    }
+                    const int rr = 16 * pw + r;
+                    t[r] = rr == c ? 1.f : (rr < c ? 0.f : -(acc0 + acc1));
+                }
+                __syncwarp();
+                if (lane < 16) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r)
+                        At[swz(16 * pw + r, c, kC)] = t[r];
+                }
+            }
+            psync();
+            { // join at 32 rows, blocks b = 0 (rows 0..31) and 1 (rows 32..63); thread:
+              // rows r0, r0 + 1 of the 16 x 16 product, columns c0, c0 + 1
+                const int b = ptid >> 6, q = ptid & 63;
+                const int o = 32 * b, r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
+                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a0 = At[swz(o + 16 + r0, o + i, kC)];
+                    const float a1 = At[swz(o + 17 + r0, o + i, kC)];
+                    const float t0 = At[swz(o + i, o + c0, kC)];
+                    const float t1 = At[swz(o + i, o + c0 + 1, kC)];
+                    y00 = fmaf(a0, t0, y00); y01 = fmaf(a0, t1, y01);
+                    y10 = fmaf(a1, t0, y10); y11 = fmaf(a1, t1, y11);
+                }
+                Y[b * 256 + r0 * 16 + c0] = y00;
+                Y[b * 256 + r0 * 16 + c0 + 1] = y01;
+                Y[b * 256 + (r0 + 1) * 16 + c0] = y10;
+                Y[b * 256 + (r0 + 1) * 16 + c0 + 1] = y11;
+                psync();
+                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float a0 = At[swz(o + 16 + r0, o + 16 + i, kC)];
+                    const float a1 = At[swz(o + 17 + r0, o + 16 + i, kC)];
+                    const float t0 = Y[b * 256 + i * 16 + c0];
+                    const float t1 = Y[b * 256 + i * 16 + c0 + 1];
+                    x00 = fmaf(a0, t0, x00); x01 = fmaf(a0, t1, x01);
+                    x10 = fmaf(a1, t0, x10); x11 = fmaf(a1, t1, x11);
+                }
+                // A21 was read only before the barrier above: overwrite it in place
+                At[swz(o + 16 + r0, o + c0, kC)] = -x00;
+                At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x01;
+                At[swz(o + 17 + r0, o + c0, kC)] = -x10;
+                At[swz(o + 17 + r0, o + c0 + 1, kC)] = -x11;
+            }
+            psync();
+            { // join at 64 rows: thread: rows r0, r0 + 1 of the 32 x 32 product, columns c0 .. + 3
+                const int r0 = 2 * (ptid >> 3), c0 = 4 * (ptid & 7);
+                float y[2][4] = {};
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const float a0 = At[swz(32 + r0, i, kC)];
+                    const float a1 = At[swz(33 + r0, i, kC)];
+                    const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(i, c0, kC));
+                    y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
+                    y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
+                    y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
+                    y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
+                }
+                *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) =
+                    make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
+                *reinterpret_cast<float4 *>(Y + (r0 + 1) * 36 + c0) =
+                    make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
+                psync();
+                float x[2][4] = {};
+#pragma unroll 8
+                for (int i = 0; i < 32; ++i) {
+                    const float a0 = At[swz(32 + r0, 32 + i, kC)];
+                    const float a1 = At[swz(33 + r0, 32 + i, kC)];
+                    const float4 t4 = *reinterpret_cast<const float4 *>(Y + i * 36 + c0);
+                    x[0][0] = fmaf(a0, t4.x, x[0][0]); x[0][1] = fmaf(a0, t4.y, x[0][1]);
+                    x[0][2] = fmaf(a0, t4.z, x[0][2]); x[0][3] = fmaf(a0, t4.w, x[0][3]);
+                    x[1][0] = fmaf(a1, t4.x, x[1][0]); x[1][1] = fmaf(a1, t4.y, x[1][1]);
+                    x[1][2] = fmaf(a1, t4.z, x[1][2]); x[1][3] = fmaf(a1, t4.w, x[1][3]);
+                }
+                *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
+                    make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
+                *reinterpret_cast<float4 *>(At + swz(33 + r0, c0, kC)) =
+                    make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
+            }
+            psync();
+            // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
+#pragma unroll 2
+            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
+                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
+                const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(r, c, kC));
+                const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][c]);
+                const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][c]);
+                const float4 tb = make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
+                *reinterpret_cast<float4 *>(sm.Tb + swz(r, c, kC)) = tf32_rna(tb);
+                *reinterpret_cast<float4 *>(sm.Tg + swz(r, c, kC)) =
+                    tf32_rna(make_float4(tb.x * g4.x, tb.y * g4.y, tb.z * g4.z, tb.w * g4.w));
+            }
+        };
+
+        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phv = 0, phk0 = 0, phk1 = 0, php = 0, pha = 0;
+        const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.VQ), 2 * kC * 128, 512); // A of MMA 1
+        const uint64_t dTb = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
+        const uint64_t dTg = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
+        const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
+        const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
+        constexpr int kVQBlk = ChunkSmem<T>::kVQBlk;
+        T av[2], bv[2]; // raw gate inputs of the next chunk to be gated
+        if (nchunks > 0) {
+            // ---- prologue: all tiles of chunk 0, its gates, T and P
+            if (leader) {
+                tma_tile(sm.VQ, &maps.v, xv, start, 4, bar_v, kVQBlk);
+                tma_tile(sm.VQ + kC * 32, &maps.q, xq, start, 4, bar_q, kVQBlk);
+                tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0, kC * 32);
+                tma_tile(sm.P, &maps.kq, xkk + kC, start, 2, bar_p, kC * 32);
+                tma_tile(sm.A, &maps.kq, xkk, start, 2, bar_a, kC * 32);
+                issue_z(0);
+            }
+            load_ab(0, av, bv);
+            gates(0, av, bv, 0);
+            ok = wait(bar_a, pha) && ok;
+            psync();
+            build_A(0);
+            psync();
+            solve(0);
+            psync(); // A is free again
+            if (leader && nchunks > 1) {
+                tma_tile(sm.K[1], &maps.k, xq, start + kC, 4, bar_k1, kC * 32);
+                tma_tile(sm.A, &maps.kq, xkk, start + kC, 2, bar_a, kC * 32);
+            }
+            ok = wait(bar_p, php) && ok;
+            build_P(0);
+            load_ab(1, av, bv);
+            fence_proxy_async_smem();
+            psync();
+            if (leader)
+                mbar_arrive(bar_prep); // chunk 0 ready
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int cur = c & 1, nxt = cur ^ 1;
+            const int64_t t0 = start + (int64_t)c * kC;
+            const bool has_next = c + 1 < nchunks;
+            // ---- MMA 1: U~^T = V^T (T diag b)^T and W^T = K^T (T diag b gamma)^T
+            if (leader) {
+                ok = wait(bar_v, phv) && ok;
+                ok = (cur ? wait(bar_k1, phk1) : wait(bar_k0, phk0)) && ok;
+                tc_fence_after();
+                const uint64_t dK = cur ? dK1 : dK0;
+                constexpr uint32_t id = idesc_tf32(128, kC, true, false);
+#pragma unroll
+                for (int s = 0; s < kC / 8; ++s) {
+                    const uint64_t ks = (uint64_t)((((s >> 2) * kC * 128) + (s & 3) * 32) >> 4);
+                    mma_tf32_ss(tmem + kColU, dV + s * 64, dTb + ks, id, s > 0);
+                    mma_tf32_ss(tmem + kColW, dK + s * 64, dTg + ks, id, s > 0);
+                }
+                mma_commit(bar_mma1);
+            }
+            gates(c + 1, av, bv, nxt);
+            ok = wait(bar_mma1, ph1) && ok; // T diag(b), T diag(b gamma) are free
+            if (has_next) {
+                ok = wait(bar_a, pha) && ok;
+                psync();
+                build_A(nxt);
+                psync();
+                solve(nxt);
+                fence_proxy_async_smem();
+                psync(); // A is free, Tb / Tg of the next chunk are written
+            }
+            ok = wait(bar_mma2, ph2) && ok; // V (then -W) and Q are free
+            if (leader && has_next) {
+                tma_tile(sm.VQ, &maps.v, xv, t0 + kC, 4, bar_v, kVQBlk);
+                tma_tile(sm.VQ + kC * 32, &maps.q, xq, t0 + kC, 4, bar_q, kVQBlk);
+            }
+            ok = wait(bar_mma3, ph3) && ok; // P, K[cur] and the U / W columns are free
+            if (leader) {
+                if (has_next)
+                    tma_tile(sm.P, &maps.kq, xkk + kC, t0 + kC, 2, bar_p, kC * 32);
+                if (c + 2 < nchunks) {
+                    tma_tile(sm.K[cur], &maps.k, xq, t0 + 2 * kC, 4, cur ? bar_k1 : bar_k0, kC * 32);
+                    tma_tile(sm.A, &maps.kq, xkk, t0 + 2 * kC, 2, bar_a, kC * 32);
+                }
+            }
+            load_ab(c + 2, av, bv);
+            if (has_next) {
+                ok = wait(bar_p, php) && ok;
+                build_P(nxt);
+                fence_proxy_async_smem();
+                psync();
+                if (leader)
+                    mbar_arrive(bar_prep); // the next chunk is ready
+            }
+            if (group_sync_or(kBarPrep, kPrepThreads, !ok || *(volatile int *)&sm.abort)) {
+                ok = false;
+                break;
+            }
+        }
+        if (!ok)
+            *(volatile int *)&sm.abort = 1;
+    } else {
+        // ================================================================ state group
+        const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
+        const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
+        const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
+        auto ssync = [&]() { group_sync(kBarState, kStateThreads); };
+        // initial state into TMEM (row vch, this half's 64 columns); O starts at zero
+        {
+            const float *src = p.init_state
+                                   ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
+                                   : nullptr;
 #pragma unroll
             for (int cb = 0; cb < 2; ++cb) {
                 float v[32];
-                tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+#pragma unroll
+                for (int i = 0; i < 32; i += 4) {
+                    float4 x = src ? *reinterpret_cast<const float4 *>(src + cb * 32 + i)
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+                    v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+                }
+                tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+            }
+            float zero[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                zero[i] = 0.f;
+            tmem_st32(tl + kColO + 32 * hf, zero); // MMA 2 accumulates onto O
+            tmem_wait_st();
+        }
+        const float wn = __ldg(p.norm_w + vch);
+        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phq = 0, phz = 0, phr = 0;
+        const uint64_t dWQ = sdesc_sw128(smem_u32(sm.VQ), 16, 1024); // B of MMA 2 (N = 128)
+        const uint64_t dP = sdesc_sw128(smem_u32(sm.P), 16, 1024);
+        const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
+        const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
+        for (int c = 0; c < nchunks; ++c) {
+            const int cur = c & 1;
+            const int nr = rows_of(c);
+            const int64_t t0 = start + (int64_t)c * kC;
+            ok = wait(bar_mma1, ph1) && ok;
+            tc_fence_after();
+            // ---- -W into rows 0..63 of VQ (K-major: rows r, columns k = vch), tf32;
+            //      this half takes rows 32 hf .. 32 hf + 31
+            {
+                float w[32];
+                tmem_ld32(tl + kColW + 32 * hf, w);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    v[i] *= gC;
-                tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+                    sm.VQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(-w[i]);
             }
-            tmem_wait_st();
-        }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        // ---- MMA 3: O^T += U^T P^T and S += (U diag(gamma_C/gamma))^T K
-        if (tid == 0) {
-            constexpr uint32_t idp = idesc_tf32(128, kC, false, false);
-            constexpr uint32_t ids = idesc_tf32(128, kD, false, true);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            ssync();
+            tc_fence_after();
+            // ---- MMA 2: [U^T | O^T] += S0 [-W; Q]^T, one N = 128 product (A = the
+            //      FP32 state in TMEM); U^T starts as U~^T, O^T as zero
+            if (tid == 0) {
+                ok = wait(bar_q, phq) && ok;
+                constexpr uint32_t id = idesc_tf32(128, 2 * kC, false, false);
 #pragma unroll
-            for (int s = 0; s < kC / 8; ++s) {
-                mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, dP + kstep(s, kBlk), idp, 1);
-                mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, ids, 1);
-            }
-            mma_commit(bar_mma);
-        }
-        ok = wait(bar_z, ph_z) && ok; // z rows of this chunk
-        ok = wait(bar_mma, ph_mma) && ok;
-        if (__syncthreads_or(!ok))
-            break;
-        tc_fence_after();
-        // P and K[cur] are free: fetch the next chunk's Q K^T rows, and the K
-        // and K K^T rows of the chunk after it
-        if (has_next)
-            tma_tile(sm.P, &maps.kq, xkk + kC, t0 + kC, 2, bar_p);
-        if (c + 2 < nchunks) {
-            tma_tile(sm.K[cur], &maps.k, xq, t0 + 2 * kC, 4, cur ? bar_k1 : bar_k0);
-            tma_tile(sm.A, &maps.kq, xkk, t0 + 2 * kC, 2, bar_a);
-        }
-        load_ab(c + 2, av, bv);
-        // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
-        //      RMSNorm over v, times w[v] SiLU(z), stored
-        {
-            float o[32], sq[32];
-            tmem_ld32(tl + kColO + 32 * hf, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                sq[i] = o[i] * o[i];
-            // reduce-scatter over the 32 lanes: lane l ends with row 32 hf + l
-#pragma unroll
-            for (int w = 16; w >= 1; w >>= 1) {
-                const bool upper = (lane & w) != 0;
-#pragma unroll
-                for (int i = 0; i < w; ++i) {
-                    const float send = upper ? sq[i] : sq[i + w];
-                    const float keep = upper ? sq[i + w] : sq[i];
-                    sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                for (int s = 0; s < kD / 8; ++s) {
+                    const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
+                    mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, dWQ + ks, id, 1);
                 }
+                mma_commit(bar_mma2);
             }
-            sm.red[lq][32 * hf + lane] = sq[0];
-            __syncthreads();
-            if (tid < kC)
-                sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
-                                       sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
-            __syncthreads();
-            // y[t0 + r][h][vch] for this half's rows r = 32 hf + i
-            T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
-            float *op = p.o_raw ? p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch : nullptr;
-            const int rows = nr - 32 * hf; // valid rows of this half (may be <= 0)
-            auto emit = [&](int i) {
-                float zv;
-                if constexpr (sizeof(T) == 2)
-                    zv = to_f(sm.Z[(32 * hf + i) * kD + vch]);
-                else
-                    zv = to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD + (int64_t)h * kD + vch]);
-                const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
-                yp[i * HD] = from_f<T>(o[i] * (sm.rstd[32 * hf + i] * wn) * gate);
-            };
-            if (rows >= 32) {
+            ok = wait(bar_mma2, ph2) && ok;
+            ok = wait(bar_prep, phr) && ok; // this chunk's gates and P
+            tc_fence_after();
+            // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
+            //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
+            {
+                float u[32], o[32];
+                tmem_ld32(tl + kColU + 32 * hf, u);
+                tmem_ld32(tl + kColO + 32 * hf, o);
+                tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    emit(i);
-            } else {
+                    o[i] *= sm.gam[cur][32 * hf + i];
+                tmem_st32(tl + kColO + 32 * hf, o);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    o[i] = tf32_rna(u[i] * sm.kd[cur][32 * hf + i]);
+                    u[i] = tf32_rna(u[i]);
+                }
+                tmem_st32(tl + kColU + 32 * hf, u);
+                tmem_st32(tl + kColUk + 32 * hf, o);
+                const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
+#pragma unroll
+                for (int cb = 0; cb < 2; ++cb) {
+                    float v[32];
+                    tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        v[i] *= gC;
+                    tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+                }
+                tmem_wait_st();
+            }
+            tc_fence_before();
+            ssync();
+            tc_fence_after();
+            // ---- MMA 3: O^T += U^T P^T and S += (U diag(gamma_C/gamma))^T K
+            if (tid == 0) {
+                const uint64_t dK = cur ? dK1 : dK0;
+                constexpr uint32_t idp = idesc_tf32(128, kC, false, false);
+                constexpr uint32_t ids = idesc_tf32(128, kD, false, true);
+#pragma unroll
+                for (int s = 0; s < kC / 8; ++s) {
+                    const uint64_t ks = (uint64_t)((((s >> 2) * kC * 128) + (s & 3) * 32) >> 4);
+                    mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, dP + ks, idp, 1);
+                    mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, ids, 1);
+                }
+                mma_commit(bar_mma3);
+            }
+            ok = wait(bar_z, phz) && ok; // z rows of this chunk
+            ok = wait(bar_mma3, ph3) && ok;
+            tc_fence_after();
+            // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
+            //      RMSNorm over v, times w[v] SiLU(z), stored; then O is zeroed
+            {
+                float o[32], sq[32];
+                tmem_ld32(tl + kColO + 32 * hf, o);
+                tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (i < rows)
+                    sq[i] = o[i] * o[i];
+                // reduce-scatter over the 32 lanes: lane l ends with row 32 hf + l
+#pragma unroll
+                for (int w = 16; w >= 1; w >>= 1) {
+                    const bool upper = (lane & w) != 0;
+#pragma unroll
+                    for (int i = 0; i < w; ++i) {
+                        const float send = upper ? sq[i] : sq[i + w];
+                        const float keep = upper ? sq[i + w] : sq[i];
+                        sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                    }
+                }
+                sm.red[lq][32 * hf + lane] = sq[0];
+                ssync();
+                if (tid < kC)
+                    sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
+                                           sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
+                ssync();
+                T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
+                float *op = p.o_raw ? p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch : nullptr;
+                const int rows = nr - 32 * hf; // valid rows of this half (may be <= 0)
+                auto emit = [&](int i) {
+                    float zv;
+                    if constexpr (sizeof(T) == 2)
+                        zv = to_f(sm.Z[(32 * hf + i) * kD + vch]);
+                    else
+                        zv = to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD + (int64_t)h * kD + vch]);
+                    const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
+                    yp[i * HD] = from_f<T>(o[i] * (sm.rstd[32 * hf + i] * wn) * gate);
+                };
+                if (rows >= 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
                         emit(i);
-            }
-            if (op != nullptr) {
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < rows)
+                            emit(i);
+                }
+                if (op != nullptr) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < rows)
+                            op[i * HD] = o[i];
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    if (i < rows)
-                        op[i * HD] = o[i];
+                    o[i] = 0.f;
+                tmem_st32(tl + kColO + 32 * hf, o); // MMA 2 accumulates onto O
+                tmem_wait_st();
             }
-            // O is consumed: zero it, since MMA 2 accumulates onto it
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                o[i] = 0.f;
-            tmem_st32(tl + kColO + 32 * hf, o);
-            tmem_wait_st();
+            tc_fence_before();
+            const bool bad = group_sync_or(kBarState, kStateThreads,
+                                           !ok || *(volatile int *)&sm.abort); // Z is read
+            tc_fence_after();
+            if (bad) {
+                ok = false;
+                break;
+            }
+            if (tid == 0 && c + 1 < nchunks)
+                issue_z(c + 1);
         }
-        __syncthreads(); // Z is read; red / rstd are reused
-        if (has_next) {
-            issue_z(c + 1);
-            // the next chunk's tiles
-            ok = wait(bar_v, ph_v) && ok;
-            ok = wait(bar_q, ph_q) && ok;
-            ok = wait(nxt ? bar_k1 : bar_k0, nxt ? ph_k1 : ph_k0) && ok;
-            ok = wait(bar_p, ph_p) && ok;
-            build_P(nxt);
-        }
+        if (!ok)
+            *(volatile int *)&sm.abort = 1;
     }
 
     ok = !__syncthreads_or(!ok); // one verdict for the whole CTA
     if (!ok) {
         if (tid == 0 && p.ws_err != nullptr)
             atomicOr(p.ws_err, 1u);
-    } else if (p.final_state != nullptr) {
+    } else if (is_state && p.final_state != nullptr) {
+        const int lq = warp & 3, hf = warp >> 2, vch = lq * 32 + lane;
+        const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
         float *dst = p.final_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf;
 #pragma unroll
         for (int cb = 0; cb < 2; ++cb) {
