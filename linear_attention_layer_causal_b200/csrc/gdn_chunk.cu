@@ -388,37 +388,56 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
             }
         };
+        // Each prep thread owns the float4 at column c = 4 (ptid % 16) of rows
+        // r = ptid / 16 + 8 k, k = 0..7, in the 64 x 64 tiles below.  Every
+        // pass loads all its inputs before its first store, so that the
+        // compiler need not order later loads behind stores it cannot
+        // disambiguate.
+        const int pc = 4 * (ptid & 15), pr = ptid >> 4;
         // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
+        // (the kq rows are 0 for s >= r and beta is 0 on padded rows; the
+        // clamp keeps the unused upper triangle finite: G_r - G_s > 0 there)
         auto build_A = [&](int sl) {
-#pragma unroll 2
-            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
-                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-                float4 *p4 = reinterpret_cast<float4 *>(sm.A + swz(r, c, kC));
-                float4 x = *p4;
-                const float br = sm.beta[sl][r], Gr = sm.G[sl][r];
-                // the kq rows are 0 for s >= r and beta is 0 on padded rows; the
-                // clamp keeps the unused upper triangle finite (G_r - G_s > 0 there)
-                x.x *= br * __expf(fminf(Gr - sm.G[sl][c], 0.f));
-                x.y *= br * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f));
-                x.z *= br * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f));
-                x.w *= br * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f));
-                *p4 = x;
+            const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][pc]);
+            float4 x[8];
+            float Gr[8], br[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                x[k] = *reinterpret_cast<const float4 *>(sm.A + swz(pr + 8 * k, pc, kC));
+                Gr[k] = sm.G[sl][pr + 8 * k];
+                br[k] = sm.beta[sl][pr + 8 * k];
             }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                x[k].x *= br[k] * __expf(fminf(Gr[k] - Gc.x, 0.f));
+                x[k].y *= br[k] * __expf(fminf(Gr[k] - Gc.y, 0.f));
+                x[k].z *= br[k] * __expf(fminf(Gr[k] - Gc.z, 0.f));
+                x[k].w *= br[k] * __expf(fminf(Gr[k] - Gc.w, 0.f));
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4 *>(sm.A + swz(pr + 8 * k, pc, kC)) = x[k];
         };
         // Q K^T rows -> P in place (K-major swizzled): P[r][s] = e^{G_r - G_s} QK[r][s], tf32
         auto build_P = [&](int sl) {
-#pragma unroll 2
-            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
-                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-                float4 *p4 = reinterpret_cast<float4 *>(sm.P + swz(r, c, kC));
-                float4 x = *p4;
-                const float Gr = sm.G[sl][r];
-                x.x = tf32_rna(x.x * __expf(fminf(Gr - sm.G[sl][c], 0.f)));
-                x.y = tf32_rna(x.y * __expf(fminf(Gr - sm.G[sl][c + 1], 0.f)));
-                x.z = tf32_rna(x.z * __expf(fminf(Gr - sm.G[sl][c + 2], 0.f)));
-                x.w = tf32_rna(x.w * __expf(fminf(Gr - sm.G[sl][c + 3], 0.f)));
-                *p4 = x;
+            const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][pc]);
+            float4 x[8];
+            float Gr[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                x[k] = *reinterpret_cast<const float4 *>(sm.P + swz(pr + 8 * k, pc, kC));
+                Gr[k] = sm.G[sl][pr + 8 * k];
             }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                x[k].x = tf32_rna(x[k].x * __expf(fminf(Gr[k] - Gc.x, 0.f)));
+                x[k].y = tf32_rna(x[k].y * __expf(fminf(Gr[k] - Gc.y, 0.f)));
+                x[k].z = tf32_rna(x[k].z * __expf(fminf(Gr[k] - Gc.z, 0.f)));
+                x[k].w = tf32_rna(x[k].w * __expf(fminf(Gr[k] - Gc.w, 0.f)));
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                *reinterpret_cast<float4 *>(sm.P + swz(pr + 8 * k, pc, kC)) = x[k];
         };
         // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A,
         // by block doubling: invert the four 16 x 16 diagonal blocks by forward
@@ -526,16 +545,22 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             psync();
             // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
-#pragma unroll 2
-            for (int e = ptid; e < kC * kC / 4; e += kPrepThreads) {
-                const int r = e / (kC / 4), c = (e % (kC / 4)) * 4;
-                const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(r, c, kC));
-                const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][c]);
-                const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][c]);
-                const float4 tb = make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w);
-                *reinterpret_cast<float4 *>(sm.Tb + swz(r, c, kC)) = tf32_rna(tb);
-                *reinterpret_cast<float4 *>(sm.Tg + swz(r, c, kC)) =
-                    tf32_rna(make_float4(tb.x * g4.x, tb.y * g4.y, tb.z * g4.z, tb.w * g4.w));
+            {
+                const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][pc]);
+                const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][pc]);
+                const float4 bg = make_float4(b4.x * g4.x, b4.y * g4.y, b4.z * g4.z, b4.w * g4.w);
+                float4 t4[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    t4[k] = *reinterpret_cast<const float4 *>(At + swz(pr + 8 * k, pc, kC));
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    const int o = swz(pr + 8 * k, pc, kC);
+                    *reinterpret_cast<float4 *>(sm.Tb + o) = tf32_rna(
+                        make_float4(t4[k].x * b4.x, t4[k].y * b4.y, t4[k].z * b4.z, t4[k].w * b4.w));
+                    *reinterpret_cast<float4 *>(sm.Tg + o) = tf32_rna(
+                        make_float4(t4[k].x * bg.x, t4[k].y * bg.y, t4[k].z * bg.z, t4[k].w * bg.w));
+                }
             }
         };
 
@@ -710,22 +735,27 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
             //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
             {
-                float u[32], o[32];
+                float u[32], o[32], gm[32], kf[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    gm[i] = sm.gam[cur][32 * hf + i];
+                    kf[i] = sm.kd[cur][32 * hf + i];
+                }
+                const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
                 tmem_ld32(tl + kColU + 32 * hf, u);
                 tmem_ld32(tl + kColO + 32 * hf, o);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    o[i] *= sm.gam[cur][32 * hf + i];
+                    o[i] *= gm[i];
                 tmem_st32(tl + kColO + 32 * hf, o);
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    o[i] = tf32_rna(u[i] * sm.kd[cur][32 * hf + i]);
+                    o[i] = tf32_rna(u[i] * kf[i]);
                     u[i] = tf32_rna(u[i]);
                 }
                 tmem_st32(tl + kColU + 32 * hf, u);
                 tmem_st32(tl + kColUk + 32 * hf, o);
-                const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
 #pragma unroll
                 for (int cb = 0; cb < 2; ++cb) {
                     float v[32];
@@ -784,32 +814,38 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                                            sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
                 ssync();
                 T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
-                float *op = p.o_raw ? p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch : nullptr;
                 const int rows = nr - 32 * hf; // valid rows of this half (may be <= 0)
-                auto emit = [&](int i) {
-                    float zv;
-                    if constexpr (sizeof(T) == 2)
-                        zv = to_f(sm.Z[(32 * hf + i) * kD + vch]);
-                    else
-                        zv = to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD + (int64_t)h * kD + vch]);
-                    const float gate = __fdividef(zv, 1.0f + __expf(-zv)); // SiLU(z)
-                    yp[i * HD] = from_f<T>(o[i] * (sm.rstd[32 * hf + i] * wn) * gate);
-                };
-                if (rows >= 32) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        emit(i);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < rows)
-                            emit(i);
-                }
-                if (op != nullptr) {
+                if (p.o_raw != nullptr) {
+                    float *op = p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
 #pragma unroll
                     for (int i = 0; i < 32; ++i)
                         if (i < rows)
                             op[i * HD] = o[i];
+                }
+                // all loads first, then the arithmetic, then the stores
+                float zr[32], sc[32];
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    if constexpr (sizeof(T) == 2)
+                        zr[i] = to_f(sm.Z[(32 * hf + i) * kD + vch]);
+                    else
+                        zr[i] = i < rows ? to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD +
+                                                                  (int64_t)h * kD + vch])
+                                         : 0.f;
+                    sc[i] = sm.rstd[32 * hf + i];
+                }
+#pragma unroll
+                for (int i = 0; i < 32; ++i) // o * rstd * w * SiLU(z)
+                    o[i] = o[i] * (sc[i] * wn) * __fdividef(zr[i], 1.0f + __expf(-zr[i]));
+                if (rows >= 32) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        yp[i * HD] = from_f<T>(o[i]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        if (i < rows)
+                            yp[i * HD] = from_f<T>(o[i]);
                 }
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
