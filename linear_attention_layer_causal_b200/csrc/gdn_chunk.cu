@@ -17,21 +17,16 @@
 // factor exceeds 1 however strong the decay.
 //
 // Mapping onto the tensor core (M = 128 = d_v is the TMEM lane dimension):
-//   U~^T = V^T (T diag b)^T          A = V  (smem, MN-major)   B = T diag b (smem)
-//   W^T  = K^T (T diag b gamma)^T    A = K  (smem, MN-major)   B = T diag b gamma
-//   U^T  = U~^T + S0 (-W)^T          A = S0 (TMEM)             B = -W (smem)
-//   O^T  = S0 Q^T, then column r * gamma_r     A = S0 (TMEM)   B = Q (smem)
-//   O^T += U^T P^T                   A = U^T (TMEM)            B = P (smem)
-//   S   <- gamma_C S + (U diag(gamma_C/gamma))^T K    A = TMEM  B = K (smem, MN-major)
-// The FP32 state lives in TMEM for the whole sequence and is itself the A
-// operand of the state products.  All products run as kind::tf32.  The
-// operands computed here (T diag b, -W, P and both forms of U) are rounded to
-// nearest before the tensor core reads them, since its own conversion
-// truncates and the resulting bias in U accumulates through the state; v is
-// rounded where it is produced; for S, q and k the truncation costs nothing
-// measurable.  The intra-chunk Gram matrices K K^T and Q K^T, to which
-// near-cancelling outputs are most sensitive, come exact in FP32 from
-// kq_prep_kernel.
+//   MMA 1  U~^T = V^T (T diag b)^T,  -W^T = K^T (-T diag b gamma)^T
+//          A = V, K (smem, MN-major), B = the two T tiles (smem, K-major)
+//   MMA 2  [U^T | O^T] += S0 [-W ; diag(gamma) Q]^T   (one N = 128 product,
+//          A = the FP32 state in TMEM; U^T starts as U~^T, O^T as zero)
+//   MMA 3  O^T += U^T P^T  and  S += (U diag(gamma_C/gamma))^T K
+// The state lives in TMEM for the whole sequence.  All products run as
+// kind::tf32; every operand computed here is rounded to nearest first (the
+// tensor core's own conversion truncates, a bias that would accumulate
+// through the state).  The Gram matrices K K^T and Q K^T come exact in FP32
+// from kq_prep_kernel: the near-cancelling outputs are sensitive to them.
 //
 // The gated RMSNorm y = o / rms(o) * w * SiLU(z) ("Qwen3.8-2.4T-A95B vs
 // Inkling", output-gate row) is fused into the output store.
@@ -169,78 +164,94 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
 
 // ------------------------------------------------------------ chunk kernel
 //
-// Two warp groups work on consecutive chunks at once:
-//   state group (warps 0..7): reads and rewrites TMEM (the W pass, the pass
-//     that rounds U and scales O and S, the gated-RMSNorm epilogue) and issues
-//     MMA 2 and MMA 3 of the current chunk; warps w and w + 4 share TMEM lanes
-//     32 (w % 4) .. + 31 (lane i = value channel i) and split the columns;
-//   prep group (warps 8..11): builds the next chunk's gates, A, T = (I+A)^-1,
-//     T diag(beta), T diag(beta gamma) and P on the CUDA cores, issues every
-//     TMA load and MMA 1.
-// They hand over through mbarriers: MMA 1/2/3 completion (tcgen05.commit), a
-// "prep ready" arrival, and the TMA transaction barriers of each tile.
+// One CTA per (value head, sequence), five roles that run consecutive chunks
+// at once and hand over through mbarriers:
+//   state group (warps 0..7): the W pass (-W^T from TMEM to shared memory),
+//     the U pass (U and U diag(gamma_C/gamma) rounded, S scaled by gamma_C)
+//     and the gated-RMSNorm epilogue; warps w and w + 4 share TMEM lanes
+//     32 (w % 4) .. + 31 (lane = value channel) and split the columns.  O and
+//     U are double-buffered in TMEM, so the epilogue of chunk c overlaps MMA 2
+//     of chunk c + 1;
+//   T team (warps 8..11): gates, A, T = (I + A)^-1 in a working tile of its
+//     own, then T diag(beta) and -T diag(beta gamma) once MMA 1 of the
+//     previous chunk has released them;
+//   P team (warps 12..13): diag(gamma) Q in place and P from the Q K^T tile;
+//   MMA warp (warp 14) and TMA warp (warp 15): one elected lane each.
+// Sixteen warps, four per scheduler, leave 128 registers a thread.
+// The per-chunk critical path is MMA 2 -> U pass -> MMA 3 -> MMA 2; MMA 1 and
+// the W pass of the next chunk run beside the U pass.
 
-constexpr int kStateThreads = 256;
-constexpr int kPrepThreads = 128;
-constexpr int kThreads = kStateThreads + kPrepThreads;
-constexpr int kBarState = 1, kBarPrep = 2; // named barriers of the two groups
+constexpr int kSG = 256;                          // state group threads
+constexpr int kTeam = 128;                        // T team threads
+constexpr int kTeamP = 64;                        // P team threads
+constexpr int kThreads = kSG + kTeam + kTeamP + 64; // + MMA warp + TMA warp: 16 warps
+constexpr int kWarpMma = (kSG + kTeam + kTeamP) / 32; // 14
+constexpr int kBarSG = 1, kBarT = 2, kBarP = 3;   // named barriers
 
-// TMEM columns
-constexpr uint32_t kColS = 0;    // state S (FP32), 128 columns; also the A operand of S [-W; Q]^T
-constexpr uint32_t kColU = 128;  // U^T (starts as U~^T), 64 columns
-constexpr uint32_t kColO = 192;  // O^T, 64 columns (directly after U^T: MMA 2 writes both)
-constexpr uint32_t kColW = 256;  // W^T, 64 columns
-constexpr uint32_t kColUk = 320; // U^T diag(gamma_C / gamma) rounded to tf32, 64 columns
+// TMEM columns: state, two [U | O] pairs (MMA 2 writes one pair with a single
+// N = 128 product), -W^T, U diag(gamma_C / gamma)
+constexpr uint32_t kColS = 0;
+constexpr uint32_t kColU0 = 128, kColU1 = 256; // O of each pair sits 64 columns on
+constexpr uint32_t kColW = 384;
+constexpr uint32_t kColUk = 448;
 constexpr uint32_t kTmemCols = 512;
 
-// Both operand layouts below split a tile of R rows along its contiguous
-// dimension into 32-float (128-byte) column blocks of R rows each.
+// Operand layouts.  Both split a tile along its contiguous dimension into
+// 32-float (128-byte) column blocks.
 //
 // K-major operand (rows = M or N, columns = K), 128-byte swizzle: the 16-byte
-// chunks of row r are XOR-swizzled by r mod 8.
+// chunks of row r are XOR-swizzled by r mod 8; blocks of R rows.
 __device__ __forceinline__ int swz(int r, int c, int R) {
     return (c >> 5) * (R * 32) + r * 32 + ((((c & 31) >> 2) ^ (r & 7)) << 2) + (c & 3);
 }
-// MN-major tf32 operand (rows = K, columns = M or N), 128-byte swizzle on a
-// 32-byte base: the 32-byte chunks of row k are XOR-swizzled by k mod 4.
-__device__ __forceinline__ int swz_mn(int k, int c, int R) {
-    return (c >> 5) * (R * 32) + k * 32 + ((((c & 31) >> 3) ^ (k & 3)) << 3) + (c & 7);
-}
+// MN-major tf32 operands (V, K) use the 128-byte swizzle on a 32-byte base,
+// written only by TMA: 32-byte chunks of row k XOR-swizzled by k mod 4.
+// Lower-triangular 64 x 64 tile in the K-major layout with its zero quadrant
+// (rows 0..31, columns 32..63) left out: column block 0 holds rows 0..63
+// (2048 floats), block 1 rows 32..63 only (1024 floats).  An MMA over the
+// tile takes block 0 with N = 64 and block 1 with N = 32 at row 32.  Element
+// (r, c) sits at swz(r, c, 64) for c < 32 and at 1024 + swz(r, c - 32, 64)
+// for c >= 32 (r >= 32); the passes below fold these into per-thread bases.
+constexpr int kTriFloats = 3 * 1024;
 
-template <typename T> struct __align__(1024) ChunkSmem {
-    // V and Q share 32-column blocks of 128 rows: rows 0..63 hold V (A,
-    // MN-major, for MMA 1), then -W; rows 64..127 hold Q; so that [-W; Q] is
-    // one K-major N = 128 operand of MMA 2
-    float VQ[2 * kC * kD];
-    float K[2][kC * kD];  // A / B, MN-major: K of this chunk and the next (ping-pong)
-    float Tb[kC * kC];    // B, K-major: T diag(beta)
-    float Tg[kC * kC];    // B, K-major: T diag(beta gamma)
-    float P[kC * kC];     // B, K-major: P (lands as raw Q K^T rows)
-    float A[kC * kC];     // the next chunk's A (lands as raw K K^T rows), then T; K-major swizzle
-    T Z[sizeof(T) == 2 ? kC * kD : 1]; // z rows of this chunk (16-bit activations only)
-    float G[2][kC], beta[2][kC];      // cumulative log-decay and beta, by chunk parity
-    float gam[2][kC], kd[2][kC];      // gamma_r = e^{G_r} and gamma_C / gamma_r
-    float red[4][kC];
-    float rstd[kC];
-    unsigned long long bar_mma1, bar_mma2, bar_mma3, bar_prep;
-    unsigned long long bar_v, bar_q, bar_k[2], bar_p, bar_a, bar_z;
+struct __align__(1024) ChunkSmem {
+    // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = -W, rows 64..127 = diag(gamma) Q
+    float WQ[2 * kC * kD];
+    float V[kC * kD];          // A of MMA 1 (MN-major)
+    float K[2][kC * kD];       // A of MMA 1 / B of MMA 3 (MN-major), by chunk parity
+    float Tb[kTriFloats];      // B of MMA 1: T diag(beta)
+    float Tg[kTriFloats];      // B of MMA 1: -T diag(beta gamma)
+    float P[kTriFloats];       // B of MMA 3: lands as Q K^T rows, becomes P
+    float Wk[kTriFloats];      // T team: lands as K K^T rows, becomes A, then T
+    // z rows of the chunk (16-bit activations).  Once the state group has formed
+    // the gate from it, its head holds the epilogue's partial sums of squares
+    // (red[4][64]) and reciprocal norms (rstd[64]).
+    __nv_bfloat16 Z[kC * kD];
+    float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
+    float beta[kC];            // T team's current chunk
+    unsigned long long bar_v, bar_q, bar_k[2], bar_kk, bar_qk, bar_z; // TMA landings
+    unsigned long long bar_m1, bar_m2, bar_m3;                  // MMA completions
+    unsigned long long bar_w, bar_u, bar_of[2];                 // state group -> MMA
+    unsigned long long bar_pT[2], bar_pQ, bar_pP, bar_wfree;    // T / P teams -> MMA, TMA
+    unsigned long long bar_fin;                                 // MMA drain on abort
     uint32_t tmem;
     int abort;
-    static constexpr int kVQBlk = 2 * kC * 32; // floats per 32-column block of VQ
 };
 
 constexpr long long kWaitLimit = 2000000000LL; // ~1 s of SM cycles
 
-// The tensor maps of one call: 64-row boxes of the workspace and of z.
+// The tensor maps of one call: 64-row boxes (32-row for the lower half of
+// the Gram tiles' second column block) of the workspace.
 struct ChunkMaps {
-    CUtensorMap v;  // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle
-    CUtensorMap k;  // normalised k, [N, Hk*128] of the q|k rows, 32-column boxes, MN-major swizzle
-    CUtensorMap q;  // normalised q, [N, Hk*128], 32-column boxes, 128-byte swizzle (K-major)
-    CUtensorMap kq; // Gram rows, [N, Hk*128] fp32, 32-column boxes, 128-byte swizzle
-    CUtensorMap z;  // z, [N, Hv*128] 16-bit, 128-column boxes, no swizzle
+    CUtensorMap v;    // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle
+    CUtensorMap k;    // normalised k, [N, Hk*128] of the q|k rows, MN-major tf32 swizzle
+    CUtensorMap q;    // normalised q, [N, Hk*128], 128-byte swizzle (K-major)
+    CUtensorMap kq;   // Gram rows, [N, Hk*128] fp32, 32 x 64 boxes, 128-byte swizzle
+    CUtensorMap kq32; // the same with 32 x 32 boxes
+    CUtensorMap z;    // z, [N, Hv*128] bf16, 128 x 64 boxes, no swizzle (bf16 activations)
 };
 
-// Barrier over the `n` threads of one warp group (named barrier `id`).
+// Barrier over the `n` threads of one group (named barrier `id`).
 __device__ __forceinline__ void group_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
@@ -261,38 +272,74 @@ __device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// L2 prefetch of one TMA box.
+__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap),
+                 "r"(x), "r"(y)
+                 : "memory");
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     using namespace sm100;
-    extern __shared__ unsigned char chunk_smem_raw[];
-    ChunkSmem<T> &sm = *reinterpret_cast<ChunkSmem<T> *>(
-        (reinterpret_cast<uintptr_t>(chunk_smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) unsigned char chunk_smem_raw[];
+    // the swizzled tiles need 1024-byte alignment, which the dynamic shared
+    // memory window provides when the kernel has no static shared memory; a
+    // misaligned window fails the call instead of corrupting the tiles
+    if ((smem_u32(chunk_smem_raw) & 1023u) != 0) {
+        if (threadIdx.x == 0 && p.ws_err != nullptr)
+            atomicOr(p.ws_err, 2u);
+        return;
+    }
+    ChunkSmem &sm = *reinterpret_cast<ChunkSmem *>(chunk_smem_raw);
 
     const int h = blockIdx.x;
     const int n = blockIdx.y;
     const int j = h / p.G;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
-    const bool is_state = tid < kStateThreads;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
     const int nchunks = (int)((len + kC - 1) / kC);
     const int64_t HD = (int64_t)p.Hv * kD;
 
-    const uint32_t bar_mma1 = smem_u32(&sm.bar_mma1), bar_mma2 = smem_u32(&sm.bar_mma2);
-    const uint32_t bar_mma3 = smem_u32(&sm.bar_mma3), bar_prep = smem_u32(&sm.bar_prep);
     const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
-    const uint32_t bar_p = smem_u32(&sm.bar_p), bar_a = smem_u32(&sm.bar_a);
-    const uint32_t bar_z = smem_u32(&sm.bar_z);
     const uint32_t bar_k0 = smem_u32(&sm.bar_k[0]), bar_k1 = smem_u32(&sm.bar_k[1]);
+    const uint32_t bar_kk = smem_u32(&sm.bar_kk), bar_qk = smem_u32(&sm.bar_qk);
+    const uint32_t bar_z = smem_u32(&sm.bar_z);
+    constexpr bool kZTile = sizeof(T) == 2; // z comes by TMA (16-bit) or from global (fp32)
+    const uint32_t bar_m1 = smem_u32(&sm.bar_m1), bar_m2 = smem_u32(&sm.bar_m2);
+    const uint32_t bar_m3 = smem_u32(&sm.bar_m3);
+    const uint32_t bar_w = smem_u32(&sm.bar_w), bar_u = smem_u32(&sm.bar_u);
+    const uint32_t bar_of0 = smem_u32(&sm.bar_of[0]), bar_of1 = smem_u32(&sm.bar_of[1]);
+    // T tiles + gates ready, by chunk parity: a waiter for chunk c must see that
+    // phase before the barrier can move on, and chunk c + 1 may finish first
+    const uint32_t bar_pT0 = smem_u32(&sm.bar_pT[0]), bar_pT1 = smem_u32(&sm.bar_pT[1]);
+    const uint32_t bar_pQ = smem_u32(&sm.bar_pQ);
+    const uint32_t bar_pP = smem_u32(&sm.bar_pP), bar_wfree = smem_u32(&sm.bar_wfree);
     if (tid == 0) {
-        const uint32_t all[11] = {bar_mma1, bar_mma2, bar_mma3, bar_prep, bar_v, bar_q,
-                                  bar_k0, bar_k1, bar_p, bar_a, bar_z};
-        for (int b = 0; b < 11; ++b)
-            mbar_init(all[b], 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_q, 1);
+        mbar_init(bar_k0, 1);
+        mbar_init(bar_k1, 1);
+        mbar_init(bar_kk, 1);
+        mbar_init(bar_qk, 1);
+        mbar_init(bar_z, 1);
+        mbar_init(bar_m1, 1);
+        mbar_init(bar_m2, 1);
+        mbar_init(bar_m3, 1);
+        mbar_init(bar_w, 1);
+        mbar_init(bar_u, 1);
+        mbar_init(bar_of0, 1);
+        mbar_init(bar_of1, 1);
+        mbar_init(bar_pT0, 1);
+        mbar_init(bar_pT1, 1);
+        mbar_init(bar_pQ, 1);
+        mbar_init(bar_pP, 1);
+        mbar_init(bar_wfree, 1);
+        mbar_init(smem_u32(&sm.bar_fin), 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -304,371 +351,45 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
-    const float negA = -expf(__ldg(p.A_log + h));
-    const float dtb = __ldg(p.dt_bias + h);
+    volatile int *abort_flag = &sm.abort;
     const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
     auto rows_of = [&](int c) {
         const int64_t left = len - (int64_t)c * kC;
         return (int)(left < kC ? left : kC);
     };
-    auto wait = [&](uint32_t bar, uint32_t &ph) {
-        const bool w = mbar_wait_bounded(bar, ph, kWaitLimit);
-        ph ^= 1u;
-        return w;
-    };
-    // TMA issue by the calling thread: nb 32-column boxes of 64 rows at
-    // x0 + 32 b, row t0, column block b landing at dst + b * bstride floats
-    auto tma_tile = [&](float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb, uint32_t bar,
-                        int bstride) {
-        mbar_arrive_expect_tx(bar, (uint32_t)(nb * kC * 32 * sizeof(float)));
-        for (int b = 0; b < nb; ++b)
-            tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, bar);
-    };
-    auto issue_z = [&](int c) { // by one thread
-        if constexpr (sizeof(T) == 2) {
-            mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
-            tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)(start + (int64_t)c * kC), bar_z);
-        } else { // float32 z is read straight from global memory
-            mbar_arrive(bar_z);
-        }
-    };
-
-    bool ok = true;
-    if (!is_state) {
-        // ================================================================ prep group
-        const int ptid = tid - kStateThreads, pw = ptid >> 5;
-        const bool leader = ptid == 0;
-        auto psync = [&]() { group_sync(kBarPrep, kPrepThreads); };
-        // raw gate inputs of chunk c, rows lane and lane + 32 (first prep warp);
-        // converted only in gates() so that the loads overlap other work
-        auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
-            if (pw == 0) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int r = lane + 32 * q;
-                    ra[q] = from_f<T>(0.f);
-                    rb[q] = from_f<T>(0.f);
-                    if (c < nchunks && r < rows_of(c)) {
-                        const int64_t t = start + (int64_t)c * kC + r;
-                        ra[q] = ((const T *)p.a)[t * p.Hv + h];
-                        rb[q] = ((const T *)p.b)[t * p.Hv + h];
-                    }
-                }
-            }
-        };
-        // g, beta, the inclusive prefix G, gamma = e^G and gamma_C / gamma of a
-        // chunk into slot `sl` (first prep warp; rows lane and lane + 32)
-        auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
-            if (pw == 0) {
-                float g[2], be[2];
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const bool in = c < nchunks && lane + 32 * q < rows_of(c);
-                    g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
-                    be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
-                }
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
-                    const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
-                    if (lane >= o) {
-                        g[0] += x0;
-                        g[1] += x1;
-                    }
-                }
-                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-                const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int r = lane + 32 * q;
-                    sm.G[sl][r] = g[q];
-                    sm.beta[sl][r] = be[q];
-                    sm.gam[sl][r] = expf(g[q]);
-                    sm.kd[sl][r] = expf(Glast - g[q]);
-                }
-            }
-        };
-        // Each prep thread owns the float4 at column c = 4 (ptid % 16) of rows
-        // r = ptid / 16 + 8 k, k = 0..7, in the 64 x 64 tiles below.  Every
-        // pass loads all its inputs before its first store, so that the
-        // compiler need not order later loads behind stores it cannot
-        // disambiguate.
-        const int pc = 4 * (ptid & 15), pr = ptid >> 4;
-        // K K^T rows -> A in place: A[r][s] = beta_r e^{G_r - G_s} KK[r][s]
-        // (the kq rows are 0 for s >= r and beta is 0 on padded rows; the
-        // clamp keeps the unused upper triangle finite: G_r - G_s > 0 there)
-        auto build_A = [&](int sl) {
-            const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][pc]);
-            float4 x[8];
-            float Gr[8], br[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                x[k] = *reinterpret_cast<const float4 *>(sm.A + swz(pr + 8 * k, pc, kC));
-                Gr[k] = sm.G[sl][pr + 8 * k];
-                br[k] = sm.beta[sl][pr + 8 * k];
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                x[k].x *= br[k] * __expf(fminf(Gr[k] - Gc.x, 0.f));
-                x[k].y *= br[k] * __expf(fminf(Gr[k] - Gc.y, 0.f));
-                x[k].z *= br[k] * __expf(fminf(Gr[k] - Gc.z, 0.f));
-                x[k].w *= br[k] * __expf(fminf(Gr[k] - Gc.w, 0.f));
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<float4 *>(sm.A + swz(pr + 8 * k, pc, kC)) = x[k];
-        };
-        // Q K^T rows -> P in place (K-major swizzled): P[r][s] = e^{G_r - G_s} QK[r][s], tf32
-        auto build_P = [&](int sl) {
-            const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][pc]);
-            float4 x[8];
-            float Gr[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                x[k] = *reinterpret_cast<const float4 *>(sm.P + swz(pr + 8 * k, pc, kC));
-                Gr[k] = sm.G[sl][pr + 8 * k];
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                x[k].x = tf32_rna(x[k].x * __expf(fminf(Gr[k] - Gc.x, 0.f)));
-                x[k].y = tf32_rna(x[k].y * __expf(fminf(Gr[k] - Gc.y, 0.f)));
-                x[k].z = tf32_rna(x[k].z * __expf(fminf(Gr[k] - Gc.z, 0.f)));
-                x[k].w = tf32_rna(x[k].w * __expf(fminf(Gr[k] - Gc.w, 0.f)));
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                *reinterpret_cast<float4 *>(sm.P + swz(pr + 8 * k, pc, kC)) = x[k];
-        };
-        // T = (I + A)^-1 for the strictly lower triangular A, in place in sm.A,
-        // by block doubling: invert the four 16 x 16 diagonal blocks by forward
-        // substitution, then join pairs of blocks with [T1 0; X T2],
-        // X = -T2 A21 T1, at 32 and at 64 rows.  Finally T diag(beta) and
-        // T diag(beta gamma) are written as tf32 B operands.  sm.Tg serves as
-        // scratch for A21 T1 (MMA 1 has finished reading it).
-        auto solve = [&](int sl) {
-            float *At = sm.A;
-            float *Y = sm.Tg;
-            { // 16 x 16 diagonal block pw; lane l < 16 owns column 16 pw + l
-                const int c = 16 * pw + (lane & 15);
-                float t[16];
-#pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                    for (int i = 0; i < r; ++i) {
-                        const float a = At[swz(16 * pw + r, 16 * pw + i, kC)];
-                        if (i & 1)
-                            acc1 = fmaf(a, t[i], acc1);
-                        else
-                            acc0 = fmaf(a, t[i], acc0);
-                    }
-                    const int rr = 16 * pw + r;
-                    t[r] = rr == c ? 1.f : (rr < c ? 0.f : -(acc0 + acc1));
-                }
-                __syncwarp();
-                if (lane < 16) {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        At[swz(16 * pw + r, c, kC)] = t[r];
-                }
-            }
-            psync();
-            { // join at 32 rows, blocks b = 0 (rows 0..31) and 1 (rows 32..63); thread:
-              // rows r0, r0 + 1 of the 16 x 16 product, columns c0, c0 + 1
-                const int b = ptid >> 6, q = ptid & 63;
-                const int o = 32 * b, r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
-                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float a0 = At[swz(o + 16 + r0, o + i, kC)];
-                    const float a1 = At[swz(o + 17 + r0, o + i, kC)];
-                    const float t0 = At[swz(o + i, o + c0, kC)];
-                    const float t1 = At[swz(o + i, o + c0 + 1, kC)];
-                    y00 = fmaf(a0, t0, y00); y01 = fmaf(a0, t1, y01);
-                    y10 = fmaf(a1, t0, y10); y11 = fmaf(a1, t1, y11);
-                }
-                Y[b * 256 + r0 * 16 + c0] = y00;
-                Y[b * 256 + r0 * 16 + c0 + 1] = y01;
-                Y[b * 256 + (r0 + 1) * 16 + c0] = y10;
-                Y[b * 256 + (r0 + 1) * 16 + c0 + 1] = y11;
-                psync();
-                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const float a0 = At[swz(o + 16 + r0, o + 16 + i, kC)];
-                    const float a1 = At[swz(o + 17 + r0, o + 16 + i, kC)];
-                    const float t0 = Y[b * 256 + i * 16 + c0];
-                    const float t1 = Y[b * 256 + i * 16 + c0 + 1];
-                    x00 = fmaf(a0, t0, x00); x01 = fmaf(a0, t1, x01);
-                    x10 = fmaf(a1, t0, x10); x11 = fmaf(a1, t1, x11);
-                }
-                // A21 was read only before the barrier above: overwrite it in place
-                At[swz(o + 16 + r0, o + c0, kC)] = -x00;
-                At[swz(o + 16 + r0, o + c0 + 1, kC)] = -x01;
-                At[swz(o + 17 + r0, o + c0, kC)] = -x10;
-                At[swz(o + 17 + r0, o + c0 + 1, kC)] = -x11;
-            }
-            psync();
-            { // join at 64 rows: thread: rows r0, r0 + 1 of the 32 x 32 product, columns c0 .. + 3
-                const int r0 = 2 * (ptid >> 3), c0 = 4 * (ptid & 7);
-                float y[2][4] = {};
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const float a0 = At[swz(32 + r0, i, kC)];
-                    const float a1 = At[swz(33 + r0, i, kC)];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(At + swz(i, c0, kC));
-                    y[0][0] = fmaf(a0, t4.x, y[0][0]); y[0][1] = fmaf(a0, t4.y, y[0][1]);
-                    y[0][2] = fmaf(a0, t4.z, y[0][2]); y[0][3] = fmaf(a0, t4.w, y[0][3]);
-                    y[1][0] = fmaf(a1, t4.x, y[1][0]); y[1][1] = fmaf(a1, t4.y, y[1][1]);
-                    y[1][2] = fmaf(a1, t4.z, y[1][2]); y[1][3] = fmaf(a1, t4.w, y[1][3]);
-                }
-                *reinterpret_cast<float4 *>(Y + r0 * 36 + c0) =
-                    make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
-                *reinterpret_cast<float4 *>(Y + (r0 + 1) * 36 + c0) =
-                    make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
-                psync();
-                float x[2][4] = {};
-#pragma unroll 8
-                for (int i = 0; i < 32; ++i) {
-                    const float a0 = At[swz(32 + r0, 32 + i, kC)];
-                    const float a1 = At[swz(33 + r0, 32 + i, kC)];
-                    const float4 t4 = *reinterpret_cast<const float4 *>(Y + i * 36 + c0);
-                    x[0][0] = fmaf(a0, t4.x, x[0][0]); x[0][1] = fmaf(a0, t4.y, x[0][1]);
-                    x[0][2] = fmaf(a0, t4.z, x[0][2]); x[0][3] = fmaf(a0, t4.w, x[0][3]);
-                    x[1][0] = fmaf(a1, t4.x, x[1][0]); x[1][1] = fmaf(a1, t4.y, x[1][1]);
-                    x[1][2] = fmaf(a1, t4.z, x[1][2]); x[1][3] = fmaf(a1, t4.w, x[1][3]);
-                }
-                *reinterpret_cast<float4 *>(At + swz(32 + r0, c0, kC)) =
-                    make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
-                *reinterpret_cast<float4 *>(At + swz(33 + r0, c0, kC)) =
-                    make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
-            }
-            psync();
-            // T diag(beta), T diag(beta gamma) -> tf32 K-major operands (rows r, columns s)
-            {
-                const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[sl][pc]);
-                const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][pc]);
-                const float4 bg = make_float4(b4.x * g4.x, b4.y * g4.y, b4.z * g4.z, b4.w * g4.w);
-                float4 t4[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k)
-                    t4[k] = *reinterpret_cast<const float4 *>(At + swz(pr + 8 * k, pc, kC));
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    const int o = swz(pr + 8 * k, pc, kC);
-                    *reinterpret_cast<float4 *>(sm.Tb + o) = tf32_rna(
-                        make_float4(t4[k].x * b4.x, t4[k].y * b4.y, t4[k].z * b4.z, t4[k].w * b4.w));
-                    *reinterpret_cast<float4 *>(sm.Tg + o) = tf32_rna(
-                        make_float4(t4[k].x * bg.x, t4[k].y * bg.y, t4[k].z * bg.z, t4[k].w * bg.w));
-                }
-            }
-        };
-
-        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phv = 0, phk0 = 0, phk1 = 0, php = 0, pha = 0;
-        const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.VQ), 2 * kC * 128, 512); // A of MMA 1
-        const uint64_t dTb = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
-        const uint64_t dTg = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
-        const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
-        const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
-        constexpr int kVQBlk = ChunkSmem<T>::kVQBlk;
-        T av[2], bv[2]; // raw gate inputs of the next chunk to be gated
-        if (nchunks > 0) {
-            // ---- prologue: all tiles of chunk 0, its gates, T and P
-            if (leader) {
-                tma_tile(sm.VQ, &maps.v, xv, start, 4, bar_v, kVQBlk);
-                tma_tile(sm.VQ + kC * 32, &maps.q, xq, start, 4, bar_q, kVQBlk);
-                tma_tile(sm.K[0], &maps.k, xq, start, 4, bar_k0, kC * 32);
-                tma_tile(sm.P, &maps.kq, xkk + kC, start, 2, bar_p, kC * 32);
-                tma_tile(sm.A, &maps.kq, xkk, start, 2, bar_a, kC * 32);
-                issue_z(0);
-            }
-            load_ab(0, av, bv);
-            gates(0, av, bv, 0);
-            ok = wait(bar_a, pha) && ok;
-            psync();
-            build_A(0);
-            psync();
-            solve(0);
-            psync(); // A is free again
-            if (leader && nchunks > 1) {
-                tma_tile(sm.K[1], &maps.k, xq, start + kC, 4, bar_k1, kC * 32);
-                tma_tile(sm.A, &maps.kq, xkk, start + kC, 2, bar_a, kC * 32);
-            }
-            ok = wait(bar_p, php) && ok;
-            build_P(0);
-            load_ab(1, av, bv);
-            fence_proxy_async_smem();
-            psync();
-            if (leader)
-                mbar_arrive(bar_prep); // chunk 0 ready
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            const int cur = c & 1, nxt = cur ^ 1;
-            const int64_t t0 = start + (int64_t)c * kC;
-            const bool has_next = c + 1 < nchunks;
-            // ---- MMA 1: U~^T = V^T (T diag b)^T and W^T = K^T (T diag b gamma)^T
-            if (leader) {
-                ok = wait(bar_v, phv) && ok;
-                ok = (cur ? wait(bar_k1, phk1) : wait(bar_k0, phk0)) && ok;
-                tc_fence_after();
-                const uint64_t dK = cur ? dK1 : dK0;
-                constexpr uint32_t id = idesc_tf32(128, kC, true, false);
-#pragma unroll
-                for (int s = 0; s < kC / 8; ++s) {
-                    const uint64_t ks = (uint64_t)((((s >> 2) * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ss(tmem + kColU, dV + s * 64, dTb + ks, id, s > 0);
-                    mma_tf32_ss(tmem + kColW, dK + s * 64, dTg + ks, id, s > 0);
-                }
-                mma_commit(bar_mma1);
-            }
-            gates(c + 1, av, bv, nxt);
-            ok = wait(bar_mma1, ph1) && ok; // T diag(b), T diag(b gamma) are free
-            if (has_next) {
-                ok = wait(bar_a, pha) && ok;
-                psync();
-                build_A(nxt);
-                psync();
-                solve(nxt);
-                fence_proxy_async_smem();
-                psync(); // A is free, Tb / Tg of the next chunk are written
-            }
-            ok = wait(bar_mma2, ph2) && ok; // V (then -W) and Q are free
-            if (leader && has_next) {
-                tma_tile(sm.VQ, &maps.v, xv, t0 + kC, 4, bar_v, kVQBlk);
-                tma_tile(sm.VQ + kC * 32, &maps.q, xq, t0 + kC, 4, bar_q, kVQBlk);
-            }
-            ok = wait(bar_mma3, ph3) && ok; // P, K[cur] and the U / W columns are free
-            if (leader) {
-                if (has_next)
-                    tma_tile(sm.P, &maps.kq, xkk + kC, t0 + kC, 2, bar_p, kC * 32);
-                if (c + 2 < nchunks) {
-                    tma_tile(sm.K[cur], &maps.k, xq, t0 + 2 * kC, 4, cur ? bar_k1 : bar_k0, kC * 32);
-                    tma_tile(sm.A, &maps.kq, xkk, t0 + 2 * kC, 2, bar_a, kC * 32);
-                }
-            }
-            load_ab(c + 2, av, bv);
-            if (has_next) {
-                ok = wait(bar_p, php) && ok;
-                build_P(nxt);
-                fence_proxy_async_smem();
-                psync();
-                if (leader)
-                    mbar_arrive(bar_prep); // the next chunk is ready
-            }
-            if (group_sync_or(kBarPrep, kPrepThreads, !ok || *(volatile int *)&sm.abort)) {
-                ok = false;
+    // bounded wait on phase `ph` of `bar` (then flips ph); false on time-out or
+    // abort.  The first wait of the call that times out records, in the second
+    // word of the workspace header, which warp gave up on which barrier:
+    // 0x80000000 | warp << 24 | barrier index << 16 | phases this thread had
+    // seen on it (low 16 bits); the status word then gets bit 0.
+    const uint32_t bar_base = smem_u32(&sm.bar_v);
+    uint32_t waits_seen = 0;
+    auto waitp = [&](uint32_t bar, uint32_t &ph) {
+        const long long t0 = clock64();
+        bool done;
+        while (!(done = mbar_try_wait(bar, ph))) {
+            if (*abort_flag)
+                break;
+            if (clock64() - t0 > kWaitLimit) {
+                if (p.ws_err != nullptr)
+                    atomicCAS(p.ws_err + 1, 0u,
+                              0x80000000u | ((uint32_t)warp << 24) | (((bar - bar_base) / 8) << 16) |
+                                  (waits_seen & 0xffffu));
                 break;
             }
         }
-        if (!ok)
-            *(volatile int *)&sm.abort = 1;
-    } else {
-        // ================================================================ state group
+        ph ^= 1u;
+        ++waits_seen;
+        return done;
+    };
+    bool ok = true;
+
+    if (warp < kSG / 32) {
+        // ==================================================== state group
         const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
         const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
-        auto ssync = [&]() { group_sync(kBarState, kStateThreads); };
-        // initial state into TMEM (row vch, this half's 64 columns); O starts at zero
+        // initial state into TMEM (row vch, this half's 64 columns); both O buffers zero
         {
             const float *src = p.init_state
                                    ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
@@ -688,191 +409,738 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
 #pragma unroll
             for (int i = 0; i < 32; ++i)
                 zero[i] = 0.f;
-            tmem_st32(tl + kColO + 32 * hf, zero); // MMA 2 accumulates onto O
+            tmem_st32(tl + kColU0 + 64 + 32 * hf, zero);
+            tmem_st32(tl + kColU1 + 64 + 32 * hf, zero);
             tmem_wait_st();
         }
         const float wn = __ldg(p.norm_w + vch);
-        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phq = 0, phz = 0, phr = 0;
-        const uint64_t dWQ = sdesc_sw128(smem_u32(sm.VQ), 16, 1024); // B of MMA 2 (N = 128)
-        const uint64_t dP = sdesc_sw128(smem_u32(sm.P), 16, 1024);
-        const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
-        const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
-        for (int c = 0; c < nchunks; ++c) {
-            const int cur = c & 1;
-            const int nr = rows_of(c);
-            const int64_t t0 = start + (int64_t)c * kC;
-            ok = wait(bar_mma1, ph1) && ok;
+        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phT0 = 0, phT1 = 0, phz = 0;
+        float *red = reinterpret_cast<float *>(sm.Z); // [4][kC], then rstd[kC]
+        float *rstd = red + 4 * kC;
+        // -W^T (TMEM, tf32-rounded) -> rows 0..63 of WQ (K-major: rows r, columns k = vch);
+        // this half takes rows 32 hf .. + 31
+        auto w_pass = [&](int c) -> bool {
+            bool good = waitp(bar_m1, ph1);
+            good = ((c & 1) ? waitp(bar_pT1, phT1) : waitp(bar_pT0, phT0)) && good; // gates
+            good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
             tc_fence_after();
-            // ---- -W into rows 0..63 of VQ (K-major: rows r, columns k = vch), tf32;
-            //      this half takes rows 32 hf .. 32 hf + 31
-            {
+            if (good) {
                 float w[32];
                 tmem_ld32(tl + kColW + 32 * hf, w);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    sm.VQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(-w[i]);
+                    sm.WQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(w[i]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            ssync();
-            tc_fence_after();
-            // ---- MMA 2: [U^T | O^T] += S0 [-W; Q]^T, one N = 128 product (A = the
-            //      FP32 state in TMEM); U^T starts as U~^T, O^T as zero
-            if (tid == 0) {
-                ok = wait(bar_q, phq) && ok;
-                constexpr uint32_t id = idesc_tf32(128, 2 * kC, false, false);
-#pragma unroll
-                for (int s = 0; s < kD / 8; ++s) {
-                    const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ts(tmem + kColU, tmem + kColS + 8 * s, dWQ + ks, id, 1);
-                }
-                mma_commit(bar_mma2);
-            }
-            ok = wait(bar_mma2, ph2) && ok;
-            ok = wait(bar_prep, phr) && ok; // this chunk's gates and P
-            tc_fence_after();
-            // ---- TMEM pass (this half's columns): U -> tf32; U diag(gamma_C/gamma)
-            //      -> tf32 copy; O columns r scaled by gamma_r; S scaled by gamma_C
+            const bool bad = group_sync_or(kBarSG, kSG, !good || *abort_flag);
+            if (!bad && tid == 0)
+                mbar_arrive(bar_w);
+            return !bad;
+        };
+        if (nchunks > 0)
+            ok = w_pass(0);
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int sl = c & 3;
+            const uint32_t cU = (c & 1) ? kColU1 : kColU0, cO = cU + 64;
+            // ---- U pass: U -> tf32 (in place), U diag(gamma_C/gamma) -> tf32 (Uk), S *= gamma_C
             {
-                float u[32], o[32], gm[32], kf[32];
+                bool good = __all_sync(0xffffffffu, waitp(bar_m2, ph2));
+                tc_fence_after();
+                if (good) {
+                    float u[32], uk[32];
+                    tmem_ld32(tl + cU + 32 * hf, u);
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    gm[i] = sm.gam[cur][32 * hf + i];
-                    kf[i] = sm.kd[cur][32 * hf + i];
-                }
-                const float gC = sm.gam[cur][kC - 1]; // padded rows carry g = 0
-                tmem_ld32(tl + kColU + 32 * hf, u);
-                tmem_ld32(tl + kColO + 32 * hf, o);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    o[i] *= gm[i];
-                tmem_st32(tl + kColO + 32 * hf, o);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    o[i] = tf32_rna(u[i] * kf[i]);
-                    u[i] = tf32_rna(u[i]);
-                }
-                tmem_st32(tl + kColU + 32 * hf, u);
-                tmem_st32(tl + kColUk + 32 * hf, o);
-#pragma unroll
-                for (int cb = 0; cb < 2; ++cb) {
-                    float v[32];
-                    tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+                    for (int i = 0; i < 32; i += 4) {
+                        const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kd[sl][32 * hf + i]);
+                        uk[i] = k4.x; uk[i + 1] = k4.y; uk[i + 2] = k4.z; uk[i + 3] = k4.w;
+                    }
+                    const float gC = expf(sm.G[sl][kC - 1]); // padded rows carry g = 0
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        v[i] *= gC;
-                    tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
-                }
-                tmem_wait_st();
-            }
-            tc_fence_before();
-            ssync();
-            tc_fence_after();
-            // ---- MMA 3: O^T += U^T P^T and S += (U diag(gamma_C/gamma))^T K
-            if (tid == 0) {
-                const uint64_t dK = cur ? dK1 : dK0;
-                constexpr uint32_t idp = idesc_tf32(128, kC, false, false);
-                constexpr uint32_t ids = idesc_tf32(128, kD, false, true);
+                    for (int i = 0; i < 32; ++i) {
+                        uk[i] = tf32_rna(u[i] * uk[i]);
+                        u[i] = tf32_rna(u[i]);
+                    }
+                    tmem_st32(tl + cU + 32 * hf, u);
+                    tmem_st32(tl + kColUk + 32 * hf, uk);
 #pragma unroll
-                for (int s = 0; s < kC / 8; ++s) {
-                    const uint64_t ks = (uint64_t)((((s >> 2) * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ts(tmem + kColO, tmem + kColU + 8 * s, dP + ks, idp, 1);
-                    mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, ids, 1);
+                    for (int cb = 0; cb < 2; ++cb) {
+                        float v[32];
+                        tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            v[i] *= gC;
+                        tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+                    }
+                    tmem_wait_st();
                 }
-                mma_commit(bar_mma3);
+                tc_fence_before();
+                if (group_sync_or(kBarSG, kSG, !good || *abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (tid == 0)
+                    mbar_arrive(bar_u);
             }
-            ok = wait(bar_z, phz) && ok; // z rows of this chunk
-            ok = wait(bar_mma3, ph3) && ok;
-            tc_fence_after();
+            // ---- W pass of the next chunk (MMA 1 of it ran beside the U pass)
+            if (c + 1 < nchunks) {
+                if (!w_pass(c + 1)) {
+                    ok = false;
+                    break;
+                }
+            }
             // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
             //      RMSNorm over v, times w[v] SiLU(z), stored; then O is zeroed
             {
-                float o[32], sq[32];
-                tmem_ld32(tl + kColO + 32 * hf, o);
-                tmem_wait_ld();
+                const int64_t t0 = start + (int64_t)c * kC;
+                const int rows = rows_of(c) - 32 * hf; // valid rows of this half (may be <= 0)
+                // the gate w[v] SiLU(z) does not depend on the state: form it while
+                // MMA 3 runs
+                float gt[32];
+                bool zok = true;
+                if constexpr (kZTile) {
+                    zok = __all_sync(0xffffffffu, waitp(bar_z, phz));
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        gt[i] = to_f(sm.Z[(32 * hf + i) * kD + vch]);
+                } else {
+                    const T *zp = (const T *)p.z + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        gt[i] = i < rows ? ld_cg(zp + i * HD) : 0.f;
+                }
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
-                    sq[i] = o[i] * o[i];
-                // reduce-scatter over the 32 lanes: lane l ends with row 32 hf + l
+                    gt[i] = wn * __fdividef(gt[i], 1.0f + __expf(-gt[i]));
+                group_sync(kBarSG, kSG); // the z tile is read: its head takes the sums below
+                bool good = zok && __all_sync(0xffffffffu, waitp(bar_m3, ph3));
+                tc_fence_after();
+                float o[32];
+                if (good) {
+                    float sq[32];
+                    tmem_ld32(tl + cO + 32 * hf, o);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int w = 16; w >= 1; w >>= 1) {
-                    const bool upper = (lane & w) != 0;
+                    for (int i = 0; i < 32; ++i)
+                        sq[i] = o[i] * o[i];
+                    // reduce-scatter over the 32 lanes: lane l ends with row 32 hf + l
 #pragma unroll
-                    for (int i = 0; i < w; ++i) {
-                        const float send = upper ? sq[i] : sq[i + w];
-                        const float keep = upper ? sq[i + w] : sq[i];
-                        sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                    for (int w = 16; w >= 1; w >>= 1) {
+                        const bool upper = (lane & w) != 0;
+#pragma unroll
+                        for (int i = 0; i < w; ++i) {
+                            const float send = upper ? sq[i] : sq[i + w];
+                            const float keep = upper ? sq[i + w] : sq[i];
+                            sq[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+                        }
+                    }
+                    red[lq * kC + 32 * hf + lane] = sq[0];
+                }
+                group_sync(kBarSG, kSG);
+                if (tid < kC)
+                    rstd[tid] = rsqrtf((red[tid] + red[kC + tid] + red[2 * kC + tid] +
+                                        red[3 * kC + tid]) * (1.0f / kD) + p.rms_eps);
+                group_sync(kBarSG, kSG);
+                if (good) {
+                    if (p.o_raw != nullptr) {
+                        float *op = p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < rows)
+                                st_cg(op + i * HD, o[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) // o * rstd * w * SiLU(z)
+                        o[i] = o[i] * rstd[32 * hf + i] * gt[i];
+                    T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
+                    if (rows >= 32) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            st_cg(yp + i * HD, o[i]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            if (i < rows)
+                                st_cg(yp + i * HD, o[i]);
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        o[i] = 0.f;
+                    tmem_st32(tl + cO + 32 * hf, o); // MMA 2 accumulates onto O
+                    tmem_wait_st();
+                }
+                tc_fence_before();
+                if (group_sync_or(kBarSG, kSG, !good || *abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (tid == 0)
+                    mbar_arrive((c & 1) ? bar_of1 : bar_of0);
+            }
+        }
+        if (!ok)
+            *abort_flag = 1;
+    } else if (warp < (kSG + kTeam) / 32) {
+        // ==================================================== T team
+        const int tt = tid - kSG, tw = tt >> 5;
+        float *Wk = sm.Wk;
+        // raw gate inputs of chunk c, rows lane and lane + 32 (first warp of the team)
+        auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
+            if (tw == 0) {
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int r = lane + 32 * q;
+                    ra[q] = from_f<T>(0.f);
+                    rb[q] = from_f<T>(0.f);
+                    if (c < nchunks && r < rows_of(c)) {
+                        const int64_t t = start + (int64_t)c * kC + r;
+                        ra[q] = ((const T *)p.a)[t * p.Hv + h];
+                        rb[q] = ((const T *)p.b)[t * p.Hv + h];
                     }
                 }
-                sm.red[lq][32 * hf + lane] = sq[0];
-                ssync();
-                if (tid < kC)
-                    sm.rstd[tid] = rsqrtf((sm.red[0][tid] + sm.red[1][tid] + sm.red[2][tid] +
-                                           sm.red[3][tid]) * (1.0f / kD) + p.rms_eps);
-                ssync();
-                T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
-                const int rows = nr - 32 * hf; // valid rows of this half (may be <= 0)
-                if (p.o_raw != nullptr) {
-                    float *op = p.o_raw + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < rows)
-                            op[i * HD] = o[i];
-                }
-                // all loads first, then the arithmetic, then the stores
-                float zr[32], sc[32];
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    if constexpr (sizeof(T) == 2)
-                        zr[i] = to_f(sm.Z[(32 * hf + i) * kD + vch]);
-                    else
-                        zr[i] = i < rows ? to_f(((const T *)p.z)[(t0 + 32 * hf + i) * HD +
-                                                                  (int64_t)h * kD + vch])
-                                         : 0.f;
-                    sc[i] = sm.rstd[32 * hf + i];
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i) // o * rstd * w * SiLU(z)
-                    o[i] = o[i] * (sc[i] * wn) * __fdividef(zr[i], 1.0f + __expf(-zr[i]));
-                if (rows >= 32) {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        yp[i * HD] = from_f<T>(o[i]);
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (i < rows)
-                            yp[i * HD] = from_f<T>(o[i]);
-                }
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    o[i] = 0.f;
-                tmem_st32(tl + kColO + 32 * hf, o); // MMA 2 accumulates onto O
-                tmem_wait_st();
             }
-            tc_fence_before();
-            const bool bad = group_sync_or(kBarState, kStateThreads,
-                                           !ok || *(volatile int *)&sm.abort); // Z is read
-            tc_fence_after();
-            if (bad) {
+        };
+        const float negA = -expf(__ldg(p.A_log + h));
+        const float dtb = __ldg(p.dt_bias + h);
+        // g, the inclusive prefix G and gamma_C / gamma of a chunk into slot
+        // `sl`, beta into the team's own row (first warp; rows lane and lane + 32)
+        auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
+            if (tw == 0) {
+                float g[2], be[2];
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const bool in = lane + 32 * q < rows_of(c);
+                    g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
+                    be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
+                }
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
+                    const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
+                    if (lane >= o) {
+                        g[0] += x0;
+                        g[1] += x1;
+                    }
+                }
+                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
+                const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
+#pragma unroll
+                for (int q = 0; q < 2; ++q) {
+                    const int r = lane + 32 * q;
+                    sm.G[sl][r] = g[q];
+                    sm.beta[r] = be[q];
+                    sm.kd[sl][r] = expf(Glast - g[q]);
+                }
+            }
+        };
+        // The six float4s of a triangular tile this thread handles: rows
+        // tt / 8 + 16 jj (jj = 0..3, column block 0, columns 4 (tt % 8)) and
+        // 32 + tt / 8 + 16 (jj - 4) (jj = 4, 5, block 1, columns 32 + 4 (tt % 8)).
+        // 16 jj keeps r mod 8, so the swizzle term is one constant per thread.
+        const int trow = tt >> 3, tcol = 4 * (tt & 7);
+        const int tbase = trow * 32 + (((tt & 7) ^ (trow & 7)) << 2);
+        auto tri_r = [&](int jj) { return jj < 4 ? trow + 16 * jj : 32 + trow + 16 * (jj - 4); };
+        auto tri_c = [&](int jj) { return jj < 4 ? tcol : 32 + tcol; };
+        auto tri_o = [&](int jj) { return tbase + (jj < 4 ? 512 * jj : 1024 + 512 * (jj - 2)); };
+        uint32_t phkk = 0, ph1 = 0;
+        T av[2], bv[2];
+        load_ab(0, av, bv);
+        for (int c = 0; c < nchunks; ++c) {
+            const int sl = c & 3;
+            gates(c, av, bv, sl);
+            load_ab(c + 1, av, bv);
+            bool good = waitp(bar_kk, phkk); // K K^T rows of this chunk are in Wk
+            if (group_sync_or(kBarT, kTeam, !good || *abort_flag)) {
                 ok = false;
                 break;
             }
-            if (tid == 0 && c + 1 < nchunks)
-                issue_z(c + 1);
+            // ---- A[r][s] = beta_r e^{G_r - G_s} KK[r][s] in place (the kq rows are
+            //      0 for s >= r and beta is 0 on padded rows; the clamp keeps the
+            //      unused upper triangle finite: G_r - G_s > 0 there)
+            {
+                float4 x[6];
+#pragma unroll
+                for (int jj = 0; jj < 6; ++jj)
+                    x[jj] = *reinterpret_cast<const float4 *>(Wk + tri_o(jj));
+#pragma unroll
+                for (int jj = 0; jj < 6; ++jj) {
+                    const float Gr = sm.G[sl][tri_r(jj)], br = sm.beta[tri_r(jj)];
+                    const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][tri_c(jj)]);
+                    x[jj].x *= br * __expf(fminf(Gr - Gc.x, 0.f));
+                    x[jj].y *= br * __expf(fminf(Gr - Gc.y, 0.f));
+                    x[jj].z *= br * __expf(fminf(Gr - Gc.z, 0.f));
+                    x[jj].w *= br * __expf(fminf(Gr - Gc.w, 0.f));
+                }
+#pragma unroll
+                for (int jj = 0; jj < 6; ++jj)
+                    *reinterpret_cast<float4 *>(Wk + tri_o(jj)) = x[jj];
+            }
+            group_sync(kBarT, kTeam);
+            // ---- T = (I + A)^-1 in place, by block doubling.  Level 1: the four
+            //      16 x 16 diagonal blocks by forward substitution, one column per
+            //      thread (threads 0..63)
+            {
+                // warp 0: blocks 0, 1 (column block 0); warp 1: blocks 2, 3 (block 1,
+                // whose rows 32.. sit at 1024 + 32 r); lanes 0..15 / 16..31 take the
+                // two blocks, R' = 0 / 16 within the column block
+                const int cl = tt & 15, Rp = 16 * ((tt >> 4) & 1), R = 32 * (tt >> 5) + Rp;
+                const float *blk = Wk + 1024 * (tt >> 5) + R * 32;
+                float x[16];
+                if (tt < 64) {
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) {
+                        float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+                        for (int m = 0; m < (r + 3) / 4; ++m) {
+                            const float4 a = *reinterpret_cast<const float4 *>(
+                                blk + r * 32 + ((((Rp >> 2) + m) ^ (r & 7)) << 2));
+                            const float av4[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                if (4 * m + e < r) {
+                                    if (e & 1)
+                                        acc1 = fmaf(av4[e], x[4 * m + e], acc1);
+                                    else
+                                        acc0 = fmaf(av4[e], x[4 * m + e], acc0);
+                                }
+                        }
+                        x[r] = r < cl ? 0.f : (r == cl ? 1.f : -(acc0 + acc1));
+                    }
+                }
+                group_sync(kBarT, kTeam); // every diagonal block of A has been read
+                if (tt < 64) {
+                    float *dst = Wk + 1024 * (tt >> 5) + R * 32 + ((Rp + cl) & 3);
+#pragma unroll
+                    for (int r = 0; r < 16; ++r)
+                        dst[r * 32 + ((((Rp + cl) >> 2) ^ (r & 7)) << 2)] = x[r];
+                }
+            }
+            group_sync(kBarT, kTeam);
+            // ---- level 2: join the 16-blocks of each 32-block p (warps 0, 1: p = 0
+            //      in column block 0; warps 2, 3: p = 1 in block 1):
+            //      T21 = -T22 (A21 T11); thread: rows r0, r0 + 1, columns c0, c0 + 1;
+            //      element (32 p + i, 32 p + j) at base + i * 32 + swizzle(i, j)
+            {
+                const int pb = tt >> 6, q = tt & 63;
+                const int r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
+                float *base = Wk + 1024 * pb + 32 * pb * 32;
+                auto at = [&](int i, int jc) { return base + i * 32 + (((jc >> 2) ^ (i & 7)) << 2) + (jc & 3); };
+                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 4 * m));
+                    const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 4 * m));
+                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 t2 = *reinterpret_cast<const float2 *>(at(4 * m + e, c0));
+                        y00 = fmaf(a0v[e], t2.x, y00); y01 = fmaf(a0v[e], t2.y, y01);
+                        y10 = fmaf(a1v[e], t2.x, y10); y11 = fmaf(a1v[e], t2.y, y11);
+                    }
+                }
+                group_sync(kBarT, kTeam); // A21 is read: Y takes its place
+                *reinterpret_cast<float2 *>(at(16 + r0, c0)) = make_float2(y00, y01);
+                *reinterpret_cast<float2 *>(at(17 + r0, c0)) = make_float2(y10, y11);
+                group_sync(kBarT, kTeam);
+                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 16 + 4 * m));
+                    const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 16 + 4 * m));
+                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 t2 = *reinterpret_cast<const float2 *>(at(16 + 4 * m + e, c0));
+                        x00 = fmaf(a0v[e], t2.x, x00); x01 = fmaf(a0v[e], t2.y, x01);
+                        x10 = fmaf(a1v[e], t2.x, x10); x11 = fmaf(a1v[e], t2.y, x11);
+                    }
+                }
+                group_sync(kBarT, kTeam); // Y is read: T21 takes its place
+                *reinterpret_cast<float2 *>(at(16 + r0, c0)) = make_float2(-x00, -x01);
+                *reinterpret_cast<float2 *>(at(17 + r0, c0)) = make_float2(-x10, -x11);
+            }
+            group_sync(kBarT, kTeam);
+            // ---- level 3: join the two 32-blocks: T21 = -T22 (A21 T11); thread:
+            //      rows r0, r0 + 1, columns c0 .. + 3 of the 32 x 32 products.  A21,
+            //      T11 and Y sit in column block 0 (offset r * 32 + chunk ^ (r & 7)),
+            //      T22 in block 1 (rows 32..63)
+            {
+                const int r0 = 2 * (tt >> 3), q0 = tt & 7; // columns c0 = 4 q0
+                const float *Ar0 = Wk + (32 + r0) * 32, *Ar1 = Ar0 + 32;   // rows 32 + r0, + 1
+                const float *Br0 = Wk + 2048 + r0 * 32, *Br1 = Br0 + 32;   // block 1 rows
+                const int x0 = r0 & 7, x1 = (r0 + 1) & 7;
+                float y[2][4] = {};
+#pragma unroll 2
+                for (int m = 0; m < 8; ++m) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(Ar0 + ((m ^ x0) << 2));
+                    const float4 a1 = *reinterpret_cast<const float4 *>(Ar1 + ((m ^ x1) << 2));
+                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 4 * m + e; // T11 row i, columns c0 .. + 3
+                        const float4 t4 =
+                            *reinterpret_cast<const float4 *>(Wk + i * 32 + ((q0 ^ (i & 7)) << 2));
+                        y[0][0] = fmaf(a0v[e], t4.x, y[0][0]); y[0][1] = fmaf(a0v[e], t4.y, y[0][1]);
+                        y[0][2] = fmaf(a0v[e], t4.z, y[0][2]); y[0][3] = fmaf(a0v[e], t4.w, y[0][3]);
+                        y[1][0] = fmaf(a1v[e], t4.x, y[1][0]); y[1][1] = fmaf(a1v[e], t4.y, y[1][1]);
+                        y[1][2] = fmaf(a1v[e], t4.z, y[1][2]); y[1][3] = fmaf(a1v[e], t4.w, y[1][3]);
+                    }
+                }
+                group_sync(kBarT, kTeam); // A21 is read: Y takes its place
+                float *Yr0 = Wk + (32 + r0) * 32 + ((q0 ^ x0) << 2);
+                float *Yr1 = Wk + (33 + r0) * 32 + ((q0 ^ x1) << 2);
+                *reinterpret_cast<float4 *>(Yr0) = make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
+                *reinterpret_cast<float4 *>(Yr1) = make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
+                group_sync(kBarT, kTeam);
+                float x[2][4] = {};
+#pragma unroll 2
+                for (int m = 0; m < 8; ++m) {
+                    const float4 a0 = *reinterpret_cast<const float4 *>(Br0 + ((m ^ x0) << 2));
+                    const float4 a1 = *reinterpret_cast<const float4 *>(Br1 + ((m ^ x1) << 2));
+                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int i = 32 + 4 * m + e; // Y row i - 32, columns c0 .. + 3
+                        const float4 t4 =
+                            *reinterpret_cast<const float4 *>(Wk + i * 32 + ((q0 ^ (i & 7)) << 2));
+                        x[0][0] = fmaf(a0v[e], t4.x, x[0][0]); x[0][1] = fmaf(a0v[e], t4.y, x[0][1]);
+                        x[0][2] = fmaf(a0v[e], t4.z, x[0][2]); x[0][3] = fmaf(a0v[e], t4.w, x[0][3]);
+                        x[1][0] = fmaf(a1v[e], t4.x, x[1][0]); x[1][1] = fmaf(a1v[e], t4.y, x[1][1]);
+                        x[1][2] = fmaf(a1v[e], t4.z, x[1][2]); x[1][3] = fmaf(a1v[e], t4.w, x[1][3]);
+                    }
+                }
+                group_sync(kBarT, kTeam); // Y is read: T21 takes its place
+                *reinterpret_cast<float4 *>(Yr0) = make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
+                *reinterpret_cast<float4 *>(Yr1) = make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
+            }
+            // ---- T diag(beta), -T diag(beta gamma) -> the tf32 B operands of MMA 1,
+            //      once MMA 1 of the previous chunk has read them
+            good = c == 0 || waitp(bar_m1, ph1);
+            group_sync(kBarT, kTeam);
+            if (good) {
+                float4 t4[6];
+#pragma unroll
+                for (int jj = 0; jj < 6; ++jj)
+                    t4[jj] = *reinterpret_cast<const float4 *>(Wk + tri_o(jj));
+#pragma unroll
+                for (int jj = 0; jj < 6; ++jj) {
+                    const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[tri_c(jj)]);
+                    const float4 G4 = *reinterpret_cast<const float4 *>(&sm.G[sl][tri_c(jj)]);
+                    const float4 g4 = make_float4(__expf(G4.x), __expf(G4.y), __expf(G4.z), __expf(G4.w));
+                    const float4 tb = make_float4(t4[jj].x * b4.x, t4[jj].y * b4.y, t4[jj].z * b4.z,
+                                                  t4[jj].w * b4.w);
+                    *reinterpret_cast<float4 *>(sm.Tb + tri_o(jj)) = tf32_rna(tb);
+                    *reinterpret_cast<float4 *>(sm.Tg + tri_o(jj)) =
+                        tf32_rna(make_float4(-tb.x * g4.x, -tb.y * g4.y, -tb.z * g4.z, -tb.w * g4.w));
+                }
+            }
+            fence_proxy_async_smem();
+            if (group_sync_or(kBarT, kTeam, !good || *abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (tt == 0) {
+                mbar_arrive((c & 1) ? bar_pT1 : bar_pT0); // T operands and gates of chunk c
+                mbar_arrive(bar_wfree); // Wk may take the next chunk's K K^T rows
+            }
         }
         if (!ok)
-            *(volatile int *)&sm.abort = 1;
+            *abort_flag = 1;
+    } else if (warp < (kSG + kTeam + kTeamP) / 32) {
+        // ==================================================== P team
+        const int pt = tid - kSG - kTeam;
+        uint32_t phT0 = 0, phT1 = 0, phq = 0, phqk = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int sl = c & 3;
+            // ---- diag(gamma) Q in place (rows 64..127 of WQ), tf32
+            bool good = (c & 1) ? waitp(bar_pT1, phT1) : waitp(bar_pT0, phT0); // gates
+            good = waitp(bar_q, phq) && good;
+            if (good) {
+#pragma unroll 1
+                for (int half = 0; half < 4; ++half) {
+                    float4 x[8];
+                    float gr[8];
+                    int off[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const int f = pt + kTeamP * (8 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
+                        off[jj] = cb * (2 * kC * 32) + (kC + r) * 32 + (((f & 7) ^ (r & 7)) << 2);
+                        x[jj] = *reinterpret_cast<const float4 *>(sm.WQ + off[jj]);
+                        gr[jj] = __expf(sm.G[sl][r]); // far inside the tf32 rounding below
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        *reinterpret_cast<float4 *>(sm.WQ + off[jj]) =
+                            tf32_rna(make_float4(x[jj].x * gr[jj], x[jj].y * gr[jj], x[jj].z * gr[jj],
+                                                 x[jj].w * gr[jj]));
+                }
+            }
+            fence_proxy_async_smem();
+            if (group_sync_or(kBarP, kTeamP, !good || *abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (pt == 0)
+                mbar_arrive(bar_pQ);
+            // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32
+            good = waitp(bar_qk, phqk);
+            if (good) {
+                // float4 k (k = 0..11) of this thread: rows prow + 8 k of column block 0
+                // (k < 8, columns pcol) or 32 + prow + 8 (k - 8) of block 1; 8 k keeps
+                // r mod 8, so the swizzle term is one constant per thread
+                const int prow = pt >> 3, pcol = 4 * (pt & 7);
+                const int pbase = prow * 32 + (((pt & 7) ^ (prow & 7)) << 2);
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    float4 x[6];
+#pragma unroll
+                    for (int jj = 0; jj < 6; ++jj) {
+                        const int k = 6 * half + jj;
+                        x[jj] = *reinterpret_cast<const float4 *>(
+                            sm.P + pbase + (k < 8 ? 256 * k : 2048 + 256 * (k - 8)));
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 6; ++jj) {
+                        const int k = 6 * half + jj;
+                        const float Gr = sm.G[sl][k < 8 ? prow + 8 * k : 32 + prow + 8 * (k - 8)];
+                        const float4 Gc =
+                            *reinterpret_cast<const float4 *>(&sm.G[sl][k < 8 ? pcol : 32 + pcol]);
+                        x[jj] = tf32_rna(make_float4(x[jj].x * __expf(fminf(Gr - Gc.x, 0.f)),
+                                                     x[jj].y * __expf(fminf(Gr - Gc.y, 0.f)),
+                                                     x[jj].z * __expf(fminf(Gr - Gc.z, 0.f)),
+                                                     x[jj].w * __expf(fminf(Gr - Gc.w, 0.f))));
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < 6; ++jj) {
+                        const int k = 6 * half + jj;
+                        *reinterpret_cast<float4 *>(sm.P + pbase +
+                                                    (k < 8 ? 256 * k : 2048 + 256 * (k - 8))) = x[jj];
+                    }
+                }
+            }
+            fence_proxy_async_smem();
+            if (group_sync_or(kBarP, kTeamP, !good || *abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (pt == 0)
+                mbar_arrive(bar_pP);
+        }
+        if (!ok)
+            *abort_flag = 1;
+    } else if (warp == kWarpMma) {
+        // ==================================================== MMA issue
+        if (lane == 0 && nchunks > 0) {
+            const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.V), kC * 128, 512);
+            const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
+            const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
+            const uint64_t dTb0 = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
+            const uint64_t dTb1 = sdesc_sw128(smem_u32(sm.Tb + 2048), 16, 1024);
+            const uint64_t dTg0 = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
+            const uint64_t dTg1 = sdesc_sw128(smem_u32(sm.Tg + 2048), 16, 1024);
+            const uint64_t dP0 = sdesc_sw128(smem_u32(sm.P), 16, 1024);
+            const uint64_t dP1 = sdesc_sw128(smem_u32(sm.P + 2048), 16, 1024);
+            const uint64_t dWQ = sdesc_sw128(smem_u32(sm.WQ), 16, 1024);
+            constexpr uint32_t id64 = idesc_tf32(128, 64, true, false);  // A MN-major (MMA 1)
+            constexpr uint32_t id32 = idesc_tf32(128, 32, true, false);
+            constexpr uint32_t id128 = idesc_tf32(128, 128, false, false); // MMA 2
+            constexpr uint32_t idO64 = idesc_tf32(128, 64, false, false);  // MMA 3, O
+            constexpr uint32_t idO32 = idesc_tf32(128, 32, false, false);
+            constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3, S (B MN-major)
+            uint32_t phT0 = 0, phT1 = 0, phv = 0, phk0 = 0, phk1 = 0, phw = 0, phQ = 0, phu = 0;
+            uint32_t phP = 0;
+            uint32_t ph2 = 0, phof0 = 0, phof1 = 0;
+            // MMA 1 of chunk c: U~^T into U_(c%2), -W^T into W.  K steps 0..3 run over
+            // column block 0 of the T tiles (N = 64), 4..7 over block 1 (rows 32..63)
+            auto mma1 = [&](int c) {
+                const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0), dW = tmem + kColW;
+                const uint64_t dK = (c & 1) ? dK1 : dK0;
+#pragma unroll 1
+                for (int s = 0; s < 4; ++s) {
+                    mma_tf32_ss(dU, dV + s * 64, dTb0 + 2 * s, id64, s > 0);
+                    mma_tf32_ss(dW, dK + s * 64, dTg0 + 2 * s, id64, s > 0);
+                }
+#pragma unroll 1
+                for (int s = 4; s < 8; ++s) {
+                    mma_tf32_ss(dU + 32, dV + s * 64, dTb1 + 2 * (s - 4), id32, 1);
+                    mma_tf32_ss(dW + 32, dK + s * 64, dTg1 + 2 * (s - 4), id32, 1);
+                }
+                mma_commit(bar_m1);
+            };
+            bool good = waitp(bar_pT0, phT0);
+            good = good && waitp(bar_v, phv);
+            good = good && waitp(bar_k0, phk0);
+            tc_fence_after();
+            if (good)
+                mma1(0);
+            for (int c = 0; good && c < nchunks; ++c) {
+                const uint32_t dUO = tmem + ((c & 1) ? kColU1 : kColU0);
+                // ---- MMA 2: [U^T | O^T] += S [-W; diag(gamma) Q]^T (A = the state in TMEM)
+                good = waitp(bar_w, phw);
+                good = good && waitp(bar_pQ, phQ);
+                if (c >= 2)
+                    good = good && ((c & 1) ? waitp(bar_of1, phof1) : waitp(bar_of0, phof0));
+                if (!good)
+                    break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int s = 0; s < kD / 8; ++s) {
+                    const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
+                    mma_tf32_ts(dUO, tmem + kColS + 8 * s, dWQ + ks, id128, 1);
+                }
+                mma_commit(bar_m2);
+                // ---- MMA 1 of the next chunk, once MMA 2 (and with it MMA 3 of the
+                //      previous chunk, the last reader of that U buffer) has finished
+                if (c + 1 < nchunks) {
+                    good = waitp(bar_m2, ph2);
+                    good = good && ((c & 1) ? waitp(bar_pT0, phT0) : waitp(bar_pT1, phT1));
+                    good = good && waitp(bar_v, phv);
+                    good = good && ((c & 1) ? waitp(bar_k0, phk0) : waitp(bar_k1, phk1));
+                    if (!good)
+                        break;
+                    tc_fence_after();
+                    mma1(c + 1);
+                }
+                // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K
+                good = waitp(bar_u, phu);
+                good = good && waitp(bar_pP, phP);
+                if (!good)
+                    break;
+                tc_fence_after();
+                {
+                    const uint64_t dK = (c & 1) ? dK1 : dK0;
+#pragma unroll 1
+                    for (int s = 0; s < 4; ++s)
+                        mma_tf32_ts(dUO + 64, dUO + 8 * s, dP0 + 2 * s, idO64, 1);
+#pragma unroll 1
+                    for (int s = 4; s < 8; ++s)
+                        mma_tf32_ts(dUO + 96, dUO + 8 * s, dP1 + 2 * (s - 4), idO32, 1);
+#pragma unroll 1
+                    for (int s = 0; s < kC / 8; ++s)
+                        mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, idS, 1);
+                }
+                mma_commit(bar_m3);
+            }
+            ok = good;
+            // let every MMA issued so far finish before the CTA releases TMEM
+            if (!ok) {
+                *abort_flag = 1;
+                uint32_t phx = 0;
+                const uint32_t bar_x = smem_u32(&sm.bar_fin);
+                mma_commit(bar_x);
+                mbar_wait_bounded(bar_x, phx, kWaitLimit);
+            }
+        }
+    } else {
+        // ==================================================== TMA issue
+        if (lane == 0 && nchunks > 0) {
+            uint32_t cnt[7] = {0, 0, 0, 0, 0, 0, 0}; // loads armed on v, q, k0, k1, kk, qk, z
+            const uint32_t lbar[7] = {bar_v, bar_q, bar_k0, bar_k1, bar_kk, bar_qk, bar_z};
+            // nb 32-column boxes of 64 rows at x0 + 32 b, row t0, block b landing at dst + b * bstride
+            auto tile = [&](int which, float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb,
+                            int bstride) {
+                mbar_arrive_expect_tx(lbar[which], (uint32_t)(nb * kC * 32 * sizeof(float)));
+                for (int b = 0; b < nb; ++b)
+                    tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, lbar[which]);
+                ++cnt[which];
+            };
+            // a lower-triangular Gram tile: block 0 (64 rows) and the lower half of block 1
+            auto gram = [&](int which, float *dst, int x0, int64_t t0) {
+                mbar_arrive_expect_tx(lbar[which], (uint32_t)(kTriFloats * sizeof(float)));
+                tma_load_2d(smem_u32(dst), &maps.kq, x0, (int)t0, lbar[which]);
+                tma_load_2d(smem_u32(dst + 2048), &maps.kq32, x0 + 32, (int)(t0 + 32), lbar[which]);
+                ++cnt[which];
+            };
+            auto t_of = [&](int c) { return start + (int64_t)c * kC; };
+            // the z rows of a chunk: one 128-column box of 64 rows
+            auto ztile = [&](int c) {
+                if constexpr (kZTile) {
+                    mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
+                    tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)t_of(c), bar_z);
+                    ++cnt[6];
+                }
+            };
+            constexpr int kBlkV = kC * 32, kBlkQ = 2 * kC * 32;
+            tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
+            tile(2, sm.K[0], &maps.k, xq, t_of(0), 4, kBlkV);
+            gram(4, sm.Wk, xkk, t_of(0));
+            tile(1, sm.WQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ);
+            gram(5, sm.P, xkk + kC, t_of(0));
+            ztile(0);
+            if (nchunks > 1) {
+                tile(3, sm.K[1], &maps.k, xq, t_of(1), 4, kBlkV);
+                tma_prefetch_2d(&maps.kq, xkk, (int)t_of(1));
+                tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(1) + 32));
+            }
+            // four event streams, each served in chunk order as it completes
+            int iw = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile ? 0 : nchunks;
+            long long t_last = clock64();
+            while (iw < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
+                bool prog = false;
+                // the epilogue of chunk iz has released the z tile
+                if (iz < nchunks && mbar_test_wait((iz & 1) ? bar_of1 : bar_of0, (iz >> 1) & 1)) {
+                    if (iz + 1 < nchunks)
+                        ztile(iz + 1);
+                    ++iz;
+                    prog = true;
+                }
+                if (iw < nchunks && mbar_test_wait(bar_wfree, iw & 1)) { // Wk is free
+                    if (iw + 1 < nchunks)
+                        gram(4, sm.Wk, xkk, t_of(iw + 1));
+                    if (iw + 2 < nchunks) {
+                        tma_prefetch_2d(&maps.kq, xkk, (int)t_of(iw + 2));
+                        tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(iw + 2) + 32));
+                    }
+                    ++iw;
+                    prog = true;
+                }
+                if (i1 < nchunks && mbar_test_wait(bar_m1, i1 & 1)) { // V is free
+                    if (i1 + 1 < nchunks)
+                        tile(0, sm.V, &maps.v, xv, t_of(i1 + 1), 4, kBlkV);
+                    ++i1;
+                    prog = true;
+                }
+                if (i2 < nchunks && mbar_test_wait(bar_m2, i2 & 1)) { // Q is free
+                    if (i2 + 1 < nchunks)
+                        tile(1, sm.WQ + kC * 32, &maps.q, xq, t_of(i2 + 1), 4, kBlkQ);
+                    ++i2;
+                    prog = true;
+                }
+                if (i3 < nchunks && mbar_test_wait(bar_m3, i3 & 1)) { // P and K[i3 % 2] are free
+                    if (i3 + 1 < nchunks)
+                        gram(5, sm.P, xkk + kC, t_of(i3 + 1));
+                    if (i3 + 2 < nchunks)
+                        tile((i3 & 1) ? 3 : 2, sm.K[i3 & 1], &maps.k, xq, t_of(i3 + 2), 4, kBlkV);
+                    ++i3;
+                    prog = true;
+                }
+                if (prog) {
+                    t_last = clock64();
+                } else if (clock64() - t_last > kWaitLimit || *abort_flag) {
+                    ok = false;
+                    break;
+                } else {
+                    __nanosleep(64); // leave the issue slots to the working warps
+                }
+            }
+            // every armed load lands before the CTA exits
+#pragma unroll
+            for (int b = 0; b < 7; ++b)
+                if (cnt[b] > 0)
+                    mbar_wait_bounded(lbar[b], (cnt[b] - 1) & 1, kWaitLimit);
+            if (!ok)
+                *abort_flag = 1;
+        }
     }
 
     ok = !__syncthreads_or(!ok); // one verdict for the whole CTA
     if (!ok) {
         if (tid == 0 && p.ws_err != nullptr)
             atomicOr(p.ws_err, 1u);
-    } else if (is_state && p.final_state != nullptr) {
+    } else if (warp < kSG / 32 && p.final_state != nullptr) {
         const int lq = warp & 3, hf = warp >> 2, vch = lq * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
         float *dst = p.final_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf;
@@ -912,24 +1180,25 @@ EncodeTiledFn encoder() {
     return fn;
 }
 
-// Row-major 2-D map over `rows` rows of `cols` elements (row pitch `pitch`
-// bytes), boxes of `box_cols` x 64 rows.
-bool encode_2d(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t cols,
-               uint64_t rows, uint64_t pitch, uint32_t box_cols, CUtensorMapSwizzle sw) {
+// Row-major 2-D map over `rows` rows of `cols` elements (row pitch
+// `pitch` bytes), boxes of `box_cols` x `box_rows`.
+bool encode_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t pitch,
+               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw,
+               CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32) {
     EncodeTiledFn enc = encoder();
     if (enc == nullptr)
         return false;
     const cuuint64_t dims[2] = {cols, rows};
     const cuuint64_t strides[1] = {pitch};
-    const cuuint32_t box[2] = {box_cols, (cuuint32_t)kC};
+    const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t es[2] = {1, 1};
-    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, es,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStream_t s) {
-    const size_t smem = sizeof(ChunkSmem<T>) + 1024;
+    const size_t smem = sizeof(ChunkSmem);
     cudaError_t e = cudaFuncSetAttribute(chunk_prefill_kernel<T>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
@@ -938,20 +1207,19 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
     memset(&maps, 0, sizeof(maps));
     if (p.N > 0) {
         const uint64_t N = (uint64_t)p.N, F = sizeof(float);
-        const uint64_t qkw = 2ull * p.Hk * kD;
+        const uint64_t qkw = 2ull * p.Hk * kD, kqw = (uint64_t)p.Hk * 2 * kC;
         const bool okm =
-            encode_2d(&maps.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_v, (uint64_t)p.Hv * kD, N,
-                      (uint64_t)p.Hv * kD * F, 32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
-            encode_2d(&maps.k, CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
-                      (const float *)p.ws_qk + (size_t)p.Hk * kD, (uint64_t)p.Hk * kD, N, qkw * F,
-                      32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
-            encode_2d(&maps.q, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_qk, (uint64_t)p.Hk * kD, N,
-                      qkw * F, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            encode_2d(&maps.kq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.ws_kq, (uint64_t)p.Hk * 2 * kC,
-                      N, (uint64_t)p.Hk * 2 * kC * F, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.v, p.ws_v, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * F, 32, kC,
+                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
+            encode_2d(&maps.k, (const float *)p.ws_qk + (size_t)p.Hk * kD, (uint64_t)p.Hk * kD, N,
+                      qkw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
+            encode_2d(&maps.q, p.ws_qk, (uint64_t)p.Hk * kD, N, qkw * F, 32, kC,
+                      CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.kq, p.ws_kq, kqw, N, kqw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.kq32, p.ws_kq, kqw, N, kqw * F, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
             (sizeof(T) != 2 ||
-             encode_2d(&maps.z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.z, (uint64_t)p.Hv * kD, N,
-                       (uint64_t)p.Hv * kD * sizeof(T), kD, CU_TENSOR_MAP_SWIZZLE_NONE));
+             encode_2d(&maps.z, p.z, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * sizeof(T), kD, kC,
+                       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16));
         if (!okm)
             return cudaErrorInvalidValue;
     }

@@ -60,6 +60,18 @@ template <typename T> __device__ __forceinline__ Vec16<T> zero16() {
     return v;
 }
 
+// Loads and stores cached in L2 only: a kernel whose shared memory takes most
+// of the L1/shared store leaves little L1, and strided element accesses that
+// allocate L1 lines then serialise.
+__device__ __forceinline__ float ld_cg(const float *p) { return __ldcg(p); }
+__device__ __forceinline__ float ld_cg(const __nv_bfloat16 *p) {
+    return __bfloat162float(__ushort_as_bfloat16(__ldcg(reinterpret_cast<const unsigned short *>(p))));
+}
+__device__ __forceinline__ void st_cg(float *p, float x) { __stcg(p, x); }
+__device__ __forceinline__ void st_cg(__nv_bfloat16 *p, float x) {
+    __stcg(reinterpret_cast<unsigned short *>(p), __bfloat16_as_ushort(__float2bfloat16_rn(x)));
+}
+
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
 __device__ __forceinline__ float siluf_(float x) { return x / (1.0f + __expf(-x)); }
 // log(1 + e^x) = max(x, 0) + log1p(e^{-|x|}), finite for every x.

@@ -30,8 +30,10 @@ conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int 
     constexpr int LANES = D / V; // lanes per head
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "head must tile a warp");
     const int C = (2 * Hk + Hv) * D;
-    if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
-        *err = 0u; // status word of this call; later kernels only set bits
+    if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+        err[0] = 0u; // status word of this call; later kernels only set bits
+        err[1] = 0u; // where the first timed-out wait gave up
+    }
     const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * V;
     const bool active = c0 < C;
     const int cc = active ? c0 : 0; // inactive lanes still join the shuffles
