@@ -45,9 +45,6 @@ constexpr int kD = 128; // head dim (d_k = d_v)
 
 // -------------------------------------------------------------- K K^T, Q K^T
 
-constexpr int kKqThreads = 256;
-constexpr int kTp = kC + 4; // row stride of the transposed tiles (16-byte aligned, banks staggered)
-
 // Chunk offsets: offs[n] = number of 64-token chunks in sequences 0 .. n-1
 // (offs[batch] = total).  One CTA of 1024 threads; each thread scans a run of
 // consecutive sequences, then the run totals are scanned across the block.
@@ -85,10 +82,23 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 // One CTA per (chunk, q/k head j): with the chunk's rows t = t0 + r, r < nr,
 //   kq[t][j][0][s] = k_t . k_{t0+s} for s < r, else 0
 //   kq[t][j][1][s] = q_t . k_{t0+s} for s <= r, else 0
-// from the normalised float32 q|k rows of the workspace.  Thread (tr, ts) of
-// a 16 x 16 grid owns rows 4 tr .. + 3 and columns 4 ts .. + 3 of both
-// products (blocks above the diagonal are zero); the chunk's q and k sit
-// transposed in shared memory so that every step reads three float4s.
+// from the normalised float32 q|k rows of the workspace, exact in FP32.  The
+// chunk's q and k sit transposed in shared memory; thread i < 136 owns the
+// lower-triangle 4 x 4 tile (tr, ts), ts <= tr, i = tr (tr + 1) / 2 + ts, of
+// both products, so that every warp but the last is full.
+constexpr int kKqThreads = 160;
+constexpr int kTp = kC + 4; // row stride of the transposed tiles (16-byte aligned, banks staggered)
+
+__device__ __forceinline__ void tri_tile(int i, int &tr, int &ts) {
+    int r = (int)((sqrtf(8.0f * (float)i + 1.0f) - 1.0f) * 0.5f);
+    while ((r + 1) * (r + 2) / 2 <= i)
+        ++r;
+    while (r * (r + 1) / 2 > i)
+        --r;
+    tr = r;
+    ts = i - r * (r + 1) / 2;
+}
+
 __global__ void __launch_bounds__(kKqThreads)
 kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int batch, int64_t N,
                int Hk, const int32_t *__restrict__ offs, float *__restrict__ kq) {
@@ -111,23 +121,37 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
     const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
     const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
     const int64_t QKW = 2 * (int64_t)Hk * kD;
-    for (int e = tid; e < kC * (kD / 4); e += kKqThreads) {
-        const int r = e % kC, d = (e / kC) * 4; // consecutive threads: consecutive rows
-        float4 q4 = make_float4(0.f, 0.f, 0.f, 0.f), k4 = q4;
-        if (r < nr) {
-            const float *row = qk + (t0 + r) * QKW + j * kD + d;
-            q4 = __ldg(reinterpret_cast<const float4 *>(row));
-            k4 = __ldg(reinterpret_cast<const float4 *>(row + Hk * kD));
+    // four rounds of loads in flight before their stores (consecutive threads:
+    // consecutive rows, so the transposed stores do not conflict)
+    for (int e0 = tid; e0 < kC * (kD / 4); e0 += 4 * kKqThreads) {
+        float4 q4[4], k4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u * kKqThreads, r = e % kC, d = (e / kC) * 4;
+            q4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            k4[u] = q4[u];
+            if (e < kC * (kD / 4) && r < nr) {
+                const float *row = qk + (t0 + r) * QKW + j * kD + d;
+                q4[u] = __ldg(reinterpret_cast<const float4 *>(row));
+                k4[u] = __ldg(reinterpret_cast<const float4 *>(row + Hk * kD));
+            }
         }
-        Qt[(d + 0) * kTp + r] = q4.x; Qt[(d + 1) * kTp + r] = q4.y;
-        Qt[(d + 2) * kTp + r] = q4.z; Qt[(d + 3) * kTp + r] = q4.w;
-        Kt[(d + 0) * kTp + r] = k4.x; Kt[(d + 1) * kTp + r] = k4.y;
-        Kt[(d + 2) * kTp + r] = k4.z; Kt[(d + 3) * kTp + r] = k4.w;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int e = e0 + u * kKqThreads, r = e % kC, d = (e / kC) * 4;
+            if (e < kC * (kD / 4)) {
+                Qt[(d + 0) * kTp + r] = q4[u].x; Qt[(d + 1) * kTp + r] = q4[u].y;
+                Qt[(d + 2) * kTp + r] = q4[u].z; Qt[(d + 3) * kTp + r] = q4[u].w;
+                Kt[(d + 0) * kTp + r] = k4[u].x; Kt[(d + 1) * kTp + r] = k4[u].y;
+                Kt[(d + 2) * kTp + r] = k4[u].z; Kt[(d + 3) * kTp + r] = k4[u].w;
+            }
+        }
     }
     __syncthreads();
-    const int tr = tid >> 4, ts = tid & 15;
-    float kk[4][4] = {}, qq[4][4] = {};
-    if (ts <= tr) {
+    if (tid < 136) {
+        int tr, ts;
+        tri_tile(tid, tr, ts);
+        float kk[4][4] = {}, qq[4][4] = {};
 #pragma unroll 4
         for (int d = 0; d < kD; ++d) {
             const float4 kr = *reinterpret_cast<const float4 *>(Kt + d * kTp + 4 * tr);
@@ -143,22 +167,31 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
                     qq[x][y] = fmaf(b[x], c[y], qq[x][y]);
                 }
         }
-    }
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const int r = 4 * tr + x;
-        if (r >= nr)
-            break;
-        float o1[4], o2[4];
+        for (int x = 0; x < 4; ++x) {
+            const int r = 4 * tr + x;
+            if (r >= nr)
+                break;
+            float o1[4], o2[4];
 #pragma unroll
-        for (int y = 0; y < 4; ++y) {
-            const int s = 4 * ts + y;
-            o1[y] = s < r ? kk[x][y] : 0.f;
-            o2[y] = s <= r ? qq[x][y] : 0.f;
+            for (int y = 0; y < 4; ++y) {
+                const int s = 4 * ts + y;
+                o1[y] = s < r ? kk[x][y] : 0.f;
+                o2[y] = s <= r ? qq[x][y] : 0.f;
+            }
+            float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
+            *reinterpret_cast<float4 *>(o + 4 * ts) = make_float4(o1[0], o1[1], o1[2], o1[3]);
+            *reinterpret_cast<float4 *>(o + kC + 4 * ts) = make_float4(o2[0], o2[1], o2[2], o2[3]);
         }
-        float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
-        *reinterpret_cast<float4 *>(o + 4 * ts) = make_float4(o1[0], o1[1], o1[2], o1[3]);
-        *reinterpret_cast<float4 *>(o + kC + 4 * ts) = make_float4(o2[0], o2[1], o2[2], o2[3]);
+    }
+    // the tiles right of each row's diagonal tile are zero
+    for (int e = tid; e < kC * 16; e += kKqThreads) {
+        const int r = e >> 4, tx = e & 15;
+        if (tx > (r >> 2) && r < nr) {
+            float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
+            *reinterpret_cast<float4 *>(o + 4 * tx) = make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(o + kC + 4 * tx) = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
     }
 }
 
@@ -1232,15 +1265,18 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 
 size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * 2 * kC * sizeof(float); }
 
-cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s) {
+cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s) {
     if (p.N == 0 || p.batch == 0)
         return cudaSuccess;
     chunk_offsets_kernel<<<1, 1024, 0, s>>>(p.cu, p.batch, p.N, p.ws_offs);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess)
-        return e;
+    return cudaGetLastError();
+}
+
+cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s) {
+    if (p.N == 0 || p.batch == 0)
+        return cudaSuccess;
     const size_t smem = sizeof(float) * 2 * kD * kTp;
-    e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     // upper bound on the chunk count: every sequence adds at most one partial chunk

@@ -73,7 +73,7 @@ __device__ __forceinline__ void st_cg(__nv_bfloat16 *p, float x) {
 }
 
 __device__ __forceinline__ float sigmoidf_(float x) { return 1.0f / (1.0f + __expf(-x)); }
-__device__ __forceinline__ float siluf_(float x) { return x / (1.0f + __expf(-x)); }
+__device__ __forceinline__ float siluf_(float x) { return __fdividef(x, 1.0f + __expf(-x)); }
 // log(1 + e^x) = max(x, 0) + log1p(e^{-|x|}), finite for every x.
 __device__ __forceinline__ float softplusf_(float x) {
     return fmaxf(x, 0.0f) + log1pf(__expf(-fabsf(x)));

@@ -45,43 +45,33 @@ conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int 
         w[i][0] = wv.x; w[i][1] = wv.y; w[i][2] = wv.z; w[i][3] = wv.w;
     }
     const int64_t t0 = (int64_t)blockIdx.x * kConvTokens;
-    for (int tt = 0; tt < kConvTokens; ++tt) {
-        const int64_t t = t0 + tt;
-        if (t >= N)
-            break; // uniform over the block
-        const int n = seq_of_token(cu, batch, t);
-        int64_t start = __ldg(cu + n);
-        start = start > t ? t : (start < 0 ? 0 : start); // malformed cu_seqlens stay in bounds
-        float acc[V];
+    // all source rows of the block's tokens first (rows t0 - 3 .. t0 + 7; rows
+    // outside [0, N) read as zero and feed no output), so that their loads overlap
+    Vec16<T> rows[kConvTokens + 3];
 #pragma unroll
-        for (int i = 0; i < V; ++i)
-            acc[i] = 0.f;
-#pragma unroll
-        for (int tap = 0; tap < 4; ++tap) {
-            const int64_t src = t - 3 + tap;
-            Vec16<T> x;
-            if (src >= start)
-                x = ld16_nc(qkv + src * C + cc);
-            else if (init_conv != nullptr)
-                x = ld16_nc(init_conv + ((int64_t)n * 3 + (3 + (src - start))) * C + cc);
-            else
-                x = zero16<T>();
-#pragma unroll
-            for (int i = 0; i < V; ++i)
-                acc[i] = fmaf(w[i][tap], x.get(i), acc[i]);
-        }
+    for (int k = 0; k < kConvTokens + 3; ++k) {
+        const int64_t src = t0 - 3 + k;
+        rows[k] = (src >= 0 && src < N) ? ld16_nc(qkv + src * C + cc) : zero16<T>();
+    }
+    int n = seq_of_token(cu, batch, t0 < N ? t0 : N - 1);
+    int64_t start = __ldg(cu + n), next = __ldg(cu + n + 1);
+    const int64_t tend = t0 + kConvTokens < N ? t0 + kConvTokens : N;
+    // q and k leave L2-normalised (the warp reduces only if some lane holds q
+    // or k), v as is; all in float32 so that no rounding is added before the
+    // recurrence, except that v, when only the tensor-core path reads it, is
+    // rounded to its tf32 operand here
+    const bool norm_warp = __any_sync(0xffffffffu, region < 2);
+    auto emit = [&](int64_t t, float (&acc)[V]) {
         float ss = 0.f;
 #pragma unroll
         for (int i = 0; i < V; ++i) {
             acc[i] = siluf_(acc[i]);
             ss = fmaf(acc[i], acc[i], ss);
         }
-        ss = group_sum<LANES>(ss);
+        if (norm_warp)
+            ss = group_sum<LANES>(ss);
         if (!active)
-            continue;
-        // q and k leave L2-normalised, v as is; all in float32 so that no
-        // rounding is added before the recurrence, except that v, when only
-        // the tensor-core path reads it, is rounded to its tf32 operand here
+            return;
         const float f = region == 2 ? 1.0f : rsqrtf(ss + l2_eps) * (region == 0 ? q_scale : 1.0f);
         if (region == 2 && round_v) {
 #pragma unroll
@@ -97,6 +87,56 @@ conv_prep_kernel(const T *__restrict__ qkv, const int32_t *__restrict__ cu, int 
         for (int i = 0; i < V; i += 4)
             *reinterpret_cast<float4 *>(dst + i) =
                 make_float4(acc[i] * f, acc[i + 1] * f, acc[i + 2] * f, acc[i + 3] * f);
+    };
+    if (start <= t0 - 3 && next >= tend) {
+        // one sequence covers every tap of every token of the block (the usual case)
+#pragma unroll
+        for (int tt = 0; tt < kConvTokens; ++tt) {
+            if (t0 + tt >= N)
+                break; // uniform over the block
+            float acc[V];
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                acc[i] = w[i][0] * rows[tt].get(i);
+#pragma unroll
+            for (int tap = 1; tap < 4; ++tap)
+#pragma unroll
+                for (int i = 0; i < V; ++i)
+                    acc[i] = fmaf(w[i][tap], rows[tt + tap].get(i), acc[i]);
+            emit(t0 + tt, acc);
+        }
+        return;
+    }
+#pragma unroll 1
+    for (int tt = 0; tt < kConvTokens; ++tt) {
+        const int64_t t = t0 + tt;
+        if (t >= N)
+            break; // uniform over the block
+        while (t >= next && n + 1 < batch) { // t starts a new sequence (after any empty ones)
+            ++n;
+            start = next;
+            next = __ldg(cu + n + 1);
+        }
+        const int64_t st = start > t ? t : (start < 0 ? 0 : start); // malformed cu_seqlens stay in bounds
+        float acc[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+            acc[i] = 0.f;
+#pragma unroll
+        for (int tap = 0; tap < 4; ++tap) {
+            const int64_t src = t - 3 + tap;
+            Vec16<T> x;
+            if (src >= st)
+                x = ld16_nc(qkv + src * C + cc); // rows[] would need a dynamic index here
+            else if (init_conv != nullptr)
+                x = ld16_nc(init_conv + ((int64_t)n * 3 + (3 + (src - st))) * C + cc);
+            else
+                x = zero16<T>();
+#pragma unroll
+            for (int i = 0; i < V; ++i)
+                acc[i] = fmaf(w[i][tap], x.get(i), acc[i]);
+        }
+        emit(t, acc);
     }
 }
 

@@ -61,6 +61,7 @@ constexpr size_t kWorkspaceHeader = 256; // holds the device status word
 cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_final_conv(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_recurrent_prefill(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_chunk_prefill(const PrefillArgs &p, cudaStream_t s);
 size_t kq_workspace_bytes(int Hk, int64_t N);
