@@ -16,12 +16,13 @@
 // Only exp(G_r - G_s) with s <= r and exp(G_C - G_s) are ever formed, so no
 // factor exceeds 1 however strong the decay.
 //
-// Mapping onto the tensor core (M = 128 = d_v is the TMEM lane dimension):
-//   MMA 1  U~^T = V^T (T diag b)^T,  -W^T = K^T (-T diag b gamma)^T
-//          A = V, K (smem, MN-major), B = the two T tiles (smem, K-major)
-//   MMA 2  [U^T | O^T] += S0 [-W ; diag(gamma) Q]^T   (one N = 128 product,
-//          A = the FP32 state in TMEM; U^T starts as U~^T, O^T as zero)
-//   MMA 3  O^T += U^T P^T  and  S += (U diag(gamma_C/gamma))^T K
+// Mapping onto the tensor core (M = 128 = d_v is the TMEM lane dimension),
+// with X = K S0^T:
+//   MMA 1   U~^T = V^T (T diag b)^T        A = V (smem, MN-major), B = T diag b
+//   MMA 2   [X^T | O^T] = S0 [K ; diag(gamma) Q]^T   (one N = 128 product; A =
+//           the FP32 state in TMEM, B = K and gamma Q, K-major)
+//   MMA 2b  U^T = U~^T + X^T (-T diag b gamma)^T     (A = X^T from TMEM)
+//   MMA 3   O^T += U^T P^T  and  S += (U diag(gamma_C/gamma))^T K   (K MN-major)
 // The state lives in TMEM for the whole sequence.  All products run as
 // kind::tf32; every operand computed here is rounded to nearest first (the
 // tensor core's own conversion truncates, a bias that would accumulate
@@ -199,20 +200,19 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
 //
 // One CTA per (value head, sequence), five roles that run consecutive chunks
 // at once and hand over through mbarriers:
-//   state group (warps 0..7): the W pass (-W^T from TMEM to shared memory),
-//     the U pass (U and U diag(gamma_C/gamma) rounded, S scaled by gamma_C)
-//     and the gated-RMSNorm epilogue; warps w and w + 4 share TMEM lanes
-//     32 (w % 4) .. + 31 (lane = value channel) and split the columns.  O and
-//     U are double-buffered in TMEM, so the epilogue of chunk c overlaps MMA 2
-//     of chunk c + 1;
+//   state group (warps 0..7): the U pass (U and U diag(gamma_C/gamma) rounded
+//     to tf32, S scaled by gamma_C) and the gated-RMSNorm epilogue; warps w and
+//     w + 4 share TMEM lanes 32 (w % 4) .. + 31 (lane = value channel) and
+//     split the columns.  X/O and U are double-buffered in TMEM, so the
+//     epilogue of chunk c overlaps MMA 2 of chunk c + 1;
 //   T team (warps 8..11): gates, A, T = (I + A)^-1 in a working tile of its
-//     own, then T diag(beta) and -T diag(beta gamma) once MMA 1 of the
-//     previous chunk has released them;
+//     own, then T diag(beta) and -T diag(beta gamma) into the tiles of the
+//     chunk's parity once MMA 1 and 2b of chunk c - 2 have read them;
 //   P team (warps 12..13): diag(gamma) Q in place and P from the Q K^T tile;
 //   MMA warp (warp 14) and TMA warp (warp 15): one elected lane each.
 // Sixteen warps, four per scheduler, leave 128 registers a thread.
-// The per-chunk critical path is MMA 2 -> U pass -> MMA 3 -> MMA 2; MMA 1 and
-// the W pass of the next chunk run beside the U pass.
+// The per-chunk critical path is MMA 2 -> MMA 2b -> U pass -> MMA 3 -> MMA 2;
+// MMA 1 of the next chunk runs beside the U pass.
 
 constexpr int kSG = 256;                          // state group threads
 constexpr int kTeam = 128;                        // T team threads
@@ -221,22 +221,20 @@ constexpr int kThreads = kSG + kTeam + kTeamP + 64; // + MMA warp + TMA warp: 16
 constexpr int kWarpMma = (kSG + kTeam + kTeamP) / 32; // 14
 constexpr int kBarSG = 1, kBarT = 2, kBarP = 3;   // named barriers
 
-// TMEM columns: state, two [U | O] pairs (MMA 2 writes one pair with a single
-// N = 128 product), -W^T, U diag(gamma_C / gamma)
+// TMEM columns: the state, two [X^T | O^T] pairs (MMA 2 writes one pair with a
+// single N = 128 product; once MMA 2b has read X^T its columns take U diag(
+// gamma_C / gamma)), two U^T buffers.  All by chunk parity.
 constexpr uint32_t kColS = 0;
-constexpr uint32_t kColU0 = 128, kColU1 = 256; // O of each pair sits 64 columns on
-constexpr uint32_t kColW = 384;
-constexpr uint32_t kColUk = 448;
+constexpr uint32_t kColX0 = 128, kColX1 = 256; // O of each pair sits 64 columns on
+constexpr uint32_t kColU0 = 384, kColU1 = 448;
 constexpr uint32_t kTmemCols = 512;
 
 // Operand layouts.  Both split a tile along its contiguous dimension into
 // 32-float (128-byte) column blocks.
 //
-// K-major operand (rows = M or N, columns = K), 128-byte swizzle: the 16-byte
-// chunks of row r are XOR-swizzled by r mod 8; blocks of R rows.
-__device__ __forceinline__ int swz(int r, int c, int R) {
-    return (c >> 5) * (R * 32) + r * 32 + ((((c & 31) >> 2) ^ (r & 7)) << 2) + (c & 3);
-}
+// K-major operands (rows = M or N, columns = K): 128-byte swizzle, the
+// 16-byte chunks of row r XOR-swizzled by r mod 8; element (r, c) of a tile of
+// R-row blocks at (c / 32) R 32 + 32 r + 4 (((c mod 32) / 4) xor (r mod 8)) + c mod 4.
 // MN-major tf32 operands (V, K) use the 128-byte swizzle on a 32-byte base,
 // written only by TMA: 32-byte chunks of row k XOR-swizzled by k mod 4.
 // Lower-triangular 64 x 64 tile in the K-major layout with its zero quadrant
@@ -248,12 +246,12 @@ __device__ __forceinline__ int swz(int r, int c, int R) {
 constexpr int kTriFloats = 3 * 1024;
 
 struct __align__(1024) ChunkSmem {
-    // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = -W, rows 64..127 = diag(gamma) Q
-    float WQ[2 * kC * kD];
+    // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = K, rows 64..127 = diag(gamma) Q
+    float KQ[2 * kC * kD];
     float V[kC * kD];          // A of MMA 1 (MN-major)
-    float K[2][kC * kD];       // A of MMA 1 / B of MMA 3 (MN-major), by chunk parity
-    float Tb[kTriFloats];      // B of MMA 1: T diag(beta)
-    float Tg[kTriFloats];      // B of MMA 1: -T diag(beta gamma)
+    float K[kC * kD];          // B of MMA 3 (MN-major)
+    float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta), by chunk parity
+    float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma), by chunk parity
     float P[kTriFloats];       // B of MMA 3: lands as Q K^T rows, becomes P
     float Wk[kTriFloats];      // T team: lands as K K^T rows, becomes A, then T
     // z rows of the chunk (16-bit activations).  Once the state group has formed
@@ -262,10 +260,10 @@ struct __align__(1024) ChunkSmem {
     __nv_bfloat16 Z[kC * kD];
     float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
     float beta[kC];            // T team's current chunk
-    unsigned long long bar_v, bar_q, bar_k[2], bar_kk, bar_qk, bar_z; // TMA landings
-    unsigned long long bar_m1, bar_m2, bar_m3;                  // MMA completions
-    unsigned long long bar_w, bar_u, bar_of[2];                 // state group -> MMA
-    unsigned long long bar_pT[2], bar_pQ, bar_pP, bar_wfree;    // T / P teams -> MMA, TMA
+    unsigned long long bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z; // TMA landings
+    unsigned long long bar_m1, bar_m2, bar_m2b[2], bar_m3;      // MMA completions
+    unsigned long long bar_u, bar_of[2];                        // state group -> MMA
+    unsigned long long bar_pT[4], bar_pQ, bar_pP, bar_wfree;    // T / P teams -> MMA, TMA
     unsigned long long bar_fin;                                 // MMA drain on abort
     uint32_t tmem;
     int abort;
@@ -279,6 +277,7 @@ struct ChunkMaps {
     CUtensorMap v;    // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle
     CUtensorMap k;    // normalised k, [N, Hk*128] of the q|k rows, MN-major tf32 swizzle
     CUtensorMap q;    // normalised q, [N, Hk*128], 128-byte swizzle (K-major)
+    CUtensorMap kmaj; // normalised k, [N, Hk*128], 128-byte swizzle (K-major)
     CUtensorMap kq;   // Gram rows, [N, Hk*128] fp32, 32 x 64 boxes, 128-byte swizzle
     CUtensorMap kq32; // the same with 32 x 32 boxes
     CUtensorMap z;    // z, [N, Hv*128] bf16, 128 x 64 boxes, no swizzle (bf16 activations)
@@ -339,40 +338,34 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     const int64_t HD = (int64_t)p.Hv * kD;
 
     const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
-    const uint32_t bar_k0 = smem_u32(&sm.bar_k[0]), bar_k1 = smem_u32(&sm.bar_k[1]);
+    const uint32_t bar_k = smem_u32(&sm.bar_k), bar_kmaj = smem_u32(&sm.bar_kmaj);
     const uint32_t bar_kk = smem_u32(&sm.bar_kk), bar_qk = smem_u32(&sm.bar_qk);
     const uint32_t bar_z = smem_u32(&sm.bar_z);
     constexpr bool kZTile = sizeof(T) == 2; // z comes by TMA (16-bit) or from global (fp32)
     const uint32_t bar_m1 = smem_u32(&sm.bar_m1), bar_m2 = smem_u32(&sm.bar_m2);
     const uint32_t bar_m3 = smem_u32(&sm.bar_m3);
-    const uint32_t bar_w = smem_u32(&sm.bar_w), bar_u = smem_u32(&sm.bar_u);
+    // MMA 2b done, by chunk parity (its waiters are a chunk apart)
+    auto bar_m2b = [&](int c) { return smem_u32(&sm.bar_m2b[c & 1]); };
+    const uint32_t bar_u = smem_u32(&sm.bar_u);
     const uint32_t bar_of0 = smem_u32(&sm.bar_of[0]), bar_of1 = smem_u32(&sm.bar_of[1]);
-    // T tiles + gates ready, by chunk parity: a waiter for chunk c must see that
-    // phase before the barrier can move on, and chunk c + 1 may finish first
-    const uint32_t bar_pT0 = smem_u32(&sm.bar_pT[0]), bar_pT1 = smem_u32(&sm.bar_pT[1]);
+    // T tiles + gates of chunk c ready, by chunk index mod 4: a waiter for chunk c
+    // must see that phase before the barrier can move on, and the T team may run
+    // up to two chunks ahead of the state group
+    auto bar_pT = [&](int c) { return smem_u32(&sm.bar_pT[c & 3]); };
     const uint32_t bar_pQ = smem_u32(&sm.bar_pQ);
     const uint32_t bar_pP = smem_u32(&sm.bar_pP), bar_wfree = smem_u32(&sm.bar_wfree);
     if (tid == 0) {
-        mbar_init(bar_v, 1);
-        mbar_init(bar_q, 1);
-        mbar_init(bar_k0, 1);
-        mbar_init(bar_k1, 1);
-        mbar_init(bar_kk, 1);
-        mbar_init(bar_qk, 1);
-        mbar_init(bar_z, 1);
-        mbar_init(bar_m1, 1);
-        mbar_init(bar_m2, 1);
-        mbar_init(bar_m3, 1);
-        mbar_init(bar_w, 1);
-        mbar_init(bar_u, 1);
-        mbar_init(bar_of0, 1);
-        mbar_init(bar_of1, 1);
-        mbar_init(bar_pT0, 1);
-        mbar_init(bar_pT1, 1);
-        mbar_init(bar_pQ, 1);
-        mbar_init(bar_pP, 1);
-        mbar_init(bar_wfree, 1);
-        mbar_init(smem_u32(&sm.bar_fin), 1);
+        const uint32_t one[] = {bar_v,  bar_q,   bar_k,   bar_kmaj, bar_kk,   bar_qk,  bar_z,
+                                bar_m1, bar_m2,  bar_m3,  bar_u,    bar_of0,  bar_of1, bar_pQ,
+                                bar_pP, bar_wfree, smem_u32(&sm.bar_fin)};
+#pragma unroll
+        for (int b = 0; b < (int)(sizeof(one) / sizeof(one[0])); ++b)
+            mbar_init(one[b], 1);
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+            mbar_init(smem_u32(&sm.bar_pT[b]), 1);
+        mbar_init(smem_u32(&sm.bar_m2b[0]), 1);
+        mbar_init(smem_u32(&sm.bar_m2b[1]), 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -415,6 +408,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         ++waits_seen;
         return done;
     };
+    // the same for an explicit phase parity (barriers split by chunk index)
+    auto waitq = [&](uint32_t bar, uint32_t parity) {
+        uint32_t ph = parity;
+        return waitp(bar, ph);
+    };
     bool ok = true;
 
     if (warp < kSG / 32) {
@@ -422,7 +420,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
         const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
-        // initial state into TMEM (row vch, this half's 64 columns); both O buffers zero
+        // initial state into TMEM (row vch, this half's 64 columns)
         {
             const float *src = p.init_state
                                    ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
@@ -438,48 +436,27 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
             }
-            float zero[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-                zero[i] = 0.f;
-            tmem_st32(tl + kColU0 + 64 + 32 * hf, zero);
-            tmem_st32(tl + kColU1 + 64 + 32 * hf, zero);
             tmem_wait_st();
         }
+        tc_fence_before();
+        if (group_sync_or(kBarSG, kSG, *abort_flag))
+            ok = false;
+        if (ok && tid == 0)
+            mbar_arrive(bar_u); // phase 0 of the U barrier: the initial state is in TMEM
         const float wn = __ldg(p.norm_w + vch);
-        uint32_t ph1 = 0, ph2 = 0, ph3 = 0, phT0 = 0, phT1 = 0, phz = 0;
+        uint32_t ph3 = 0, phz = 0;
         float *red = reinterpret_cast<float *>(sm.Z); // [4][kC], then rstd[kC]
         float *rstd = red + 4 * kC;
-        // -W^T (TMEM, tf32-rounded) -> rows 0..63 of WQ (K-major: rows r, columns k = vch);
-        // this half takes rows 32 hf .. + 31
-        auto w_pass = [&](int c) -> bool {
-            bool good = waitp(bar_m1, ph1);
-            good = ((c & 1) ? waitp(bar_pT1, phT1) : waitp(bar_pT0, phT0)) && good; // gates
-            good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
-            tc_fence_after();
-            if (good) {
-                float w[32];
-                tmem_ld32(tl + kColW + 32 * hf, w);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    sm.WQ[swz(32 * hf + i, vch, 2 * kC)] = tf32_rna(w[i]);
-            }
-            fence_proxy_async_smem();
-            tc_fence_before();
-            const bool bad = group_sync_or(kBarSG, kSG, !good || *abort_flag);
-            if (!bad && tid == 0)
-                mbar_arrive(bar_w);
-            return !bad;
-        };
-        if (nchunks > 0)
-            ok = w_pass(0);
         for (int c = 0; ok && c < nchunks; ++c) {
             const int sl = c & 3;
-            const uint32_t cU = (c & 1) ? kColU1 : kColU0, cO = cU + 64;
-            // ---- U pass: U -> tf32 (in place), U diag(gamma_C/gamma) -> tf32 (Uk), S *= gamma_C
+            const uint32_t cU = (c & 1) ? kColU1 : kColU0, cX = (c & 1) ? kColX1 : kColX0;
+            const uint32_t cO = cX + 64;
+            // ---- U pass: U -> tf32 (in place), U diag(gamma_C/gamma) -> tf32 into the
+            //      X columns (MMA 2b has read them), S *= gamma_C
             {
-                bool good = __all_sync(0xffffffffu, waitp(bar_m2, ph2));
+                bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
+                good = waitq(bar_m2b(c), (c >> 1) & 1) && good;
+                good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
                 tc_fence_after();
                 if (good) {
                     float u[32], uk[32];
@@ -497,7 +474,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                         u[i] = tf32_rna(u[i]);
                     }
                     tmem_st32(tl + cU + 32 * hf, u);
-                    tmem_st32(tl + kColUk + 32 * hf, uk);
+                    tmem_st32(tl + cX + 32 * hf, uk);
 #pragma unroll
                     for (int cb = 0; cb < 2; ++cb) {
                         float v[32];
@@ -518,15 +495,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 if (tid == 0)
                     mbar_arrive(bar_u);
             }
-            // ---- W pass of the next chunk (MMA 1 of it ran beside the U pass)
-            if (c + 1 < nchunks) {
-                if (!w_pass(c + 1)) {
-                    ok = false;
-                    break;
-                }
-            }
             // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
-            //      RMSNorm over v, times w[v] SiLU(z), stored; then O is zeroed
+            //      RMSNorm over v, times w[v] SiLU(z), stored
             {
                 const int64_t t0 = start + (int64_t)c * kC;
                 const int rows = rows_of(c) - 32 * hf; // valid rows of this half (may be <= 0)
@@ -599,11 +569,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                             if (i < rows)
                                 st_cg(yp + i * HD, o[i]);
                     }
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        o[i] = 0.f;
-                    tmem_st32(tl + cO + 32 * hf, o); // MMA 2 accumulates onto O
-                    tmem_wait_st();
                 }
                 tc_fence_before();
                 if (group_sync_or(kBarSG, kSG, !good || *abort_flag)) {
@@ -678,7 +643,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         auto tri_r = [&](int jj) { return jj < 4 ? trow + 16 * jj : 32 + trow + 16 * (jj - 4); };
         auto tri_c = [&](int jj) { return jj < 4 ? tcol : 32 + tcol; };
         auto tri_o = [&](int jj) { return tbase + (jj < 4 ? 512 * jj : 1024 + 512 * (jj - 2)); };
-        uint32_t phkk = 0, ph1 = 0;
+        uint32_t phkk = 0;
         T av[2], bv[2];
         load_ab(0, av, bv);
         for (int c = 0; c < nchunks; ++c) {
@@ -849,9 +814,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 *reinterpret_cast<float4 *>(Yr0) = make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
                 *reinterpret_cast<float4 *>(Yr1) = make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
             }
-            // ---- T diag(beta), -T diag(beta gamma) -> the tf32 B operands of MMA 1,
-            //      once MMA 1 of the previous chunk has read them
-            good = c == 0 || waitp(bar_m1, ph1);
+            // ---- T diag(beta), -T diag(beta gamma) -> the tf32 B operands of MMA 1 and
+            //      2b in the tiles of this chunk's parity, once MMA 2b (and with it
+            //      MMA 1) of chunk c - 2 has read them
+            good = c < 2 || waitq(bar_m2b(c), ((c - 2) >> 1) & 1);
             group_sync(kBarT, kTeam);
             if (good) {
                 float4 t4[6];
@@ -865,8 +831,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     const float4 g4 = make_float4(__expf(G4.x), __expf(G4.y), __expf(G4.z), __expf(G4.w));
                     const float4 tb = make_float4(t4[jj].x * b4.x, t4[jj].y * b4.y, t4[jj].z * b4.z,
                                                   t4[jj].w * b4.w);
-                    *reinterpret_cast<float4 *>(sm.Tb + tri_o(jj)) = tf32_rna(tb);
-                    *reinterpret_cast<float4 *>(sm.Tg + tri_o(jj)) =
+                    *reinterpret_cast<float4 *>(sm.Tb[c & 1] + tri_o(jj)) = tf32_rna(tb);
+                    *reinterpret_cast<float4 *>(sm.Tg[c & 1] + tri_o(jj)) =
                         tf32_rna(make_float4(-tb.x * g4.x, -tb.y * g4.y, -tb.z * g4.z, -tb.w * g4.w));
                 }
             }
@@ -876,7 +842,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 break;
             }
             if (tt == 0) {
-                mbar_arrive((c & 1) ? bar_pT1 : bar_pT0); // T operands and gates of chunk c
+                mbar_arrive(bar_pT(c)); // T operands and gates of chunk c
                 mbar_arrive(bar_wfree); // Wk may take the next chunk's K K^T rows
             }
         }
@@ -885,11 +851,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     } else if (warp < (kSG + kTeam + kTeamP) / 32) {
         // ==================================================== P team
         const int pt = tid - kSG - kTeam;
-        uint32_t phT0 = 0, phT1 = 0, phq = 0, phqk = 0;
+        uint32_t phq = 0, phqk = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int sl = c & 3;
-            // ---- diag(gamma) Q in place (rows 64..127 of WQ), tf32
-            bool good = (c & 1) ? waitp(bar_pT1, phT1) : waitp(bar_pT0, phT0); // gates
+            // ---- diag(gamma) Q in place (rows 64..127 of KQ)
+            bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
             good = waitp(bar_q, phq) && good;
             if (good) {
 #pragma unroll 1
@@ -901,12 +867,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     for (int jj = 0; jj < 8; ++jj) {
                         const int f = pt + kTeamP * (8 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
                         off[jj] = cb * (2 * kC * 32) + (kC + r) * 32 + (((f & 7) ^ (r & 7)) << 2);
-                        x[jj] = *reinterpret_cast<const float4 *>(sm.WQ + off[jj]);
+                        x[jj] = *reinterpret_cast<const float4 *>(sm.KQ + off[jj]);
                         gr[jj] = __expf(sm.G[sl][r]); // far inside the tf32 rounding below
                     }
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj)
-                        *reinterpret_cast<float4 *>(sm.WQ + off[jj]) =
+                        *reinterpret_cast<float4 *>(sm.KQ + off[jj]) =
                             tf32_rna(make_float4(x[jj].x * gr[jj], x[jj].y * gr[jj], x[jj].z * gr[jj],
                                                  x[jj].w * gr[jj]));
                 }
@@ -968,94 +934,117 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         // ==================================================== MMA issue
         if (lane == 0 && nchunks > 0) {
             const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.V), kC * 128, 512);
-            const uint64_t dK0 = sdesc_sw128_b32(smem_u32(sm.K[0]), kC * 128, 512);
-            const uint64_t dK1 = sdesc_sw128_b32(smem_u32(sm.K[1]), kC * 128, 512);
-            const uint64_t dTb0 = sdesc_sw128(smem_u32(sm.Tb), 16, 1024);
-            const uint64_t dTb1 = sdesc_sw128(smem_u32(sm.Tb + 2048), 16, 1024);
-            const uint64_t dTg0 = sdesc_sw128(smem_u32(sm.Tg), 16, 1024);
-            const uint64_t dTg1 = sdesc_sw128(smem_u32(sm.Tg + 2048), 16, 1024);
+            const uint64_t dK = sdesc_sw128_b32(smem_u32(sm.K), kC * 128, 512);
+            const uint64_t dKQ = sdesc_sw128(smem_u32(sm.KQ), 16, 1024);
             const uint64_t dP0 = sdesc_sw128(smem_u32(sm.P), 16, 1024);
             const uint64_t dP1 = sdesc_sw128(smem_u32(sm.P + 2048), 16, 1024);
-            const uint64_t dWQ = sdesc_sw128(smem_u32(sm.WQ), 16, 1024);
-            constexpr uint32_t id64 = idesc_tf32(128, 64, true, false);  // A MN-major (MMA 1)
+            auto tb0 = [&](int c) { return sdesc_sw128(smem_u32(sm.Tb[c & 1]), 16, 1024); };
+            auto tb1 = [&](int c) { return sdesc_sw128(smem_u32(sm.Tb[c & 1] + 2048), 16, 1024); };
+            auto tg0 = [&](int c) { return sdesc_sw128(smem_u32(sm.Tg[c & 1]), 16, 1024); };
+            auto tg1 = [&](int c) { return sdesc_sw128(smem_u32(sm.Tg[c & 1] + 2048), 16, 1024); };
+            constexpr uint32_t id64 = idesc_tf32(128, 64, true, false);    // MMA 1 (A MN-major)
             constexpr uint32_t id32 = idesc_tf32(128, 32, true, false);
             constexpr uint32_t id128 = idesc_tf32(128, 128, false, false); // MMA 2
-            constexpr uint32_t idO64 = idesc_tf32(128, 64, false, false);  // MMA 3, O
-            constexpr uint32_t idO32 = idesc_tf32(128, 32, false, false);
-            constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3, S (B MN-major)
-            uint32_t phT0 = 0, phT1 = 0, phv = 0, phk0 = 0, phk1 = 0, phw = 0, phQ = 0, phu = 0;
-            uint32_t phP = 0;
-            uint32_t ph2 = 0, phof0 = 0, phof1 = 0;
-            // MMA 1 of chunk c: U~^T into U_(c%2), -W^T into W.  K steps 0..3 run over
-            // column block 0 of the T tiles (N = 64), 4..7 over block 1 (rows 32..63)
+            constexpr uint32_t idT64 = idesc_tf32(128, 64, false, false);  // MMA 2b, MMA 3 O
+            constexpr uint32_t idT32 = idesc_tf32(128, 32, false, false);
+            constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3 S (B MN-major)
+            uint32_t phv = 0, phkm = 0, phk = 0, phQ = 0, phu = 0, phP = 0, ph2 = 0;
+            // MMA 1 of chunk c: U~^T into U_(c%2).  K steps 0..3 run over column
+            // block 0 of the T tile (N = 64), 4..7 over block 1 (rows 32..63)
             auto mma1 = [&](int c) {
-                const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0), dW = tmem + kColW;
-                const uint64_t dK = (c & 1) ? dK1 : dK0;
+                const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0);
+                const uint64_t b0 = tb0(c), b1 = tb1(c);
 #pragma unroll 1
-                for (int s = 0; s < 4; ++s) {
-                    mma_tf32_ss(dU, dV + s * 64, dTb0 + 2 * s, id64, s > 0);
-                    mma_tf32_ss(dW, dK + s * 64, dTg0 + 2 * s, id64, s > 0);
-                }
+                for (int s = 0; s < 4; ++s)
+                    mma_tf32_ss(dU, dV + s * 64, b0 + 2 * s, id64, s > 0);
 #pragma unroll 1
-                for (int s = 4; s < 8; ++s) {
-                    mma_tf32_ss(dU + 32, dV + s * 64, dTb1 + 2 * (s - 4), id32, 1);
-                    mma_tf32_ss(dW + 32, dK + s * 64, dTg1 + 2 * (s - 4), id32, 1);
-                }
+                for (int s = 4; s < 8; ++s)
+                    mma_tf32_ss(dU + 32, dV + s * 64, b1 + 2 * (s - 4), id32, 1);
                 mma_commit(bar_m1);
             };
-            bool good = waitp(bar_pT0, phT0);
-            good = good && waitp(bar_v, phv);
-            good = good && waitp(bar_k0, phk0);
+            // the inputs of MMA 1 of chunk c: its T tiles (and gates) and V
+            auto m1_ready = [&](int c, bool block) {
+                if (!block)
+                    return mbar_test_wait(bar_pT(c), (c >> 2) & 1) && mbar_test_wait(bar_v, phv);
+                bool g = waitq(bar_pT(c), (c >> 2) & 1);
+                g = g && waitq(bar_v, phv);
+                return g;
+            };
+            bool good = m1_ready(0, true) && waitp(bar_u, phu); // phase 0 of U: the initial state
+            phv ^= 1u;
             tc_fence_after();
             if (good)
                 mma1(0);
             for (int c = 0; good && c < nchunks; ++c) {
-                const uint32_t dUO = tmem + ((c & 1) ? kColU1 : kColU0);
-                // ---- MMA 2: [U^T | O^T] += S [-W; diag(gamma) Q]^T (A = the state in TMEM)
-                good = waitp(bar_w, phw);
-                good = good && waitp(bar_pQ, phQ);
+                const uint32_t dXO = tmem + ((c & 1) ? kColX1 : kColX0);
+                const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0);
+                // ---- MMA 2: [X^T | O^T] = S [K; diag(gamma) Q]^T (A = the state in TMEM)
+                good = waitp(bar_pQ, phQ);
+                good = good && waitp(bar_kmaj, phkm);
                 if (c >= 2)
-                    good = good && ((c & 1) ? waitp(bar_of1, phof1) : waitp(bar_of0, phof0));
+                    good = good && ((c & 1) ? waitq(bar_of1, ((c >> 1) - 1) & 1)
+                                            : waitq(bar_of0, ((c >> 1) - 1) & 1));
                 if (!good)
                     break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int s = 0; s < kD / 8; ++s) {
                     const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ts(dUO, tmem + kColS + 8 * s, dWQ + ks, id128, 1);
+                    mma_tf32_ts(dXO, tmem + kColS + 8 * s, dKQ + ks, id128, s > 0);
                 }
                 mma_commit(bar_m2);
-                // ---- MMA 1 of the next chunk, once MMA 2 (and with it MMA 3 of the
-                //      previous chunk, the last reader of that U buffer) has finished
-                if (c + 1 < nchunks) {
-                    good = waitp(bar_m2, ph2);
-                    good = good && ((c & 1) ? waitp(bar_pT0, phT0) : waitp(bar_pT1, phT1));
-                    good = good && waitp(bar_v, phv);
-                    good = good && ((c & 1) ? waitp(bar_k0, phk0) : waitp(bar_k1, phk1));
+                // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
+                good = waitp(bar_m2, ph2);
+                if (!good)
+                    break;
+                tc_fence_after();
+                {
+                    const uint64_t g0 = tg0(c), g1 = tg1(c);
+#pragma unroll 1
+                    for (int s = 0; s < 4; ++s)
+                        mma_tf32_ts(dU, dXO + 8 * s, g0 + 2 * s, idT64, 1);
+#pragma unroll 1
+                    for (int s = 4; s < 8; ++s)
+                        mma_tf32_ts(dU + 32, dXO + 8 * s, g1 + 2 * (s - 4), idT32, 1);
+                }
+                mma_commit(bar_m2b(c));
+                // ---- MMA 1 of the next chunk beside the U pass, if its inputs are in
+                //      (its U buffer was last read by MMA 3 of chunk c - 1)
+                bool m1_issued = false;
+                if (c + 1 < nchunks && m1_ready(c + 1, false)) {
+                    phv ^= 1u;
+                    tc_fence_after();
+                    mma1(c + 1);
+                    m1_issued = true;
+                }
+                // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K
+                good = waitp(bar_u, phu);
+                good = good && waitp(bar_pP, phP);
+                good = good && waitp(bar_k, phk);
+                if (!good)
+                    break;
+                tc_fence_after();
+                {
+                    const uint32_t dO = dXO + 64;
+#pragma unroll 1
+                    for (int s = 0; s < 4; ++s)
+                        mma_tf32_ts(dO, dU + 8 * s, dP0 + 2 * s, idT64, 1);
+#pragma unroll 1
+                    for (int s = 4; s < 8; ++s)
+                        mma_tf32_ts(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1);
+#pragma unroll 1
+                    for (int s = 0; s < kC / 8; ++s)
+                        mma_tf32_ts(tmem + kColS, dXO + 8 * s, dK + s * 64, idS, 1);
+                }
+                mma_commit(bar_m3);
+                if (c + 1 < nchunks && !m1_issued) {
+                    good = m1_ready(c + 1, true);
+                    phv ^= 1u;
                     if (!good)
                         break;
                     tc_fence_after();
                     mma1(c + 1);
                 }
-                // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K
-                good = waitp(bar_u, phu);
-                good = good && waitp(bar_pP, phP);
-                if (!good)
-                    break;
-                tc_fence_after();
-                {
-                    const uint64_t dK = (c & 1) ? dK1 : dK0;
-#pragma unroll 1
-                    for (int s = 0; s < 4; ++s)
-                        mma_tf32_ts(dUO + 64, dUO + 8 * s, dP0 + 2 * s, idO64, 1);
-#pragma unroll 1
-                    for (int s = 4; s < 8; ++s)
-                        mma_tf32_ts(dUO + 96, dUO + 8 * s, dP1 + 2 * (s - 4), idO32, 1);
-#pragma unroll 1
-                    for (int s = 0; s < kC / 8; ++s)
-                        mma_tf32_ts(tmem + kColS, tmem + kColUk + 8 * s, dK + s * 64, idS, 1);
-                }
-                mma_commit(bar_m3);
             }
             ok = good;
             // let every MMA issued so far finish before the CTA releases TMEM
@@ -1070,8 +1059,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     } else {
         // ==================================================== TMA issue
         if (lane == 0 && nchunks > 0) {
-            uint32_t cnt[7] = {0, 0, 0, 0, 0, 0, 0}; // loads armed on v, q, k0, k1, kk, qk, z
-            const uint32_t lbar[7] = {bar_v, bar_q, bar_k0, bar_k1, bar_kk, bar_qk, bar_z};
+            uint32_t cnt[7] = {0, 0, 0, 0, 0, 0, 0}; // loads armed on v, q, k, kmaj, kk, qk, z
+            const uint32_t lbar[7] = {bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z};
             // nb 32-column boxes of 64 rows at x0 + 32 b, row t0, block b landing at dst + b * bstride
             auto tile = [&](int which, float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb,
                             int bstride) {
@@ -1098,17 +1087,17 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             };
             constexpr int kBlkV = kC * 32, kBlkQ = 2 * kC * 32;
             tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
-            tile(2, sm.K[0], &maps.k, xq, t_of(0), 4, kBlkV);
+            tile(3, sm.KQ, &maps.kmaj, xq, t_of(0), 4, kBlkQ);        // rows 0..63 of KQ
             gram(4, sm.Wk, xkk, t_of(0));
-            tile(1, sm.WQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ);
+            tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ); // rows 64..127
+            tile(2, sm.K, &maps.k, xq, t_of(0), 4, kBlkV);
             gram(5, sm.P, xkk + kC, t_of(0));
             ztile(0);
             if (nchunks > 1) {
-                tile(3, sm.K[1], &maps.k, xq, t_of(1), 4, kBlkV);
                 tma_prefetch_2d(&maps.kq, xkk, (int)t_of(1));
                 tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(1) + 32));
             }
-            // four event streams, each served in chunk order as it completes
+            // five event streams, each served in chunk order as it completes
             int iw = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile ? 0 : nchunks;
             long long t_last = clock64();
             while (iw < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
@@ -1136,17 +1125,19 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     ++i1;
                     prog = true;
                 }
-                if (i2 < nchunks && mbar_test_wait(bar_m2, i2 & 1)) { // Q is free
-                    if (i2 + 1 < nchunks)
-                        tile(1, sm.WQ + kC * 32, &maps.q, xq, t_of(i2 + 1), 4, kBlkQ);
+                if (i2 < nchunks && mbar_test_wait(bar_m2, i2 & 1)) { // K (K-major) and Q are free
+                    if (i2 + 1 < nchunks) {
+                        tile(3, sm.KQ, &maps.kmaj, xq, t_of(i2 + 1), 4, kBlkQ);
+                        tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(i2 + 1), 4, kBlkQ);
+                    }
                     ++i2;
                     prog = true;
                 }
-                if (i3 < nchunks && mbar_test_wait(bar_m3, i3 & 1)) { // P and K[i3 % 2] are free
-                    if (i3 + 1 < nchunks)
+                if (i3 < nchunks && mbar_test_wait(bar_m3, i3 & 1)) { // P and K (MN-major) are free
+                    if (i3 + 1 < nchunks) {
                         gram(5, sm.P, xkk + kC, t_of(i3 + 1));
-                    if (i3 + 2 < nchunks)
-                        tile((i3 & 1) ? 3 : 2, sm.K[i3 & 1], &maps.k, xq, t_of(i3 + 2), 4, kBlkV);
+                        tile(2, sm.K, &maps.k, xq, t_of(i3 + 1), 4, kBlkV);
+                    }
                     ++i3;
                     prog = true;
                 }
@@ -1248,6 +1239,8 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
                       qkw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
             encode_2d(&maps.q, p.ws_qk, (uint64_t)p.Hk * kD, N, qkw * F, 32, kC,
                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.kmaj, (const float *)p.ws_qk + (size_t)p.Hk * kD, (uint64_t)p.Hk * kD, N,
+                      qkw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&maps.kq, p.ws_kq, kqw, N, kqw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&maps.kq32, p.ws_kq, kqw, N, kqw * F, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
             (sizeof(T) != 2 ||
