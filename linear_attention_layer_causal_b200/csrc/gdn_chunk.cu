@@ -43,6 +43,7 @@ namespace {
 
 constexpr int kC = 64;  // chunk length
 constexpr int kD = 128; // head dim (d_k = d_v)
+constexpr long long kWaitLimit = 2000000000LL; // bounded waits: ~1 s of SM cycles
 
 // -------------------------------------------------------------- K K^T, Q K^T
 
@@ -83,32 +84,38 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 // One CTA per (chunk, q/k head j): with the chunk's rows t = t0 + r, r < nr,
 //   kq[t][j][0][s] = k_t . k_{t0+s} for s < r, else 0
 //   kq[t][j][1][s] = q_t . k_{t0+s} for s <= r, else 0
-// from the normalised float32 q|k rows of the workspace, exact in FP32.  The
-// chunk's q and k sit transposed in shared memory; thread i < 136 owns the
-// lower-triangle 4 x 4 tile (tr, ts), ts <= tr, i = tr (tr + 1) / 2 + ts, of
-// both products, so that every warp but the last is full.
-constexpr int kKqThreads = 160;
-constexpr int kTp = kC + 4; // row stride of the transposed tiles (16-byte aligned, banks staggered)
+// from the normalised float32 q|k rows of the workspace, on the tensor core:
+// D = [K; Q] K^T (M = 128: the chunk's 64 k rows then its 64 q rows, N = 64).
+// Every operand is split into tf32 hi + lo parts and D = hi hi^T + hi lo^T +
+// lo hi^T (the lo lo^T term is below 2^-21 relative), which is FP32-accurate:
+// the near-cancelling outputs of the layer are sensitive to these products,
+// and one tf32 pass is not enough.  The 128 columns (d) go in two halves of
+// 64, each staged as hi and lo tiles (K-major, 128-byte swizzle) in 64 KB of
+// shared memory.
+constexpr int kKqThreads = 128;
 
-__device__ __forceinline__ void tri_tile(int i, int &tr, int &ts) {
-    int r = (int)((sqrtf(8.0f * (float)i + 1.0f) - 1.0f) * 0.5f);
-    while ((r + 1) * (r + 2) / 2 <= i)
-        ++r;
-    while (r * (r + 1) / 2 > i)
-        --r;
-    tr = r;
-    ts = i - r * (r + 1) / 2;
-}
+struct __align__(1024) KqSmem {
+    float hi[128 * 64]; // [K; Q] hi parts, two 32-column blocks of 128 rows
+    float lo[128 * 64];
+    unsigned long long bar;
+    uint32_t tmem;
+};
 
 __global__ void __launch_bounds__(kKqThreads)
 kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int batch, int64_t N,
-               int Hk, const int32_t *__restrict__ offs, float *__restrict__ kq) {
-    extern __shared__ __align__(16) float kq_smem[];
-    float *Kt = kq_smem;        // Kt[d][r] = k_{t0+r}[d]
-    float *Qt = Kt + kD * kTp;  // Qt[d][r] = q_{t0+r}[d]
-    const int ci = blockIdx.x, j = blockIdx.y, tid = threadIdx.x;
+               int Hk, const int32_t *__restrict__ offs, float *__restrict__ kq,
+               unsigned int *__restrict__ err) {
+    using namespace sm100;
+    extern __shared__ __align__(1024) unsigned char kq_smem_raw[];
+    const int ci = blockIdx.x, j = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (ci >= __ldg(offs + batch))
         return;
+    if ((smem_u32(kq_smem_raw) & 1023u) != 0) { // swizzled tiles need 1024-byte alignment
+        if (tid == 0 && err != nullptr)
+            atomicOr(err, 2u);
+        return;
+    }
+    KqSmem &sm = *reinterpret_cast<KqSmem *>(kq_smem_raw);
     int lo = 0, hi = batch - 1; // the sequence n with offs[n] <= ci < offs[n+1]
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -122,78 +129,93 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
     const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
     const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
     const int64_t QKW = 2 * (int64_t)Hk * kD;
-    // four rounds of loads in flight before their stores (consecutive threads:
-    // consecutive rows, so the transposed stores do not conflict)
-    for (int e0 = tid; e0 < kC * (kD / 4); e0 += 4 * kKqThreads) {
-        float4 q4[4], k4[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = e0 + u * kKqThreads, r = e % kC, d = (e / kC) * 4;
-            q4[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-            k4[u] = q4[u];
-            if (e < kC * (kD / 4) && r < nr) {
-                const float *row = qk + (t0 + r) * QKW + j * kD + d;
-                q4[u] = __ldg(reinterpret_cast<const float4 *>(row));
-                k4[u] = __ldg(reinterpret_cast<const float4 *>(row + Hk * kD));
-            }
+    const uint32_t bar = smem_u32(&sm.bar);
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        tmem_alloc(smem_u32(&sm.tmem), 64);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem;
+    bool ok = true;
+    uint32_t ph = 0;
+    constexpr uint32_t id = idesc_tf32(128, 64, false, false);
+    for (int half = 0; half < 2; ++half) {
+        if (half == 1) { // MMAs of half 0 read the tiles: wait before overwriting them
+            ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
+            ph ^= 1u;
         }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int e = e0 + u * kKqThreads, r = e % kC, d = (e / kC) * 4;
-            if (e < kC * (kD / 4)) {
-                Qt[(d + 0) * kTp + r] = q4[u].x; Qt[(d + 1) * kTp + r] = q4[u].y;
-                Qt[(d + 2) * kTp + r] = q4[u].z; Qt[(d + 3) * kTp + r] = q4[u].w;
-                Kt[(d + 0) * kTp + r] = k4[u].x; Kt[(d + 1) * kTp + r] = k4[u].y;
-                Kt[(d + 2) * kTp + r] = k4[u].z; Kt[(d + 3) * kTp + r] = k4[u].w;
+        // row r < 64: k of token t0 + r; r >= 64: q of token t0 + r - 64 (zeros past nr)
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+            const int f = tid + kKqThreads * i, r = f >> 4, c = 4 * (f & 15); // c: column in the half
+            const int rr = r & 63;
+            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (rr < nr)
+                x = __ldg(reinterpret_cast<const float4 *>(
+                    qk + (t0 + rr) * QKW + (r < 64 ? Hk * kD : 0) + j * kD + 64 * half + c));
+            const float4 h4 = tf32_rna(x);
+            const float4 l4 = tf32_rna(make_float4(x.x - h4.x, x.y - h4.y, x.z - h4.z, x.w - h4.w));
+            const int o = (c >> 5) * (128 * 32) + r * 32 + ((((c & 31) >> 2) ^ (r & 7)) << 2);
+            *reinterpret_cast<float4 *>(sm.hi + o) = h4;
+            *reinterpret_cast<float4 *>(sm.lo + o) = l4;
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+        if (tid == 0 && ok) {
+            // A = [K; Q] (128 rows), B = its first 64 rows (K), K-major, 8 columns a step
+            const uint64_t aH = sdesc_sw128(smem_u32(sm.hi), 16, 1024);
+            const uint64_t aL = sdesc_sw128(smem_u32(sm.lo), 16, 1024);
+#pragma unroll 1
+            for (int s = 0; s < 8; ++s) {
+                const uint64_t ks = (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4);
+                mma_tf32_ss(tmem, aH + ks, aH + ks, id, (half > 0 || s > 0) ? 1u : 0u);
+                mma_tf32_ss(tmem, aH + ks, aL + ks, id, 1);
+                mma_tf32_ss(tmem, aL + ks, aH + ks, id, 1);
             }
+            mma_commit(bar);
         }
     }
-    __syncthreads();
-    if (tid < 136) {
-        int tr, ts;
-        tri_tile(tid, tr, ts);
-        float kk[4][4] = {}, qq[4][4] = {};
-#pragma unroll 4
-        for (int d = 0; d < kD; ++d) {
-            const float4 kr = *reinterpret_cast<const float4 *>(Kt + d * kTp + 4 * tr);
-            const float4 qr = *reinterpret_cast<const float4 *>(Qt + d * kTp + 4 * tr);
-            const float4 ks = *reinterpret_cast<const float4 *>(Kt + d * kTp + 4 * ts);
-            const float a[4] = {kr.x, kr.y, kr.z, kr.w}, b[4] = {qr.x, qr.y, qr.z, qr.w};
-            const float c[4] = {ks.x, ks.y, ks.z, ks.w};
+    ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
+    tc_fence_after();
+    // TMEM lane r = row r of D; columns s.  Warp w reads lanes 32 w .. + 31.
+    {
+        const int r = 32 * warp + lane, rr = r & 63;
+        const bool isq = r >= 64;
+        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
+        float v[2][32];
+        tmem_ld32(tl, v[0]);
+        tmem_ld32(tl + 32, v[1]);
+        tmem_wait_ld();
+        if (ok && rr < nr) {
+            float *o = kq + ((t0 + rr) * Hk + j) * (2 * kC) + (isq ? kC : 0);
 #pragma unroll
-            for (int x = 0; x < 4; ++x)
+            for (int b = 0; b < 2; ++b)
 #pragma unroll
-                for (int y = 0; y < 4; ++y) {
-                    kk[x][y] = fmaf(a[x], c[y], kk[x][y]);
-                    qq[x][y] = fmaf(b[x], c[y], qq[x][y]);
+                for (int i = 0; i < 32; i += 4) {
+                    const int s = 32 * b + i;
+                    float4 w4;
+                    w4.x = (isq ? s <= rr : s < rr) ? v[b][i] : 0.f;
+                    w4.y = (isq ? s + 1 <= rr : s + 1 < rr) ? v[b][i + 1] : 0.f;
+                    w4.z = (isq ? s + 2 <= rr : s + 2 < rr) ? v[b][i + 2] : 0.f;
+                    w4.w = (isq ? s + 3 <= rr : s + 3 < rr) ? v[b][i + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(o + s) = w4;
                 }
         }
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            const int r = 4 * tr + x;
-            if (r >= nr)
-                break;
-            float o1[4], o2[4];
-#pragma unroll
-            for (int y = 0; y < 4; ++y) {
-                const int s = 4 * ts + y;
-                o1[y] = s < r ? kk[x][y] : 0.f;
-                o2[y] = s <= r ? qq[x][y] : 0.f;
-            }
-            float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
-            *reinterpret_cast<float4 *>(o + 4 * ts) = make_float4(o1[0], o1[1], o1[2], o1[3]);
-            *reinterpret_cast<float4 *>(o + kC + 4 * ts) = make_float4(o2[0], o2[1], o2[2], o2[3]);
-        }
     }
-    // the tiles right of each row's diagonal tile are zero
-    for (int e = tid; e < kC * 16; e += kKqThreads) {
-        const int r = e >> 4, tx = e & 15;
-        if (tx > (r >> 2) && r < nr) {
-            float *o = kq + ((t0 + r) * Hk + j) * (2 * kC);
-            *reinterpret_cast<float4 *>(o + 4 * tx) = make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(o + kC + 4 * tx) = make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-    }
+    if (__syncthreads_or(!ok) && tid == 0 && err != nullptr)
+        atomicOr(err, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        tmem_dealloc(tmem, 64);
 }
 
 // ------------------------------------------------------------ chunk kernel
@@ -269,7 +291,6 @@ struct __align__(1024) ChunkSmem {
     int abort;
 };
 
-constexpr long long kWaitLimit = 2000000000LL; // ~1 s of SM cycles
 
 // The tensor maps of one call: 64-row boxes (32-row for the lower half of
 // the Gram tiles' second column block) of the workspace.
@@ -390,10 +411,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     // seen on it (low 16 bits); the status word then gets bit 0.
     const uint32_t bar_base = smem_u32(&sm.bar_v);
     uint32_t waits_seen = 0;
+    // every wait polls: sleeping on the barrier (a suspend hint) measured slower
     auto waitp = [&](uint32_t bar, uint32_t &ph) {
         const long long t0 = clock64();
         bool done;
-        while (!(done = mbar_try_wait(bar, ph))) {
+        while (!(done = mbar_try_wait_spin(bar, ph))) {
             if (*abort_flag)
                 break;
             if (clock64() - t0 > kWaitLimit) {
@@ -1268,14 +1290,14 @@ cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s) {
 cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s) {
     if (p.N == 0 || p.batch == 0)
         return cudaSuccess;
-    const size_t smem = sizeof(float) * 2 * kD * kTp;
+    const size_t smem = sizeof(KqSmem);
     cudaError_t e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
     // upper bound on the chunk count: every sequence adds at most one partial chunk
     dim3 grid((unsigned)((p.N + kC - 1) / kC + p.batch), p.Hk);
     kq_prep_kernel<<<grid, kKqThreads, smem, s>>>((const float *)p.ws_qk, p.cu, p.batch, p.N, p.Hk,
-                                                  p.ws_offs, (float *)p.ws_kq);
+                                                  p.ws_offs, (float *)p.ws_kq, p.ws_err);
     return cudaGetLastError();
 }
 
