@@ -192,11 +192,12 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     const ProfileHook hook = take_profile_hook();
     if (batch == 0)
         return GDN_OK;
-    // conv / SiLU / L2 front end, then for the chunked path the chunk offsets
-    // and the intra-chunk Gram rows
-    cudaError_t e = launch_conv_prep(p, s);
-    if (e == cudaSuccess && p.chunked)
-        e = launch_chunk_offsets(p, s);
+    // conv / SiLU / L2 front end; the chunked path first computes the chunk
+    // offsets (and clears the status words), and after the conv the
+    // intra-chunk Gram rows
+    cudaError_t e = p.chunked ? launch_chunk_offsets(p, s) : cudaSuccess;
+    if (e == cudaSuccess)
+        e = launch_conv_prep(p, s);
     if (e == cudaSuccess && p.chunked)
         e = launch_kq_prep(p, s);
     if (e == cudaSuccess)

@@ -27,7 +27,8 @@
 // kind::tf32; every operand computed here is rounded to nearest first (the
 // tensor core's own conversion truncates, a bias that would accumulate
 // through the state).  The Gram matrices K K^T and Q K^T come exact in FP32
-// from kq_prep_kernel: the near-cancelling outputs are sensitive to them.
+// from the front kernel (gdn_front.cu): the near-cancelling outputs are
+// sensitive to them.
 //
 // The gated RMSNorm y = o / rms(o) * w * SiLU(z) ("Qwen3.8-2.4T-A95B vs
 // Inkling", output-gate row) is fused into the output store.
@@ -36,6 +37,7 @@
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
+#include "gdn_tmap.h"
 
 namespace gdn {
 
@@ -45,15 +47,22 @@ constexpr int kC = 64;  // chunk length
 constexpr int kD = 128; // head dim (d_k = d_v)
 constexpr long long kWaitLimit = 2000000000LL; // bounded waits: ~1 s of SM cycles
 
-// -------------------------------------------------------------- K K^T, Q K^T
+// ------------------------------------------------------------ chunk offsets
 
 // Chunk offsets: offs[n] = number of 64-token chunks in sequences 0 .. n-1
 // (offs[batch] = total).  One CTA of 1024 threads; each thread scans a run of
 // consecutive sequences, then the run totals are scanned across the block.
+// It is the first kernel of a chunked prefill call, so it also clears the
+// call's status words.
 __global__ void __launch_bounds__(1024)
-chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32_t *__restrict__ offs) {
+chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32_t *__restrict__ offs,
+                     unsigned int *__restrict__ err) {
     __shared__ int32_t part[1024];
     const int tid = threadIdx.x;
+    if (tid == 0 && err != nullptr) {
+        err[0] = 0u; // status word of this call; later kernels only set bits
+        err[1] = 0u; // where the first timed-out wait gave up
+    }
     const int per = (batch + 1023) / 1024;
     const int b0 = tid * per, b1 = b0 + per < batch ? b0 + per : batch;
     int32_t sum = 0;
@@ -79,143 +88,6 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
     }
     if (tid == 1023)
         offs[batch] = part[1023];
-}
-
-// One CTA per (chunk, q/k head j): with the chunk's rows t = t0 + r, r < nr,
-//   kq[t][j][0][s] = k_t . k_{t0+s} for s < r, else 0
-//   kq[t][j][1][s] = q_t . k_{t0+s} for s <= r, else 0
-// from the normalised float32 q|k rows of the workspace, on the tensor core:
-// D = [K; Q] K^T (M = 128: the chunk's 64 k rows then its 64 q rows, N = 64).
-// Every operand is split into tf32 hi + lo parts and D = hi hi^T + hi lo^T +
-// lo hi^T (the lo lo^T term is below 2^-21 relative), which is FP32-accurate:
-// the near-cancelling outputs of the layer are sensitive to these products,
-// and one tf32 pass is not enough.  The 128 columns (d) go in two halves of
-// 64, each staged as hi and lo tiles (K-major, 128-byte swizzle) in 64 KB of
-// shared memory.
-constexpr int kKqThreads = 128;
-
-struct __align__(1024) KqSmem {
-    float hi[128 * 64]; // [K; Q] hi parts, two 32-column blocks of 128 rows
-    float lo[128 * 64];
-    unsigned long long bar;
-    uint32_t tmem;
-};
-
-__global__ void __launch_bounds__(kKqThreads)
-kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int batch, int64_t N,
-               int Hk, const int32_t *__restrict__ offs, float *__restrict__ kq,
-               unsigned int *__restrict__ err) {
-    using namespace sm100;
-    extern __shared__ __align__(1024) unsigned char kq_smem_raw[];
-    const int ci = blockIdx.x, j = blockIdx.y, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if (ci >= __ldg(offs + batch))
-        return;
-    if ((smem_u32(kq_smem_raw) & 1023u) != 0) { // swizzled tiles need 1024-byte alignment
-        if (tid == 0 && err != nullptr)
-            atomicOr(err, 2u);
-        return;
-    }
-    KqSmem &sm = *reinterpret_cast<KqSmem *>(kq_smem_raw);
-    int lo = 0, hi = batch - 1; // the sequence n with offs[n] <= ci < offs[n+1]
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (__ldg(offs + mid) <= ci)
-            lo = mid;
-        else
-            hi = mid - 1;
-    }
-    int64_t s0, e0;
-    seq_bounds(cu, lo, N, s0, e0);
-    const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
-    const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
-    const int64_t QKW = 2 * (int64_t)Hk * kD;
-    const uint32_t bar = smem_u32(&sm.bar);
-    if (tid == 0) {
-        mbar_init(bar, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    if (warp == 0) {
-        tmem_alloc(smem_u32(&sm.tmem), 64);
-        tmem_relinquish();
-    }
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    const uint32_t tmem = sm.tmem;
-    bool ok = true;
-    uint32_t ph = 0;
-    constexpr uint32_t id = idesc_tf32(128, 64, false, false);
-    for (int half = 0; half < 2; ++half) {
-        if (half == 1) { // MMAs of half 0 read the tiles: wait before overwriting them
-            ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
-            ph ^= 1u;
-        }
-        // row r < 64: k of token t0 + r; r >= 64: q of token t0 + r - 64 (zeros past nr)
-#pragma unroll 4
-        for (int i = 0; i < 16; ++i) {
-            const int f = tid + kKqThreads * i, r = f >> 4, c = 4 * (f & 15); // c: column in the half
-            const int rr = r & 63;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (rr < nr)
-                x = __ldg(reinterpret_cast<const float4 *>(
-                    qk + (t0 + rr) * QKW + (r < 64 ? Hk * kD : 0) + j * kD + 64 * half + c));
-            const float4 h4 = tf32_rna(x);
-            const float4 l4 = tf32_rna(make_float4(x.x - h4.x, x.y - h4.y, x.z - h4.z, x.w - h4.w));
-            const int o = (c >> 5) * (128 * 32) + r * 32 + ((((c & 31) >> 2) ^ (r & 7)) << 2);
-            *reinterpret_cast<float4 *>(sm.hi + o) = h4;
-            *reinterpret_cast<float4 *>(sm.lo + o) = l4;
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0 && ok) {
-            // A = [K; Q] (128 rows), B = its first 64 rows (K), K-major, 8 columns a step
-            const uint64_t aH = sdesc_sw128(smem_u32(sm.hi), 16, 1024);
-            const uint64_t aL = sdesc_sw128(smem_u32(sm.lo), 16, 1024);
-#pragma unroll 1
-            for (int s = 0; s < 8; ++s) {
-                const uint64_t ks = (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4);
-                mma_tf32_ss(tmem, aH + ks, aH + ks, id, (half > 0 || s > 0) ? 1u : 0u);
-                mma_tf32_ss(tmem, aH + ks, aL + ks, id, 1);
-                mma_tf32_ss(tmem, aL + ks, aH + ks, id, 1);
-            }
-            mma_commit(bar);
-        }
-    }
-    ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
-    tc_fence_after();
-    // TMEM lane r = row r of D; columns s.  Warp w reads lanes 32 w .. + 31.
-    {
-        const int r = 32 * warp + lane, rr = r & 63;
-        const bool isq = r >= 64;
-        const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-        float v[2][32];
-        tmem_ld32(tl, v[0]);
-        tmem_ld32(tl + 32, v[1]);
-        tmem_wait_ld();
-        if (ok && rr < nr) {
-            float *o = kq + ((t0 + rr) * Hk + j) * (2 * kC) + (isq ? kC : 0);
-#pragma unroll
-            for (int b = 0; b < 2; ++b)
-#pragma unroll
-                for (int i = 0; i < 32; i += 4) {
-                    const int s = 32 * b + i;
-                    float4 w4;
-                    w4.x = (isq ? s <= rr : s < rr) ? v[b][i] : 0.f;
-                    w4.y = (isq ? s + 1 <= rr : s + 1 < rr) ? v[b][i + 1] : 0.f;
-                    w4.z = (isq ? s + 2 <= rr : s + 2 < rr) ? v[b][i + 2] : 0.f;
-                    w4.w = (isq ? s + 3 <= rr : s + 3 < rr) ? v[b][i + 3] : 0.f;
-                    *reinterpret_cast<float4 *>(o + s) = w4;
-                }
-        }
-    }
-    if (__syncthreads_or(!ok) && tid == 0 && err != nullptr)
-        atomicOr(err, 1u);
-    tc_fence_before();
-    __syncthreads();
-    if (warp == 0)
-        tmem_dealloc(tmem, 64);
 }
 
 // ------------------------------------------------------------ chunk kernel
@@ -1207,42 +1079,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         tmem_dealloc(tmem, kTmemCols);
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-// The driver's tensor-map encoder, looked up once through the runtime.
-EncodeTiledFn encoder() {
-    static EncodeTiledFn fn = []() -> EncodeTiledFn {
-        void *f = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
-                cudaSuccess ||
-            q != cudaDriverEntryPointSuccess)
-            return nullptr;
-        return reinterpret_cast<EncodeTiledFn>(f);
-    }();
-    return fn;
-}
-
-// Row-major 2-D map over `rows` rows of `cols` elements (row pitch
-// `pitch` bytes), boxes of `box_cols` x `box_rows`.
-bool encode_2d(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint64_t pitch,
-               uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle sw,
-               CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_FLOAT32) {
-    EncodeTiledFn enc = encoder();
-    if (enc == nullptr)
-        return false;
-    const cuuint64_t dims[2] = {cols, rows};
-    const cuuint64_t strides[1] = {pitch};
-    const cuuint32_t box[2] = {box_cols, box_rows};
-    const cuuint32_t es[2] = {1, 1};
-    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box,
-               es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStream_t s) {
     const size_t smem = sizeof(ChunkSmem);
     cudaError_t e = cudaFuncSetAttribute(chunk_prefill_kernel<T>,
@@ -1281,23 +1117,9 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * 2 * kC * sizeof(float); }
 
 cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s) {
-    if (p.N == 0 || p.batch == 0)
+    if (p.batch == 0)
         return cudaSuccess;
-    chunk_offsets_kernel<<<1, 1024, 0, s>>>(p.cu, p.batch, p.N, p.ws_offs);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s) {
-    if (p.N == 0 || p.batch == 0)
-        return cudaSuccess;
-    const size_t smem = sizeof(KqSmem);
-    cudaError_t e = cudaFuncSetAttribute(kq_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess)
-        return e;
-    // upper bound on the chunk count: every sequence adds at most one partial chunk
-    dim3 grid((unsigned)((p.N + kC - 1) / kC + p.batch), p.Hk);
-    kq_prep_kernel<<<grid, kKqThreads, smem, s>>>((const float *)p.ws_qk, p.cu, p.batch, p.N, p.Hk,
-                                                  p.ws_offs, (float *)p.ws_kq, p.ws_err);
+    chunk_offsets_kernel<<<1, 1024, 0, s>>>(p.cu, p.batch, p.N, p.ws_offs, p.ws_err);
     return cudaGetLastError();
 }
 
