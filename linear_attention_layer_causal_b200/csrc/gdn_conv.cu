@@ -10,14 +10,15 @@ namespace {
 
 constexpr int kConvThreads = 256;
 
-// One CTA: kConvTokens consecutive packed tokens x kConvThreads 16-byte
-// channel vectors.  The lanes covering one head are consecutive and the head
+// One CTA: kConvTokens consecutive packed tokens x kConvThreads channel
+// vectors (8 bytes = 4 channels for bf16 at head dim 128, whose lighter
+// threads fit three CTAs on an SM; 16 bytes otherwise).  The lanes covering one head are consecutive and the head
 // width d / V divides 32, so the L2 reduction is a shuffle within an aligned
 // lane group.
-template <typename T, int D>
+template <typename T, int D, typename VecT = Vec16<T>>
 __global__ void __launch_bounds__(kConvThreads)
 conv_prep_kernel(ConvIO<T> io, unsigned int *__restrict__ err) {
-    constexpr int V = Vec16<T>::N;
+    constexpr int V = VecT::N;
     const int C = (2 * io.Hk + io.Hv) * D;
     if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         err[0] = 0u; // status word of this call; later kernels only set bits
@@ -30,9 +31,9 @@ conv_prep_kernel(ConvIO<T> io, unsigned int *__restrict__ err) {
     const int n = seq_of_token(io.cu, io.batch, t0 < io.N ? t0 : io.N - 1);
     // a block whose channels all lie in v skips the norm code (uniform branch)
     if ((int)blockIdx.y * kConvThreads * V >= 2 * io.Hk * D)
-        conv_thread<T, D, true>(io, active ? c0 : 2 * io.Hk * D, active, t0, tend, n);
+        conv_thread<T, D, true, VecT>(io, active ? c0 : 2 * io.Hk * D, active, t0, tend, n);
     else
-        conv_thread<T, D>(io, active ? c0 : 0, active, t0, tend, n);
+        conv_thread<T, D, false, VecT>(io, active ? c0 : 0, active, t0, tend, n);
 }
 
 // final_conv[n] = the last 3 pre-conv rows of [init_conv[n]; sequence n].
@@ -83,13 +84,13 @@ ConvIO<T> conv_io(const PrefillArgs &p) {
     return io;
 }
 
-template <typename T, int D>
+template <typename T, int D, typename VecT = Vec16<T>>
 cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
-    constexpr int V = Vec16<T>::N;
+    constexpr int V = VecT::N;
     const int C = (2 * p.Hk + p.Hv) * D;
     dim3 grid((unsigned)((p.N + kConvTokens - 1) / kConvTokens),
               (C / V + kConvThreads - 1) / kConvThreads);
-    conv_prep_kernel<T, D><<<grid, kConvThreads, 0, s>>>(conv_io<T>(p), p.ws_err);
+    conv_prep_kernel<T, D, VecT><<<grid, kConvThreads, 0, s>>>(conv_io<T>(p), p.ws_err);
     return cudaGetLastError();
 }
 
@@ -108,7 +109,7 @@ cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s) {
     if (p.N == 0)
         return cudaSuccess;
     if (p.bf16)
-        return p.D == 128 ? launch_conv_prep_t<__nv_bfloat16, 128>(p, s)
+        return p.D == 128 ? launch_conv_prep_t<__nv_bfloat16, 128, Vec8bf>(p, s)
                           : launch_conv_prep_t<__nv_bfloat16, 32>(p, s);
     return p.D == 128 ? launch_conv_prep_t<float, 128>(p, s) : launch_conv_prep_t<float, 32>(p, s);
 }

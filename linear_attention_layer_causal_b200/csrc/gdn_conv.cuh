@@ -14,6 +14,25 @@ namespace gdn {
 
 constexpr int kConvTokens = 8; // tokens per thread
 
+// Loads of one thread's channel vector: Vec16<T> (16 bytes) or Vec8bf (8 bytes of bf16).
+template <typename VecT, typename T> struct VecIO;
+template <typename T> struct VecIO<Vec16<T>, T> {
+    static __device__ __forceinline__ Vec16<T> load(const T *p) { return ld16_nc(p); }
+    static __device__ __forceinline__ Vec16<T> zero() { return zero16<T>(); }
+};
+template <> struct VecIO<Vec8bf, __nv_bfloat16> {
+    static __device__ __forceinline__ Vec8bf load(const __nv_bfloat16 *p) {
+        Vec8bf v;
+        v.raw = __ldg(reinterpret_cast<const uint2 *>(p));
+        return v;
+    }
+    static __device__ __forceinline__ Vec8bf zero() {
+        Vec8bf v;
+        v.raw = make_uint2(0u, 0u);
+        return v;
+    }
+};
+
 template <typename T> struct ConvIO {
     const T *qkv;          // [N, C] pre-conv q|k|v rows
     const int32_t *cu;     // [batch + 1] sequence offsets
@@ -38,10 +57,10 @@ template <typename T> struct ConvIO {
 // Inactive lanes (active = false, cc any valid channel) join the shuffles only.
 // V_ONLY: the caller guarantees that every lane of the warp holds v channels
 // (no norm, no reduction).
-template <typename T, int D, bool V_ONLY = false>
+template <typename T, int D, bool V_ONLY = false, typename VecT = Vec16<T>>
 __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool active, int64_t t0,
-                                          int64_t tend, int n, const Vec16<T> (&rows)[kConvTokens + 3]) {
-    constexpr int V = Vec16<T>::N;
+                                          int64_t tend, int n, const VecT (&rows)[kConvTokens + 3]) {
+    constexpr int V = VecT::N;
     constexpr int LANES = D / V; // lanes per head
     static_assert(LANES >= 1 && LANES <= 32 && (32 % LANES) == 0, "head must tile a warp");
     const int C = (2 * io.Hk + io.Hv) * D;
@@ -140,13 +159,13 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
 #pragma unroll
         for (int tap = 0; tap < 4; ++tap) {
             const int64_t src = t - 3 + tap;
-            Vec16<T> x;
+            VecT x;
             if (src >= st)
-                x = ld16_nc(io.qkv + src * C + cc); // rows[] would need a dynamic index here
+                x = VecIO<VecT, T>::load(io.qkv + src * C + cc); // rows[] would need a dynamic index here
             else if (io.init_conv != nullptr)
-                x = ld16_nc(io.init_conv + ((int64_t)n * 3 + (3 + (src - st))) * C + cc);
+                x = VecIO<VecT, T>::load(io.init_conv + ((int64_t)n * 3 + (3 + (src - st))) * C + cc);
             else
-                x = zero16<T>();
+                x = VecIO<VecT, T>::zero();
 #pragma unroll
             for (int i = 0; i < V; ++i)
                 acc[i] = fmaf(w[i][tap], x.get(i), acc[i]);
@@ -157,17 +176,18 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
 
 // conv_emit with the rows loaded from global memory first, so that all their
 // loads overlap.
-template <typename T, int D, bool V_ONLY = false>
+template <typename T, int D, bool V_ONLY = false, typename VecT = Vec16<T>>
 __device__ __forceinline__ void conv_thread(const ConvIO<T> &io, int cc, bool active, int64_t t0,
                                             int64_t tend, int n) {
     const int C = (2 * io.Hk + io.Hv) * D;
-    Vec16<T> rows[kConvTokens + 3];
+    VecT rows[kConvTokens + 3];
 #pragma unroll
     for (int k = 0; k < kConvTokens + 3; ++k) {
         const int64_t src = t0 - 3 + k;
-        rows[k] = (src >= 0 && src < io.N) ? ld16_nc(io.qkv + src * C + cc) : zero16<T>();
+        rows[k] = (src >= 0 && src < io.N) ? VecIO<VecT, T>::load(io.qkv + src * C + cc)
+                                          : VecIO<VecT, T>::zero();
     }
-    conv_emit<T, D, V_ONLY>(io, cc, active, t0, tend, n, rows);
+    conv_emit<T, D, V_ONLY, VecT>(io, cc, active, t0, tend, n, rows);
 }
 
 } // namespace gdn
