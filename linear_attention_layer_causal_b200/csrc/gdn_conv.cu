@@ -12,11 +12,11 @@ constexpr int kConvThreads = 256;
 
 // One CTA: kConvTokens consecutive packed tokens x kConvThreads channel
 // vectors (8 bytes = 4 channels for bf16 at head dim 128, whose lighter
-// threads fit three CTAs on an SM; 16 bytes otherwise).  The lanes covering one head are consecutive and the head
+// threads fit four CTAs on an SM; 16 bytes otherwise).  The lanes covering one head are consecutive and the head
 // width d / V divides 32, so the L2 reduction is a shuffle within an aligned
 // lane group.
 template <typename T, int D, typename VecT = Vec16<T>>
-__global__ void __launch_bounds__(kConvThreads)
+__global__ void __launch_bounds__(kConvThreads, sizeof(VecT) == 8 ? 4 : 1) // 8-byte units: 64 registers
 conv_prep_kernel(ConvIO<T> io, unsigned int *__restrict__ err) {
     constexpr int V = VecT::N;
     const int C = (2 * io.Hk + io.Hv) * D;
