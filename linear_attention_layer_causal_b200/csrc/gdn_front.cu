@@ -22,15 +22,16 @@ constexpr long long kWaitLimit = 2000000000LL; // bounded waits: ~1 s of SM cycl
 // Every operand is split into tf32 hi + lo parts and D = hi hi^T + hi lo^T +
 // lo hi^T (the lo lo^T term is below 2^-21 relative), which is FP32-accurate:
 // the near-cancelling outputs of the layer are sensitive to these products,
-// and one tf32 pass is not enough.  The 128 columns (d) go in two halves of
-// 64, each staged as hi and lo tiles (K-major, 128-byte swizzle) in 64 KB of
-// shared memory.
+// and one tf32 pass is not enough.  The 128 columns (d) go in four blocks of
+// 32, staged as hi and lo tiles (K-major, 128-byte swizzle) in two stages of
+// 32 KB: each thread loads the next block while it splits the current one,
+// and the MMAs of a block overlap the loads of the next.
 constexpr int kKqThreads = 128;
 
 struct __align__(1024) KqSmem {
-    float hi[128 * 64]; // [K; Q] hi parts, two 32-column blocks of 128 rows
-    float lo[128 * 64];
-    unsigned long long bar;
+    float hi[2][128 * 32]; // [K; Q] hi parts of a 32-column block, by stage
+    float lo[2][128 * 32];
+    unsigned long long bar[2]; // the MMAs of the stage's block are done
     uint32_t tmem;
 };
 
@@ -62,9 +63,10 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
     const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
     const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
     const int64_t QKW = 2 * (int64_t)Hk * kD;
-    const uint32_t bar = smem_u32(&sm.bar);
+    const uint32_t bar0 = smem_u32(&sm.bar[0]), bar1 = smem_u32(&sm.bar[1]);
     if (tid == 0) {
-        mbar_init(bar, 1);
+        mbar_init(bar0, 1);
+        mbar_init(bar1, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -76,28 +78,41 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     bool ok = true;
-    uint32_t ph = 0;
     constexpr uint32_t id = idesc_tf32(128, 64, false, false);
-    for (int half = 0; half < 2; ++half) {
-        if (half == 1) { // MMAs of half 0 read the tiles: wait before overwriting them
-            ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
-            ph ^= 1u;
-        }
-        // row r < 64: k of token t0 + r; r >= 64: q of token t0 + r - 64 (zeros past
-        // nr); all 16 loads of a thread are issued before the first split
+    // row r < 64: k of token t0 + r; r >= 64: q of token t0 + r - 64 (zeros past
+    // nr); columns 32 q .. + 31 of the head; thread tid takes the float4 f =
+    // tid + 128 i (row f / 8, column 4 (f % 8))
+    auto load_block = [&](int q, float4 (&x)[8]) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int f = tid + kKqThreads * i, r = f >> 4, c = 4 * (f & 15); // c: column in the half
-            const int rr = r & 63;
-            float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int i = 0; i < 8; ++i) {
+            const int f = tid + kKqThreads * i, r = f >> 3, c = 4 * (f & 7), rr = r & 63;
+            x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (rr < nr)
-                x = __ldg(reinterpret_cast<const float4 *>(
-                    qk + (t0 + rr) * QKW + (r < 64 ? Hk * kD : 0) + j * kD + 64 * half + c));
-            const float4 h4 = tf32_rna(x);
-            const float4 l4 = tf32_rna(make_float4(x.x - h4.x, x.y - h4.y, x.z - h4.z, x.w - h4.w));
-            const int o = (c >> 5) * (128 * 32) + r * 32 + ((((c & 31) >> 2) ^ (r & 7)) << 2);
-            *reinterpret_cast<float4 *>(sm.hi + o) = h4;
-            *reinterpret_cast<float4 *>(sm.lo + o) = l4;
+                x[i] = __ldg(reinterpret_cast<const float4 *>(
+                    qk + (t0 + rr) * QKW + (r < 64 ? Hk * kD : 0) + j * kD + 32 * q + c));
+        }
+    };
+    float4 xn[8];
+    load_block(0, xn);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float4 x[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            x[i] = xn[i];
+        if (q < 3)
+            load_block(q + 1, xn);
+        const int st = q & 1;
+        if (q >= 2) // the MMAs of block q - 2 read this stage
+            ok = mbar_wait_bounded(st ? bar1 : bar0, 0u, kWaitLimit) && ok;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int f = tid + kKqThreads * i, r = f >> 3, c = 4 * (f & 7);
+            const float4 h4 = tf32_rna(x[i]);
+            const float4 l4 = tf32_rna(make_float4(x[i].x - h4.x, x[i].y - h4.y, x[i].z - h4.z, x[i].w - h4.w));
+            const int o = r * 32 + (((c >> 2) ^ (r & 7)) << 2);
+            *reinterpret_cast<float4 *>(sm.hi[st] + o) = h4;
+            *reinterpret_cast<float4 *>(sm.lo[st] + o) = l4;
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -105,19 +120,19 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
         tc_fence_after();
         if (tid == 0 && ok) {
             // A = [K; Q] (128 rows), B = its first 64 rows (K), K-major, 8 columns a step
-            const uint64_t aH = sdesc_sw128(smem_u32(sm.hi), 16, 1024);
-            const uint64_t aL = sdesc_sw128(smem_u32(sm.lo), 16, 1024);
+            const uint64_t aH = sdesc_sw128(smem_u32(sm.hi[st]), 16, 1024);
+            const uint64_t aL = sdesc_sw128(smem_u32(sm.lo[st]), 16, 1024);
 #pragma unroll 1
-            for (int s = 0; s < 8; ++s) {
-                const uint64_t ks = (uint64_t)((((s >> 2) * 128 * 128) + (s & 3) * 32) >> 4);
-                mma_tf32_ss(tmem, aH + ks, aH + ks, id, (half > 0 || s > 0) ? 1u : 0u);
+            for (int s = 0; s < 4; ++s) {
+                const uint64_t ks = (uint64_t)(s * 32 >> 4);
+                mma_tf32_ss(tmem, aH + ks, aH + ks, id, (q > 0 || s > 0) ? 1u : 0u);
                 mma_tf32_ss(tmem, aH + ks, aL + ks, id, 1);
                 mma_tf32_ss(tmem, aL + ks, aH + ks, id, 1);
             }
-            mma_commit(bar);
+            mma_commit(st ? bar1 : bar0);
         }
     }
-    ok = mbar_wait_bounded(bar, ph, kWaitLimit) && ok;
+    ok = mbar_wait_bounded(bar1, 1u, kWaitLimit) && ok; // block 3, and with it every MMA
     tc_fence_after();
     // TMEM lane r = row r of D; columns s.  Warp w reads lanes 32 w .. + 31.
     {
