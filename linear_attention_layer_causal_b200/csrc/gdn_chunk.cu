@@ -621,7 +621,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 float *base = Wk + 1024 * pb + 32 * pb * 32;
                 auto at = [&](int i, int jc) { return base + i * 32 + (((jc >> 2) ^ (i & 7)) << 2) + (jc & 3); };
                 float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll
+#pragma unroll 1
                 for (int m = 0; m < 4; ++m) {
                     const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 4 * m));
                     const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 4 * m));
@@ -638,7 +638,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 *reinterpret_cast<float2 *>(at(17 + r0, c0)) = make_float2(y10, y11);
                 group_sync(kBarT, kTeam);
                 float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-#pragma unroll
+#pragma unroll 1
                 for (int m = 0; m < 4; ++m) {
                     const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 16 + 4 * m));
                     const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 16 + 4 * m));
@@ -665,7 +665,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 const float *Br0 = Wk + 2048 + r0 * 32, *Br1 = Br0 + 32;   // block 1 rows
                 const int x0 = r0 & 7, x1 = (r0 + 1) & 7;
                 float y[2][4] = {};
-#pragma unroll 2
+#pragma unroll 1
                 for (int m = 0; m < 8; ++m) {
                     const float4 a0 = *reinterpret_cast<const float4 *>(Ar0 + ((m ^ x0) << 2));
                     const float4 a1 = *reinterpret_cast<const float4 *>(Ar1 + ((m ^ x1) << 2));
@@ -688,7 +688,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 *reinterpret_cast<float4 *>(Yr1) = make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
                 group_sync(kBarT, kTeam);
                 float x[2][4] = {};
-#pragma unroll 2
+#pragma unroll 1
                 for (int m = 0; m < 8; ++m) {
                     const float4 a0 = *reinterpret_cast<const float4 *>(Br0 + ((m ^ x0) << 2));
                     const float4 a1 = *reinterpret_cast<const float4 *>(Br1 + ((m ^ x1) << 2));
@@ -787,17 +787,17 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 const int prow = pt >> 3, pcol = 4 * (pt & 7);
                 const int pbase = prow * 32 + (((pt & 7) ^ (prow & 7)) << 2);
 #pragma unroll 1
-                for (int half = 0; half < 2; ++half) {
-                    float4 x[6];
+                for (int half = 0; half < 4; ++half) {
+                    float4 x[3];
 #pragma unroll
-                    for (int jj = 0; jj < 6; ++jj) {
-                        const int k = 6 * half + jj;
+                    for (int jj = 0; jj < 3; ++jj) {
+                        const int k = 3 * half + jj;
                         x[jj] = *reinterpret_cast<const float4 *>(
                             sm.P + pbase + (k < 8 ? 256 * k : 2048 + 256 * (k - 8)));
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 6; ++jj) {
-                        const int k = 6 * half + jj;
+                    for (int jj = 0; jj < 3; ++jj) {
+                        const int k = 3 * half + jj;
                         const float Gr = sm.G[sl][k < 8 ? prow + 8 * k : 32 + prow + 8 * (k - 8)];
                         const float4 Gc =
                             *reinterpret_cast<const float4 *>(&sm.G[sl][k < 8 ? pcol : 32 + pcol]);
@@ -807,8 +807,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                                                      x[jj].w * __expf(fminf(Gr - Gc.w, 0.f))));
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 6; ++jj) {
-                        const int k = 6 * half + jj;
+                    for (int jj = 0; jj < 3; ++jj) {
+                        const int k = 3 * half + jj;
                         *reinterpret_cast<float4 *>(sm.P + pbase +
                                                     (k < 8 ? 256 * k : 2048 + 256 * (k - 8))) = x[jj];
                     }
