@@ -353,31 +353,34 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
                 tc_fence_after();
                 if (good) {
-                    float u[32], uk[32];
-                    tmem_ld32(tl + cU + 32 * hf, u);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kd[sl][32 * hf + i]);
-                        uk[i] = k4.x; uk[i + 1] = k4.y; uk[i + 2] = k4.z; uk[i + 3] = k4.w;
-                    }
                     const float gC = expf(sm.G[sl][kC - 1]); // padded rows carry g = 0
-                    tmem_wait_ld();
+#pragma unroll 1
+                    for (int q = 0; q < 2; ++q) {
+                        float u[16], uk[16];
+                        tmem_ld16(tl + cU + 32 * hf + 16 * q, u);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        uk[i] = tf32_rna(u[i] * uk[i]);
-                        u[i] = tf32_rna(u[i]);
-                    }
-                    tmem_st32(tl + cU + 32 * hf, u);
-                    tmem_st32(tl + cX + 32 * hf, uk);
-#pragma unroll
-                    for (int cb = 0; cb < 2; ++cb) {
-                        float v[32];
-                        tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kd[sl][32 * hf + 16 * q + i]);
+                            uk[i] = k4.x; uk[i + 1] = k4.y; uk[i + 2] = k4.z; uk[i + 3] = k4.w;
+                        }
                         tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i)
+                        for (int i = 0; i < 16; ++i) {
+                            uk[i] = tf32_rna(u[i] * uk[i]);
+                            u[i] = tf32_rna(u[i]);
+                        }
+                        tmem_st16(tl + cU + 32 * hf + 16 * q, u);
+                        tmem_st16(tl + cX + 32 * hf + 16 * q, uk);
+                    }
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        float v[16];
+                        tmem_ld16(tl + kColS + 64 * hf + 16 * q, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
                             v[i] *= gC;
-                        tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+                        tmem_st16(tl + kColS + 64 * hf + 16 * q, v);
                     }
                     tmem_wait_st();
                 }
