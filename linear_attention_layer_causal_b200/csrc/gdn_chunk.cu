@@ -176,6 +176,24 @@ struct ChunkMaps {
     CUtensorMap z;    // z, [N, Hv*128] bf16, 128 x 64 boxes, no swizzle (bf16 activations)
 };
 
+// The rest of a bounded wait whose first try failed: polls until the phase
+// completes, another role aborts, or about 1 s passes; on a time-out records
+// `diag` (the first one only) in err[1].  Out of line: every wait site shares it.
+__device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t ph, volatile int *abort_flag,
+                                       unsigned int *err, uint32_t diag) {
+    const long long t0 = clock64();
+    while (!sm100::mbar_try_wait_spin(bar, ph)) {
+        if (*abort_flag)
+            return false;
+        if (clock64() - t0 > kWaitLimit) {
+            if (err != nullptr)
+                atomicCAS(err + 1, 0u, diag);
+            return false;
+        }
+    }
+    return true;
+}
+
 // Barrier over the `n` threads of one group (named barrier `id`).
 __device__ __forceinline__ void group_sync(int id, int n) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
@@ -285,19 +303,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     uint32_t waits_seen = 0;
     // every wait polls: sleeping on the barrier (a suspend hint) measured slower
     auto waitp = [&](uint32_t bar, uint32_t &ph) {
-        const long long t0 = clock64();
-        bool done;
-        while (!(done = mbar_try_wait_spin(bar, ph))) {
-            if (*abort_flag)
-                break;
-            if (clock64() - t0 > kWaitLimit) {
-                if (p.ws_err != nullptr)
-                    atomicCAS(p.ws_err + 1, 0u,
-                              0x80000000u | ((uint32_t)warp << 24) | (((bar - bar_base) / 8) << 16) |
-                                  (waits_seen & 0xffffu));
-                break;
-            }
-        }
+        bool done = mbar_try_wait_spin(bar, ph);
+        if (!done)
+            done = wait_slow(bar, ph, abort_flag, p.ws_err,
+                             0x80000000u | ((uint32_t)warp << 24) | (((bar - bar_base) / 8) << 16) |
+                                 (waits_seen & 0xffffu));
         ph ^= 1u;
         ++waits_seen;
         return done;
