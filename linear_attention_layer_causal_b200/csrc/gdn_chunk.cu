@@ -766,19 +766,19 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             good = waitp(bar_q, phq) && good;
             if (good) {
 #pragma unroll 1
-                for (int half = 0; half < 4; ++half) {
-                    float4 x[8];
-                    float gr[8];
-                    int off[8];
+                for (int half = 0; half < 16; ++half) {
+                    float4 x[2];
+                    float gr[2];
+                    int off[2];
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const int f = pt + kTeamP * (8 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int f = pt + kTeamP * (2 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
                         off[jj] = cb * (2 * kC * 32) + (kC + r) * 32 + (((f & 7) ^ (r & 7)) << 2);
                         x[jj] = *reinterpret_cast<const float4 *>(sm.KQ + off[jj]);
                         gr[jj] = __expf(sm.G[sl][r]); // far inside the tf32 rounding below
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
+                    for (int jj = 0; jj < 2; ++jj)
                         *reinterpret_cast<float4 *>(sm.KQ + off[jj]) =
                             tf32_rna(make_float4(x[jj].x * gr[jj], x[jj].y * gr[jj], x[jj].z * gr[jj],
                                                  x[jj].w * gr[jj]));
