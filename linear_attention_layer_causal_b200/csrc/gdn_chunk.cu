@@ -800,17 +800,17 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 const int prow = pt >> 3, pcol = 4 * (pt & 7);
                 const int pbase = prow * 32 + (((pt & 7) ^ (prow & 7)) << 2);
 #pragma unroll 1
-                for (int half = 0; half < 4; ++half) {
-                    float4 x[3];
+                for (int half = 0; half < 12; ++half) {
+                    float4 x[1];
 #pragma unroll
-                    for (int jj = 0; jj < 3; ++jj) {
-                        const int k = 3 * half + jj;
+                    for (int jj = 0; jj < 1; ++jj) {
+                        const int k = half + jj;
                         x[jj] = *reinterpret_cast<const float4 *>(
                             sm.P + pbase + (k < 8 ? 256 * k : 2048 + 256 * (k - 8)));
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 3; ++jj) {
-                        const int k = 3 * half + jj;
+                    for (int jj = 0; jj < 1; ++jj) {
+                        const int k = half + jj;
                         const float Gr = sm.G[sl][k < 8 ? prow + 8 * k : 32 + prow + 8 * (k - 8)];
                         const float4 Gc =
                             *reinterpret_cast<const float4 *>(&sm.G[sl][k < 8 ? pcol : 32 + pcol]);
@@ -820,8 +820,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                                                      x[jj].w * __expf(fminf(Gr - Gc.w, 0.f))));
                     }
 #pragma unroll
-                    for (int jj = 0; jj < 3; ++jj) {
-                        const int k = 3 * half + jj;
+                    for (int jj = 0; jj < 1; ++jj) {
+                        const int k = half + jj;
                         *reinterpret_cast<float4 *>(sm.P + pbase +
                                                     (k < 8 ? 256 * k : 2048 + 256 * (k - 8))) = x[jj];
                     }
