@@ -153,6 +153,7 @@ struct __align__(1024) ChunkSmem {
     // (red[4][64]) and reciprocal norms (rstd[64]).
     __nv_bfloat16 Z[kC * kD];
     float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
+    float gam[4][kC];          // gamma = e^G (fast exponential), by chunk index mod 4
     float beta[kC];            // T team's current chunk
     unsigned long long bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z; // TMA landings
     unsigned long long bar_m1, bar_m2, bar_m2b[2], bar_m3;      // MMA completions
@@ -538,6 +539,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     sm.G[sl][r] = g[q];
                     sm.beta[r] = be[q];
                     sm.kd[sl][r] = expf(Glast - g[q]);
+                    sm.gam[sl][r] = __expf(g[q]); // far inside the tf32 rounding of its users
                 }
             }
         };
@@ -734,8 +736,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
 #pragma unroll
                 for (int jj = 0; jj < 6; ++jj) {
                     const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[tri_c(jj)]);
-                    const float4 G4 = *reinterpret_cast<const float4 *>(&sm.G[sl][tri_c(jj)]);
-                    const float4 g4 = make_float4(__expf(G4.x), __expf(G4.y), __expf(G4.z), __expf(G4.w));
+                    const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][tri_c(jj)]);
                     const float4 tb = make_float4(t4[jj].x * b4.x, t4[jj].y * b4.y, t4[jj].z * b4.z,
                                                   t4[jj].w * b4.w);
                     *reinterpret_cast<float4 *>(sm.Tb[c & 1] + tri_o(jj)) = tf32_rna(tb);
@@ -775,7 +776,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                         const int f = pt + kTeamP * (2 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
                         off[jj] = cb * (2 * kC * 32) + (kC + r) * 32 + (((f & 7) ^ (r & 7)) << 2);
                         x[jj] = *reinterpret_cast<const float4 *>(sm.KQ + off[jj]);
-                        gr[jj] = __expf(sm.G[sl][r]); // far inside the tf32 rounding below
+                        gr[jj] = sm.gam[sl][r];
                     }
 #pragma unroll
                     for (int jj = 0; jj < 2; ++jj)
