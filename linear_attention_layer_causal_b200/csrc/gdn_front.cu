@@ -23,15 +23,15 @@ constexpr long long kWaitLimit = 2000000000LL; // bounded waits: ~1 s of SM cycl
 // lo hi^T (the lo lo^T term is below 2^-21 relative), which is FP32-accurate:
 // the near-cancelling outputs of the layer are sensitive to these products,
 // and one tf32 pass is not enough.  The 128 columns (d) go in four blocks of
-// 32, staged as hi and lo tiles (K-major, 128-byte swizzle) in two stages of
-// 32 KB: each thread loads the next block while it splits the current one,
-// and the MMAs of a block overlap the loads of the next.
+// 32, staged as hi and lo tiles (K-major, 128-byte swizzle) in 32 KB of shared
+// memory: each thread loads the next block into registers while the MMAs of
+// the current one run, and the small stage lets four CTAs share an SM.
 constexpr int kKqThreads = 128;
 
 struct __align__(1024) KqSmem {
-    float hi[2][128 * 32]; // [K; Q] hi parts of a 32-column block, by stage
-    float lo[2][128 * 32];
-    unsigned long long bar[2]; // the MMAs of the stage's block are done
+    float hi[1][128 * 32]; // [K; Q] hi parts of a 32-column block
+    float lo[1][128 * 32];
+    unsigned long long bar[2]; // bar[0]: the MMAs of the staged block are done (bar[1] unused)
     uint32_t tmem;
 };
 
@@ -102,9 +102,9 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
             x[i] = xn[i];
         if (q < 3)
             load_block(q + 1, xn);
-        const int st = q & 1;
-        if (q >= 2) // the MMAs of block q - 2 read this stage
-            ok = mbar_wait_bounded(st ? bar1 : bar0, 0u, kWaitLimit) && ok;
+        const int st = 0;
+        if (q >= 1) // the MMAs of block q - 1 read the stage
+            ok = mbar_wait_bounded(bar0, (uint32_t)((q - 1) & 1), kWaitLimit) && ok;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const int f = tid + kKqThreads * i, r = f >> 3, c = 4 * (f & 7);
@@ -129,10 +129,10 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
                 mma_tf32_ss(tmem, aH + ks, aL + ks, id, 1);
                 mma_tf32_ss(tmem, aL + ks, aH + ks, id, 1);
             }
-            mma_commit(st ? bar1 : bar0);
+            mma_commit(bar0);
         }
     }
-    ok = mbar_wait_bounded(bar1, 1u, kWaitLimit) && ok; // block 3, and with it every MMA
+    ok = mbar_wait_bounded(bar0, 1u, kWaitLimit) && ok; // block 3, and with it every MMA
     tc_fence_after();
     // TMEM lane r = row r of D; columns s.  Warp w reads lanes 32 w .. + 31.
     {
