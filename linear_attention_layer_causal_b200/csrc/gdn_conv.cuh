@@ -14,6 +14,12 @@ namespace gdn {
 
 constexpr int kConvTokens = 8; // tokens per thread
 
+// float32 -> tf32, round to nearest with ties away from zero (the same rule
+// as tf32_rna of gdn_sm100.cuh, without needing that header here)
+__device__ __forceinline__ float round_tf32(float x) {
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
+}
+
 // Loads of one thread's channel vector: Vec16<T> (16 bytes) or Vec8bf (8 bytes of bf16).
 template <typename VecT, typename T> struct VecIO;
 template <typename T> struct VecIO<Vec16<T>, T> {
@@ -86,9 +92,7 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
             for (int i = 0; i < V; ++i) {
                 acc[i] = siluf_(acc[i]);
                 if (io.round_v) {
-                    uint32_t r;
-                    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(acc[i]));
-                    acc[i] = __uint_as_float(r);
+                    acc[i] = round_tf32(acc[i]);
                 }
             }
 #pragma unroll
@@ -110,9 +114,7 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
         if (region == 2 && io.round_v) {
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                uint32_t r;
-                asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(acc[i]));
-                acc[i] = __uint_as_float(r);
+                acc[i] = round_tf32(acc[i]);
             }
         }
         float *dst = region < 2 ? io.qk_out + t * (2 * io.Hk * D) + cc

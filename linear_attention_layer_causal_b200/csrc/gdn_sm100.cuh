@@ -185,11 +185,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
 
 // float32 -> tf32 with round-to-nearest (ties away from zero); the result is a
 // float whose 13 low mantissa bits are zero.  The tensor core would otherwise
-// drop those bits (a biased truncation).
+// drop those bits (a biased truncation).  On the sign-magnitude bit pattern,
+// adding half of the dropped unit (2^12) and clearing the 13 low bits rounds
+// the magnitude half-up, carrying into the exponent when the mantissa fills:
+// two integer operations (tests/test_tf32_rounding.py checks it against the
+// nearest-tf32 definition).
 __device__ __forceinline__ float tf32_rna(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+    return __uint_as_float((__float_as_uint(x) + 0x1000u) & 0xffffe000u);
 }
 __device__ __forceinline__ float4 tf32_rna(float4 v) {
     return make_float4(tf32_rna(v.x), tf32_rna(v.y), tf32_rna(v.z), tf32_rna(v.w));
