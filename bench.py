@@ -198,6 +198,30 @@ def oracle_throughput(wl, inp, budget_s=10.0, max_tokens=None):
 # ----------------------------------------------------------------- our arm
 
 
+# ------------------------------------------------------------------ ranks
+# One process per GPU, replicas only: every rank runs its own seeded copy of
+# the workload and the ranks meet only for a barrier and the max of the times.
+
+def rank_seed(base, rank):
+    """Seed of this rank's synthetic inputs (distinct per rank)."""
+    return base + 7919 * rank
+
+
+def reduce_max(dist, x, device):
+    """Max of the float x over all ranks (x itself without a process group)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_step, world, steps, max_ms):
+    """Whole-job throughput: the units all ranks processed over the slowest rank's time."""
+    return units_per_step * world * steps / (max_ms / 1e3)
+
+
 def run_ours(args, rank, world, dev, dist):
     import torch
 
@@ -207,7 +231,7 @@ def run_ours(args, rank, world, dev, dist):
     pk = peaks()
     wl = W.QWEN38_PREFILL
     cfg = gdn.Config.of(wl, args.algo)
-    inp = W.make_prefill(wl, dev, seed=wl.seed + 7919 * rank)
+    inp = W.make_prefill(wl, dev, seed=rank_seed(wl.seed, rank))
     P = [inp[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
     N, B = sum(inp["seqlens"]), len(inp["seqlens"])
     y = torch.empty((N, cfg.num_v_heads, cfg.head_dim), dtype=torch.bfloat16, device=dev)
@@ -223,11 +247,7 @@ def run_ours(args, rank, world, dev, dist):
             dist.barrier()
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(dist, x, dev)
 
     window = {}
 
@@ -261,7 +281,7 @@ def run_ours(args, rank, world, dev, dist):
     total_ms = max_over_ranks(total_ms)
     kern_ms_max = max_over_ranks(kern_ms)
     ms_per_step = total_ms / args.steps
-    value = N * world * args.steps / (total_ms / 1e3)
+    value = job_rate(N, world, args.steps, total_ms)
 
     flops = prefill_flops_per_token(cfg.num_qk_heads, cfg.num_v_heads, cfg.head_dim) * N
     byts = prefill_bytes(cfg.num_qk_heads, cfg.num_v_heads, cfg.head_dim, N, B)
@@ -329,7 +349,7 @@ def run_ours(args, rank, world, dev, dist):
         e2e_step()
     etot, _ = timed(e2e_step, args.steps)
     etot = max_over_ranks(etot)
-    e2e = {"value": N * world * args.steps / (etot / 1e3), "unit": UNIT,
+    e2e = {"value": job_rate(N, world, args.steps, etot), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -356,7 +376,7 @@ def run_decode(args, rank, world, dev, pk, timed, max_over_ranks):
     dwl = W.QWEN38_DECODE
     dcfg = gdn.Config.of(dwl)
     dB = args.decode_batch
-    d = W.make_decode(dwl, dev, batch=dB, seed=dwl.seed + 7919 * rank)
+    d = W.make_decode(dwl, dev, batch=dB, seed=rank_seed(dwl.seed, rank))
     DP = [d[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
     dy = torch.empty((dB, dcfg.num_v_heads, dcfg.head_dim), dtype=torch.bfloat16, device=dev)
 
@@ -370,7 +390,7 @@ def run_decode(args, rank, world, dev, pk, timed, max_over_ranks):
     dbytes = decode_bytes(dcfg.num_qk_heads, dcfg.num_v_heads, dcfg.head_dim, dB)
     dgbs = dbytes / (dkern / 1e3) / 1e9
     return {"metric": "GDN decode tokens/s at Qwen3.8 layer shape", "unit": "tokens/s",
-            "value": dB * world * args.steps / (dtot / 1e3), "ms_per_step": dtot / args.steps,
+            "value": job_rate(dB, world, args.steps, dtot), "ms_per_step": dtot / args.steps,
             "config": {"workload": dwl.name, "batch": dB, "state_gib": 4 * dB * 128 ** 3 / 2 ** 30},
             "roofline": {"kernel": "decode_kernel", "bound": "hbm", "achieved": round(dgbs, 1),
                          "peak": pk["hbm_gbs"], "unit": "GB/s",

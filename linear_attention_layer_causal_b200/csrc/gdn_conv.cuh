@@ -1,6 +1,7 @@
 // gdn_conv.cuh -- the per-thread body of the prefill front end: depthwise causal
-// conv (kernel 4) + SiLU over 16 bytes of q|k|v channels for up to 8 tokens,
-// L2 normalisation of q and k per q/k head, FP32 results into the workspace.
+// conv (kernel 4) + SiLU over one vector of q|k|v channels (8 or 16 bytes) for
+// up to 8 tokens, L2 normalisation of q and k per q/k head, FP32 results into
+// the workspace.
 //
 // The conv, its kernel size and the SiLU follow the Gated DeltaNet row of the
 // component table on "Qwen3.8-2.4T-A95B vs Inkling" (and linear_conv_kernel_dim
@@ -53,7 +54,7 @@ template <typename T> struct ConvIO {
     bool round_v;          // v to its tf32 operand (tensor-core path)
 };
 
-// One thread: channels cc .. cc + V - 1 (V = 16 bytes of T) for the tokens
+// One thread: channels cc .. cc + V - 1 (V = the vector's elements) for the tokens
 // t0 .. tend - 1 (at most kConvTokens; tend <= N), n = the sequence of t0,
 // given rows[k] = the pre-conv row t0 - 3 + k of those channels (zero outside
 // [0, N)).  Tokens whose taps reach before the start of their sequence read

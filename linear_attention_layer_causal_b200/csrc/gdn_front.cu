@@ -31,7 +31,7 @@ constexpr int kKqThreads = 128;
 struct __align__(1024) KqSmem {
     float hi[1][128 * 32]; // [K; Q] hi parts of a 32-column block
     float lo[1][128 * 32];
-    unsigned long long bar[2]; // bar[0]: the MMAs of the staged block are done (bar[1] unused)
+    unsigned long long bar[1]; // the MMAs of the staged block are done
     uint32_t tmem;
 };
 
@@ -63,10 +63,9 @@ kq_prep_kernel(const float *__restrict__ qk, const int32_t *__restrict__ cu, int
     const int64_t t0 = s0 + (int64_t)(ci - __ldg(offs + lo)) * kC;
     const int nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
     const int64_t QKW = 2 * (int64_t)Hk * kD;
-    const uint32_t bar0 = smem_u32(&sm.bar[0]), bar1 = smem_u32(&sm.bar[1]);
+    const uint32_t bar0 = smem_u32(&sm.bar[0]);
     if (tid == 0) {
         mbar_init(bar0, 1);
-        mbar_init(bar1, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
