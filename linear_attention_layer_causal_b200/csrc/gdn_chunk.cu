@@ -356,15 +356,33 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             const int sl = c & 3;
             const uint32_t cU = (c & 1) ? kColU1 : kColU0, cX = (c & 1) ? kColX1 : kColX0;
             const uint32_t cO = cX + 64;
-            // ---- U pass: U -> tf32 (in place), U diag(gamma_C/gamma) -> tf32 into the
-            //      X columns (MMA 2b has read them), S *= gamma_C
+            // ---- U pass: S *= gamma_C once MMA 2 is done; then, once MMA 2b is done,
+            //      U -> tf32 (in place) and U diag(gamma_C/gamma) -> tf32 into the
+            //      X columns (MMA 2b has read them)
             {
                 bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
-                good = waitq(bar_m2b(c), (c >> 1) & 1) && good;
+                // S *= gamma_C as soon as MMA 2 (the last reader of S0) is done,
+                // beside MMA 2b, which does not touch S
+                good = waitq(bar_m2, c & 1) && good;
                 good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
                 tc_fence_after();
                 if (good) {
                     const float gC = expf(sm.G[sl][kC - 1]); // padded rows carry g = 0
+#pragma unroll 1
+                    for (int q = 0; q < 4; ++q) {
+                        float v[16];
+                        tmem_ld16(tl + kColS + 64 * hf + 16 * q, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            v[i] *= gC;
+                        tmem_st16(tl + kColS + 64 * hf + 16 * q, v);
+                    }
+                }
+                good = waitq(bar_m2b(c), (c >> 1) & 1) && good;
+                good = __all_sync(0xffffffffu, good);
+                tc_fence_after();
+                if (good) {
 #pragma unroll 1
                     for (int q = 0; q < 2; ++q) {
                         float u[16], uk[16];
@@ -382,16 +400,6 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                         }
                         tmem_st16(tl + cU + 32 * hf + 16 * q, u);
                         tmem_st16(tl + cX + 32 * hf + 16 * q, uk);
-                    }
-#pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        float v[16];
-                        tmem_ld16(tl + kColS + 64 * hf + 16 * q, v);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            v[i] *= gC;
-                        tmem_st16(tl + kColS + 64 * hf + 16 * q, v);
                     }
                     tmem_wait_st();
                 }
