@@ -173,6 +173,31 @@ def test_edge_lengths_full(cuda_device, with_conv, algo):
         assert torch.equal(out["final_state"][n], inp["initial_state"][n])
 
 
+EDGE_F32 = W.Workload("edge_f32", 2, 4, 128, dtype="f32", seqlens=(0, 5, 64, 100, 31),
+                      state_std=0.02, seed=78)
+
+
+@ALGOS
+def test_float32_activations_head_dim_128(cuda_device, algo):
+    """fp32 activations at head dim 128 (the float instantiation of every kernel of both
+    paths), with empty and ragged sequences."""
+    wl = EDGE_F32
+    cfg = gdn.Config.of(wl, algo)
+    inp = W.make_prefill(wl, cuda_device)
+    assert inp["qkv"].dtype == torch.float32
+    B = len(wl.seqlens)
+    out = _gpu_prefill(cfg, inp, return_final_state=True, return_o_raw=True)
+    torch.cuda.synchronize()
+    cu = inp["cu_seqlens"].tolist()
+    for n in range(B):
+        ref = _oracle_seq(wl, inp, n)
+        s, e = cu[n], cu[n + 1]
+        if e > s:
+            assert_output_close(out["y"][s:e], ref["y"], f"y seq {n}")
+            assert_output_close(out["o_raw"][s:e], ref["o"], f"o seq {n}")
+        assert_state_close(out["final_state"][n], ref["state"], f"state seq {n}")
+
+
 @ALGOS
 def test_in_place_state_and_conv(cuda_device, algo):
     """final_state = initial_state and final_conv = initial_conv give the out-of-place result."""
