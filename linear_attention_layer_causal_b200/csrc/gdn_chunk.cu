@@ -94,19 +94,24 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 //
 // One CTA per (value head, sequence), five roles that run consecutive chunks
 // at once and hand over through mbarriers:
-//   state group (warps 0..7): the U pass (U and U diag(gamma_C/gamma) rounded
-//     to tf32, S scaled by gamma_C) and the gated-RMSNorm epilogue; warps w and
-//     w + 4 share TMEM lanes 32 (w % 4) .. + 31 (lane = value channel) and
-//     split the columns.  X/O and U are double-buffered in TMEM, so the
-//     epilogue of chunk c overlaps MMA 2 of chunk c + 1;
-//   T team (warps 8..11): gates, A, T = (I + A)^-1 in a working tile of its
-//     own, then T diag(beta) and -T diag(beta gamma) into the tiles of the
-//     chunk's parity once MMA 1 and 2b of chunk c - 2 have read them;
-//   P team (warps 12..13): diag(gamma) Q in place and P from the Q K^T tile;
+//   state group (warps 0..7): S scaled by gamma_C once MMA 2 has read it, the
+//     U pass (U and U diag(gamma_C/gamma) rounded to tf32) once MMA 2b is done,
+//     and the gated-RMSNorm epilogue; warps w and w + 4 share TMEM lanes
+//     32 (w % 4) .. + 31 (lane = value channel) and split the columns.  X/O
+//     and U are double-buffered in TMEM, so the epilogue of chunk c overlaps
+//     MMA 2 of chunk c + 1;
+//   T team (warps 8..11): gates (G, beta, gamma_C / gamma, gamma), A,
+//     T = (I + A)^-1 in a working tile of its own, then T diag(beta) and
+//     -T diag(beta gamma) into the tiles of the chunk's parity once MMA 1 and
+//     2b of chunk c - 2 have read them;
+//   P team (warps 12..13): diag(gamma) Q in place (MMA 2 waits for it) and P
+//     from the Q K^T tile (MMA 3 waits for it);
 //   MMA warp (warp 14) and TMA warp (warp 15): one elected lane each.
-// Sixteen warps, four per scheduler, leave 128 registers a thread.
-// The per-chunk critical path is MMA 2 -> MMA 2b -> U pass -> MMA 3 -> MMA 2;
-// MMA 1 of the next chunk runs beside the U pass.
+// Sixteen warps, four per scheduler, leave 128 registers a thread.  The
+// per-chunk critical path is MMA 2 -> MMA 2b -> U pass -> MMA 3 -> MMA 2, with
+// the P team's two passes gating MMA 2 and MMA 3; MMA 1 of the next chunk runs
+// beside the U pass.  The roles' loops are rolled where that measured faster:
+// the SMs fetch the kernel's code from L2, and smaller hot code runs faster.
 
 constexpr int kSG = 256;                          // state group threads
 constexpr int kTeam = 128;                        // T team threads
