@@ -78,8 +78,8 @@ typedef enum gdn_dtype {
 typedef struct gdn_config {
     int32_t num_qk_heads; /* H_k >= 1 */
     int32_t num_v_heads;  /* H_v, a multiple of H_k (G = H_v / H_k value heads per q/k head) */
-    int32_t head_dim;     /* d = d_k = d_v; this build supports 32 and 128 */
-    int32_t conv_kernel;  /* causal conv width; this build supports 4 */
+    int32_t head_dim;     /* d = d_k = d_v; the library supports 32 and 128 */
+    int32_t conv_kernel;  /* causal conv width; the library supports 4 */
     float rms_eps;        /* epsilon of the gated RMSNorm (1e-6 for Qwen3.8) */
     float l2_eps;         /* epsilon inside the q/k L2 norm: x / sqrt(sum x^2 + l2_eps) */
     float q_scale;        /* extra factor on normalised q (1.0 = none) */

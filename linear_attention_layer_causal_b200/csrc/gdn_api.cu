@@ -104,7 +104,7 @@ const char *gdn_status_string(gdn_status s) {
     switch (s) {
     case GDN_OK: return "success";
     case GDN_ERR_INVALID_ARG: return "invalid argument (pointer, alignment, size or shape)";
-    case GDN_ERR_UNSUPPORTED: return "unsupported shape for this build";
+    case GDN_ERR_UNSUPPORTED: return "configuration or size outside what the library supports";
     case GDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case GDN_ERR_CUDA: return "CUDA launch or runtime error";
     }
