@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 1
+#define GDN_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -66,7 +66,9 @@ typedef enum gdn_status {
     GDN_ERR_INVALID_ARG = 1, /* NULL/misaligned pointer, bad size or inconsistent shape */
     GDN_ERR_UNSUPPORTED = 2, /* well-formed, but no kernel for this shape (head_dim, kernel) */
     GDN_ERR_WORKSPACE = 3,   /* workspace NULL, misaligned or smaller than the size query says */
-    GDN_ERR_CUDA = 4         /* a CUDA launch or runtime call failed */
+    GDN_ERR_CUDA = 4,        /* a CUDA launch or runtime call failed */
+    GDN_ERR_TIMEOUT = 5      /* a bounded wait inside a kernel gave up (device status word);
+                                returned only by the status queries below */
 } gdn_status;
 
 typedef enum gdn_dtype {
@@ -135,8 +137,7 @@ GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t bat
  *                 256-byte aligned; its contents on entry do not matter.  Its
  *                 first 4 bytes become a status word: 0 after a successful
  *                 call; nonzero if a wait inside a kernel gave up (the call's
- *                 outputs are then invalid).  Read it after the stream work
- *                 has completed.
+ *                 outputs are then invalid).  gdn_prefill_status reads it.
  * The values of cu_seqlens are read on the device only; a cu_seqlens array
  * that breaks the rules above gives unspecified output (never an
  * out-of-bounds access outside [0, N) rows).
@@ -146,6 +147,39 @@ GDN_API gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, 
                        int32_t batch, int64_t total_tokens, const float *initial_state,
                        const void *initial_conv, void *y, float *final_state, void *final_conv,
                        float *o_raw, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Device-side outcome of the last gdn_prefill that used `workspace`.
+ *
+ * The chunked kernels hand work between warps through barriers whose waits
+ * are bounded (about one second of SM clock); a wait that gives up makes the
+ * whole call abort cleanly (no fault, no hang) and leaves bits in the status
+ * word at the start of the workspace.  This call waits for `stream` (the
+ * stream the prefill ran on) to finish, then reads that word:
+ *   GDN_OK           the call completed normally,
+ *   GDN_ERR_TIMEOUT  a bounded wait gave up; the call's outputs are invalid,
+ *   GDN_ERR_CUDA     the stream reported an error, or a kernel found its
+ *                    shared-memory window misaligned,
+ *   GDN_ERR_INVALID_ARG  workspace NULL or shorter than the 8-byte header.
+ * `detail` (host, may be NULL) receives the second word of the header: 0, or
+ * where the first timed-out wait gave up (0x80000000 | warp << 24 | barrier
+ * index << 16 | waits that warp had completed).  A workspace that no prefill
+ * has used holds unspecified bytes.  Synchronises the host with `stream`.
+ */
+GDN_API gdn_status gdn_prefill_status(const void *workspace, size_t workspace_bytes,
+                                      uint32_t *detail, void *stream);
+
+/*
+ * Testing hook for the bounded waits above.  Arms a one-shot on the calling
+ * host thread: the next gdn_prefill or gdn_prefill_noalloc call made by this
+ * thread gives each wait between the warps of its chunked kernel `cycles` SM
+ * cycles instead of the default of 2e9 (about one second), so that a test can
+ * make a wait run out and check the abort path and gdn_prefill_status.  The
+ * waits that let a kernel's own in-flight copies and tensor-core work finish
+ * before it exits keep the default.  cycles = 0 disarms.  Returns
+ * GDN_ERR_INVALID_ARG for a negative value.
+ */
+GDN_API gdn_status gdn_wait_limit_next_call(int64_t cycles);
 
 /*
  * Decode: one new token for each of `batch` sequences against their resident
@@ -164,6 +198,58 @@ GDN_API gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, 
 GDN_API gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, const void *qkv,
                       const void *a, const void *b, const void *z, float *state,
                       void *conv_cache, int32_t batch, void *y, void *stream);
+
+/*
+ * Multi-token decode: num_tokens (k, 1..8) new tokens for each of `batch`
+ * sequences against their resident states, applied in order; state and conv
+ * cache advance by all k tokens, in place.  This is what decoding several
+ * tokens per step needs, e.g. the draft tokens of the multi-token-prediction
+ * layer of Qwen3.8 ("Qwen3.8 2.4T A95B", key facts: one extra MTP layer used
+ * to accelerate decoding; raw config field mtp_num_hidden_layers 1) once they
+ * are all accepted.  Each state row is read once and written once for the k
+ * tokens.  The result equals k calls of gdn_decode, and a prefill of the same
+ * k tokens continuing the sequence.
+ *
+ *   qkv        [batch, k, conv_dim]   act_dtype
+ *   a, b       [batch, k, H_v]        act_dtype
+ *   z          [batch, k, H_v, d]     act_dtype
+ *   state      [batch, H_v, d, d]     float32, in/out
+ *   conv_cache [batch, K-1, conv_dim] act_dtype, in/out
+ *   y          [batch, k, H_v, d]     act_dtype   output of every token
+ * Returns GDN_ERR_UNSUPPORTED for k > 8, or when k tokens of one q/k head
+ * group do not fit the kernel's shared memory (k * G * d * 8 bytes and a
+ * little more; every G <= 16 at d = 128 fits k = 8).  Needs no workspace.
+ */
+GDN_API gdn_status gdn_decode_multi(const gdn_config *cfg, const gdn_params *params,
+                                    const void *qkv, const void *a, const void *b, const void *z,
+                                    float *state, void *conv_cache, int32_t batch,
+                                    int32_t num_tokens, void *y, void *stream);
+
+/*
+ * Speculative decoding, step 1 of 2: the outputs y of k draft tokens per
+ * sequence (layout as gdn_decode_multi), computed against the resident state
+ * and conv cache WITHOUT changing either (both are only read).  The state is
+ * read once for all k tokens.  After the caller has decided how many leading
+ * tokens of each sequence it keeps, gdn_decode_commit takes exactly those.
+ */
+GDN_API gdn_status gdn_decode_verify(const gdn_config *cfg, const gdn_params *params,
+                                     const void *qkv, const void *a, const void *b, const void *z,
+                                     const float *state, const void *conv_cache, int32_t batch,
+                                     int32_t num_tokens, void *y, void *stream);
+
+/*
+ * Speculative decoding, step 2 of 2: advance each sequence's state and conv
+ * cache, in place, by its first accepted[n] of the num_tokens tokens given
+ * (the same qkv, a, b as the verify call; z is not needed).  accepted is a
+ * DEVICE int32 array [batch]; values are clamped to [0, num_tokens], and a
+ * sequence with 0 is left untouched.  Rejected draft tokens never reach the
+ * state, so nothing has to be rolled back.  The result equals gdn_decode_multi
+ * over the accepted tokens.
+ */
+GDN_API gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *params,
+                                     const void *qkv, const void *a, const void *b, float *state,
+                                     void *conv_cache, int32_t batch, int32_t num_tokens,
+                                     const int32_t *accepted, void *stream);
 
 /*
  * Size of the fixed device scratch array used by gdn_prefill_noalloc:
@@ -193,8 +279,15 @@ GDN_API gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, c
  *     last call's contents.  Nothing in it needs to start at zero.  Calls
  *     whose work overlaps on the GPU (different streams or host threads on
  *     the same device) race on the array and give wrong results: order them.
- * Returns what gdn_prefill returns, or GDN_ERR_CUDA if the address look-up
- * fails.
+ *   - Device status: the status word that gdn_prefill leaves in its
+ *     workspace lives here in the fixed array, out of the caller's reach;
+ *     read it with gdn_prefill_noalloc_status.
+ *   - A device reset (cudaDeviceReset) after the first call on that device
+ *     is not supported: the cached address would be stale.
+ * Validates its arguments exactly as gdn_prefill does (same codes, same
+ * order); only then a call that needs more than the fixed array returns
+ * GDN_ERR_WORKSPACE.  Nothing is launched by a rejected call.  Returns
+ * GDN_ERR_CUDA if the address look-up fails.
  */
 GDN_API gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_params *params,
                                        const void *qkv, const void *a, const void *b,
@@ -202,6 +295,14 @@ GDN_API gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_params *
                                        int64_t total_tokens, const float *initial_state,
                                        const void *initial_conv, void *y, float *final_state,
                                        void *final_conv, float *o_raw, void *stream);
+
+/*
+ * gdn_prefill_status for gdn_prefill_noalloc: waits for `stream`, then reads
+ * the status word of the fixed scratch array on the current device (the
+ * outcome of the last gdn_prefill_noalloc call there).  Returns GDN_OK when
+ * no such call has been made on this device.  Allocates nothing.
+ */
+GDN_API gdn_status gdn_prefill_noalloc_status(uint32_t *detail, void *stream);
 
 /*
  * Timing hook for benchmarks.  Arms a one-shot on the calling host thread:

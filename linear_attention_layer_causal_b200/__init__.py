@@ -28,11 +28,14 @@ from dataclasses import dataclass
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libgdn.so")
 
-GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA = range(5)
+(GDN_OK, GDN_ERR_INVALID_ARG, GDN_ERR_UNSUPPORTED, GDN_ERR_WORKSPACE, GDN_ERR_CUDA,
+ GDN_ERR_TIMEOUT) = range(6)
 GDN_F32, GDN_BF16 = 0, 1
 
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_status_string",
-            "gdn_abi_version", "gdn_profile_next_call", "gdn_prefill_noalloc")
+            "gdn_abi_version", "gdn_profile_next_call", "gdn_prefill_noalloc",
+            "gdn_prefill_status", "gdn_prefill_noalloc_status", "gdn_wait_limit_next_call",
+            "gdn_decode_multi", "gdn_decode_verify", "gdn_decode_commit")
 
 # Fixed scratch of gdn_prefill_noalloc (GDN_NOALLOC_SCRATCH_BYTES in include/gdn.h).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -110,10 +113,23 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill_noalloc.restype = ctypes.c_int
         L.gdn_decode.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
         L.gdn_decode.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_decode_verify.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.gdn_decode_verify.restype = ctypes.c_int
+        L.gdn_decode_commit.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.gdn_decode_commit.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_profile_next_call.argtypes = [vp, vp]
         L.gdn_profile_next_call.restype = ctypes.c_int
+        u32p = ctypes.POINTER(ctypes.c_uint32)
+        L.gdn_prefill_status.argtypes = [vp, sz, u32p, vp]
+        L.gdn_prefill_status.restype = ctypes.c_int
+        L.gdn_prefill_noalloc_status.argtypes = [u32p, vp]
+        L.gdn_prefill_noalloc_status.restype = ctypes.c_int
+        L.gdn_wait_limit_next_call.argtypes = [i64]
+        L.gdn_wait_limit_next_call.restype = ctypes.c_int
         L.gdn_abi_version.argtypes = []
         L.gdn_abi_version.restype = ctypes.c_int32
         _lib = L
@@ -162,12 +178,32 @@ def profile_next_call(begin_event, end_event) -> None:
         raise GdnError(st, "gdn_profile_next_call")
 
 
-def workspace_status(workspace) -> int:
-    """The status word a prefill call left in its workspace (0 = ok); synchronises."""
-    import torch
-    if workspace is None or workspace.numel() < 4:
-        return 0
-    return int(workspace[:4].view(torch.int32).item())
+def prefill_status(workspace, stream=None) -> tuple[int, int]:
+    """(status, detail) of the last prefill that used `workspace` (gdn_prefill_status):
+    GDN_OK, GDN_ERR_TIMEOUT when a bounded wait inside a kernel gave up, or
+    GDN_ERR_CUDA; detail says where the first timed-out wait gave up.  Waits for
+    the stream."""
+    if workspace is None or workspace.numel() < 8:
+        return GDN_OK, 0
+    d = ctypes.c_uint32(0)
+    st = lib().gdn_prefill_status(_ptr(workspace), workspace.numel(), ctypes.byref(d),
+                                  _stream(stream))
+    return st, d.value
+
+
+def prefill_noalloc_status(stream=None) -> tuple[int, int]:
+    """(status, detail) of the last gdn_prefill_noalloc call on the current device."""
+    d = ctypes.c_uint32(0)
+    st = lib().gdn_prefill_noalloc_status(ctypes.byref(d), _stream(stream))
+    return st, d.value
+
+
+def wait_limit_next_call(cycles: int) -> None:
+    """Testing hook: the next prefill call on this thread bounds each wait between
+    the warps of its chunked kernel by `cycles` SM cycles (0 = default, ~1 s)."""
+    st = lib().gdn_wait_limit_next_call(int(cycles))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_wait_limit_next_call")
 
 
 def prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
@@ -216,8 +252,10 @@ def prefill(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bias, norm_
                            _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill")
-    if check_status and workspace_status(workspace) != 0:
-        raise GdnError(GDN_ERR_CUDA, f"gdn_prefill: device status {workspace_status(workspace)}")
+    if check_status:
+        dst, detail = prefill_status(workspace, stream)
+        if dst != GDN_OK:
+            raise GdnError(dst, f"gdn_prefill (device status, detail {detail:#010x})")
     out = {"y": y}
     if final_state is not None:
         out["final_state"] = final_state
@@ -239,7 +277,8 @@ def prefill_noalloc(cfg: Config, qkv, a, b, z, cu_seqlens, conv_w, A_log, dt_bia
     Calls on one device share the scratch: calls that overlap on the GPU race.
     The first call on a device looks up the scratch's address; make it before
     any stream capture.  Raises GdnError if the call needs more than
-    NOALLOC_SCRATCH_BYTES of scratch (see prefill_workspace_size)."""
+    NOALLOC_SCRATCH_BYTES of scratch (see prefill_workspace_size).  The device
+    status of the call is read with prefill_noalloc_status()."""
     N = qkv.shape[0]
     B = cu_seqlens.shape[0] - 1
     st = lib().gdn_prefill_noalloc(ctypes.byref(cfg._c()),
@@ -269,3 +308,52 @@ def decode(cfg: Config, qkv, a, b, z, state, conv_cache, conv_w, A_log, dt_bias,
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode")
     return y
+
+
+def _multi_y(cfg, qkv, y):
+    import torch
+    if y is None:
+        B, k = qkv.shape[0], qkv.shape[1]
+        y = torch.empty((B, k, cfg.num_v_heads, cfg.head_dim), dtype=_act(cfg), device=qkv.device)
+    return y
+
+
+def decode_multi(cfg: Config, qkv, a, b, z, state, conv_cache, conv_w, A_log, dt_bias, norm_w,
+                 *, y=None, stream=None):
+    """k tokens per sequence (qkv [B, k, conv_dim], a, b [B, k, H_v], z [B, k, H_v, d]);
+    `state` and `conv_cache` advance by all k tokens in place.  Returns y [B, k, H_v, d]."""
+    y = _multi_y(cfg, qkv, y)
+    st = lib().gdn_decode_multi(ctypes.byref(cfg._c()),
+                                ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                                _ptr(qkv), _ptr(a), _ptr(b), _ptr(z), _ptr(state),
+                                _ptr(conv_cache), qkv.shape[0], qkv.shape[1], _ptr(y),
+                                _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_multi")
+    return y
+
+
+def decode_verify(cfg: Config, qkv, a, b, z, state, conv_cache, conv_w, A_log, dt_bias, norm_w,
+                  *, y=None, stream=None):
+    """Outputs of k draft tokens per sequence; `state` and `conv_cache` are only read."""
+    y = _multi_y(cfg, qkv, y)
+    st = lib().gdn_decode_verify(ctypes.byref(cfg._c()),
+                                 ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                                 _ptr(qkv), _ptr(a), _ptr(b), _ptr(z), _ptr(state),
+                                 _ptr(conv_cache), qkv.shape[0], qkv.shape[1], _ptr(y),
+                                 _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_verify")
+    return y
+
+
+def decode_commit(cfg: Config, qkv, a, b, state, conv_cache, accepted, conv_w, A_log, dt_bias,
+                  norm_w, *, stream=None) -> None:
+    """Advance `state` and `conv_cache` in place by the first accepted[n] tokens of each
+    sequence (accepted: int32 tensor [B] on the device)."""
+    st = lib().gdn_decode_commit(ctypes.byref(cfg._c()),
+                                 ctypes.byref(_params(conv_w, A_log, dt_bias, norm_w)),
+                                 _ptr(qkv), _ptr(a), _ptr(b), _ptr(state), _ptr(conv_cache),
+                                 qkv.shape[0], qkv.shape[1], _ptr(accepted), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_decode_commit")

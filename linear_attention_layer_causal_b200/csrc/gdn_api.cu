@@ -62,6 +62,7 @@ bool elem_aligned(const void *p, bool bf16) {
 gdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
 thread_local ProfileHook tl_hook;
+thread_local long long tl_wait_limit = 0; // 0 = not armed
 
 } // namespace
 
@@ -69,6 +70,56 @@ ProfileHook take_profile_hook() {
     ProfileHook h = tl_hook;
     tl_hook = ProfileHook{};
     return h;
+}
+
+long long take_wait_limit() {
+    const long long w = tl_wait_limit;
+    tl_wait_limit = 0;
+    return w > 0 ? w : kDefaultWaitLimit;
+}
+
+gdn_status validate_prefill(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                            const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                            int32_t batch, int64_t total_tokens, const float *initial_state,
+                            const void *initial_conv, const void *y, const float *final_state,
+                            const void *final_conv, const float *o_raw, size_t *need) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if ((st = check_params(params)) != GDN_OK)
+        return st;
+    if (batch < 0 || total_tokens < 0 || batch > 65535)
+        return batch > 65535 ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID_ARG;
+    if (batch == 0 && total_tokens > 0)
+        return GDN_ERR_INVALID_ARG;
+    if (batch > 0 && cu_seqlens == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    const bool bf16 = cfg->act_dtype == GDN_BF16;
+    if (total_tokens > 0 && (qkv == nullptr || a == nullptr || b == nullptr || z == nullptr ||
+                             y == nullptr))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(z) || !aligned16(y) || !aligned16(initial_state) ||
+        !aligned16(initial_conv) || !aligned16(final_state) || !aligned16(final_conv) ||
+        !aligned16(o_raw) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    *need = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads, cfg->head_dim, bf16,
+                                    total_tokens, batch);
+    return GDN_OK;
+}
+
+gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t stream) {
+    uint32_t w[2] = {0u, 0u};
+    cudaError_t e = cudaMemcpyAsync(w, header, sizeof(w), cudaMemcpyDeviceToHost, stream);
+    if (e == cudaSuccess)
+        e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess)
+        return GDN_ERR_CUDA;
+    if (detail != nullptr)
+        *detail = w[1];
+    if (w[0] & 1u)
+        return GDN_ERR_TIMEOUT;
+    return w[0] != 0u ? GDN_ERR_CUDA : GDN_OK;
 }
 
 // Header (status word), float32 normalised q|k, float32 convolved v and, for
@@ -100,6 +151,20 @@ gdn_status gdn_profile_next_call(void *begin_event, void *end_event) {
     return GDN_OK;
 }
 
+gdn_status gdn_wait_limit_next_call(int64_t cycles) {
+    if (cycles < 0)
+        return GDN_ERR_INVALID_ARG;
+    tl_wait_limit = (long long)cycles;
+    return GDN_OK;
+}
+
+gdn_status gdn_prefill_status(const void *workspace, size_t workspace_bytes, uint32_t *detail,
+                              void *stream) {
+    if (workspace == nullptr || workspace_bytes < 2 * sizeof(uint32_t))
+        return GDN_ERR_INVALID_ARG;
+    return read_status_words(workspace, detail, (cudaStream_t)stream);
+}
+
 const char *gdn_status_string(gdn_status s) {
     switch (s) {
     case GDN_OK: return "success";
@@ -107,6 +172,7 @@ const char *gdn_status_string(gdn_status s) {
     case GDN_ERR_UNSUPPORTED: return "configuration or size outside what the library supports";
     case GDN_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     case GDN_ERR_CUDA: return "CUDA launch or runtime error";
+    case GDN_ERR_TIMEOUT: return "a bounded wait inside a kernel gave up; the outputs are invalid";
     }
     return "unknown status";
 }
@@ -128,28 +194,13 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
                        int32_t batch, int64_t total_tokens, const float *initial_state,
                        const void *initial_conv, void *y, float *final_state, void *final_conv,
                        float *o_raw, void *workspace, size_t workspace_bytes, void *stream) {
-    gdn_status st = check_config(cfg);
+    size_t need = 0;
+    gdn_status st = validate_prefill(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens,
+                                     initial_state, initial_conv, y, final_state, final_conv,
+                                     o_raw, &need);
     if (st != GDN_OK)
         return st;
-    if ((st = check_params(params)) != GDN_OK)
-        return st;
-    if (batch < 0 || total_tokens < 0 || batch > 65535)
-        return batch > 65535 ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID_ARG;
-    if (batch == 0 && total_tokens > 0)
-        return GDN_ERR_INVALID_ARG;
-    if (batch > 0 && cu_seqlens == nullptr)
-        return GDN_ERR_INVALID_ARG;
     const bool bf16 = cfg->act_dtype == GDN_BF16;
-    if (total_tokens > 0 && (qkv == nullptr || a == nullptr || b == nullptr || z == nullptr ||
-                             y == nullptr))
-        return GDN_ERR_INVALID_ARG;
-    if (!aligned16(qkv) || !aligned16(z) || !aligned16(y) || !aligned16(initial_state) ||
-        !aligned16(initial_conv) || !aligned16(final_state) || !aligned16(final_conv) ||
-        !aligned16(o_raw) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
-        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
-        return GDN_ERR_INVALID_ARG;
-    const size_t need = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads,
-                                                cfg->head_dim, bf16, total_tokens, batch);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
                      (reinterpret_cast<uintptr_t>(workspace) & 255u)))
         return GDN_ERR_WORKSPACE;
@@ -190,16 +241,18 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
 
     cudaStream_t s = (cudaStream_t)stream;
     const ProfileHook hook = take_profile_hook();
+    p.wait_limit = take_wait_limit();
     if (batch == 0)
         return GDN_OK;
-    // conv / SiLU / L2 front end; the chunked path first computes the chunk
-    // offsets (and clears the status words), and after the conv the
-    // intra-chunk Gram rows
+    // front end.  Chunked path: chunk offsets (which also clear the status
+    // words), the fused q/k kernel (conv, SiLU, L2 norm and the intra-chunk
+    // Gram rows), then the conv of the v channels.  Token-serial path: the conv
+    // of every channel.
     cudaError_t e = p.chunked ? launch_chunk_offsets(p, s) : cudaSuccess;
+    if (e == cudaSuccess && p.chunked)
+        e = launch_qk_front(p, s);
     if (e == cudaSuccess)
         e = launch_conv_prep(p, s);
-    if (e == cudaSuccess && p.chunked)
-        e = launch_kq_prep(p, s);
     if (e == cudaSuccess)
         e = record_if(hook.begin, s);
     if (e == cudaSuccess)
@@ -211,55 +264,108 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     return cuda_status(e);
 }
 
-gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, const void *qkv,
-                      const void *a, const void *b, const void *z, float *state,
-                      void *conv_cache, int32_t batch, void *y, void *stream) {
+}
+
+namespace gdn {
+namespace {
+
+// The checks and launch shared by the decode entry points.  mode < 0: the
+// one-token kernel; otherwise a multi-token mode with `k` tokens per sequence.
+gdn_status decode_call(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                       const void *a, const void *b, const void *z, const float *state,
+                       const void *conv_cache, int32_t batch, int32_t k, const int32_t *accepted,
+                       void *y, void *stream, int mode) {
     gdn_status st = check_config(cfg);
     if (st != GDN_OK)
         return st;
     if ((st = check_params(params)) != GDN_OK)
         return st;
-    if (batch < 0)
+    if (batch < 0 || k < 1)
         return GDN_ERR_INVALID_ARG;
-    if (batch > 65535)
+    if (batch > 65535 || k > kDecodeMaxTokens)
+        return GDN_ERR_UNSUPPORTED;
+    const int G = cfg->num_v_heads / cfg->num_qk_heads;
+    if (mode >= 0 && decode_multi_smem_bytes(G, cfg->head_dim, k, mode) > kDecodeMaxSmem)
         return GDN_ERR_UNSUPPORTED;
     if (batch == 0) {
         take_profile_hook();
         return GDN_OK;
     }
     const bool bf16 = cfg->act_dtype == GDN_BF16;
-    if (qkv == nullptr || a == nullptr || b == nullptr || z == nullptr || state == nullptr ||
-        conv_cache == nullptr || y == nullptr)
+    const bool want_y = mode != kDecodeCommit;
+    const bool want_z = want_y;
+    if (qkv == nullptr || a == nullptr || b == nullptr || (want_z && z == nullptr) ||
+        state == nullptr || conv_cache == nullptr || (want_y && y == nullptr) ||
+        (mode == kDecodeCommit && accepted == nullptr))
         return GDN_ERR_INVALID_ARG;
     if (!aligned16(qkv) || !aligned16(z) || !aligned16(y) || !aligned16(state) ||
-        !aligned16(conv_cache) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16))
+        !aligned16(conv_cache) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
+        (reinterpret_cast<uintptr_t>(accepted) & 3u))
         return GDN_ERR_INVALID_ARG;
     DecodeArgs p{};
     p.Hk = cfg->num_qk_heads;
     p.Hv = cfg->num_v_heads;
     p.D = cfg->head_dim;
-    p.G = p.Hv / p.Hk;
+    p.G = G;
     p.bf16 = bf16;
     p.rms_eps = cfg->rms_eps;
     p.l2_eps = cfg->l2_eps;
     p.q_scale = cfg->q_scale;
     p.qkv = qkv; p.a = a; p.b = b; p.z = z;
-    p.state = state;
-    p.conv_cache = conv_cache;
+    p.state = const_cast<float *>(state); // written only by the updating modes
+    p.conv_cache = const_cast<void *>(conv_cache);
     p.batch = batch;
     p.y = y;
     p.conv_w = params->conv_w;
     p.A_log = params->A_log;
     p.dt_bias = params->dt_bias;
     p.norm_w = params->norm_w;
+    p.k = k;
+    p.accepted = accepted;
     cudaStream_t s = (cudaStream_t)stream;
     const ProfileHook hook = take_profile_hook();
     cudaError_t e = record_if(hook.begin, s);
     if (e == cudaSuccess)
-        e = launch_decode(p, s);
+        e = mode < 0 ? launch_decode(p, s) : launch_decode_multi(p, mode, s);
     if (e == cudaSuccess)
         e = record_if(hook.end, s);
     return cuda_status(e);
+}
+
+} // namespace
+} // namespace gdn
+
+extern "C" {
+
+gdn_status gdn_decode(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                      const void *a, const void *b, const void *z, float *state,
+                      void *conv_cache, int32_t batch, void *y, void *stream) {
+    return decode_call(cfg, params, qkv, a, b, z, state, conv_cache, batch, 1, nullptr, y, stream,
+                       -1);
+}
+
+gdn_status gdn_decode_multi(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                            const void *a, const void *b, const void *z, float *state,
+                            void *conv_cache, int32_t batch, int32_t num_tokens, void *y,
+                            void *stream) {
+    return decode_call(cfg, params, qkv, a, b, z, state, conv_cache, batch, num_tokens, nullptr, y,
+                       stream, kDecodeMulti);
+}
+
+gdn_status gdn_decode_verify(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                             const void *a, const void *b, const void *z, const float *state,
+                             const void *conv_cache, int32_t batch, int32_t num_tokens, void *y,
+                             void *stream) {
+    return decode_call(cfg, params, qkv, a, b, z, state, conv_cache, batch, num_tokens, nullptr, y,
+                       stream, kDecodeVerify);
+}
+
+gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                             const void *a, const void *b, float *state, void *conv_cache,
+                             int32_t batch, int32_t num_tokens, const int32_t *accepted,
+                             void *stream) {
+    return decode_call(cfg, params, qkv, a, b, nullptr, state, conv_cache, batch, num_tokens,
+                       accepted, nullptr, stream, kDecodeCommit);
 }
 
 } // extern "C"

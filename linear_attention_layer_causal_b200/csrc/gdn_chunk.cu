@@ -19,16 +19,20 @@
 // Mapping onto the tensor core (M = 128 = d_v is the TMEM lane dimension),
 // with X = K S0^T:
 //   MMA 1   U~^T = V^T (T diag b)^T        A = V (smem, MN-major), B = T diag b
-//   MMA 2   [X^T | O^T] = S0 [K ; diag(gamma) Q]^T   (one N = 128 product; A =
-//           the FP32 state in TMEM, B = K and gamma Q, K-major)
+//   MMA 2   [X^T | O^T] = S0 [K ; Q]^T     (one N = 128 product; A = the FP32
+//           state in TMEM, B = K and Q, K-major); then, in FP32 on the CUDA
+//           cores, O^T *= diag(gamma) and S *= gamma_C
 //   MMA 2b  U^T = U~^T + X^T (-T diag b gamma)^T     (A = X^T from TMEM)
-//   MMA 3   O^T += U^T P^T  and  S += (U diag(gamma_C/gamma))^T K   (K MN-major)
+//   MMA 3   O^T += U^T P^T  and  S += U^T (diag(gamma_C/gamma) K)   (K MN-major)
 // The state lives in TMEM for the whole sequence.  All products run as
-// kind::tf32; every operand computed here is rounded to nearest first (the
-// tensor core's own conversion truncates, a bias that would accumulate
-// through the state).  The Gram matrices K K^T and Q K^T come exact in FP32
-// from the front kernel (gdn_front.cu): the near-cancelling outputs are
-// sensitive to them.
+// kind::tf32 on operands rounded to nearest beforehand (the tensor core's own
+// conversion truncates, a bias that would accumulate through the state): q
+// and k leave the front kernel rounded, V leaves the conv rounded, and every
+// operand formed here (T diag b, -T diag b gamma, P, diag(gamma_C/gamma) K, U)
+// is rounded where it is formed; only S0 and X, which the tensor core reads
+// straight from TMEM, are truncated.  The Gram matrices K K^T and Q K^T come
+// exact in FP32 from the front kernel (gdn_front.cu): the near-cancelling
+// outputs are sensitive to them.
 //
 // The gated RMSNorm y = o / rms(o) * w * SiLU(z) ("Qwen3.8-2.4T-A95B vs
 // Inkling", output-gate row) is fused into the output store.
@@ -45,7 +49,10 @@ namespace {
 
 constexpr int kC = 64;  // chunk length
 constexpr int kD = 128; // head dim (d_k = d_v)
-constexpr long long kWaitLimit = 2000000000LL; // bounded waits: ~1 s of SM cycles
+// The waits that let this CTA's own TMA copies and MMAs finish before it
+// releases shared memory and TMEM always get the default bound (~1 s of SM
+// cycles); the waits between roles get the call's bound (p.wait_limit).
+constexpr long long kWaitLimit = kDefaultWaitLimit;
 
 // ------------------------------------------------------------ chunk offsets
 
@@ -94,24 +101,25 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 //
 // One CTA per (value head, sequence), five roles that run consecutive chunks
 // at once and hand over through mbarriers:
-//   state group (warps 0..7): S scaled by gamma_C once MMA 2 has read it, the
-//     U pass (U and U diag(gamma_C/gamma) rounded to tf32) once MMA 2b is done,
-//     and the gated-RMSNorm epilogue; warps w and w + 4 share TMEM lanes
-//     32 (w % 4) .. + 31 (lane = value channel) and split the columns.  X/O
-//     and U are double-buffered in TMEM, so the epilogue of chunk c overlaps
-//     MMA 2 of chunk c + 1;
+//   state group (warps 0..7): once MMA 2 is done, S *= gamma_C and O^T *=
+//     diag(gamma); once MMA 2b is done, U rounded to tf32 in place; then the
+//     gated-RMSNorm epilogue.  Warps w and w + 4 share TMEM lanes 32 (w % 4) ..
+//     + 31 (lane = value channel) and split the columns.  X/O and U are
+//     double-buffered in TMEM, so the epilogue of chunk c overlaps MMA 2 of
+//     chunk c + 1;
 //   T team (warps 8..11): gates (G, beta, gamma_C / gamma, gamma), A,
 //     T = (I + A)^-1 in a working tile of its own, then T diag(beta) and
 //     -T diag(beta gamma) into the tiles of the chunk's parity once MMA 1 and
 //     2b of chunk c - 2 have read them;
-//   P team (warps 12..13): diag(gamma) Q in place (MMA 2 waits for it) and P
-//     from the Q K^T tile (MMA 3 waits for it);
-//   MMA warp (warp 14) and TMA warp (warp 15): one elected lane each.
+//   P team (warps 12..13): diag(gamma_C / gamma) K in place on the MN-major K
+//     tile and P from the Q K^T tile (MMA 3 waits for both);
+//   MMA warp (warp 14): the whole warp runs the issue loop, one elected lane
+//     issues; TMA warp (warp 15): one lane.
 // Sixteen warps, four per scheduler, leave 128 registers a thread.  The
-// per-chunk critical path is MMA 2 -> MMA 2b -> U pass -> MMA 3 -> MMA 2, with
-// the P team's two passes gating MMA 2 and MMA 3; MMA 1 of the next chunk runs
-// beside the U pass.  The roles' loops are rolled where that measured faster:
-// the SMs fetch the kernel's code from L2, and smaller hot code runs faster.
+// per-chunk critical path is MMA 2 -> MMA 2b -> U rounding -> MMA 3 -> MMA 2;
+// MMA 1 of the next chunk runs beside the U rounding.  The roles' loops are
+// rolled where that measured faster: the SMs fetch the kernel's code from L2,
+// and smaller hot code runs faster.
 
 constexpr int kSG = 256;                          // state group threads
 constexpr int kTeam = 128;                        // T team threads
@@ -121,8 +129,7 @@ constexpr int kWarpMma = (kSG + kTeam + kTeamP) / 32; // 14
 constexpr int kBarSG = 1, kBarT = 2, kBarP = 3;   // named barriers
 
 // TMEM columns: the state, two [X^T | O^T] pairs (MMA 2 writes one pair with a
-// single N = 128 product; once MMA 2b has read X^T its columns take U diag(
-// gamma_C / gamma)), two U^T buffers.  All by chunk parity.
+// single N = 128 product), two U^T buffers.  All by chunk parity.
 constexpr uint32_t kColS = 0;
 constexpr uint32_t kColX0 = 128, kColX1 = 256; // O of each pair sits 64 columns on
 constexpr uint32_t kColU0 = 384, kColU1 = 448;
@@ -145,25 +152,26 @@ constexpr uint32_t kTmemCols = 512;
 constexpr int kTriFloats = 3 * 1024;
 
 struct __align__(1024) ChunkSmem {
-    // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = K, rows 64..127 = diag(gamma) Q
+    // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = K, rows 64..127 = Q
     float KQ[2 * kC * kD];
     float V[kC * kD];          // A of MMA 1 (MN-major)
-    float K[kC * kD];          // B of MMA 3 (MN-major)
+    float K[kC * kD];          // B of MMA 3 (MN-major): lands as K, becomes diag(gamma_C/gamma) K
     float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta), by chunk parity
     float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma), by chunk parity
     float P[kTriFloats];       // B of MMA 3: lands as Q K^T rows, becomes P
     float Wk[kTriFloats];      // T team: lands as K K^T rows, becomes A, then T
     // z rows of the chunk (16-bit activations).  Once the state group has formed
-    // the gate from it, its head holds the epilogue's partial sums of squares
-    // (red[4][64]) and reciprocal norms (rstd[64]).
+    // the gate from it, it stages the chunk's y rows for one TMA store.
     __nv_bfloat16 Z[kC * kD];
+    float red[4][kC];          // epilogue: partial sums of o^2 per TMEM lane quarter
+    float rstd[kC];            // epilogue: reciprocal RMS of each row
     float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
     float gam[4][kC];          // gamma = e^G (fast exponential), by chunk index mod 4
     float beta[kC];            // T team's current chunk
     unsigned long long bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z; // TMA landings
     unsigned long long bar_m1, bar_m2, bar_m2b[2], bar_m3;      // MMA completions
     unsigned long long bar_u, bar_of[2];                        // state group -> MMA
-    unsigned long long bar_pT[4], bar_pQ, bar_pP, bar_wfree;    // T / P teams -> MMA, TMA
+    unsigned long long bar_pT[4], bar_pP, bar_wfree;            // T / P teams -> MMA, TMA
     unsigned long long bar_fin;                                 // MMA drain on abort
     uint32_t tmem;
     int abort;
@@ -180,18 +188,20 @@ struct ChunkMaps {
     CUtensorMap kq;   // Gram rows, [N, Hk*128] fp32, 32 x 64 boxes, 128-byte swizzle
     CUtensorMap kq32; // the same with 32 x 32 boxes
     CUtensorMap z;    // z, [N, Hv*128] bf16, 128 x 64 boxes, no swizzle (bf16 activations)
+    CUtensorMap y;    // y, the same layout (bf16 activations): the store of a full chunk
 };
 
 // The rest of a bounded wait whose first try failed: polls until the phase
-// completes, another role aborts, or about 1 s passes; on a time-out records
-// `diag` (the first one only) in err[1].  Out of line: every wait site shares it.
+// completes, another role aborts, or `limit` SM cycles pass (about 1 s by
+// default); on a time-out records `diag` (the first one only) in err[1].  Out
+// of line: every wait site shares it.
 __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t ph, volatile int *abort_flag,
-                                       unsigned int *err, uint32_t diag) {
+                                       unsigned int *err, uint32_t diag, long long limit) {
     const long long t0 = clock64();
     while (!sm100::mbar_try_wait_spin(bar, ph)) {
         if (*abort_flag)
             return false;
-        if (clock64() - t0 > kWaitLimit) {
+        if (clock64() - t0 > limit) {
             if (err != nullptr)
                 atomicCAS(err + 1, 0u, diag);
             return false;
@@ -269,12 +279,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     // must see that phase before the barrier can move on, and the T team may run
     // up to two chunks ahead of the state group
     auto bar_pT = [&](int c) { return smem_u32(&sm.bar_pT[c & 3]); };
-    const uint32_t bar_pQ = smem_u32(&sm.bar_pQ);
     const uint32_t bar_pP = smem_u32(&sm.bar_pP), bar_wfree = smem_u32(&sm.bar_wfree);
     if (tid == 0) {
         const uint32_t one[] = {bar_v,  bar_q,   bar_k,   bar_kmaj, bar_kk,   bar_qk,  bar_z,
-                                bar_m1, bar_m2,  bar_m3,  bar_u,    bar_of0,  bar_of1, bar_pQ,
-                                bar_pP, bar_wfree, smem_u32(&sm.bar_fin)};
+                                bar_m1, bar_m2,  bar_m3,  bar_u,    bar_of0,  bar_of1, bar_pP,
+                                bar_wfree, smem_u32(&sm.bar_fin)};
 #pragma unroll
         for (int b = 0; b < (int)(sizeof(one) / sizeof(one[0])); ++b)
             mbar_init(one[b], 1);
@@ -313,7 +322,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         if (!done)
             done = wait_slow(bar, ph, abort_flag, p.ws_err,
                              0x80000000u | ((uint32_t)warp << 24) | (((bar - bar_base) / 8) << 16) |
-                                 (waits_seen & 0xffffu));
+                                 (waits_seen & 0xffffu),
+                             p.wait_limit);
         ph ^= 1u;
         ++waits_seen;
         return done;
@@ -355,59 +365,69 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             mbar_arrive(bar_u); // phase 0 of the U barrier: the initial state is in TMEM
         const float wn = __ldg(p.norm_w + vch);
         uint32_t ph3 = 0, phz = 0;
-        float *red = reinterpret_cast<float *>(sm.Z); // [4][kC], then rstd[kC]
-        float *rstd = red + 4 * kC;
+        float *red = &sm.red[0][0];
+        float *rstd = sm.rstd;
         for (int c = 0; ok && c < nchunks; ++c) {
             const int sl = c & 3;
             const uint32_t cU = (c & 1) ? kColU1 : kColU0, cX = (c & 1) ? kColX1 : kColX0;
             const uint32_t cO = cX + 64;
-            // ---- U pass: S *= gamma_C once MMA 2 is done; then, once MMA 2b is done,
-            //      U -> tf32 (in place) and U diag(gamma_C/gamma) -> tf32 into the
-            //      X columns (MMA 2b has read them)
+            // ---- once MMA 2 is done: S *= gamma_C and O^T *= diag(gamma) (MMA 2 left
+            //      S0 Q^T there; MMA 3 adds U^T P^T), beside MMA 2b, which touches
+            //      neither; then, once MMA 2b is done, U -> tf32 in place (the A
+            //      operand of both parts of MMA 3)
             {
                 bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
-                // S *= gamma_C as soon as MMA 2 (the last reader of S0) is done,
-                // beside MMA 2b, which does not touch S
                 good = waitq(bar_m2, c & 1) && good;
                 good = __all_sync(0xffffffffu, good); // TMEM loads are warp-wide
                 tc_fence_after();
                 if (good) {
                     const float gC = expf(sm.G[sl][kC - 1]); // padded rows carry g = 0
+                    // three rounds of two TMEM loads in flight: S columns 0..31 and
+                    // 32..63 of this half, then O rows r = 32 hf + 16 q + i
 #pragma unroll 1
-                    for (int q = 0; q < 4; ++q) {
-                        float v[16];
-                        tmem_ld16(tl + kColS + 64 * hf + 16 * q, v);
+                    for (int rd = 0; rd < 3; ++rd) {
+                        float v[2][16];
+                        const uint32_t col = rd < 2 ? kColS + 64 * hf + 32 * rd : cO + 32 * hf;
+                        tmem_ld16(tl + col, v[0]);
+                        tmem_ld16(tl + col + 16, v[1]);
                         tmem_wait_ld();
+                        if (rd < 2) {
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            v[i] *= gC;
-                        tmem_st16(tl + kColS + 64 * hf + 16 * q, v);
+                            for (int i = 0; i < 16; ++i) {
+                                v[0][i] *= gC;
+                                v[1][i] *= gC;
+                            }
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 2; ++q)
+#pragma unroll
+                                for (int i = 0; i < 16; i += 4) {
+                                    const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][32 * hf + 16 * q + i]);
+                                    v[q][i] *= g4.x; v[q][i + 1] *= g4.y;
+                                    v[q][i + 2] *= g4.z; v[q][i + 3] *= g4.w;
+                                }
+                        }
+                        tmem_st16(tl + col, v[0]);
+                        tmem_st16(tl + col + 16, v[1]);
                     }
                 }
                 good = waitq(bar_m2b(c), (c >> 1) & 1) && good;
                 good = __all_sync(0xffffffffu, good);
                 tc_fence_after();
                 if (good) {
-#pragma unroll 1
-                    for (int q = 0; q < 2; ++q) {
-                        float u[16], uk[16];
-                        tmem_ld16(tl + cU + 32 * hf + 16 * q, u);
+                    float u[2][16];
+                    tmem_ld16(tl + cU + 32 * hf, u[0]);
+                    tmem_ld16(tl + cU + 32 * hf + 16, u[1]);
+                    tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; i += 4) {
-                            const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kd[sl][32 * hf + 16 * q + i]);
-                            uk[i] = k4.x; uk[i + 1] = k4.y; uk[i + 2] = k4.z; uk[i + 3] = k4.w;
-                        }
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            uk[i] = tf32_rna(u[i] * uk[i]);
-                            u[i] = tf32_rna(u[i]);
-                        }
-                        tmem_st16(tl + cU + 32 * hf + 16 * q, u);
-                        tmem_st16(tl + cX + 32 * hf + 16 * q, uk);
+                    for (int i = 0; i < 16; ++i) {
+                        u[0][i] = tf32_rna(u[0][i]);
+                        u[1][i] = tf32_rna(u[1][i]);
                     }
-                    tmem_wait_st();
+                    tmem_st16(tl + cU + 32 * hf, u[0]);
+                    tmem_st16(tl + cU + 32 * hf + 16, u[1]);
                 }
+                tmem_wait_st();
                 tc_fence_before();
                 if (group_sync_or(kBarSG, kSG, !good || *abort_flag)) {
                     ok = false;
@@ -421,6 +441,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             {
                 const int64_t t0 = start + (int64_t)c * kC;
                 const int rows = rows_of(c) - 32 * hf; // valid rows of this half (may be <= 0)
+                const bool full = rows_of(c) == kC;
                 // the gate w[v] SiLU(z) does not depend on the state: form it while
                 // MMA 3 runs
                 float gt[32];
@@ -439,7 +460,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
 #pragma unroll
                 for (int i = 0; i < 32; ++i)
                     gt[i] = wn * __fdividef(gt[i], 1.0f + __expf(-gt[i]));
-                group_sync(kBarSG, kSG); // the z tile is read: its head takes the sums below
+                group_sync(kBarSG, kSG); // the z tile is read: it takes the y rows below
                 bool good = zok && __all_sync(0xffffffffu, waitp(bar_m3, ph3));
                 tc_fence_after();
                 float o[32];
@@ -479,16 +500,26 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
 #pragma unroll
                     for (int i = 0; i < 32; ++i) // o * rstd * w * SiLU(z)
                         o[i] = o[i] * rstd[32 * hf + i] * gt[i];
-                    T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
-                    if (rows >= 32) {
+                    if (kZTile && full) { // y rows into the z tile, then one TMA store
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
-                            st_cg(yp + i * HD, o[i]);
+                            reinterpret_cast<__nv_bfloat16 *>(sm.Z)[(32 * hf + i) * kD + vch] =
+                                __float2bfloat16_rn(o[i]);
                     } else {
+                        T *yp = (T *)p.y + (t0 + 32 * hf) * HD + (int64_t)h * kD + vch;
 #pragma unroll
                         for (int i = 0; i < 32; ++i)
                             if (i < rows)
                                 st_cg(yp + i * HD, o[i]);
+                    }
+                }
+                if (kZTile && full) {
+                    fence_proxy_async_smem();
+                    group_sync(kBarSG, kSG);
+                    if (tid == 0 && good) {
+                        tma_store_2d(&maps.y, h * kD, (int)t0, smem_u32(sm.Z));
+                        bulk_commit();
+                        bulk_wait_read(); // the z tile may take the next chunk's rows
                     }
                 }
                 tc_fence_before();
@@ -772,39 +803,36 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     } else if (warp < (kSG + kTeam + kTeamP) / 32) {
         // ==================================================== P team
         const int pt = tid - kSG - kTeam;
-        uint32_t phq = 0, phqk = 0;
+        uint32_t phk = 0, phqk = 0;
         for (int c = 0; c < nchunks; ++c) {
             const int sl = c & 3;
-            // ---- diag(gamma) Q in place (rows 64..127 of KQ)
+            // ---- diag(gamma_C / gamma) K in place on the MN-major K tile (the B operand
+            //      of MMA 3's state part), tf32: token row s of every 32-column
+            //      block is 32 consecutive floats (their 32-byte chunks swizzled
+            //      within the row), all scaled by kd[s]
             bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
-            good = waitp(bar_q, phq) && good;
+            good = waitp(bar_k, phk) && good;
             if (good) {
+                // eight float4s in flight a thread: the pass is latency-bound otherwise
 #pragma unroll 1
-                for (int half = 0; half < 16; ++half) {
-                    float4 x[2];
-                    float gr[2];
-                    int off[2];
+                for (int it = 0; it < 4; ++it) {
+                    float4 x[8];
 #pragma unroll
-                    for (int jj = 0; jj < 2; ++jj) {
-                        const int f = pt + kTeamP * (2 * half + jj), r = f >> 5, cb = (f >> 3) & 3;
-                        off[jj] = cb * (2 * kC * 32) + (kC + r) * 32 + (((f & 7) ^ (r & 7)) << 2);
-                        x[jj] = *reinterpret_cast<const float4 *>(sm.KQ + off[jj]);
-                        gr[jj] = sm.gam[sl][r];
+                    for (int jj = 0; jj < 8; ++jj)
+                        x[jj] = *reinterpret_cast<const float4 *>(sm.K + 4 * (pt + kTeamP * (8 * it + jj)));
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        const int e = pt + kTeamP * (8 * it + jj); // float4 index 0..2047
+                        const float f = sm.kd[sl][(e >> 3) & (kC - 1)];
+                        *reinterpret_cast<float4 *>(sm.K + 4 * e) =
+                            tf32_rna(make_float4(x[jj].x * f, x[jj].y * f, x[jj].z * f, x[jj].w * f));
                     }
-#pragma unroll
-                    for (int jj = 0; jj < 2; ++jj)
-                        *reinterpret_cast<float4 *>(sm.KQ + off[jj]) =
-                            tf32_rna(make_float4(x[jj].x * gr[jj], x[jj].y * gr[jj], x[jj].z * gr[jj],
-                                                 x[jj].w * gr[jj]));
                 }
             }
-            fence_proxy_async_smem();
             if (group_sync_or(kBarP, kTeamP, !good || *abort_flag)) {
                 ok = false;
                 break;
             }
-            if (pt == 0)
-                mbar_arrive(bar_pQ);
             // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32
             good = waitp(bar_qk, phqk);
             if (good) {
@@ -813,31 +841,24 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 // r mod 8, so the swizzle term is one constant per thread
                 const int prow = pt >> 3, pcol = 4 * (pt & 7);
                 const int pbase = prow * 32 + (((pt & 7) ^ (prow & 7)) << 2);
-#pragma unroll 1
-                for (int half = 0; half < 12; ++half) {
-                    float4 x[1];
+                // six float4s in flight a round: the pass is latency-bound otherwise
 #pragma unroll
-                    for (int jj = 0; jj < 1; ++jj) {
-                        const int k = half + jj;
-                        x[jj] = *reinterpret_cast<const float4 *>(
-                            sm.P + pbase + (k < 8 ? 256 * k : 2048 + 256 * (k - 8)));
-                    }
+                for (int h6 = 0; h6 < 12; h6 += 6) {
+                    float4 x[6];
 #pragma unroll
-                    for (int jj = 0; jj < 1; ++jj) {
-                        const int k = half + jj;
-                        const float Gr = sm.G[sl][k < 8 ? prow + 8 * k : 32 + prow + 8 * (k - 8)];
-                        const float4 Gc =
-                            *reinterpret_cast<const float4 *>(&sm.G[sl][k < 8 ? pcol : 32 + pcol]);
-                        x[jj] = tf32_rna(make_float4(x[jj].x * __expf(fminf(Gr - Gc.x, 0.f)),
-                                                     x[jj].y * __expf(fminf(Gr - Gc.y, 0.f)),
-                                                     x[jj].z * __expf(fminf(Gr - Gc.z, 0.f)),
-                                                     x[jj].w * __expf(fminf(Gr - Gc.w, 0.f))));
-                    }
+                    for (int k = 0; k < 6; ++k)
+                        x[k] = *reinterpret_cast<const float4 *>(
+                            sm.P + pbase + (h6 + k < 8 ? 256 * (h6 + k) : 2048 + 256 * (h6 + k - 8)));
 #pragma unroll
-                    for (int jj = 0; jj < 1; ++jj) {
-                        const int k = half + jj;
-                        *reinterpret_cast<float4 *>(sm.P + pbase +
-                                                    (k < 8 ? 256 * k : 2048 + 256 * (k - 8))) = x[jj];
+                    for (int k = 0; k < 6; ++k) {
+                        const int kk = h6 + k;
+                        const float Gr = sm.G[sl][kk < 8 ? prow + 8 * kk : 32 + prow + 8 * (kk - 8)];
+                        const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][kk < 8 ? pcol : 32 + pcol]);
+                        *reinterpret_cast<float4 *>(sm.P + pbase + (kk < 8 ? 256 * kk : 2048 + 256 * (kk - 8))) =
+                            tf32_rna(make_float4(x[k].x * __expf(fminf(Gr - Gc.x, 0.f)),
+                                                 x[k].y * __expf(fminf(Gr - Gc.y, 0.f)),
+                                                 x[k].z * __expf(fminf(Gr - Gc.z, 0.f)),
+                                                 x[k].w * __expf(fminf(Gr - Gc.w, 0.f))));
                     }
                 }
             }
@@ -853,7 +874,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             *abort_flag = 1;
     } else if (warp == kWarpMma) {
         // ==================================================== MMA issue
-        if (lane == 0 && nchunks > 0) {
+        // The whole warp runs this loop in uniform control flow (so the
+        // descriptor arithmetic stays warp-uniform) and the elected lane issues
+        // the MMAs and commits; every decision is taken by all lanes alike.
+        if (nchunks > 0) {
+            const uint32_t is = elect_one();
+            auto all = [&](bool g) { return __all_sync(0xffffffffu, g) != 0; };
             const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.V), kC * 128, 512);
             const uint64_t dK = sdesc_sw128_b32(smem_u32(sm.K), kC * 128, 512);
             const uint64_t dKQ = sdesc_sw128(smem_u32(sm.KQ), 16, 1024);
@@ -869,7 +895,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             constexpr uint32_t idT64 = idesc_tf32(128, 64, false, false);  // MMA 2b, MMA 3 O
             constexpr uint32_t idT32 = idesc_tf32(128, 32, false, false);
             constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3 S (B MN-major)
-            uint32_t phv = 0, phkm = 0, phk = 0, phQ = 0, phu = 0, phP = 0, ph2 = 0;
+            uint32_t phv = 0, phkm = 0, phq = 0, phu = 0, phP = 0, ph2 = 0;
             // MMA 1 of chunk c: U~^T into U_(c%2).  K steps 0..3 run over column
             // block 0 of the T tile (N = 64), 4..7 over block 1 (rows 32..63)
             auto mma1 = [&](int c) {
@@ -877,21 +903,26 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 const uint64_t b0 = tb0(c), b1 = tb1(c);
 #pragma unroll 1
                 for (int s = 0; s < 4; ++s)
-                    mma_tf32_ss(dU, dV + s * 64, b0 + 2 * s, id64, s > 0);
+                    mma_tf32_ss_if(dU, dV + s * 64, b0 + 2 * s, id64, s > 0, is);
 #pragma unroll 1
                 for (int s = 4; s < 8; ++s)
-                    mma_tf32_ss(dU + 32, dV + s * 64, b1 + 2 * (s - 4), id32, 1);
-                mma_commit(bar_m1);
+                    mma_tf32_ss_if(dU + 32, dV + s * 64, b1 + 2 * (s - 4), id32, 1, is);
+                mma_commit_if(bar_m1, is);
             };
-            // the inputs of MMA 1 of chunk c: its T tiles (and gates) and V
+            // the inputs of MMA 1 of chunk c: its T tiles (and gates) and V; the
+            // non-blocking form takes lane 0's view, so that all lanes agree
             auto m1_ready = [&](int c, bool block) {
                 if (!block)
-                    return mbar_test_wait(bar_pT(c), (c >> 2) & 1) && mbar_test_wait(bar_v, phv);
+                    return __shfl_sync(0xffffffffu,
+                                       (int)(mbar_test_wait(bar_pT(c), (c >> 2) & 1) &&
+                                             mbar_test_wait(bar_v, phv)),
+                                       0) != 0;
                 bool g = waitq(bar_pT(c), (c >> 2) & 1);
                 g = g && waitq(bar_v, phv);
-                return g;
+                return all(g);
             };
-            bool good = m1_ready(0, true) && waitp(bar_u, phu); // phase 0 of U: the initial state
+            bool good = m1_ready(0, true);
+            good = all(waitp(bar_u, phu) && good); // phase 0 of U: the initial state
             phv ^= 1u;
             tc_fence_after();
             if (good)
@@ -899,23 +930,23 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             for (int c = 0; good && c < nchunks; ++c) {
                 const uint32_t dXO = tmem + ((c & 1) ? kColX1 : kColX0);
                 const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0);
-                // ---- MMA 2: [X^T | O^T] = S [K; diag(gamma) Q]^T (A = the state in TMEM)
-                good = waitp(bar_pQ, phQ);
-                good = good && waitp(bar_kmaj, phkm);
+                // ---- MMA 2: [X^T | O^T] = S [K; Q]^T (A = the state in TMEM)
+                good = waitp(bar_q, phq);
+                good = waitp(bar_kmaj, phkm) && good;
                 if (c >= 2)
-                    good = good && ((c & 1) ? waitq(bar_of1, ((c >> 1) - 1) & 1)
-                                            : waitq(bar_of0, ((c >> 1) - 1) & 1));
-                if (!good)
+                    good = ((c & 1) ? waitq(bar_of1, ((c >> 1) - 1) & 1)
+                                    : waitq(bar_of0, ((c >> 1) - 1) & 1)) && good;
+                if (!all(good))
                     break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int s = 0; s < kD / 8; ++s) {
                     const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ts(dXO, tmem + kColS + 8 * s, dKQ + ks, id128, s > 0);
+                    mma_tf32_ts_if(dXO, tmem + kColS + 8 * s, dKQ + ks, id128, s > 0, is);
                 }
-                mma_commit(bar_m2);
+                mma_commit_if(bar_m2, is);
                 // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
-                good = waitp(bar_m2, ph2);
+                good = all(waitp(bar_m2, ph2));
                 if (!good)
                     break;
                 tc_fence_after();
@@ -923,12 +954,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     const uint64_t g0 = tg0(c), g1 = tg1(c);
 #pragma unroll 1
                     for (int s = 0; s < 4; ++s)
-                        mma_tf32_ts(dU, dXO + 8 * s, g0 + 2 * s, idT64, 1);
+                        mma_tf32_ts_if(dU, dXO + 8 * s, g0 + 2 * s, idT64, 1, is);
 #pragma unroll 1
                     for (int s = 4; s < 8; ++s)
-                        mma_tf32_ts(dU + 32, dXO + 8 * s, g1 + 2 * (s - 4), idT32, 1);
+                        mma_tf32_ts_if(dU + 32, dXO + 8 * s, g1 + 2 * (s - 4), idT32, 1, is);
                 }
-                mma_commit(bar_m2b(c));
+                mma_commit_if(bar_m2b(c), is);
                 // ---- MMA 1 of the next chunk beside the U pass, if its inputs are in
                 //      (its U buffer was last read by MMA 3 of chunk c - 1)
                 bool m1_issued = false;
@@ -938,26 +969,25 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     mma1(c + 1);
                     m1_issued = true;
                 }
-                // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K
+                // ---- MMA 3: O^T += U^T P^T, S += U^T (diag(gamma_C/gamma) K) (K MN-major)
                 good = waitp(bar_u, phu);
-                good = good && waitp(bar_pP, phP);
-                good = good && waitp(bar_k, phk);
-                if (!good)
+                good = waitp(bar_pP, phP) && good; // P and the scaled K tile
+                if (!all(good))
                     break;
                 tc_fence_after();
                 {
                     const uint32_t dO = dXO + 64;
 #pragma unroll 1
                     for (int s = 0; s < 4; ++s)
-                        mma_tf32_ts(dO, dU + 8 * s, dP0 + 2 * s, idT64, 1);
+                        mma_tf32_ts_if(dO, dU + 8 * s, dP0 + 2 * s, idT64, 1, is);
 #pragma unroll 1
                     for (int s = 4; s < 8; ++s)
-                        mma_tf32_ts(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1);
+                        mma_tf32_ts_if(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1, is);
 #pragma unroll 1
                     for (int s = 0; s < kC / 8; ++s)
-                        mma_tf32_ts(tmem + kColS, dXO + 8 * s, dK + s * 64, idS, 1);
+                        mma_tf32_ts_if(tmem + kColS, dU + 8 * s, dK + s * 64, idS, 1, is);
                 }
-                mma_commit(bar_m3);
+                mma_commit_if(bar_m3, is);
                 if (c + 1 < nchunks && !m1_issued) {
                     good = m1_ready(c + 1, true);
                     phv ^= 1u;
@@ -973,7 +1003,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 *abort_flag = 1;
                 uint32_t phx = 0;
                 const uint32_t bar_x = smem_u32(&sm.bar_fin);
-                mma_commit(bar_x);
+                mma_commit_if(bar_x, is);
                 mbar_wait_bounded(bar_x, phx, kWaitLimit);
             }
         }
@@ -1064,7 +1094,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 if (prog) {
                     t_last = clock64();
-                } else if (clock64() - t_last > kWaitLimit || *abort_flag) {
+                } else if (clock64() - t_last > p.wait_limit || *abort_flag) {
                     ok = false;
                     break;
                 } else {
@@ -1081,6 +1111,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         }
     }
 
+    if (tid == 0)
+        bulk_wait_all(); // the epilogue's y stores are complete
     ok = !__syncthreads_or(!ok); // one verdict for the whole CTA
     if (!ok) {
         if (tid == 0 && p.ws_err != nullptr)
@@ -1129,8 +1161,10 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
             encode_2d(&maps.kq, p.ws_kq, kqw, N, kqw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&maps.kq32, p.ws_kq, kqw, N, kqw * F, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
             (sizeof(T) != 2 ||
-             encode_2d(&maps.z, p.z, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * sizeof(T), kD, kC,
-                       CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16));
+             (encode_2d(&maps.z, p.z, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * sizeof(T), kD, kC,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) &&
+              encode_2d(&maps.y, p.y, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * sizeof(T), kD, kC,
+                        CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)));
         if (!okm)
             return cudaErrorInvalidValue;
     }
@@ -1144,7 +1178,9 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * 2 * kC * sizeof(float); }
 
 cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s) {
-    if (p.batch == 0)
+    // no tokens: no workspace (the offsets and status words have no home) and
+    // no chunk to count; the chunk kernel then only passes the states through
+    if (p.batch == 0 || p.N == 0)
         return cudaSuccess;
     chunk_offsets_kernel<<<1, 1024, 0, s>>>(p.cu, p.batch, p.N, p.ws_offs, p.ws_err);
     return cudaGetLastError();

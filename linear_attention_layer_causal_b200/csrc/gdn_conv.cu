@@ -1,6 +1,8 @@
-// gdn_conv.cu -- prefill front end: conv + SiLU + L2 norm of every q|k|v
-// channel (the per-thread body is in gdn_conv.cuh), and the final conv window
-// of every sequence.
+// gdn_conv.cu -- prefill front end: conv + SiLU (+ L2 norm of q and k) of the
+// pre-conv channels (the per-thread body is in gdn_conv.cuh) -- every channel
+// for the token-serial path, the v channels for the tensor-core path, whose q
+// and k go through the fused q/k front kernel -- and the final conv window of
+// every sequence.
 #include "gdn_conv.cuh"
 #include "gdn_internal.h"
 
@@ -20,17 +22,20 @@ __global__ void __launch_bounds__(kConvThreads, sizeof(VecT) == 8 ? 4 : 1) // 8-
 conv_prep_kernel(ConvIO<T> io, unsigned int *__restrict__ err) {
     constexpr int V = VecT::N;
     const int C = (2 * io.Hk + io.Hv) * D;
-    if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    // on the token-serial path this is the first kernel of a call: it clears the
+    // call's status words (the chunked path clears them in its offsets kernel)
+    if (err != nullptr && !io.v_only && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         err[0] = 0u; // status word of this call; later kernels only set bits
         err[1] = 0u; // where the first timed-out wait gave up
     }
-    const int c0 = (blockIdx.y * kConvThreads + threadIdx.x) * V;
+    const int by = (int)blockIdx.y + io.block_y0;
+    const int c0 = (by * kConvThreads + threadIdx.x) * V;
     const bool active = c0 < C;
     const int64_t t0 = (int64_t)blockIdx.x * kConvTokens;
     const int64_t tend = t0 + kConvTokens < io.N ? t0 + kConvTokens : io.N;
     const int n = seq_of_token(io.cu, io.batch, t0 < io.N ? t0 : io.N - 1);
     // a block whose channels all lie in v skips the norm code (uniform branch)
-    if ((int)blockIdx.y * kConvThreads * V >= 2 * io.Hk * D)
+    if (by * kConvThreads * V >= 2 * io.Hk * D)
         conv_thread<T, D, true, VecT>(io, active ? c0 : 2 * io.Hk * D, active, t0, tend, n);
     else
         conv_thread<T, D, false, VecT>(io, active ? c0 : 0, active, t0, tend, n);
@@ -81,6 +86,8 @@ ConvIO<T> conv_io(const PrefillArgs &p) {
     io.qk_out = (float *)p.ws_qk;
     io.v_out = (float *)p.ws_v;
     io.round_v = p.chunked;
+    io.v_only = false;
+    io.block_y0 = 0;
     return io;
 }
 
@@ -88,9 +95,17 @@ template <typename T, int D, typename VecT = Vec16<T>>
 cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
     constexpr int V = VecT::N;
     const int C = (2 * p.Hk + p.Hv) * D;
-    dim3 grid((unsigned)((p.N + kConvTokens - 1) / kConvTokens),
-              (C / V + kConvThreads - 1) / kConvThreads);
-    conv_prep_kernel<T, D, VecT><<<grid, kConvThreads, 0, s>>>(conv_io<T>(p), p.ws_err);
+    ConvIO<T> io = conv_io<T>(p);
+    // the tensor-core path takes q and k from the fused q/k front kernel: only
+    // the blocks holding v channels run, and a block that straddles the q/k | v
+    // boundary writes only its v channels
+    if (p.chunked) {
+        io.v_only = true;
+        io.block_y0 = 2 * p.Hk * D / V / kConvThreads;
+    }
+    const int nby = (C / V + kConvThreads - 1) / kConvThreads - io.block_y0;
+    dim3 grid((unsigned)((p.N + kConvTokens - 1) / kConvTokens), nby);
+    conv_prep_kernel<T, D, VecT><<<grid, kConvThreads, 0, s>>>(io, p.ws_err);
     return cudaGetLastError();
 }
 

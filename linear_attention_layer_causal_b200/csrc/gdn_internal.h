@@ -5,6 +5,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "gdn.h"
+
 namespace gdn {
 
 struct PrefillArgs {
@@ -23,6 +25,7 @@ struct PrefillArgs {
     float *o_raw;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
     bool chunked;            // tensor-core chunked path (head_dim 128) or token-serial
+    long long wait_limit;    // SM cycles a wait between warps may take before the call aborts
     // workspace carve-up
     unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)
     void *ws_qk;             // [N, 2*Hk*D] float32: normalised q | k
@@ -41,13 +44,37 @@ struct DecodeArgs {
     int batch;
     void *y;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
+    int k = 1;                         // tokens per sequence (multi-token decode)
+    const int32_t *accepted = nullptr; // [batch] tokens to take (commit mode)
 };
+
+// Multi-token decode: modes and the most tokens per sequence one call takes.
+constexpr int kDecodeMulti = 0, kDecodeVerify = 1, kDecodeCommit = 2;
+constexpr int kDecodeMaxTokens = 8;
+constexpr size_t kDecodeMaxSmem = 227 * 1024;
 
 // One-shot events around the main kernel of the next call on this host thread.
 struct ProfileHook {
     cudaEvent_t begin = nullptr, end = nullptr;
 };
 ProfileHook take_profile_hook(); // returns the armed events and disarms
+
+// Default bound of a wait between the warps of a kernel (about one second of
+// SM clock), and the one-shot override of the calling host thread (armed by
+// gdn_wait_limit_next_call): returns the limit for this call and disarms.
+constexpr long long kDefaultWaitLimit = 2000000000LL;
+long long take_wait_limit();
+
+// The argument checks of gdn_prefill, in its order, minus the workspace; on
+// success *need holds the workspace bytes the call requires.
+gdn_status validate_prefill(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                            const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                            int32_t batch, int64_t total_tokens, const float *initial_state,
+                            const void *initial_conv, const void *y, const float *final_state,
+                            const void *final_conv, const float *o_raw, size_t *need);
+
+// Reads the two status words at `header` (device) after `stream` completes.
+gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t stream);
 
 // Records `ev` on `s` when it is non-null.
 inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
@@ -62,9 +89,11 @@ cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_final_conv(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_recurrent_prefill(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s);
-cudaError_t launch_kq_prep(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_qk_front(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_chunk_prefill(const PrefillArgs &p, cudaStream_t s);
 size_t kq_workspace_bytes(int Hk, int64_t N);
 cudaError_t launch_decode(const DecodeArgs &p, cudaStream_t s);
+cudaError_t launch_decode_multi(const DecodeArgs &p, int mode, cudaStream_t s);
+size_t decode_multi_smem_bytes(int G, int D, int k, int mode);
 
 } // namespace gdn

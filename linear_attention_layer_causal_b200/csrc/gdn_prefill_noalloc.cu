@@ -59,10 +59,13 @@ extern "C" gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_param
                                           int64_t total_tokens, const float *initial_state,
                                           const void *initial_conv, void *y, float *final_state,
                                           void *final_conv, float *o_raw, void *stream) {
-    // Size check on the host first: a call that needs more than the fixed
-    // array is rejected before any CUDA call.
+    // The argument checks of gdn_prefill first (same codes, same order), then
+    // the size check: a call that needs more than the fixed array is rejected
+    // before any CUDA call.
     size_t need = 0;
-    gdn_status st = gdn_prefill_workspace_size(cfg, batch, total_tokens, &need);
+    gdn_status st = gdn::validate_prefill(cfg, params, qkv, a, b, z, cu_seqlens, batch,
+                                          total_tokens, initial_state, initial_conv, y,
+                                          final_state, final_conv, o_raw, &need);
     if (st != GDN_OK)
         return st;
     if (need > kScratchBytes)
@@ -70,10 +73,27 @@ extern "C" gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_param
     void *scratch = nullptr;
     if (need > 0 && (st = scratch_on_current_device(&scratch)) != GDN_OK)
         return st;
-    // Nothing in the scratch has to start at zero: the conv kernel writes
-    // every element the recurrence later reads, so the previous call's
-    // contents never leak into this one.
+    // Nothing in the scratch has to start at zero: the first kernel of the
+    // call clears the status words, and the front-end kernels write every
+    // element the recurrence later reads, so the previous call's contents
+    // never leak into this one.
     return gdn_prefill(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens, initial_state,
                        initial_conv, y, final_state, final_conv, o_raw, scratch,
                        scratch ? kScratchBytes : 0, stream);
+}
+
+extern "C" gdn_status gdn_prefill_noalloc_status(uint32_t *detail, void *stream) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0)
+        return GDN_ERR_CUDA;
+    void *addr = nullptr;
+    if (dev < kMaxDevices) {
+        std::lock_guard<std::mutex> lock(g_scratch_mu);
+        addr = g_scratch_addr[dev];
+    }
+    if (detail != nullptr)
+        *detail = 0u;
+    if (addr == nullptr) // no gdn_prefill_noalloc call has used the array on this device
+        return GDN_OK;
+    return gdn::read_status_words(addr, detail, (cudaStream_t)stream);
 }

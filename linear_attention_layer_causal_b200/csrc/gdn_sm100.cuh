@@ -83,6 +83,22 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
                  : "memory");
 }
 
+// 2-D tiled TMA store of the shared-memory tile at `src` to the box at (x, y)
+// of `tmap` (bulk-group completion).  x, y >= 0; x times the element size a
+// multiple of 16 bytes.  Elements outside the tensor are not written.
+__device__ __forceinline__ void tma_store_2d(const void *tmap, int x, int y, uint32_t src) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(tmap),
+                 "r"(x), "r"(y), "r"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until every committed bulk store of this thread has read its shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+// Wait until every committed bulk store of this thread has completed.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Asynchronous 16-byte global -> shared copy; with zfill the destination is
 // zero-filled and nothing is read.
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool zfill) {
@@ -255,10 +271,51 @@ __device__ __forceinline__ void mma_tf32_ts(uint32_t d_tmem, uint32_t a_tmem, ui
                  : "memory");
 }
 
+// The same two products, issued only where `issue` is nonzero: a whole warp runs
+// the issue loop in uniform control flow (so that the descriptors stay
+// warp-uniform) and one elected lane passes issue = 1.
+__device__ __forceinline__ void mma_tf32_ss_if(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate, uint32_t issue) {
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "setp.ne.b32 q, %5, 0;\n\t"
+                 "@q tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(issue)
+                 : "memory");
+}
+__device__ __forceinline__ void mma_tf32_ts_if(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate, uint32_t issue) {
+    asm volatile("{\n\t.reg .pred p, q;\n\t"
+                 "setp.ne.b32 p, %4, 0;\n\t"
+                 "setp.ne.b32 q, %5, 0;\n\t"
+                 "@q tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+                 "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(issue)
+                 : "memory");
+}
+
+// 1 on one lane of the (fully active) warp, 0 on the others.
+__device__ __forceinline__ uint32_t elect_one() {
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "elect.sync _|p, 0xffffffff;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(r));
+    return r;
+}
+
 // Arrive on the mbarrier once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                      bar)
+                 : "memory");
+}
+
+// mma_commit where `issue` is nonzero (the elected lane of an issuing warp).
+__device__ __forceinline__ void mma_commit_if(uint32_t bar, uint32_t issue) {
+    asm volatile("{\n\t.reg .pred q;\n\t"
+                 "setp.ne.b32 q, %1, 0;\n\t"
+                 "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}"
+                 ::"r"(bar), "r"(issue)
                  : "memory");
 }
 

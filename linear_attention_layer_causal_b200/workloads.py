@@ -7,9 +7,12 @@ inputs from here, so that both sides see identical bytes.
 Shapes are the layer shapes the pages give: the Qwen3.8 Gated DeltaNet layer
 (16 q/k heads, 128 value heads, head dim 128, conv kernel 4; "Qwen3.8 2.4T
 A95B", raw config fields linear_num_key_heads, linear_num_value_heads,
-linear_key_head_dim, linear_value_head_dim, linear_conv_kernel_dim) and the
+linear_key_head_dim, linear_value_head_dim, linear_conv_kernel_dim), the
 Qwen3.6-35B-A3B linear layer (16 key heads, 32 value heads; same page,
-field-level comparison table).  No public dataset is involved.
+field-level comparison table) and the Qwen3.5-397B-A17B Gated DeltaNet layer
+(16 q/k heads, 64 value heads, 4 per q/k head; "Qwen3.5-397B-A17B vs
+Inkling", component table, Gated DeltaNet row).  No public dataset is
+involved.
 
 Distributions (all draws from one seeded generator, in the order listed):
   sequence lengths (varlen only) ~ integer U[lo, hi]
@@ -20,6 +23,13 @@ Distributions (all draws from one seeded generator, in the order listed):
   norm_w                        = 1 + 0.1 N(0, 1)
   initial states                ~ N(0, 0.02^2) (where the workload has them)
   conv cache (decode)           ~ N(0, 1), activation dtype
+
+Long-memory gates (gates="long_memory:<dt_bias>"): A_log = 0 and dt_bias =
+the given constant instead of the draws above, and b ~ N(2, 0.5^2), so that
+g = -softplus(a + dt_bias) is small (about -0.018 per token at dt_bias = -4,
+-3e-4 at -8) and beta = sigmoid(b) is about 0.88: the state keeps its past
+for hundreds to thousands of tokens, where the default draws (exp(A_log) in
+[1, 16]) forget within a few tokens.
 """
 from __future__ import annotations
 
@@ -42,6 +52,7 @@ class Workload:
     state_every: int = 1                 # sequences n with n % state_every == 0 get a state
     seed: int = 0
     conv_kernel: int = 4
+    gates: str = "default"               # or "long_memory:<dt_bias>" (see the module docstring)
     notes: str = field(default="", compare=False)
 
     @property
@@ -69,7 +80,22 @@ QWEN36_VARLEN = Workload("qwen36_varlen", 16, 32, 128, varlen=(64, 256, 8192), s
                          state_every=2, seed=1004,
                          notes="Qwen3.6-35B-A3B linear-layer shape, 64 packed sequences")
 
-WORKLOADS = {w.name: w for w in (TINY, QWEN38_PREFILL, QWEN38_LONG, QWEN38_DECODE, QWEN36_VARLEN)}
+# Beyond the five: the Qwen3.5-397B-A17B layer shape (G = 4), and long-memory
+# gates at the Qwen3.8 shape.
+QWEN35_PREFILL = Workload("qwen35_prefill", 16, 64, 128, seqlens=(4096, 4096), state_std=0.02,
+                          seed=1005, notes="Qwen3.5-397B-A17B layer prefill, B=2 T=4096")
+QWEN35_DECODE = Workload("qwen35_decode", 16, 64, 128, decode_batch=256, state_std=0.02,
+                         seed=1006, notes="Qwen3.5-397B-A17B layer decode, 256 sequences")
+QWEN38_LONG_MEMORY = Workload("qwen38_long_memory", 16, 128, 128, seqlens=(16384,) * 3,
+                              state_std=0.02, seed=1007, gates="long_memory:-4",
+                              notes="Qwen3.8 layer, B=3 T=16384, slowly decaying state")
+QWEN38_VERY_LONG_MEMORY = Workload("qwen38_very_long_memory", 16, 128, 128, seqlens=(16384,) * 3,
+                                   state_std=0.02, seed=1008, gates="long_memory:-8",
+                                   notes="Qwen3.8 layer, B=3 T=16384, nearly undecaying state")
+
+WORKLOADS = {w.name: w for w in (TINY, QWEN38_PREFILL, QWEN38_LONG, QWEN38_DECODE, QWEN36_VARLEN,
+                                 QWEN35_PREFILL, QWEN35_DECODE, QWEN38_LONG_MEMORY,
+                                 QWEN38_VERY_LONG_MEMORY)}
 
 
 def _gen(device, seed):
@@ -91,6 +117,9 @@ def _params(wl: Workload, g, device):
     A_log = torch.log(torch.rand(H, generator=g, device=device) * 15.0 + 1.0)
     dt_bias = _normal((H,), 0.5, g, device)
     norm_w = 1.0 + _normal((wl.head_dim,), 0.1, g, device)
+    if wl.gates.startswith("long_memory"):
+        A_log.zero_()
+        dt_bias.fill_(float(wl.gates.split(":")[1]))
     return {"conv_w": conv_w.contiguous(), "A_log": A_log.contiguous(),
             "dt_bias": dt_bias.contiguous(), "norm_w": norm_w.contiguous()}
 
@@ -121,6 +150,8 @@ def make_prefill(wl: Workload, device="cpu", seqlens=None, seed=None):
     out["qkv"] = _normal((N, wl.conv_dim), 1.0, g, device, dt)
     out["a"] = _normal((N, H), 1.0, g, device, dt)
     out["b"] = _normal((N, H), 1.0, g, device, dt)
+    if wl.gates.startswith("long_memory"):
+        out["b"] = (out["b"].float() * 0.5 + 2.0).to(dt)
     out["z"] = _normal((N, H, d), 1.0, g, device, dt)
     out.update(_params(wl, g, device))
     if wl.state_std > 0:
@@ -134,21 +165,23 @@ def make_prefill(wl: Workload, device="cpu", seqlens=None, seed=None):
     return out
 
 
-def make_decode(wl: Workload, device="cpu", batch=None, seed=None):
+def make_decode(wl: Workload, device="cpu", batch=None, seed=None, tokens=None):
     """Inputs of one decode call: one new token for each of B sequences.
 
     Returns qkv [B, conv_dim], a, b [B, H_v], z [B, H_v, d], conv_cache
     [B, K-1, conv_dim] (activation dtype), state [B, H_v, d, d] float32 and the
-    float32 parameters.
+    float32 parameters.  With `tokens` = k, every sequence gets k new tokens
+    instead: qkv [B, k, conv_dim], a, b [B, k, H_v], z [B, k, H_v, d].
     """
     g = _gen(device, wl.seed if seed is None else seed)
     B = batch or wl.decode_batch
     H, d, dt = wl.num_v_heads, wl.head_dim, wl.torch_dtype
+    lead = (B,) if tokens is None else (B, tokens)
     out = {}
-    out["qkv"] = _normal((B, wl.conv_dim), 1.0, g, device, dt)
-    out["a"] = _normal((B, H), 1.0, g, device, dt)
-    out["b"] = _normal((B, H), 1.0, g, device, dt)
-    out["z"] = _normal((B, H, d), 1.0, g, device, dt)
+    out["qkv"] = _normal(lead + (wl.conv_dim,), 1.0, g, device, dt)
+    out["a"] = _normal(lead + (H,), 1.0, g, device, dt)
+    out["b"] = _normal(lead + (H,), 1.0, g, device, dt)
+    out["z"] = _normal(lead + (H, d), 1.0, g, device, dt)
     out.update(_params(wl, g, device))
     out["state"] = _normal((B, H, d, d), wl.state_std if wl.state_std > 0 else 0.02, g, device)
     out["conv_cache"] = _normal((B, wl.conv_kernel - 1, wl.conv_dim), 1.0, g, device, dt)

@@ -31,12 +31,13 @@ def test_library_exports_every_declared_symbol():
     assert set(gdn.EXPORTED) <= set(declared)
     for name in declared:
         assert hasattr(L, name), f"{name} declared in include/ but not exported"
-    assert L.gdn_abi_version() == 1
+    assert L.gdn_abi_version() == 2
 
 
 def test_status_strings():
-    for s in range(5):
+    for s in range(6):
         assert gdn.status_string(s)
+    assert "wait" in gdn.status_string(gdn.GDN_ERR_TIMEOUT)
     assert gdn.status_string(99) == "unknown status"
 
 
@@ -51,6 +52,10 @@ def test_workspace_size_arithmetic():
     assert n == 256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 2 * 64 * 4 + 256
     assert gdn.prefill_workspace_size(QWEN38, 100, 4096) == n + 256  # 101 offsets: 512 bytes
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
+    # sequences but no tokens: nothing for a kernel to stage, and no workspace (the
+    # launches that would need one -- chunk offsets, status words -- are skipped)
+    assert gdn.prefill_workspace_size(QWEN38, 3, 0) == 0
+    assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 5, 0) == 0
     tiny = gdn.Config(2, 4, 32, act_dtype="f32")
     assert gdn.prefill_workspace_size(tiny, 1, 3) == 256 + 1536 + 1536
     assert gdn.prefill_workspace_size(tiny, 1, 1) == 256 + 512 + 512
@@ -141,6 +146,33 @@ def test_decode_argument_errors():
 
 
 @no_gpu
+def test_multi_token_decode_argument_errors():
+    L = gdn.lib()
+    cfg = gdn.Config(16, 128, 128)
+    par = gdn._Params(1 << 20, (1 << 20) + 256, (1 << 20) + 512, (1 << 20) + 768)
+    P = 1 << 24
+    c, p_ = ctypes.byref(cfg._c()), ctypes.byref(par)
+    # qkv, a, b, z, state, conv_cache, batch, k, y
+    ok = [P, P * 2, P * 3, P * 4, P * 5, P * 6, 3, 2, P * 7, None]
+    assert L.gdn_decode_multi(c, p_, *ok[:7], 0, *ok[8:]) == gdn.GDN_ERR_INVALID_ARG   # k = 0
+    assert L.gdn_decode_multi(c, p_, *ok[:7], 9, *ok[8:]) == gdn.GDN_ERR_UNSUPPORTED   # k > 8
+    assert L.gdn_decode_verify(c, p_, *ok[:8], None, None) == gdn.GDN_ERR_INVALID_ARG  # no y
+    assert L.gdn_decode_multi(c, p_, *ok[:7], 2, P * 7 + 8, None) == gdn.GDN_ERR_INVALID_ARG
+    # commit: qkv, a, b, state, conv_cache, batch, k, accepted
+    assert L.gdn_decode_commit(c, p_, P, P * 2, P * 3, P * 5, P * 6, 3, 2, None, None) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_decode_commit(c, p_, P, P * 2, P * 3, P * 5, P * 6, 3, 2, P * 8 + 2, None) == \
+        gdn.GDN_ERR_INVALID_ARG                                                      # misaligned
+    assert L.gdn_decode_commit(c, p_, P, P * 2, P * 3, P * 5, P * 6, 0, 2, None, None) == \
+        gdn.GDN_OK                                                                   # no sequences
+    # G = 64 at d = 128: k = 8 tokens of a group need more shared memory than a CTA has
+    wide = gdn.Config(1, 64, 128)
+    assert L.gdn_decode_multi(ctypes.byref(wide._c()), p_, *ok[:7], 8, *ok[8:]) == \
+        gdn.GDN_ERR_UNSUPPORTED
+    assert L.gdn_decode_multi(ctypes.byref(wide._c()), p_, *ok[:6], 0, 2, *ok[8:]) == gdn.GDN_OK
+
+
+@no_gpu
 def test_noalloc_rejects_oversized_calls_on_the_host():
     """The fixed-scratch prefill refuses, before any CUDA call, a call that needs
     more than GDN_NOALLOC_SCRATCH_BYTES of scratch."""
@@ -154,6 +186,37 @@ def test_noalloc_rejects_oversized_calls_on_the_host():
     bad = gdn.Config(3, 4, 32)
     assert L.gdn_prefill_noalloc(ctypes.byref(bad._c()), ctypes.byref(par), *args) == \
         gdn.GDN_ERR_INVALID_ARG
+
+
+@no_gpu
+def test_noalloc_checks_arguments_before_the_scratch_size():
+    """gdn_prefill_noalloc validates like gdn_prefill (same codes, same order) and only
+    then refuses a call that is too large for its fixed scratch."""
+    L = gdn.lib()
+    cfg = gdn.Config(16, 128, 128)
+    P = 1 << 20
+    par = gdn._Params(P, P + 256, P + 512, P + 768)
+    big = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, 100000, None, None, P * 7, None, None, None,
+           None]
+    bad_qkv = list(big)
+    bad_qkv[0] = None
+    assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *bad_qkv) == \
+        gdn.GDN_ERR_INVALID_ARG
+    misaligned = list(big)
+    misaligned[9] = P * 7 + 8  # y only 8-byte aligned
+    assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *misaligned) == \
+        gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *big) == \
+        gdn.GDN_ERR_WORKSPACE
+
+
+def test_status_query_and_wait_limit_argument_errors():
+    L = gdn.lib()
+    d = ctypes.c_uint32(7)
+    assert L.gdn_prefill_status(None, 1 << 20, ctypes.byref(d), None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_prefill_status(1 << 20, 4, ctypes.byref(d), None) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_wait_limit_next_call(-1) == gdn.GDN_ERR_INVALID_ARG
+    assert L.gdn_wait_limit_next_call(0) == gdn.GDN_OK  # disarmed
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

@@ -14,7 +14,7 @@ import torch
 import linear_attention_layer_causal_b200 as gdn
 import oracle
 from linear_attention_layer_causal_b200 import workloads as W
-from parity_util import assert_output_close, assert_state_close, to64
+from parity_util import assert_output_close, assert_state_close, report, to64
 
 pytestmark = pytest.mark.gpu
 
@@ -89,13 +89,18 @@ def test_qwen38_long_prefill_sampled(cuda_device, algo):
     torch.cuda.synchronize()
     assert torch.isfinite(out["y"].float()).all()
     cu = inp["cu_seqlens"].tolist()
-    for n, group, heads in [(0, 0, [0, 7]), (1, 9, [75]), (3, 15, [120, 127])]:
-        ref = _oracle_seq(wl, inp, n, group, heads)
+    G = wl.num_v_heads // wl.num_qk_heads
+    # one whole q/k group (all G value heads) of each of three sequences
+    for n, group in [(0, 0), (1, 9), (3, 15)]:
+        heads = list(range(group * G, (group + 1) * G))
+        ref = _oracle_seq(wl, inp, n, group)
         s, e = cu[n], cu[n + 1]
-        assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} heads {heads}")
-        assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
-        last = inp["qkv"][e - 3:e]
-        assert torch.equal(out["final_conv"][n], last)
+        r, m = assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} group {group}")
+        rs = assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
+        report(f"qwen38_long[{algo}] seq {n} group {group}", r, m, rs)
+    for n in range(len(cu) - 1):
+        e = cu[n + 1]
+        assert torch.equal(out["final_conv"][n], inp["qkv"][e - 3:e])
 
 
 def test_qwen38_decode_sampled(cuda_device):
@@ -103,7 +108,7 @@ def test_qwen38_decode_sampled(cuda_device):
     wl = W.QWEN38_DECODE
     cfg = gdn.Config.of(wl)
     inp = W.make_decode(wl, cuda_device)
-    seqs = [0, 1, 100, 255]
+    seqs = list(range(0, 256, 8)) + [1, 100, 255]
     S_before = inp["state"][seqs].cpu()
     C_before = inp["conv_cache"][seqs].cpu()
     y = gdn.decode(cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["state"],
@@ -114,8 +119,9 @@ def test_qwen38_decode_sampled(cuda_device):
            ("qkv", "a", "b", "z") + PARAMS}
     ref = oracle.decode(_shape(wl), sub["qkv"], sub["a"], sub["b"], sub["z"],
                         *[sub[k] for k in PARAMS], state=S_before, conv_cache=C_before)
-    assert_output_close(y[seqs], ref["y"])
-    assert_state_close(inp["state"][seqs], ref["state"])
+    r, m = assert_output_close(y[seqs], ref["y"])
+    rs = assert_state_close(inp["state"][seqs], ref["state"])
+    report(f"qwen38_decode ({len(seqs)} of 256 sequences)", r, m, rs)
     np.testing.assert_array_equal(to64(inp["conv_cache"][seqs]), ref["conv_window"])
 
 
@@ -131,13 +137,16 @@ def test_qwen36_varlen_sampled(cuda_device, algo):
     assert torch.isfinite(out["y"].float()).all()
     cu = inp["cu_seqlens"].tolist()
     order = np.argsort(lens)
-    picks = [(int(order[0]), 0), (int(order[-1]), 15), (2, 7), (5, 3)]  # shortest, longest, S0 / no S0
+    # shortest, longest, with and without an initial state; each pick checks one
+    # whole q/k group (both of its value heads)
+    picks = [(int(order[0]), 0), (int(order[-1]), 15), (2, 7), (5, 3), (int(order[32]), 11)]
     for n, group in picks:
         ref = _oracle_seq(wl, inp, n, group)
         s, e = cu[n], cu[n + 1]
         heads = [2 * group, 2 * group + 1]
-        assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} (len {lens[n]})")
-        assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
+        r, m = assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} (len {lens[n]})")
+        rs = assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
+        report(f"qwen36_varlen[{algo}] seq {n} len {lens[n]} group {group}", r, m, rs)
 
 
 EDGE = W.Workload("edge", 2, 4, 128, seqlens=(0, 1, 2, 3, 5, 33, 64, 0, 100, 31), state_std=0.02,
@@ -253,3 +262,113 @@ def test_split_prefill_and_decode_continue_the_sequence(cuda_device, algo):
                         mx=1e-2 if tight else 2e-2)
     assert_state_close(state, whole["final_state"], "continued state", rel=1e-4 if tight else 2e-3)
     assert torch.equal(cache[0], inp["qkv"][T - 2:T + 1])
+
+
+@ALGOS
+@pytest.mark.parametrize("wl", [W.QWEN38_LONG_MEMORY, W.QWEN38_VERY_LONG_MEMORY],
+                         ids=lambda w: w.name)
+def test_long_memory_full_groups(cuda_device, wl, algo):
+    """Slowly decaying states (A_log = 0, dt_bias = -4 or -8, beta ~ 0.88) over
+    B = 3 x T = 16384: the state carries its past across hundreds of chunks, so
+    any bias in the chunked path's operand rounding would accumulate instead of
+    being forgotten within a chunk.  One whole q/k group of each sequence,
+    element by element against the oracle, with the stated bounds."""
+    cfg = gdn.Config.of(wl, algo)
+    inp = W.make_prefill(wl, cuda_device)
+    out = _gpu_prefill(cfg, inp, return_final_state=True, return_o_raw=True)
+    torch.cuda.synchronize()
+    cu = inp["cu_seqlens"].tolist()
+    G = wl.num_v_heads // wl.num_qk_heads
+    for n, group in [(0, 3), (1, 8), (2, 14)]:
+        heads = list(range(group * G, (group + 1) * G))
+        ref = _oracle_seq(wl, inp, n, group)
+        s, e = cu[n], cu[n + 1]
+        r, m = assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} group {group}")
+        ro, mo = assert_output_close(out["o_raw"][s:e, heads], ref["o"], f"o seq {n}")
+        rs = assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
+        report(f"{wl.name}[{algo}] seq {n} group {group}", r, m, rs)
+        report(f"{wl.name}[{algo}] seq {n} group {group} o_raw", ro, mo)
+
+
+@ALGOS
+def test_all_sequences_empty(cuda_device, algo):
+    """A batch of sequences with no tokens at all: nothing is computed, every state
+    and conv window passes through unchanged, and no workspace is needed."""
+    wl = W.Workload("empty", 2, 4, 128, seqlens=(0, 0, 0), state_std=0.02, seed=5)
+    cfg = gdn.Config.of(wl, algo)
+    assert gdn.prefill_workspace_size(cfg, 3, 0) == 0
+    inp = W.make_prefill(wl, cuda_device)
+    g = torch.Generator(device=cuda_device).manual_seed(9)
+    conv = torch.randn((3, 3, wl.conv_dim), generator=g, device=cuda_device).to(torch.bfloat16)
+    out = _gpu_prefill(cfg, inp, initial_conv=conv, return_final_state=True,
+                       return_final_conv=True, check_status=False)
+    torch.cuda.synchronize()
+    assert out["y"].numel() == 0
+    assert torch.equal(out["final_state"], inp["initial_state"])
+    assert torch.equal(out["final_conv"], conv)
+
+
+def test_bounded_wait_timeout_aborts_cleanly(cuda_device):
+    """A wait between the chunk kernel's warps that runs out (here: forced by a
+    limit of 100 SM cycles, far below any real hand-over) makes the call abort
+    without a fault or a hang: the status query reports GDN_ERR_TIMEOUT, and the
+    next call on the same workspace and context is clean and correct."""
+    wl = W.Workload("timeout", 1, 2, 128, seqlens=(300, 77), state_std=0.02, seed=17)
+    cfg = gdn.Config.of(wl, "chunked")
+    inp = W.make_prefill(wl, cuda_device)
+    B, N = 2, 377
+    ws = torch.empty(gdn.prefill_workspace_size(cfg, B, N), dtype=torch.uint8, device=cuda_device)
+    ref = _gpu_prefill(cfg, inp, return_final_state=True, workspace=ws)
+    assert gdn.prefill_status(ws) == (gdn.GDN_OK, 0)
+    gdn.wait_limit_next_call(100)
+    _gpu_prefill(cfg, inp, return_final_state=True, workspace=ws, check_status=False)
+    st, detail = gdn.prefill_status(ws)
+    assert st == gdn.GDN_ERR_TIMEOUT
+    assert detail == 0 or (detail & 0x80000000), f"detail {detail:#x}"
+    again = _gpu_prefill(cfg, inp, return_final_state=True, workspace=ws)
+    torch.cuda.synchronize()
+    assert gdn.prefill_status(ws) == (gdn.GDN_OK, 0)
+    assert torch.equal(again["y"], ref["y"])
+    assert torch.equal(again["final_state"], ref["final_state"])
+
+
+@ALGOS
+def test_qwen35_prefill_sampled_groups(cuda_device, algo):
+    """The Qwen3.5-397B-A17B layer shape (16 q/k heads, 64 value heads, G = 4),
+    B = 2 x T = 4096 with initial states: whole q/k groups against the oracle."""
+    wl = W.QWEN35_PREFILL
+    cfg = gdn.Config.of(wl, algo)
+    inp = W.make_prefill(wl, cuda_device)
+    out = _gpu_prefill(cfg, inp, return_final_state=True, return_final_conv=True)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out["y"].float()).all()
+    cu = inp["cu_seqlens"].tolist()
+    for n, group in [(0, 0), (0, 10), (1, 5), (1, 15)]:
+        heads = list(range(4 * group, 4 * group + 4))
+        ref = _oracle_seq(wl, inp, n, group)
+        s, e = cu[n], cu[n + 1]
+        r, m = assert_output_close(out["y"][s:e, heads], ref["y"], f"y seq {n} group {group}")
+        rs = assert_state_close(out["final_state"][n, heads], ref["state"], f"state seq {n}")
+        report(f"qwen35_prefill[{algo}] seq {n} group {group}", r, m, rs)
+    for n in range(2):
+        assert torch.equal(out["final_conv"][n], inp["qkv"][cu[n + 1] - 3:cu[n + 1]])
+
+
+def test_qwen35_decode_sampled(cuda_device):
+    """Decode at the Qwen3.5-397B-A17B shape: 256 sequences, sampled ones against the oracle."""
+    wl = W.QWEN35_DECODE
+    cfg = gdn.Config.of(wl)
+    inp = W.make_decode(wl, cuda_device)
+    seqs = [0, 31, 128, 255]
+    S_before = inp["state"][seqs].cpu()
+    C_before = inp["conv_cache"][seqs].cpu()
+    y = gdn.decode(cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["state"],
+                   inp["conv_cache"], *[inp[k] for k in PARAMS])
+    torch.cuda.synchronize()
+    sub = {k: inp[k][seqs].cpu() for k in ("qkv", "a", "b", "z")}
+    ref = oracle.decode(_shape(wl), sub["qkv"], sub["a"], sub["b"], sub["z"],
+                        *[inp[k].cpu() for k in PARAMS], state=S_before, conv_cache=C_before)
+    r, m = assert_output_close(y[seqs], ref["y"])
+    rs = assert_state_close(inp["state"][seqs], ref["state"])
+    report("qwen35_decode", r, m, rs)
+    np.testing.assert_array_equal(to64(inp["conv_cache"][seqs]), ref["conv_window"])

@@ -36,6 +36,7 @@ def _both(cfg, inp, conv=None):
 
 
 def _check(ref, out):
+    assert gdn.prefill_noalloc_status() == (gdn.GDN_OK, 0)
     assert_output_close(out["y"], ref["y"])
     assert_output_close(out["o_raw"], ref["o_raw"], "o_raw")
     assert_state_close(out["final_state"], ref["final_state"])
@@ -70,3 +71,21 @@ def test_noalloc_largest_call_and_limit(cuda_device):
                             *[big[k] for k in P], y=y)
     assert e.value.status == gdn.GDN_ERR_WORKSPACE
     assert "scratch" in str(e.value)
+
+
+def test_noalloc_reports_device_status(cuda_device):
+    """The device status of a gdn_prefill_noalloc call sits in the library's own
+    scratch, out of the caller's reach; gdn_prefill_noalloc_status reads it.  A
+    call whose bounded waits are forced to run out reports GDN_ERR_TIMEOUT there,
+    and the next call is clean and matches gdn_prefill again."""
+    cfg = gdn.Config.of(LAYER)
+    inp = W.make_prefill(LAYER, cuda_device, seed=21, seqlens=(150, 40))
+    y = torch.empty((190, 16, 128), dtype=torch.bfloat16, device=cuda_device)
+    args = (cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["cu_seqlens"],
+            *[inp[k] for k in P])
+    gdn.wait_limit_next_call(100)
+    gdn.prefill_noalloc(*args, y=y, initial_state=inp["initial_state"])
+    st, detail = gdn.prefill_noalloc_status()
+    assert st == gdn.GDN_ERR_TIMEOUT
+    assert detail == 0 or (detail & 0x80000000)
+    _check(*_both(cfg, inp))
