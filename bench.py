@@ -303,6 +303,8 @@ def run_ours(args, rank, world, dev, dist):
         return {"metric": METRIC, "value": value, "unit": UNIT, "ms_per_step": ms_per_step,
                 "roofline": roof, "clocks": clk}
     decode = run_decode(args, rank, world, dev, pk, timed, max_over_ranks)
+    decode_k = run_decode_k(args, rank, world, dev, pk, timed, max_over_ranks)
+    qwen35 = run_prefill_shape(args, rank, world, dev, pk, timed, max_over_ranks, "qwen35_prefill")
 
     # ---- end to end through the public API from pinned host buffers.  Every
     # step uploads its inputs, runs the layer and reads back y and the final
@@ -361,10 +363,108 @@ def run_ours(args, rank, world, dev, dist):
                        "arith": "bf16 activations in/out, tf32 tensor-core products with FP32 "
                                 "accumulation, FP32 state and CUDA-core math",
                        "l2": "no flush: inputs of one step (~447 MB) exceed the 126 MB L2"},
-            "roofline": roof, "decode": decode, "e2e": e2e,
-            "gpu_launches": (4 if kname == "chunk_prefill_kernel" else 2) * args.steps,
+            "roofline": roof, "decode": decode, "decode_k": decode_k, "qwen35_prefill": qwen35,
+            "e2e": e2e,
+            # chunked: offsets, conv of q|k and of v (side stream), Gram, inverses, chunk kernel
+            "gpu_launches": (6 if kname == "chunk_prefill_kernel" else 2) * args.steps,
             "clocks": clk}
     return line
+
+
+def decode_k_bytes(Hk, Hv, d, B, k, act_bytes=2, K=4, read_state=True, write_state=True, y=True):
+    """HBM bytes of one multi-token call: the state read and/or written once for all
+    k tokens, k tokens' q|k|v, a, b (and z, y when outputs are formed) and the conv
+    cache (read, and written when the state is)."""
+    conv_dim = (2 * Hk + Hv) * d
+    st = 4 * Hv * d * d * (int(read_state) + int(write_state))
+    tok = act_bytes * k * (conv_dim + 2 * Hv + (2 * Hv * d if y else 0))
+    cache = act_bytes * (K - 1) * conv_dim * (1 + int(write_state))
+    return (st + tok + cache) * B
+
+
+def run_decode_k(args, rank, world, dev, pk, timed, max_over_ranks):
+    """Multi-token decode at the Qwen3.8 shape: k = 2 tokens per sequence (the one
+    draft of the MTP layer and the token after it) against resident states: plain
+    multi-token decode (state updated by both), and the speculative pair -- verify
+    (outputs of both, state read only) then commit (state advanced by the accepted
+    tokens, here all of them)."""
+    import torch
+
+    import linear_attention_layer_causal_b200 as gdn
+    from linear_attention_layer_causal_b200 import workloads as W
+    dwl = W.QWEN38_DECODE
+    cfg = gdn.Config.of(dwl)
+    B, k = args.decode_batch, 2
+    d = W.make_decode(dwl, dev, batch=B, seed=rank_seed(dwl.seed, rank) + 1, tokens=k)
+    P = [d[x] for x in ("conv_w", "A_log", "dt_bias", "norm_w")]
+    y = torch.empty((B, k, cfg.num_v_heads, cfg.head_dim), dtype=torch.bfloat16, device=dev)
+    acc = torch.full((B,), k, dtype=torch.int32, device=dev)
+    out = {"metric": "GDN multi-token decode tokens/s at Qwen3.8 layer shape", "unit": "tokens/s",
+           "config": {"workload": dwl.name, "batch": B, "tokens_per_sequence": k}}
+    Hk, Hv, D = cfg.num_qk_heads, cfg.num_v_heads, cfg.head_dim
+
+    def multi():
+        gdn.decode_multi(cfg, d["qkv"], d["a"], d["b"], d["z"], d["state"], d["conv_cache"], *P, y=y)
+
+    def verify():
+        gdn.decode_verify(cfg, d["qkv"], d["a"], d["b"], d["z"], d["state"], d["conv_cache"], *P, y=y)
+
+    def commit():
+        gdn.decode_commit(cfg, d["qkv"], d["a"], d["b"], d["state"], d["conv_cache"], acc, *P)
+
+    for name, fn, nbytes in [
+            ("multi", multi, decode_k_bytes(Hk, Hv, D, B, k)),
+            ("verify", verify, decode_k_bytes(Hk, Hv, D, B, k, write_state=False)),
+            ("commit", commit, decode_k_bytes(Hk, Hv, D, B, k, y=False))]:
+        for _ in range(args.warmup):
+            fn()
+        tot, kern = timed(fn, args.steps)
+        tot, kern = max_over_ranks(tot), max_over_ranks(kern)
+        gbs = nbytes / (kern / 1e3) / 1e9
+        out[name] = {"value": job_rate(B * k, world, args.steps, tot), "ms_per_step": tot / args.steps,
+                     "roofline": {"kernel": "decode_multi_kernel", "bound": "hbm",
+                                  "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                  "frac": round(gbs / pk["hbm_gbs"], 4), "algorithmic_bytes": nbytes,
+                                  "kernel_ms": round(kern, 4), "peak_source": pk["source"] + " copy"}}
+    # a speculative step of k tokens: verify + commit
+    out["value"] = job_rate(B * k, world, 1, out["verify"]["ms_per_step"] + out["commit"]["ms_per_step"])
+    return out
+
+
+def run_prefill_shape(args, rank, world, dev, pk, timed, max_over_ranks, name):
+    """Prefill at another layer shape of the family (tokens/s and the chunk kernel's
+    tensor roofline), e.g. the Qwen3.5-397B-A17B layer: 16 q/k heads, 64 value heads."""
+    import torch
+
+    import linear_attention_layer_causal_b200 as gdn
+    from linear_attention_layer_causal_b200 import workloads as W
+    wl = W.WORKLOADS[name]
+    cfg = gdn.Config.of(wl)
+    inp = W.make_prefill(wl, dev, seed=rank_seed(wl.seed, rank))
+    P = [inp[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
+    N, B = sum(inp["seqlens"]), len(inp["seqlens"])
+    y = torch.empty((N, cfg.num_v_heads, cfg.head_dim), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((B, cfg.num_v_heads, cfg.head_dim, cfg.head_dim), device=dev)
+    ws = torch.empty(max(gdn.prefill_workspace_size(cfg, B, N), 1), dtype=torch.uint8, device=dev)
+
+    def step():
+        gdn.prefill(cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["cu_seqlens"], *P, y=y,
+                    final_state=fs, initial_state=inp["initial_state"], workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    tot, kern = timed(step, args.steps)
+    tot, kern = max_over_ranks(tot), max_over_ranks(kern)
+    flops = prefill_flops_per_token(cfg.num_qk_heads, cfg.num_v_heads, cfg.head_dim) * N
+    tf32_peak = round(pk["bf16_tflops"] * TF32_PER_BF16, 1)
+    tf = flops / (kern / 1e3) / 1e12
+    return {"metric": f"GDN prefill tokens/s, {wl.notes}", "unit": "tokens/s",
+            "value": job_rate(N, world, args.steps, tot), "ms_per_step": tot / args.steps,
+            "config": {"workload": name, "batch": B, "seq_len": N // B, "num_qk_heads": cfg.num_qk_heads,
+                       "num_v_heads": cfg.num_v_heads},
+            "roofline": {"kernel": "chunk_prefill_kernel", "bound": "tensor", "achieved": round(tf, 2),
+                         "peak": tf32_peak, "unit": "TFLOP/s", "frac": round(tf / tf32_peak, 4),
+                         "kernel_ms": round(kern, 4)}}
 
 
 def run_decode(args, rank, world, dev, pk, timed, max_over_ranks):

@@ -271,7 +271,8 @@ GDN_API gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *pa
  *
  *   - Limit: a call whose gdn_prefill_workspace_size exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_WORKSPACE before any CUDA
- *     call (at the Qwen3.8 layer shape, 88 KiB per token: up to 744 tokens).
+ *     call (at the Qwen3.8 layer shape, about 108 KiB per token plus
+ *     1.7 MiB per sequence: up to 574 tokens of one sequence).
  *   - Set-up: the first call on a device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
  *     that first call before any stream capture.

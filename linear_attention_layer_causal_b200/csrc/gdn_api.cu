@@ -62,6 +62,40 @@ bool elem_aligned(const void *p, bool bf16) {
 gdn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA; }
 
 thread_local ProfileHook tl_hook;
+
+// A second stream per host thread and device, with a fork and a join event:
+// the chunked prefill runs the (bandwidth-bound) conv of the v channels on it,
+// beside the (latency-bound) q/k conv, Gram and inverse kernels on the
+// caller's stream.  Created on the first chunked call of the thread on that
+// device and kept until the process exits; thread-local, so calls from several
+// host threads never share one.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+};
+constexpr int kMaxSideDevices = 64;
+thread_local SideStream tl_side[kMaxSideDevices];
+
+cudaError_t side_stream(SideStream **out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxSideDevices)
+        return cudaErrorInvalidDevice;
+    SideStream &ss = tl_side[dev];
+    if (ss.stream == nullptr) {
+        e = cudaStreamCreateWithFlags(&ss.stream, cudaStreamNonBlocking);
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming);
+        if (e == cudaSuccess)
+            e = cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming);
+        if (e != cudaSuccess)
+            return e;
+    }
+    *out = &ss;
+    return cudaSuccess;
+}
 thread_local long long tl_wait_limit = 0; // 0 = not armed
 
 } // namespace
@@ -123,15 +157,16 @@ gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t 
 }
 
 // Header (status word), float32 normalised q|k, float32 convolved v and, for
-// head_dim 128, the chunk Gram rows and the per-sequence chunk offsets of the
-// chunked path.
+// head_dim 128, the chunked path's Q K^T rows, T diag(beta) tiles and
+// per-sequence chunk offsets.
 size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N, int batch) {
     if (N == 0)
         return 0;
     size_t b = kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4) +
                round_up((size_t)N * Hv * D * 4);
     if (D == 128)
-        b += round_up(kq_workspace_bytes(Hk, N)) + round_up(((size_t)batch + 1) * sizeof(int32_t));
+        b += round_up(kq_workspace_bytes(Hk, N)) + round_up(kk_workspace_bytes(Hk, N, batch)) +
+             round_up(tb_workspace_bytes(Hv, N, batch)) + round_up(((size_t)batch + 1) * sizeof(int32_t));
     return b;
 }
 
@@ -194,6 +229,21 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
                        int32_t batch, int64_t total_tokens, const float *initial_state,
                        const void *initial_conv, void *y, float *final_state, void *final_conv,
                        float *o_raw, void *workspace, size_t workspace_bytes, void *stream) {
+    return prefill_impl(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens, initial_state,
+                        initial_conv, y, final_state, final_conv, o_raw, workspace, workspace_bytes,
+                        stream, true);
+}
+
+} // extern "C"
+
+namespace gdn {
+
+gdn_status prefill_impl(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                        const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                        int32_t batch, int64_t total_tokens, const float *initial_state,
+                        const void *initial_conv, void *y, float *final_state, void *final_conv,
+                        float *o_raw, void *workspace, size_t workspace_bytes, void *stream,
+                        bool side) {
     size_t need = 0;
     gdn_status st = validate_prefill(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens,
                                      initial_state, initial_conv, y, final_state, final_conv,
@@ -235,8 +285,12 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
         p.ws_qk = w + kWorkspaceHeader;
         p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
         p.ws_kq = (char *)p.ws_v + round_up((size_t)total_tokens * p.Hv * p.D * 4);
-        if (p.D == 128)
-            p.ws_offs = (int32_t *)((char *)p.ws_kq + round_up(kq_workspace_bytes(p.Hk, total_tokens)));
+        if (p.D == 128) {
+            p.ws_kk = (char *)p.ws_kq + round_up(kq_workspace_bytes(p.Hk, total_tokens));
+            p.ws_tb = (char *)p.ws_kk + round_up(kk_workspace_bytes(p.Hk, total_tokens, batch));
+            p.ws_offs = (int32_t *)((char *)p.ws_tb +
+                                    round_up(tb_workspace_bytes(p.Hv, total_tokens, batch)));
+        }
     }
 
     cudaStream_t s = (cudaStream_t)stream;
@@ -244,15 +298,49 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     p.wait_limit = take_wait_limit();
     if (batch == 0)
         return GDN_OK;
-    // front end.  Chunked path: chunk offsets (which also clear the status
-    // words), the fused q/k kernel (conv, SiLU, L2 norm and the intra-chunk
-    // Gram rows), then the conv of the v channels.  Token-serial path: the conv
-    // of every channel.
-    cudaError_t e = p.chunked ? launch_chunk_offsets(p, s) : cudaSuccess;
-    if (e == cudaSuccess && p.chunked)
-        e = launch_qk_front(p, s);
-    if (e == cudaSuccess)
-        e = launch_conv_prep(p, s);
+    // front end.  Token-serial path: conv, SiLU and q/k L2 norm of every
+    // channel.  Chunked path: the chunk offsets (which also clear the status
+    // words); then, on the side stream, the conv of the v channels, and on the
+    // caller's stream the conv of q and k, the intra-chunk Gram rows and the
+    // triangular inverses; the chunk kernel waits for both.
+    cudaError_t e = cudaSuccess;
+    if (!p.chunked) {
+        e = launch_conv_prep(p, ConvPart::kAll, s);
+    } else if (!side) { // everything on the caller's stream, in order
+        e = launch_chunk_offsets(p, s);
+        if (e == cudaSuccess)
+            e = launch_conv_prep(p, ConvPart::kAll, s);
+        if (e == cudaSuccess)
+            e = launch_gram(p, s);
+        if (e == cudaSuccess)
+            e = launch_tri(p, s);
+    } else {
+        SideStream *ss = nullptr;
+        e = launch_chunk_offsets(p, s);
+        if (e == cudaSuccess)
+            e = side_stream(&ss);
+        if (e == cudaSuccess)
+            e = cudaEventRecord(ss->fork, s);
+        if (e == cudaSuccess)
+            e = cudaStreamWaitEvent(ss->stream, ss->fork, 0);
+        if (e == cudaSuccess) {
+            e = launch_conv_prep(p, ConvPart::kV, ss->stream);
+            // the join is recorded (and waited for) whatever the launch did, so
+            // that the caller's stream never runs ahead of the side stream
+            const cudaError_t e2 = cudaEventRecord(ss->join, ss->stream);
+            if (e == cudaSuccess)
+                e = e2;
+            if (e == cudaSuccess)
+                e = launch_conv_prep(p, ConvPart::kQK, s);
+            if (e == cudaSuccess)
+                e = launch_gram(p, s);
+            if (e == cudaSuccess)
+                e = launch_tri(p, s);
+            const cudaError_t e3 = e2 == cudaSuccess ? cudaStreamWaitEvent(s, ss->join, 0) : e2;
+            if (e == cudaSuccess)
+                e = e3;
+        }
+    }
     if (e == cudaSuccess)
         e = record_if(hook.begin, s);
     if (e == cudaSuccess)
@@ -264,7 +352,7 @@ gdn_status gdn_prefill(const gdn_config *cfg, const gdn_params *params, const vo
     return cuda_status(e);
 }
 
-}
+} // namespace gdn
 
 namespace gdn {
 namespace {

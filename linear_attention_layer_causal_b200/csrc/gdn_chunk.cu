@@ -42,6 +42,7 @@
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
 #include "gdn_tmap.h"
+#include "gdn_tri.cuh"
 
 namespace gdn {
 
@@ -122,11 +123,10 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 // and smaller hot code runs faster.
 
 constexpr int kSG = 256;                          // state group threads
-constexpr int kTeam = 128;                        // T team threads
-constexpr int kTeamP = 64;                        // P team threads
-constexpr int kThreads = kSG + kTeam + kTeamP + 64; // + MMA warp + TMA warp: 16 warps
-constexpr int kWarpMma = (kSG + kTeam + kTeamP) / 32; // 14
-constexpr int kBarSG = 1, kBarT = 2, kBarP = 3;   // named barriers
+constexpr int kTeam = 128;                        // prep team threads
+constexpr int kThreads = kSG + kTeam + 64;        // + MMA warp + TMA warp: 14 warps
+constexpr int kWarpMma = (kSG + kTeam) / 32;      // 12
+constexpr int kBarSG = 1, kBarT = 2;              // named barriers
 
 // TMEM columns: the state, two [X^T | O^T] pairs (MMA 2 writes one pair with a
 // single N = 128 product), two U^T buffers.  All by chunk parity.
@@ -143,23 +143,16 @@ constexpr uint32_t kTmemCols = 512;
 // R-row blocks at (c / 32) R 32 + 32 r + 4 (((c mod 32) / 4) xor (r mod 8)) + c mod 4.
 // MN-major tf32 operands (V, K) use the 128-byte swizzle on a 32-byte base,
 // written only by TMA: 32-byte chunks of row k XOR-swizzled by k mod 4.
-// Lower-triangular 64 x 64 tile in the K-major layout with its zero quadrant
-// (rows 0..31, columns 32..63) left out: column block 0 holds rows 0..63
-// (2048 floats), block 1 rows 32..63 only (1024 floats).  An MMA over the
-// tile takes block 0 with N = 64 and block 1 with N = 32 at row 32.  Element
-// (r, c) sits at swz(r, c, 64) for c < 32 and at 1024 + swz(r, c - 32, 64)
-// for c >= 32 (r >= 32); the passes below fold these into per-thread bases.
-constexpr int kTriFloats = 3 * 1024;
+// Lower-triangular 64 x 64 tiles use the triangular-tile layout of gdn_tri.cuh.
 
 struct __align__(1024) ChunkSmem {
     // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = K, rows 64..127 = Q
     float KQ[2 * kC * kD];
     float V[kC * kD];          // A of MMA 1 (MN-major)
     float K[kC * kD];          // B of MMA 3 (MN-major): lands as K, becomes diag(gamma_C/gamma) K
-    float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta), by chunk parity
+    float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta) (from the front kernel, by TMA), by chunk parity
     float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma), by chunk parity
     float P[kTriFloats];       // B of MMA 3: lands as Q K^T rows, becomes P
-    float Wk[kTriFloats];      // T team: lands as K K^T rows, becomes A, then T
     // z rows of the chunk (16-bit activations).  Once the state group has formed
     // the gate from it, it stages the chunk's y rows for one TMA store.
     __nv_bfloat16 Z[kC * kD];
@@ -167,11 +160,12 @@ struct __align__(1024) ChunkSmem {
     float rstd[kC];            // epilogue: reciprocal RMS of each row
     float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
     float gam[4][kC];          // gamma = e^G (fast exponential), by chunk index mod 4
-    float beta[kC];            // T team's current chunk
-    unsigned long long bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z; // TMA landings
+    unsigned long long bar_v, bar_q, bar_k, bar_kmaj, bar_qk, bar_z; // TMA landings
+    unsigned long long bar_tb[2];                               // TMA landing of T diag(beta), by parity
     unsigned long long bar_m1, bar_m2, bar_m2b[2], bar_m3;      // MMA completions
     unsigned long long bar_u, bar_of[2];                        // state group -> MMA
-    unsigned long long bar_pT[4], bar_pP, bar_wfree;            // T / P teams -> MMA, TMA
+    unsigned long long bar_zf;                                  // state group -> TMA: z tile free
+    unsigned long long bar_pT[4], bar_pP;                       // prep team -> MMA, TMA, state group
     unsigned long long bar_fin;                                 // MMA drain on abort
     uint32_t tmem;
     int abort;
@@ -185,8 +179,9 @@ struct ChunkMaps {
     CUtensorMap k;    // normalised k, [N, Hk*128] of the q|k rows, MN-major tf32 swizzle
     CUtensorMap q;    // normalised q, [N, Hk*128], 128-byte swizzle (K-major)
     CUtensorMap kmaj; // normalised k, [N, Hk*128], 128-byte swizzle (K-major)
-    CUtensorMap kq;   // Gram rows, [N, Hk*128] fp32, 32 x 64 boxes, 128-byte swizzle
+    CUtensorMap kq;   // Q K^T rows, [N, Hk*64] fp32, 32 x 64 boxes, 128-byte swizzle
     CUtensorMap kq32; // the same with 32 x 32 boxes
+    CUtensorMap tb;   // T diag(beta) tiles, [chunks * Hv * 96, 32] fp32, 32 x 96 boxes, 128-byte swizzle
     CUtensorMap z;    // z, [N, Hv*128] bf16, 128 x 64 boxes, no swizzle (bf16 activations)
     CUtensorMap y;    // y, the same layout (bf16 activations): the store of a full chunk
 };
@@ -210,10 +205,6 @@ __device__ __noinline__ bool wait_slow(uint32_t bar, uint32_t ph, volatile int *
     return true;
 }
 
-// Barrier over the `n` threads of one group (named barrier `id`).
-__device__ __forceinline__ void group_sync(int id, int n) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
 // The same, returning whether `pred` held on any of the group's threads.
 __device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
     uint32_t r;
@@ -231,13 +222,6 @@ __device__ __forceinline__ bool group_sync_or(int id, int n, bool pred) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-// L2 prefetch of one TMA box.
-__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {
-    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(tmap),
-                 "r"(x), "r"(y)
-                 : "memory");
-}
-
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
@@ -266,7 +250,9 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
 
     const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
     const uint32_t bar_k = smem_u32(&sm.bar_k), bar_kmaj = smem_u32(&sm.bar_kmaj);
-    const uint32_t bar_kk = smem_u32(&sm.bar_kk), bar_qk = smem_u32(&sm.bar_qk);
+    const uint32_t bar_qk = smem_u32(&sm.bar_qk);
+    // T diag(beta) of chunk c landed, by chunk parity
+    auto bar_tb = [&](int c) { return smem_u32(&sm.bar_tb[c & 1]); };
     const uint32_t bar_z = smem_u32(&sm.bar_z);
     constexpr bool kZTile = sizeof(T) == 2; // z comes by TMA (16-bit) or from global (fp32)
     const uint32_t bar_m1 = smem_u32(&sm.bar_m1), bar_m2 = smem_u32(&sm.bar_m2);
@@ -275,15 +261,16 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     auto bar_m2b = [&](int c) { return smem_u32(&sm.bar_m2b[c & 1]); };
     const uint32_t bar_u = smem_u32(&sm.bar_u);
     const uint32_t bar_of0 = smem_u32(&sm.bar_of[0]), bar_of1 = smem_u32(&sm.bar_of[1]);
+    const uint32_t bar_zf = smem_u32(&sm.bar_zf);
     // T tiles + gates of chunk c ready, by chunk index mod 4: a waiter for chunk c
     // must see that phase before the barrier can move on, and the T team may run
     // up to two chunks ahead of the state group
     auto bar_pT = [&](int c) { return smem_u32(&sm.bar_pT[c & 3]); };
-    const uint32_t bar_pP = smem_u32(&sm.bar_pP), bar_wfree = smem_u32(&sm.bar_wfree);
+    const uint32_t bar_pP = smem_u32(&sm.bar_pP);
     if (tid == 0) {
-        const uint32_t one[] = {bar_v,  bar_q,   bar_k,   bar_kmaj, bar_kk,   bar_qk,  bar_z,
-                                bar_m1, bar_m2,  bar_m3,  bar_u,    bar_of0,  bar_of1, bar_pP,
-                                bar_wfree, smem_u32(&sm.bar_fin)};
+        const uint32_t one[] = {bar_v,  bar_q,  bar_k,   bar_kmaj, bar_qk,  bar_z,  bar_m1,
+                                bar_m2, bar_m3, bar_u,   bar_of0,  bar_of1, bar_pP, bar_zf,
+                                smem_u32(&sm.bar_fin)};
 #pragma unroll
         for (int b = 0; b < (int)(sizeof(one) / sizeof(one[0])); ++b)
             mbar_init(one[b], 1);
@@ -292,6 +279,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             mbar_init(smem_u32(&sm.bar_pT[b]), 1);
         mbar_init(smem_u32(&sm.bar_m2b[0]), 1);
         mbar_init(smem_u32(&sm.bar_m2b[1]), 1);
+        mbar_init(smem_u32(&sm.bar_tb[0]), 1);
+        mbar_init(smem_u32(&sm.bar_tb[1]), 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -304,7 +293,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     tc_fence_after();
     const uint32_t tmem = sm.tmem;
     volatile int *abort_flag = &sm.abort;
-    const int xq = j * kD, xv = h * kD, xkk = j * 2 * kC;
+    const int xq = j * kD, xv = h * kD, xkk = j * kC;
     auto rows_of = [&](int c) {
         const int64_t left = len - (int64_t)c * kC;
         return (int)(left < kC ? left : kC);
@@ -367,14 +356,23 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         uint32_t ph3 = 0, phz = 0;
         float *red = &sm.red[0][0];
         float *rstd = sm.rstd;
+        bool zpend = false; // a y store from the z tile is in flight (uniform over the group)
+        // once the y store has read the z tile, the tile may take the next chunk's z
+        auto release_z = [&]() {
+            if (zpend && tid == 0) {
+                bulk_wait_read();
+                mbar_arrive(bar_zf);
+            }
+            zpend = false;
+        };
         for (int c = 0; ok && c < nchunks; ++c) {
+            release_z();
             const int sl = c & 3;
             const uint32_t cU = (c & 1) ? kColU1 : kColU0, cX = (c & 1) ? kColX1 : kColX0;
             const uint32_t cO = cX + 64;
             // ---- once MMA 2 is done: S *= gamma_C and O^T *= diag(gamma) (MMA 2 left
             //      S0 Q^T there; MMA 3 adds U^T P^T), beside MMA 2b, which touches
-            //      neither; then, once MMA 2b is done, U -> tf32 in place (the A
-            //      operand of both parts of MMA 3)
+            //      neither; then, once MMA 2b is done, the U pass
             {
                 bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
                 good = waitq(bar_m2, c & 1) && good;
@@ -415,17 +413,29 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 good = __all_sync(0xffffffffu, good);
                 tc_fence_after();
                 if (good) {
+                    // U -> tf32 in place (A of MMA 3's O part) and U diag(gamma_C / gamma)
+                    // -> tf32 into the X columns, which MMA 2b has read (A of its state part)
                     float u[2][16];
                     tmem_ld16(tl + cU + 32 * hf, u[0]);
                     tmem_ld16(tl + cU + 32 * hf + 16, u[1]);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        u[0][i] = tf32_rna(u[0][i]);
-                        u[1][i] = tf32_rna(u[1][i]);
+                    for (int q = 0; q < 2; ++q) {
+                        float uk[16];
+#pragma unroll
+                        for (int i = 0; i < 16; i += 4) {
+                            const float4 k4 = *reinterpret_cast<const float4 *>(&sm.kd[sl][32 * hf + 16 * q + i]);
+                            uk[i] = tf32_rna(u[q][i] * k4.x);
+                            uk[i + 1] = tf32_rna(u[q][i + 1] * k4.y);
+                            uk[i + 2] = tf32_rna(u[q][i + 2] * k4.z);
+                            uk[i + 3] = tf32_rna(u[q][i + 3] * k4.w);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            u[q][i] = tf32_rna(u[q][i]);
+                        tmem_st16(tl + cU + 32 * hf + 16 * q, u[q]);
+                        tmem_st16(tl + cX + 32 * hf + 16 * q, uk);
                     }
-                    tmem_st16(tl + cU + 32 * hf, u[0]);
-                    tmem_st16(tl + cU + 32 * hf + 16, u[1]);
                 }
                 tmem_wait_st();
                 tc_fence_before();
@@ -519,8 +529,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     if (tid == 0 && good) {
                         tma_store_2d(&maps.y, h * kD, (int)t0, smem_u32(sm.Z));
                         bulk_commit();
-                        bulk_wait_read(); // the z tile may take the next chunk's rows
                     }
+                    zpend = true; // released at the top of the next chunk
+                } else if (kZTile && tid == 0) {
+                    mbar_arrive(bar_zf); // read by the gate step (before the sums above)
                 }
                 tc_fence_before();
                 if (group_sync_or(kBarSG, kSG, !good || *abort_flag)) {
@@ -531,12 +543,16 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     mbar_arrive((c & 1) ? bar_of1 : bar_of0);
             }
         }
+        release_z();
         if (!ok)
             *abort_flag = 1;
     } else if (warp < (kSG + kTeam) / 32) {
-        // ==================================================== T team
+        // ==================================================== prep team
+        // Per chunk: the gates; -T diag(beta gamma) from the T diag(beta) tile that
+        // the front kernel formed (the B operands of MMA 2b and MMA 1); P from the
+        // Q K^T rows.  All tf32, in the triangular-tile layout.
         const int tt = tid - kSG, tw = tt >> 5;
-        float *Wk = sm.Wk;
+        const TriThread tr(tt);
         // raw gate inputs of chunk c, rows lane and lane + 32 (first warp of the team)
         auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
             if (tw == 0) {
@@ -555,16 +571,16 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         };
         const float negA = -expf(__ldg(p.A_log + h));
         const float dtb = __ldg(p.dt_bias + h);
-        // g, the inclusive prefix G and gamma_C / gamma of a chunk into slot
-        // `sl`, beta into the team's own row (first warp; rows lane and lane + 32)
-        auto gates = [&](int c, const T (&ra)[2], const T (&rb)[2], int sl) {
+        // g, the inclusive prefix G, gamma_C / gamma and gamma of a chunk into slot
+        // `sl` (first warp; rows lane and lane + 32).  The same arithmetic as the
+        // front kernel's, so that both see the same G.
+        auto gates = [&](int c, const T (&ra)[2], int sl) {
             if (tw == 0) {
-                float g[2], be[2];
+                float g[2];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     const bool in = lane + 32 * q < rows_of(c);
                     g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
-                    be[q] = in ? sigmoidf_(to_f(rb[q])) : 0.f;
                 }
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
@@ -581,211 +597,36 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 for (int q = 0; q < 2; ++q) {
                     const int r = lane + 32 * q;
                     sm.G[sl][r] = g[q];
-                    sm.beta[r] = be[q];
                     sm.kd[sl][r] = expf(Glast - g[q]);
-                    sm.gam[sl][r] = __expf(g[q]); // far inside the tf32 rounding of its users
+                    sm.gam[sl][r] = __expf(g[q]);
                 }
             }
         };
-        // The six float4s of a triangular tile this thread handles: rows
-        // tt / 8 + 16 jj (jj = 0..3, column block 0, columns 4 (tt % 8)) and
-        // 32 + tt / 8 + 16 (jj - 4) (jj = 4, 5, block 1, columns 32 + 4 (tt % 8)).
-        // 16 jj keeps r mod 8, so the swizzle term is one constant per thread.
-        const int trow = tt >> 3, tcol = 4 * (tt & 7);
-        const int tbase = trow * 32 + (((tt & 7) ^ (trow & 7)) << 2);
-        auto tri_r = [&](int jj) { return jj < 4 ? trow + 16 * jj : 32 + trow + 16 * (jj - 4); };
-        auto tri_c = [&](int jj) { return jj < 4 ? tcol : 32 + tcol; };
-        auto tri_o = [&](int jj) { return tbase + (jj < 4 ? 512 * jj : 1024 + 512 * (jj - 2)); };
-        uint32_t phkk = 0;
+        uint32_t phqk = 0;
         T av[2], bv[2];
         load_ab(0, av, bv);
         for (int c = 0; c < nchunks; ++c) {
             const int sl = c & 3;
-            gates(c, av, bv, sl);
+            gates(c, av, sl);
             load_ab(c + 1, av, bv);
-            bool good = waitp(bar_kk, phkk); // K K^T rows of this chunk are in Wk
-            if (group_sync_or(kBarT, kTeam, !good || *abort_flag)) {
-                ok = false;
-                break;
-            }
-            // ---- A[r][s] = beta_r e^{G_r - G_s} KK[r][s] in place (the kq rows are
-            //      0 for s >= r and beta is 0 on padded rows; the clamp keeps the
-            //      unused upper triangle finite: G_r - G_s > 0 there)
-            {
-                float4 x[6];
-#pragma unroll
-                for (int jj = 0; jj < 6; ++jj)
-                    x[jj] = *reinterpret_cast<const float4 *>(Wk + tri_o(jj));
-#pragma unroll
-                for (int jj = 0; jj < 6; ++jj) {
-                    const float Gr = sm.G[sl][tri_r(jj)], br = sm.beta[tri_r(jj)];
-                    const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][tri_c(jj)]);
-                    x[jj].x *= br * __expf(fminf(Gr - Gc.x, 0.f));
-                    x[jj].y *= br * __expf(fminf(Gr - Gc.y, 0.f));
-                    x[jj].z *= br * __expf(fminf(Gr - Gc.z, 0.f));
-                    x[jj].w *= br * __expf(fminf(Gr - Gc.w, 0.f));
-                }
-#pragma unroll
-                for (int jj = 0; jj < 6; ++jj)
-                    *reinterpret_cast<float4 *>(Wk + tri_o(jj)) = x[jj];
-            }
-            group_sync(kBarT, kTeam);
-            // ---- T = (I + A)^-1 in place, by block doubling.  Level 1: the four
-            //      16 x 16 diagonal blocks by forward substitution, one column per
-            //      thread (threads 0..63)
-            {
-                // warp 0: blocks 0, 1 (column block 0); warp 1: blocks 2, 3 (block 1,
-                // whose rows 32.. sit at 1024 + 32 r); lanes 0..15 / 16..31 take the
-                // two blocks, R' = 0 / 16 within the column block
-                const int cl = tt & 15, Rp = 16 * ((tt >> 4) & 1), R = 32 * (tt >> 5) + Rp;
-                const float *blk = Wk + 1024 * (tt >> 5) + R * 32;
-                float x[16];
-                if (tt < 64) {
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-                        for (int m = 0; m < (r + 3) / 4; ++m) {
-                            const float4 a = *reinterpret_cast<const float4 *>(
-                                blk + r * 32 + ((((Rp >> 2) + m) ^ (r & 7)) << 2));
-                            const float av4[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                if (4 * m + e < r) {
-                                    if (e & 1)
-                                        acc1 = fmaf(av4[e], x[4 * m + e], acc1);
-                                    else
-                                        acc0 = fmaf(av4[e], x[4 * m + e], acc0);
-                                }
-                        }
-                        x[r] = r < cl ? 0.f : (r == cl ? 1.f : -(acc0 + acc1));
-                    }
-                }
-                group_sync(kBarT, kTeam); // every diagonal block of A has been read
-                if (tt < 64) {
-                    float *dst = Wk + 1024 * (tt >> 5) + R * 32 + ((Rp + cl) & 3);
-#pragma unroll
-                    for (int r = 0; r < 16; ++r)
-                        dst[r * 32 + ((((Rp + cl) >> 2) ^ (r & 7)) << 2)] = x[r];
-                }
-            }
-            group_sync(kBarT, kTeam);
-            // ---- level 2: join the 16-blocks of each 32-block p (warps 0, 1: p = 0
-            //      in column block 0; warps 2, 3: p = 1 in block 1):
-            //      T21 = -T22 (A21 T11); thread: rows r0, r0 + 1, columns c0, c0 + 1;
-            //      element (32 p + i, 32 p + j) at base + i * 32 + swizzle(i, j)
-            {
-                const int pb = tt >> 6, q = tt & 63;
-                const int r0 = 2 * (q >> 3), c0 = 2 * (q & 7);
-                float *base = Wk + 1024 * pb + 32 * pb * 32;
-                auto at = [&](int i, int jc) { return base + i * 32 + (((jc >> 2) ^ (i & 7)) << 2) + (jc & 3); };
-                float y00 = 0.f, y01 = 0.f, y10 = 0.f, y11 = 0.f;
-#pragma unroll 1
-                for (int m = 0; m < 4; ++m) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 4 * m));
-                    const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 4 * m));
-                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 t2 = *reinterpret_cast<const float2 *>(at(4 * m + e, c0));
-                        y00 = fmaf(a0v[e], t2.x, y00); y01 = fmaf(a0v[e], t2.y, y01);
-                        y10 = fmaf(a1v[e], t2.x, y10); y11 = fmaf(a1v[e], t2.y, y11);
-                    }
-                }
-                group_sync(kBarT, kTeam); // A21 is read: Y takes its place
-                *reinterpret_cast<float2 *>(at(16 + r0, c0)) = make_float2(y00, y01);
-                *reinterpret_cast<float2 *>(at(17 + r0, c0)) = make_float2(y10, y11);
-                group_sync(kBarT, kTeam);
-                float x00 = 0.f, x01 = 0.f, x10 = 0.f, x11 = 0.f;
-#pragma unroll 1
-                for (int m = 0; m < 4; ++m) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(at(16 + r0, 16 + 4 * m));
-                    const float4 a1 = *reinterpret_cast<const float4 *>(at(17 + r0, 16 + 4 * m));
-                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 t2 = *reinterpret_cast<const float2 *>(at(16 + 4 * m + e, c0));
-                        x00 = fmaf(a0v[e], t2.x, x00); x01 = fmaf(a0v[e], t2.y, x01);
-                        x10 = fmaf(a1v[e], t2.x, x10); x11 = fmaf(a1v[e], t2.y, x11);
-                    }
-                }
-                group_sync(kBarT, kTeam); // Y is read: T21 takes its place
-                *reinterpret_cast<float2 *>(at(16 + r0, c0)) = make_float2(-x00, -x01);
-                *reinterpret_cast<float2 *>(at(17 + r0, c0)) = make_float2(-x10, -x11);
-            }
-            group_sync(kBarT, kTeam);
-            // ---- level 3: join the two 32-blocks: T21 = -T22 (A21 T11); thread:
-            //      rows r0, r0 + 1, columns c0 .. + 3 of the 32 x 32 products.  A21,
-            //      T11 and Y sit in column block 0 (offset r * 32 + chunk ^ (r & 7)),
-            //      T22 in block 1 (rows 32..63)
-            {
-                const int r0 = 2 * (tt >> 3), q0 = tt & 7; // columns c0 = 4 q0
-                const float *Ar0 = Wk + (32 + r0) * 32, *Ar1 = Ar0 + 32;   // rows 32 + r0, + 1
-                const float *Br0 = Wk + 2048 + r0 * 32, *Br1 = Br0 + 32;   // block 1 rows
-                const int x0 = r0 & 7, x1 = (r0 + 1) & 7;
-                float y[2][4] = {};
-#pragma unroll 1
-                for (int m = 0; m < 8; ++m) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(Ar0 + ((m ^ x0) << 2));
-                    const float4 a1 = *reinterpret_cast<const float4 *>(Ar1 + ((m ^ x1) << 2));
-                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 4 * m + e; // T11 row i, columns c0 .. + 3
-                        const float4 t4 =
-                            *reinterpret_cast<const float4 *>(Wk + i * 32 + ((q0 ^ (i & 7)) << 2));
-                        y[0][0] = fmaf(a0v[e], t4.x, y[0][0]); y[0][1] = fmaf(a0v[e], t4.y, y[0][1]);
-                        y[0][2] = fmaf(a0v[e], t4.z, y[0][2]); y[0][3] = fmaf(a0v[e], t4.w, y[0][3]);
-                        y[1][0] = fmaf(a1v[e], t4.x, y[1][0]); y[1][1] = fmaf(a1v[e], t4.y, y[1][1]);
-                        y[1][2] = fmaf(a1v[e], t4.z, y[1][2]); y[1][3] = fmaf(a1v[e], t4.w, y[1][3]);
-                    }
-                }
-                group_sync(kBarT, kTeam); // A21 is read: Y takes its place
-                float *Yr0 = Wk + (32 + r0) * 32 + ((q0 ^ x0) << 2);
-                float *Yr1 = Wk + (33 + r0) * 32 + ((q0 ^ x1) << 2);
-                *reinterpret_cast<float4 *>(Yr0) = make_float4(y[0][0], y[0][1], y[0][2], y[0][3]);
-                *reinterpret_cast<float4 *>(Yr1) = make_float4(y[1][0], y[1][1], y[1][2], y[1][3]);
-                group_sync(kBarT, kTeam);
-                float x[2][4] = {};
-#pragma unroll 1
-                for (int m = 0; m < 8; ++m) {
-                    const float4 a0 = *reinterpret_cast<const float4 *>(Br0 + ((m ^ x0) << 2));
-                    const float4 a1 = *reinterpret_cast<const float4 *>(Br1 + ((m ^ x1) << 2));
-                    const float a0v[4] = {a0.x, a0.y, a0.z, a0.w}, a1v[4] = {a1.x, a1.y, a1.z, a1.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int i = 32 + 4 * m + e; // Y row i - 32, columns c0 .. + 3
-                        const float4 t4 =
-                            *reinterpret_cast<const float4 *>(Wk + i * 32 + ((q0 ^ (i & 7)) << 2));
-                        x[0][0] = fmaf(a0v[e], t4.x, x[0][0]); x[0][1] = fmaf(a0v[e], t4.y, x[0][1]);
-                        x[0][2] = fmaf(a0v[e], t4.z, x[0][2]); x[0][3] = fmaf(a0v[e], t4.w, x[0][3]);
-                        x[1][0] = fmaf(a1v[e], t4.x, x[1][0]); x[1][1] = fmaf(a1v[e], t4.y, x[1][1]);
-                        x[1][2] = fmaf(a1v[e], t4.z, x[1][2]); x[1][3] = fmaf(a1v[e], t4.w, x[1][3]);
-                    }
-                }
-                group_sync(kBarT, kTeam); // Y is read: T21 takes its place
-                *reinterpret_cast<float4 *>(Yr0) = make_float4(-x[0][0], -x[0][1], -x[0][2], -x[0][3]);
-                *reinterpret_cast<float4 *>(Yr1) = make_float4(-x[1][0], -x[1][1], -x[1][2], -x[1][3]);
-            }
-            // ---- T diag(beta), -T diag(beta gamma) -> the tf32 B operands of MMA 1 and
-            //      2b in the tiles of this chunk's parity, once MMA 2b (and with it
-            //      MMA 1) of chunk c - 2 has read them
-            good = c < 2 || waitq(bar_m2b(c), ((c - 2) >> 1) & 1);
-            group_sync(kBarT, kTeam);
+            group_sync(kBarT, kTeam); // the gates are in
+            // ---- -T diag(beta gamma) = -(T diag beta) diag(gamma) into this chunk's
+            //      parity slot once MMA 2b of chunk c - 2 has read it
+            bool good = waitq(bar_tb(c), (c >> 1) & 1); // T diag(beta) of chunk c landed
+            good = (c < 2 || waitq(bar_m2b(c), ((c - 2) >> 1) & 1)) && good;
             if (good) {
+                const float *tb = sm.Tb[c & 1];
+                float *tg = sm.Tg[c & 1];
                 float4 t4[6];
 #pragma unroll
                 for (int jj = 0; jj < 6; ++jj)
-                    t4[jj] = *reinterpret_cast<const float4 *>(Wk + tri_o(jj));
+                    t4[jj] = *reinterpret_cast<const float4 *>(tb + tr.o(jj));
 #pragma unroll
                 for (int jj = 0; jj < 6; ++jj) {
-                    const float4 b4 = *reinterpret_cast<const float4 *>(&sm.beta[tri_c(jj)]);
-                    const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][tri_c(jj)]);
-                    const float4 tb = make_float4(t4[jj].x * b4.x, t4[jj].y * b4.y, t4[jj].z * b4.z,
-                                                  t4[jj].w * b4.w);
-                    *reinterpret_cast<float4 *>(sm.Tb[c & 1] + tri_o(jj)) = tf32_rna(tb);
-                    *reinterpret_cast<float4 *>(sm.Tg[c & 1] + tri_o(jj)) =
-                        tf32_rna(make_float4(-tb.x * g4.x, -tb.y * g4.y, -tb.z * g4.z, -tb.w * g4.w));
+                    const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][tr.c(jj)]);
+                    *reinterpret_cast<float4 *>(tg + tr.o(jj)) =
+                        tf32_rna(make_float4(-t4[jj].x * g4.x, -t4[jj].y * g4.y, -t4[jj].z * g4.z,
+                                             -t4[jj].w * g4.w));
                 }
             }
             fence_proxy_async_smem();
@@ -793,82 +634,34 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 ok = false;
                 break;
             }
-            if (tt == 0) {
-                mbar_arrive(bar_pT(c)); // T operands and gates of chunk c
-                mbar_arrive(bar_wfree); // Wk may take the next chunk's K K^T rows
-            }
-        }
-        if (!ok)
-            *abort_flag = 1;
-    } else if (warp < (kSG + kTeam + kTeamP) / 32) {
-        // ==================================================== P team
-        const int pt = tid - kSG - kTeam;
-        uint32_t phk = 0, phqk = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int sl = c & 3;
-            // ---- diag(gamma_C / gamma) K in place on the MN-major K tile (the B operand
-            //      of MMA 3's state part), tf32: token row s of every 32-column
-            //      block is 32 consecutive floats (their 32-byte chunks swizzled
-            //      within the row), all scaled by kd[s]
-            bool good = waitq(bar_pT(c), (c >> 2) & 1); // this chunk's gates
-            good = waitp(bar_k, phk) && good;
-            if (good) {
-                // eight float4s in flight a thread: the pass is latency-bound otherwise
-#pragma unroll 1
-                for (int it = 0; it < 4; ++it) {
-                    float4 x[8];
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj)
-                        x[jj] = *reinterpret_cast<const float4 *>(sm.K + 4 * (pt + kTeamP * (8 * it + jj)));
-#pragma unroll
-                    for (int jj = 0; jj < 8; ++jj) {
-                        const int e = pt + kTeamP * (8 * it + jj); // float4 index 0..2047
-                        const float f = sm.kd[sl][(e >> 3) & (kC - 1)];
-                        *reinterpret_cast<float4 *>(sm.K + 4 * e) =
-                            tf32_rna(make_float4(x[jj].x * f, x[jj].y * f, x[jj].z * f, x[jj].w * f));
-                    }
-                }
-            }
-            if (group_sync_or(kBarP, kTeamP, !good || *abort_flag)) {
-                ok = false;
-                break;
-            }
-            // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32
+            if (tt == 0)
+                mbar_arrive(bar_pT(c)); // gates and -T diag(beta gamma) of chunk c
+            // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32 (the Q K^T rows are
+            //      0 for s > r; the clamp keeps the unused upper triangle finite)
             good = waitp(bar_qk, phqk);
             if (good) {
-                // float4 k (k = 0..11) of this thread: rows prow + 8 k of column block 0
-                // (k < 8, columns pcol) or 32 + prow + 8 (k - 8) of block 1; 8 k keeps
-                // r mod 8, so the swizzle term is one constant per thread
-                const int prow = pt >> 3, pcol = 4 * (pt & 7);
-                const int pbase = prow * 32 + (((pt & 7) ^ (prow & 7)) << 2);
-                // six float4s in flight a round: the pass is latency-bound otherwise
+                float4 x[6];
 #pragma unroll
-                for (int h6 = 0; h6 < 12; h6 += 6) {
-                    float4 x[6];
+                for (int jj = 0; jj < 6; ++jj)
+                    x[jj] = *reinterpret_cast<const float4 *>(sm.P + tr.o(jj));
 #pragma unroll
-                    for (int k = 0; k < 6; ++k)
-                        x[k] = *reinterpret_cast<const float4 *>(
-                            sm.P + pbase + (h6 + k < 8 ? 256 * (h6 + k) : 2048 + 256 * (h6 + k - 8)));
-#pragma unroll
-                    for (int k = 0; k < 6; ++k) {
-                        const int kk = h6 + k;
-                        const float Gr = sm.G[sl][kk < 8 ? prow + 8 * kk : 32 + prow + 8 * (kk - 8)];
-                        const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][kk < 8 ? pcol : 32 + pcol]);
-                        *reinterpret_cast<float4 *>(sm.P + pbase + (kk < 8 ? 256 * kk : 2048 + 256 * (kk - 8))) =
-                            tf32_rna(make_float4(x[k].x * __expf(fminf(Gr - Gc.x, 0.f)),
-                                                 x[k].y * __expf(fminf(Gr - Gc.y, 0.f)),
-                                                 x[k].z * __expf(fminf(Gr - Gc.z, 0.f)),
-                                                 x[k].w * __expf(fminf(Gr - Gc.w, 0.f))));
-                    }
+                for (int jj = 0; jj < 6; ++jj) {
+                    const float Gr = sm.G[sl][tr.r(jj)];
+                    const float4 Gc = *reinterpret_cast<const float4 *>(&sm.G[sl][tr.c(jj)]);
+                    *reinterpret_cast<float4 *>(sm.P + tr.o(jj)) =
+                        tf32_rna(make_float4(x[jj].x * __expf(fminf(Gr - Gc.x, 0.f)),
+                                             x[jj].y * __expf(fminf(Gr - Gc.y, 0.f)),
+                                             x[jj].z * __expf(fminf(Gr - Gc.z, 0.f)),
+                                             x[jj].w * __expf(fminf(Gr - Gc.w, 0.f))));
                 }
             }
             fence_proxy_async_smem();
-            if (group_sync_or(kBarP, kTeamP, !good || *abort_flag)) {
+            if (group_sync_or(kBarT, kTeam, !good || *abort_flag)) {
                 ok = false;
                 break;
             }
-            if (pt == 0)
-                mbar_arrive(bar_pP);
+            if (tt == 0)
+                mbar_arrive(bar_pP); // P of chunk c
         }
         if (!ok)
             *abort_flag = 1;
@@ -895,7 +688,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             constexpr uint32_t idT64 = idesc_tf32(128, 64, false, false);  // MMA 2b, MMA 3 O
             constexpr uint32_t idT32 = idesc_tf32(128, 32, false, false);
             constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3 S (B MN-major)
-            uint32_t phv = 0, phkm = 0, phq = 0, phu = 0, phP = 0, ph2 = 0;
+            uint32_t phv = 0, phkm = 0, phq = 0, phu = 0, phP = 0, ph2 = 0, phk = 0;
             // MMA 1 of chunk c: U~^T into U_(c%2).  K steps 0..3 run over column
             // block 0 of the T tile (N = 64), 4..7 over block 1 (rows 32..63)
             auto mma1 = [&](int c) {
@@ -909,15 +702,15 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     mma_tf32_ss_if(dU + 32, dV + s * 64, b1 + 2 * (s - 4), id32, 1, is);
                 mma_commit_if(bar_m1, is);
             };
-            // the inputs of MMA 1 of chunk c: its T tiles (and gates) and V; the
-            // non-blocking form takes lane 0's view, so that all lanes agree
+            // the inputs of MMA 1 of chunk c: its T diag(beta) tile and V (both by TMA);
+            // the non-blocking form takes lane 0's view, so that all lanes agree
             auto m1_ready = [&](int c, bool block) {
                 if (!block)
                     return __shfl_sync(0xffffffffu,
-                                       (int)(mbar_test_wait(bar_pT(c), (c >> 2) & 1) &&
+                                       (int)(mbar_test_wait(bar_tb(c), (c >> 1) & 1) &&
                                              mbar_test_wait(bar_v, phv)),
                                        0) != 0;
-                bool g = waitq(bar_pT(c), (c >> 2) & 1);
+                bool g = waitq(bar_tb(c), (c >> 1) & 1);
                 g = g && waitq(bar_v, phv);
                 return all(g);
             };
@@ -946,8 +739,9 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 mma_commit_if(bar_m2, is);
                 // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
-                good = all(waitp(bar_m2, ph2));
-                if (!good)
+                good = waitp(bar_m2, ph2);
+                good = waitq(bar_pT(c), (c >> 2) & 1) && good; // -T diag(b gamma) of chunk c
+                if (!all(good))
                     break;
                 tc_fence_after();
                 {
@@ -969,9 +763,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     mma1(c + 1);
                     m1_issued = true;
                 }
-                // ---- MMA 3: O^T += U^T P^T, S += U^T (diag(gamma_C/gamma) K) (K MN-major)
+                // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K (K MN-major)
                 good = waitp(bar_u, phu);
-                good = waitp(bar_pP, phP) && good; // P and the scaled K tile
+                good = waitp(bar_pP, phP) && good;
+                good = waitp(bar_k, phk) && good;
                 if (!all(good))
                     break;
                 tc_fence_after();
@@ -985,7 +780,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                         mma_tf32_ts_if(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1, is);
 #pragma unroll 1
                     for (int s = 0; s < kC / 8; ++s)
-                        mma_tf32_ts_if(tmem + kColS, dU + 8 * s, dK + s * 64, idS, 1, is);
+                        mma_tf32_ts_if(tmem + kColS, dXO + 8 * s, dK + s * 64, idS, 1, is);
                 }
                 mma_commit_if(bar_m3, is);
                 if (c + 1 < nchunks && !m1_issued) {
@@ -1010,8 +805,9 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     } else {
         // ==================================================== TMA issue
         if (lane == 0 && nchunks > 0) {
-            uint32_t cnt[7] = {0, 0, 0, 0, 0, 0, 0}; // loads armed on v, q, k, kmaj, kk, qk, z
-            const uint32_t lbar[7] = {bar_v, bar_q, bar_k, bar_kmaj, bar_kk, bar_qk, bar_z};
+            // loads armed on v, q, k, kmaj, tb (parity 0, 1), qk, z
+            uint32_t cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+            const uint32_t lbar[8] = {bar_v, bar_q, bar_k, bar_kmaj, bar_tb(0), bar_tb(1), bar_qk, bar_z};
             // nb 32-column boxes of 64 rows at x0 + 32 b, row t0, block b landing at dst + b * bstride
             auto tile = [&](int which, float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb,
                             int bstride) {
@@ -1020,54 +816,59 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, lbar[which]);
                 ++cnt[which];
             };
-            // a lower-triangular Gram tile: block 0 (64 rows) and the lower half of block 1
-            auto gram = [&](int which, float *dst, int x0, int64_t t0) {
-                mbar_arrive_expect_tx(lbar[which], (uint32_t)(kTriFloats * sizeof(float)));
-                tma_load_2d(smem_u32(dst), &maps.kq, x0, (int)t0, lbar[which]);
-                tma_load_2d(smem_u32(dst + 2048), &maps.kq32, x0 + 32, (int)(t0 + 32), lbar[which]);
-                ++cnt[which];
-            };
             auto t_of = [&](int c) { return start + (int64_t)c * kC; };
+            // the Q K^T rows of chunk c as a triangular tile: block 0 (64 rows) and the
+            // lower half of block 1
+            auto qktile = [&](int c) {
+                mbar_arrive_expect_tx(bar_qk, (uint32_t)(kTriFloats * sizeof(float)));
+                tma_load_2d(smem_u32(sm.P), &maps.kq, xkk, (int)t_of(c), bar_qk);
+                tma_load_2d(smem_u32(sm.P + 2048), &maps.kq32, xkk + 32, (int)(t_of(c) + 32), bar_qk);
+                ++cnt[6];
+            };
+            // T diag(beta) of chunk c: one box of 96 rows (the triangular tile)
+            const int chunk0 = __ldg(p.ws_offs + n); // global index of this sequence's first chunk
+            auto tbtile = [&](int c) {
+                mbar_arrive_expect_tx(bar_tb(c), (uint32_t)(kTriFloats * sizeof(float)));
+                tma_load_2d(smem_u32(sm.Tb[c & 1]), &maps.tb, 0,
+                            (int)(((int64_t)(chunk0 + c) * p.Hv + h) * 96), bar_tb(c));
+                ++cnt[4 + (c & 1)];
+            };
             // the z rows of a chunk: one 128-column box of 64 rows
             auto ztile = [&](int c) {
                 if constexpr (kZTile) {
                     mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
                     tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)t_of(c), bar_z);
-                    ++cnt[6];
+                    ++cnt[7];
                 }
             };
             constexpr int kBlkV = kC * 32, kBlkQ = 2 * kC * 32;
+            tbtile(0);
             tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
             tile(3, sm.KQ, &maps.kmaj, xq, t_of(0), 4, kBlkQ);        // rows 0..63 of KQ
-            gram(4, sm.Wk, xkk, t_of(0));
             tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ); // rows 64..127
+            qktile(0);
             tile(2, sm.K, &maps.k, xq, t_of(0), 4, kBlkV);
-            gram(5, sm.P, xkk + kC, t_of(0));
             ztile(0);
-            if (nchunks > 1) {
-                tma_prefetch_2d(&maps.kq, xkk, (int)t_of(1));
-                tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(1) + 32));
-            }
-            // five event streams, each served in chunk order as it completes
-            int iw = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile ? 0 : nchunks;
+            if (nchunks > 1)
+                tbtile(1);
+            // six event streams, each served in chunk order as it completes
+            int ib = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile ? 0 : nchunks;
             long long t_last = clock64();
-            while (iw < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
+            while (ib < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
                 bool prog = false;
                 // the epilogue of chunk iz has released the z tile
-                if (iz < nchunks && mbar_test_wait((iz & 1) ? bar_of1 : bar_of0, (iz >> 1) & 1)) {
+                if (iz < nchunks && mbar_test_wait(bar_zf, iz & 1)) {
                     if (iz + 1 < nchunks)
                         ztile(iz + 1);
                     ++iz;
                     prog = true;
                 }
-                if (iw < nchunks && mbar_test_wait(bar_wfree, iw & 1)) { // Wk is free
-                    if (iw + 1 < nchunks)
-                        gram(4, sm.Wk, xkk, t_of(iw + 1));
-                    if (iw + 2 < nchunks) {
-                        tma_prefetch_2d(&maps.kq, xkk, (int)t_of(iw + 2));
-                        tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(iw + 2) + 32));
-                    }
-                    ++iw;
+                // MMA 1 (seen below, i1 > ib) and the prep team (its gates-and-Tg
+                // arrival) have read T diag(beta) of chunk ib: its slot takes chunk ib + 2
+                if (ib < nchunks && i1 > ib && mbar_test_wait(bar_pT(ib), (ib >> 2) & 1)) {
+                    if (ib + 2 < nchunks)
+                        tbtile(ib + 2);
+                    ++ib;
                     prog = true;
                 }
                 if (i1 < nchunks && mbar_test_wait(bar_m1, i1 & 1)) { // V is free
@@ -1086,7 +887,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 if (i3 < nchunks && mbar_test_wait(bar_m3, i3 & 1)) { // P and K (MN-major) are free
                     if (i3 + 1 < nchunks) {
-                        gram(5, sm.P, xkk + kC, t_of(i3 + 1));
+                        qktile(i3 + 1);
                         tile(2, sm.K, &maps.k, xq, t_of(i3 + 1), 4, kBlkV);
                     }
                     ++i3;
@@ -1103,7 +904,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             // every armed load lands before the CTA exits
 #pragma unroll
-            for (int b = 0; b < 7; ++b)
+            for (int b = 0; b < 8; ++b)
                 if (cnt[b] > 0)
                     mbar_wait_bounded(lbar[b], (cnt[b] - 1) & 1, kWaitLimit);
             if (!ok)
@@ -1148,7 +949,8 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
     memset(&maps, 0, sizeof(maps));
     if (p.N > 0) {
         const uint64_t N = (uint64_t)p.N, F = sizeof(float);
-        const uint64_t qkw = 2ull * p.Hk * kD, kqw = (uint64_t)p.Hk * 2 * kC;
+        const uint64_t qkw = 2ull * p.Hk * kD, kqw = (uint64_t)p.Hk * kC;
+        const uint64_t tb_rows = (uint64_t)((p.N + kC - 1) / kC + p.batch) * p.Hv * 96;
         const bool okm =
             encode_2d(&maps.v, p.ws_v, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * F, 32, kC,
                       CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
@@ -1160,6 +962,7 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
                       qkw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&maps.kq, p.ws_kq, kqw, N, kqw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B) &&
             encode_2d(&maps.kq32, p.ws_kq, kqw, N, kqw * F, 32, 32, CU_TENSOR_MAP_SWIZZLE_128B) &&
+            encode_2d(&maps.tb, p.ws_tb, 32, tb_rows, 32 * F, 32, 96, CU_TENSOR_MAP_SWIZZLE_128B) &&
             (sizeof(T) != 2 ||
              (encode_2d(&maps.z, p.z, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * sizeof(T), kD, kC,
                         CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) &&
@@ -1175,7 +978,18 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 
 } // namespace
 
-size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * 2 * kC * sizeof(float); }
+size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * kC * sizeof(float); }
+
+// T diag(beta) tiles: one per (chunk, value head), 96 rows of 32 floats; every
+// sequence adds at most one partial chunk to the N / 64 full ones.
+size_t tb_workspace_bytes(int Hv, int64_t N, int batch) {
+    return (size_t)((N + kC - 1) / kC + batch) * Hv * 96 * 32 * sizeof(float);
+}
+
+// K K^T triangular tiles: one per (chunk, q/k head).
+size_t kk_workspace_bytes(int Hk, int64_t N, int batch) {
+    return (size_t)((N + kC - 1) / kC + batch) * Hk * kTriFloats * sizeof(float);
+}
 
 cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s) {
     // no tokens: no workspace (the offsets and status words have no home) and

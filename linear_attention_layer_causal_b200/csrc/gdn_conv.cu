@@ -1,8 +1,6 @@
-// gdn_conv.cu -- prefill front end: conv + SiLU (+ L2 norm of q and k) of the
-// pre-conv channels (the per-thread body is in gdn_conv.cuh) -- every channel
-// for the token-serial path, the v channels for the tensor-core path, whose q
-// and k go through the fused q/k front kernel -- and the final conv window of
-// every sequence.
+// gdn_conv.cu -- prefill front end: conv + SiLU + L2 norm of every q|k|v
+// channel (the per-thread body is in gdn_conv.cuh), and the final conv window
+// of every sequence.
 #include "gdn_conv.cuh"
 #include "gdn_internal.h"
 
@@ -22,9 +20,8 @@ __global__ void __launch_bounds__(kConvThreads, sizeof(VecT) == 8 ? 4 : 1) // 8-
 conv_prep_kernel(ConvIO<T> io, unsigned int *__restrict__ err) {
     constexpr int V = VecT::N;
     const int C = (2 * io.Hk + io.Hv) * D;
-    // on the token-serial path this is the first kernel of a call: it clears the
-    // call's status words (the chunked path clears them in its offsets kernel)
-    if (err != nullptr && !io.v_only && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
+    // the first kernel of a token-serial call clears the call's status words
+    if (err != nullptr && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) {
         err[0] = 0u; // status word of this call; later kernels only set bits
         err[1] = 0u; // where the first timed-out wait gave up
     }
@@ -86,26 +83,27 @@ ConvIO<T> conv_io(const PrefillArgs &p) {
     io.qk_out = (float *)p.ws_qk;
     io.v_out = (float *)p.ws_v;
     io.round_v = p.chunked;
-    io.v_only = false;
     io.block_y0 = 0;
     return io;
 }
 
 template <typename T, int D, typename VecT = Vec16<T>>
-cudaError_t launch_conv_prep_t(const PrefillArgs &p, cudaStream_t s) {
+cudaError_t launch_conv_prep_t(const PrefillArgs &p, ConvPart part, cudaStream_t s) {
     constexpr int V = VecT::N;
     const int C = (2 * p.Hk + p.Hv) * D;
     ConvIO<T> io = conv_io<T>(p);
-    // the tensor-core path takes q and k from the fused q/k front kernel: only
-    // the blocks holding v channels run, and a block that straddles the q/k | v
-    // boundary writes only its v channels
-    if (p.chunked) {
-        io.v_only = true;
-        io.block_y0 = 2 * p.Hk * D / V / kConvThreads;
-    }
-    const int nby = (C / V + kConvThreads - 1) / kConvThreads - io.block_y0;
+    // channel blocks: those holding any q or k channel come first (a block that
+    // straddles the q/k | v boundary belongs to them and writes its v channels too)
+    const int nb = (C / V + kConvThreads - 1) / kConvThreads;
+    const int nqk = (2 * p.Hk * D / V + kConvThreads - 1) / kConvThreads;
+    io.block_y0 = part == ConvPart::kV ? nqk : 0;
+    const int nby = part == ConvPart::kAll ? nb : (part == ConvPart::kQK ? nqk : nb - nqk);
+    if (nby <= 0)
+        return cudaSuccess;
     dim3 grid((unsigned)((p.N + kConvTokens - 1) / kConvTokens), nby);
-    conv_prep_kernel<T, D, VecT><<<grid, kConvThreads, 0, s>>>(io, p.ws_err);
+    // the chunked path's offsets kernel clears the status words; the token-serial
+    // path's single conv launch does
+    conv_prep_kernel<T, D, VecT><<<grid, kConvThreads, 0, s>>>(io, p.chunked ? nullptr : p.ws_err);
     return cudaGetLastError();
 }
 
@@ -120,13 +118,14 @@ template <typename T> cudaError_t launch_final_conv_t(const PrefillArgs &p, cuda
 
 } // namespace
 
-cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s) {
+cudaError_t launch_conv_prep(const PrefillArgs &p, ConvPart part, cudaStream_t s) {
     if (p.N == 0)
         return cudaSuccess;
     if (p.bf16)
-        return p.D == 128 ? launch_conv_prep_t<__nv_bfloat16, 128, Vec8bf>(p, s)
-                          : launch_conv_prep_t<__nv_bfloat16, 32>(p, s);
-    return p.D == 128 ? launch_conv_prep_t<float, 128>(p, s) : launch_conv_prep_t<float, 32>(p, s);
+        return p.D == 128 ? launch_conv_prep_t<__nv_bfloat16, 128, Vec8bf>(p, part, s)
+                          : launch_conv_prep_t<__nv_bfloat16, 32>(p, part, s);
+    return p.D == 128 ? launch_conv_prep_t<float, 128>(p, part, s)
+                      : launch_conv_prep_t<float, 32>(p, part, s);
 }
 
 cudaError_t launch_final_conv(const PrefillArgs &p, cudaStream_t s) {

@@ -52,7 +52,6 @@ template <typename T> struct ConvIO {
     float *qk_out;         // [N, 2 Hk D] normalised q | k
     float *v_out;          // [N, Hv D] convolved v
     bool round_v;          // v to its tf32 operand (tensor-core path)
-    bool v_only;           // only the v channels: q and k come from the fused q/k front kernel
     int block_y0;          // channel block of blockIdx.y = 0 (skips the q/k-only blocks)
 };
 
@@ -111,7 +110,7 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
         }
         if (norm_warp)
             ss = group_sum<LANES>(ss);
-        if (!active || (io.v_only && region < 2))
+        if (!active)
             return;
         const float f = region == 2 ? 1.0f : rsqrtf(ss + io.l2_eps) * (region == 0 ? io.q_scale : 1.0f);
         if (region == 2 && io.round_v) {

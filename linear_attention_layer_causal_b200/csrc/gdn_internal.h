@@ -30,7 +30,9 @@ struct PrefillArgs {
     unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)
     void *ws_qk;             // [N, 2*Hk*D] float32: normalised q | k
     void *ws_v;              // [N, Hv*D]   float32: convolved v
-    void *ws_kq;             // [N, Hk, 2, 64] float32: chunk Gram rows (chunked path)
+    void *ws_kq;             // [N, Hk, 64] float32: chunk Q K^T rows (chunked path)
+    void *ws_kk;             // [chunks, Hk, 3072] float32: K K^T triangular tiles (chunked path)
+    void *ws_tb;             // [chunks, Hv, 96, 32] float32: T diag(beta) tiles (chunked path)
     int32_t *ws_offs;        // [batch + 1] chunk offsets per sequence (chunked path)
 };
 
@@ -73,6 +75,16 @@ gdn_status validate_prefill(const gdn_config *cfg, const gdn_params *params, con
                             const void *initial_conv, const void *y, const float *final_state,
                             const void *final_conv, const float *o_raw, size_t *need);
 
+// gdn_prefill itself; `side` allows the chunked path to run the v conv on a
+// second stream of its own (gdn_prefill_noalloc passes false: it creates
+// nothing, and runs every kernel on the caller's stream in order).
+gdn_status prefill_impl(const gdn_config *cfg, const gdn_params *params, const void *qkv,
+                        const void *a, const void *b, const void *z, const int32_t *cu_seqlens,
+                        int32_t batch, int64_t total_tokens, const float *initial_state,
+                        const void *initial_conv, void *y, float *final_state, void *final_conv,
+                        float *o_raw, void *workspace, size_t workspace_bytes, void *stream,
+                        bool side);
+
 // Reads the two status words at `header` (device) after `stream` completes.
 gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t stream);
 
@@ -85,13 +97,19 @@ inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
 size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N, int batch);
 constexpr size_t kWorkspaceHeader = 256; // holds the device status word
 
-cudaError_t launch_conv_prep(const PrefillArgs &p, cudaStream_t s);
+// Which channels a conv launch covers: all, the channel blocks holding q or k
+// (and the v channels of a block that straddles the boundary), or the rest.
+enum class ConvPart { kAll, kQK, kV };
+cudaError_t launch_conv_prep(const PrefillArgs &p, ConvPart part, cudaStream_t s);
 cudaError_t launch_final_conv(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_recurrent_prefill(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_chunk_offsets(const PrefillArgs &p, cudaStream_t s);
-cudaError_t launch_qk_front(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_gram(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_tri(const PrefillArgs &p, cudaStream_t s);
 cudaError_t launch_chunk_prefill(const PrefillArgs &p, cudaStream_t s);
 size_t kq_workspace_bytes(int Hk, int64_t N);
+size_t tb_workspace_bytes(int Hv, int64_t N, int batch);
+size_t kk_workspace_bytes(int Hk, int64_t N, int batch);
 cudaError_t launch_decode(const DecodeArgs &p, cudaStream_t s);
 cudaError_t launch_decode_multi(const DecodeArgs &p, int mode, cudaStream_t s);
 size_t decode_multi_smem_bytes(int G, int D, int k, int mode);

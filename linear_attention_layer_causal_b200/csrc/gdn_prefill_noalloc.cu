@@ -77,9 +77,10 @@ extern "C" gdn_status gdn_prefill_noalloc(const gdn_config *cfg, const gdn_param
     // call clears the status words, and the front-end kernels write every
     // element the recurrence later reads, so the previous call's contents
     // never leak into this one.
-    return gdn_prefill(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens, initial_state,
-                       initial_conv, y, final_state, final_conv, o_raw, scratch,
-                       scratch ? kScratchBytes : 0, stream);
+    // every kernel on the caller's stream: no second stream is created here
+    return gdn::prefill_impl(cfg, params, qkv, a, b, z, cu_seqlens, batch, total_tokens,
+                             initial_state, initial_conv, y, final_state, final_conv, o_raw,
+                             scratch, scratch ? kScratchBytes : 0, stream, false);
 }
 
 extern "C" gdn_status gdn_prefill_noalloc_status(uint32_t *detail, void *stream) {

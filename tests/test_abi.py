@@ -47,10 +47,14 @@ QWEN38 = gdn.Config(16, 128, 128)
 def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
     # 256-byte header (status word), float32 normalised q|k and convolved v, and
-    # for head_dim 128 the chunk Gram rows [N, H_k, 2, 64] and the chunk offsets
-    # [batch + 1]; regions rounded to 256 B
-    assert n == 256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 2 * 64 * 4 + 256
-    assert gdn.prefill_workspace_size(QWEN38, 100, 4096) == n + 256  # 101 offsets: 512 bytes
+    # for head_dim 128 the chunks' Q K^T rows [N, H_k, 64], K K^T tiles
+    # [N / 64 + batch chunks, H_k, 3072], T diag(beta) tiles [chunks, H_v, 96, 32]
+    # and the chunk offsets [batch + 1]; regions rounded to 256 B
+    tile = 128 * 96 * 32 * 4 + 16 * 3072 * 4  # one chunk's tiles, all heads
+    assert n == (256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 64 * 4 +
+                 (64 + 1) * tile + 256)
+    # 99 more sequences: at most 99 more (partial) chunks, and 512 bytes of offsets
+    assert gdn.prefill_workspace_size(QWEN38, 100, 4096) == n + 99 * tile + 256
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
     # sequences but no tokens: nothing for a kernel to stage, and no workspace (the
     # launches that would need one -- chunk offsets, status words -- are skipped)

@@ -55,17 +55,26 @@ def test_noalloc_matches_prefill_on_consecutive_calls(cuda_device):
         _check(*_both(cfg, inp, conv))
 
 
+def _limit(cfg):
+    """The most tokens one sequence can have within the fixed scratch."""
+    n = 1
+    while gdn.prefill_workspace_size(cfg, 1, n + 1) <= gdn.NOALLOC_SCRATCH_BYTES:
+        n += 1
+    return n
+
+
 def test_noalloc_largest_call_and_limit(cuda_device):
-    """At the Qwen3.8 layer shape the fixed scratch holds 744 tokens: 744 runs and
-    matches gdn_prefill, 745 is rejected before anything is launched."""
-    wl = W.Workload("noalloc_max", 16, 128, 128, seqlens=(744,), state_std=0.02, seed=3)
-    cfg = gdn.Config.of(wl)
-    assert gdn.prefill_workspace_size(cfg, 1, 744) <= gdn.NOALLOC_SCRATCH_BYTES
-    assert gdn.prefill_workspace_size(cfg, 1, 745) > gdn.NOALLOC_SCRATCH_BYTES
+    """At the Qwen3.8 layer shape the fixed scratch holds a few hundred tokens of
+    one sequence: the largest such call runs and matches gdn_prefill, one token
+    more is rejected before anything is launched."""
+    cfg = gdn.Config(16, 128, 128)
+    lim = _limit(cfg)
+    assert lim >= 512
+    wl = W.Workload("noalloc_max", 16, 128, 128, seqlens=(lim,), state_std=0.02, seed=3)
     inp = W.make_prefill(wl, cuda_device)
     _check(*_both(cfg, inp))
-    big = W.make_prefill(wl, cuda_device, seqlens=(745,), seed=4)
-    y = torch.empty((745, 128, 128), dtype=torch.bfloat16, device=cuda_device)
+    big = W.make_prefill(wl, cuda_device, seqlens=(lim + 1,), seed=4)
+    y = torch.empty((lim + 1, 128, 128), dtype=torch.bfloat16, device=cuda_device)
     with pytest.raises(gdn.GdnError) as e:
         gdn.prefill_noalloc(cfg, big["qkv"], big["a"], big["b"], big["z"], big["cu_seqlens"],
                             *[big[k] for k in P], y=y)
