@@ -252,6 +252,56 @@ GDN_API gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *pa
                                      const int32_t *accepted, void *stream);
 
 /*
+ * Kimi Delta Attention (KDA), the per-channel-decay variant of the mixer
+ * ("Inkling vs Kimi K3", component table, linear-attention row: 96 heads of
+ * dimension 128, kernel-4 conv + SiLU on q, k and v, L2-normalised q and k,
+ * per-channel log-decay g = -5 sigmoid(exp(A) z); output-gate row: the
+ * head-wise RMSNorm of the recurrent output times a full-rank channel-wise
+ * sigmoid gate).  Per head (one q, k and v head each: cfg->num_qk_heads must
+ * equal cfg->num_v_heads) and token, with alpha = exp(g) in R^{d_k}:
+ *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *     o_t = S_t q_t,   beta_t = sigmoid(b_t),
+ *     y_t = o_t / sqrt(mean(o_t^2) + rms_eps) * norm_w * sigmoid(gate_t).
+ * Arithmetic is FP32 on CUDA cores (token-serial prefill, one-token decode).
+ */
+typedef struct gdn_kda_params {
+    const float *conv_w; /* [3 H d, conv_kernel] (q heads, k heads, v heads) */
+    const float *A_log;  /* [H]: the decay scale exp(A_log[h]) of head h */
+    const float *norm_w; /* [d], shared by all heads */
+} gdn_kda_params;
+
+/* Workspace bytes of gdn_kda_prefill (as gdn_prefill_workspace_size). */
+GDN_API gdn_status gdn_kda_prefill_workspace_size(const gdn_config *cfg, int32_t batch,
+                                                  int64_t total_tokens, size_t *bytes);
+
+/*
+ * KDA prefill over a packed varlen batch; conventions, cu_seqlens, states,
+ * conv windows, o_raw and workspace as in gdn_prefill.
+ *   qkv   [N, 3 H d]  act_dtype   pre-conv q|k|v rows
+ *   zdec  [N, H, d]   act_dtype   per-channel decay inputs z
+ *   b     [N, H]      act_dtype   write-strength inputs
+ *   gate  [N, H, d]   act_dtype   output-gate inputs (sigmoid applied here)
+ *   y     [N, H, d]   act_dtype   output
+ */
+GDN_API gdn_status gdn_kda_prefill(const gdn_config *cfg, const gdn_kda_params *params,
+                                   const void *qkv, const void *zdec, const void *b,
+                                   const void *gate, const int32_t *cu_seqlens, int32_t batch,
+                                   int64_t total_tokens, const float *initial_state,
+                                   const void *initial_conv, void *y, float *final_state,
+                                   void *final_conv, float *o_raw, void *workspace,
+                                   size_t workspace_bytes, void *stream);
+
+/*
+ * KDA decode: one token per sequence against resident states, which are
+ * updated in place, as is the conv cache (layouts as gdn_decode, with zdec
+ * [batch, H, d], b [batch, H] and gate [batch, H, d]).  Needs no workspace.
+ */
+GDN_API gdn_status gdn_kda_decode(const gdn_config *cfg, const gdn_kda_params *params,
+                                  const void *qkv, const void *zdec, const void *b,
+                                  const void *gate, float *state, void *conv_cache, int32_t batch,
+                                  void *y, void *stream);
+
+/*
  * Size of the fixed device scratch array used by gdn_prefill_noalloc:
  * 64 MiB, held on every GPU that loads the library until the process exits.
  */

@@ -35,7 +35,8 @@ GDN_F32, GDN_BF16 = 0, 1
 EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_status_string",
             "gdn_abi_version", "gdn_profile_next_call", "gdn_prefill_noalloc",
             "gdn_prefill_status", "gdn_prefill_noalloc_status", "gdn_wait_limit_next_call",
-            "gdn_decode_multi", "gdn_decode_verify", "gdn_decode_commit")
+            "gdn_decode_multi", "gdn_decode_verify", "gdn_decode_commit",
+            "gdn_kda_prefill_workspace_size", "gdn_kda_prefill", "gdn_kda_decode")
 
 # Fixed scratch of gdn_prefill_noalloc (GDN_NOALLOC_SCRATCH_BYTES in include/gdn.h).
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -53,6 +54,11 @@ class _Config(ctypes.Structure):
                 ("rms_eps", ctypes.c_float), ("l2_eps", ctypes.c_float),
                 ("q_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32),
                 ("algo", ctypes.c_int32)]
+
+
+class _KdaParams(ctypes.Structure):
+    _fields_ = [("conv_w", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
+                ("norm_w", ctypes.c_void_p)]
 
 
 class _Params(ctypes.Structure):
@@ -119,6 +125,14 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode_verify.restype = ctypes.c_int
         L.gdn_decode_commit.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i32, vp, vp]
         L.gdn_decode_commit.restype = ctypes.c_int
+        kpp = ctypes.POINTER(_KdaParams)
+        L.gdn_kda_prefill_workspace_size.argtypes = [cfgp, i32, i64, ctypes.POINTER(sz)]
+        L.gdn_kda_prefill_workspace_size.restype = ctypes.c_int
+        L.gdn_kda_prefill.argtypes = [cfgp, kpp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, vp,
+                                      vp, vp, sz, vp]
+        L.gdn_kda_prefill.restype = ctypes.c_int
+        L.gdn_kda_decode.argtypes = [cfgp, kpp, vp, vp, vp, vp, vp, vp, i32, vp, vp]
+        L.gdn_kda_decode.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
         L.gdn_profile_next_call.argtypes = [vp, vp]
@@ -357,3 +371,68 @@ def decode_commit(cfg: Config, qkv, a, b, state, conv_cache, accepted, conv_w, A
                                  qkv.shape[0], qkv.shape[1], _ptr(accepted), _stream(stream))
     if st != GDN_OK:
         raise GdnError(st, "gdn_decode_commit")
+
+
+# ------------------------------------------------------------------ KDA
+
+
+def kda_prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    st = lib().gdn_kda_prefill_workspace_size(ctypes.byref(cfg._c()), batch, total_tokens,
+                                              ctypes.byref(n))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_kda_prefill_workspace_size")
+    return n.value
+
+
+def kda_prefill(cfg: Config, qkv, zdec, b, gate, cu_seqlens, conv_w, A_log, norm_w, *,
+                initial_state=None, initial_conv=None, return_final_state=False,
+                return_final_conv=False, return_o_raw=False, y=None, final_state=None,
+                final_conv=None, workspace=None, stream=None) -> dict:
+    """Kimi Delta Attention prefill (gdn_kda_prefill): per-key-channel decay
+    g = -5 sigmoid(exp(A_log) zdec), y = RMSNorm(o) * norm_w * sigmoid(gate)."""
+    import torch
+    N = qkv.shape[0]
+    B = cu_seqlens.shape[0] - 1
+    H, d, dev = cfg.num_v_heads, cfg.head_dim, qkv.device
+    if y is None:
+        y = torch.empty((N, H, d), dtype=_act(cfg), device=dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, d, d), dtype=torch.float32, device=dev)
+    if final_conv is None and return_final_conv:
+        final_conv = torch.empty((B, cfg.conv_kernel - 1, cfg.conv_dim), dtype=_act(cfg), device=dev)
+    o_raw = torch.empty((N, H, d), dtype=torch.float32, device=dev) if return_o_raw else None
+    if workspace is None:
+        workspace = torch.empty(max(kda_prefill_workspace_size(cfg, B, N), 1), dtype=torch.uint8,
+                                device=dev)
+    par = _KdaParams(_ptr(conv_w), _ptr(A_log), _ptr(norm_w))
+    st = lib().gdn_kda_prefill(ctypes.byref(cfg._c()), ctypes.byref(par), _ptr(qkv), _ptr(zdec),
+                               _ptr(b), _ptr(gate), _ptr(cu_seqlens), B, N, _ptr(initial_state),
+                               _ptr(initial_conv), _ptr(y), _ptr(final_state), _ptr(final_conv),
+                               _ptr(o_raw), _ptr(workspace), workspace.numel(), _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_kda_prefill")
+    out = {"y": y}
+    if final_state is not None:
+        out["final_state"] = final_state
+    if final_conv is not None:
+        out["final_conv"] = final_conv
+    if o_raw is not None:
+        out["o_raw"] = o_raw
+    return out
+
+
+def kda_decode(cfg: Config, qkv, zdec, b, gate, state, conv_cache, conv_w, A_log, norm_w, *,
+               y=None, stream=None):
+    """One KDA token per sequence; `state` and `conv_cache` are updated in place.  Returns y."""
+    import torch
+    B = qkv.shape[0]
+    if y is None:
+        y = torch.empty((B, cfg.num_v_heads, cfg.head_dim), dtype=_act(cfg), device=qkv.device)
+    par = _KdaParams(_ptr(conv_w), _ptr(A_log), _ptr(norm_w))
+    st = lib().gdn_kda_decode(ctypes.byref(cfg._c()), ctypes.byref(par), _ptr(qkv), _ptr(zdec),
+                              _ptr(b), _ptr(gate), _ptr(state), _ptr(conv_cache), B, _ptr(y),
+                              _stream(stream))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_kda_decode")
+    return y

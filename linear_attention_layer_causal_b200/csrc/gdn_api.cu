@@ -456,4 +456,162 @@ gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *params, co
                        accepted, nullptr, stream, kDecodeCommit);
 }
 
+// ------------------------------------------------------------------- KDA
+
+namespace {
+
+gdn_status kda_check(const gdn_config *cfg, const gdn_kda_params *params) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if (cfg->num_qk_heads != cfg->num_v_heads) // one q and one k per head
+        return GDN_ERR_INVALID_ARG;
+    if (params == nullptr || params->conv_w == nullptr || params->A_log == nullptr ||
+        params->norm_w == nullptr || !aligned16(params->conv_w) || !aligned16(params->norm_w) ||
+        (reinterpret_cast<uintptr_t>(params->A_log) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+} // namespace
+
+gdn_status gdn_kda_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
+                                          size_t *bytes) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if (cfg->num_qk_heads != cfg->num_v_heads)
+        return GDN_ERR_INVALID_ARG;
+    if (bytes == nullptr || batch < 0 || total_tokens < 0)
+        return GDN_ERR_INVALID_ARG;
+    // the token-serial path's regions: header, normalised q|k, convolved v
+    *bytes = total_tokens == 0 ? 0
+                               : kWorkspaceHeader + round_up((size_t)total_tokens * 2 * cfg->num_qk_heads * cfg->head_dim * 4) +
+                                     round_up((size_t)total_tokens * cfg->num_v_heads * cfg->head_dim * 4);
+    return GDN_OK;
+}
+
+gdn_status gdn_kda_prefill(const gdn_config *cfg, const gdn_kda_params *params, const void *qkv,
+                           const void *zdec, const void *b, const void *gate,
+                           const int32_t *cu_seqlens, int32_t batch, int64_t total_tokens,
+                           const float *initial_state, const void *initial_conv, void *y,
+                           float *final_state, void *final_conv, float *o_raw, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+    gdn_status st = kda_check(cfg, params);
+    if (st != GDN_OK)
+        return st;
+    if (batch < 0 || total_tokens < 0 || batch > 65535)
+        return batch > 65535 ? GDN_ERR_UNSUPPORTED : GDN_ERR_INVALID_ARG;
+    if ((batch == 0 && total_tokens > 0) || (batch > 0 && cu_seqlens == nullptr))
+        return GDN_ERR_INVALID_ARG;
+    const bool bf16 = cfg->act_dtype == GDN_BF16;
+    if (total_tokens > 0 && (qkv == nullptr || zdec == nullptr || b == nullptr || gate == nullptr ||
+                             y == nullptr))
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(zdec) || !aligned16(gate) || !aligned16(y) ||
+        !aligned16(initial_state) || !aligned16(initial_conv) || !aligned16(final_state) ||
+        !aligned16(final_conv) || !aligned16(o_raw) || !elem_aligned(b, bf16) ||
+        (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
+        return GDN_ERR_INVALID_ARG;
+    size_t need = 0;
+    gdn_kda_prefill_workspace_size(cfg, batch, total_tokens, &need);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need ||
+                     (reinterpret_cast<uintptr_t>(workspace) & 255u)))
+        return GDN_ERR_WORKSPACE;
+    PrefillArgs p{};
+    p.Hk = cfg->num_qk_heads;
+    p.Hv = cfg->num_v_heads;
+    p.D = cfg->head_dim;
+    p.G = 1;
+    p.bf16 = bf16;
+    p.rms_eps = cfg->rms_eps;
+    p.l2_eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale;
+    p.qkv = qkv; p.b = b; p.z = gate;
+    p.kda_zdec = zdec;
+    p.cu = cu_seqlens;
+    p.batch = batch;
+    p.N = total_tokens;
+    p.init_state = initial_state;
+    p.init_conv = initial_conv;
+    p.y = y;
+    p.final_state = final_state;
+    p.final_conv = final_conv;
+    p.o_raw = o_raw;
+    p.conv_w = params->conv_w;
+    p.A_log = params->A_log;
+    p.norm_w = params->norm_w;
+    p.chunked = false;
+    p.wait_limit = kDefaultWaitLimit;
+    if (need > 0) {
+        char *w = (char *)workspace;
+        p.ws_err = (unsigned int *)w;
+        p.ws_qk = w + kWorkspaceHeader;
+        p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    const ProfileHook hook = take_profile_hook();
+    if (batch == 0)
+        return GDN_OK;
+    cudaError_t e = launch_conv_prep(p, ConvPart::kAll, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.begin, s);
+    if (e == cudaSuccess)
+        e = launch_kda_prefill(p, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.end, s);
+    if (e == cudaSuccess)
+        e = launch_final_conv(p, s);
+    return cuda_status(e);
+}
+
+gdn_status gdn_kda_decode(const gdn_config *cfg, const gdn_kda_params *params, const void *qkv,
+                          const void *zdec, const void *b, const void *gate, float *state,
+                          void *conv_cache, int32_t batch, void *y, void *stream) {
+    gdn_status st = kda_check(cfg, params);
+    if (st != GDN_OK)
+        return st;
+    if (batch < 0)
+        return GDN_ERR_INVALID_ARG;
+    if (batch > 65535)
+        return GDN_ERR_UNSUPPORTED;
+    if (batch == 0) {
+        take_profile_hook();
+        return GDN_OK;
+    }
+    const bool bf16 = cfg->act_dtype == GDN_BF16;
+    if (qkv == nullptr || zdec == nullptr || b == nullptr || gate == nullptr || state == nullptr ||
+        conv_cache == nullptr || y == nullptr)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned16(qkv) || !aligned16(zdec) || !aligned16(gate) || !aligned16(y) ||
+        !aligned16(state) || !aligned16(conv_cache) || !elem_aligned(b, bf16))
+        return GDN_ERR_INVALID_ARG;
+    DecodeArgs p{};
+    p.Hk = cfg->num_qk_heads;
+    p.Hv = cfg->num_v_heads;
+    p.D = cfg->head_dim;
+    p.G = 1;
+    p.bf16 = bf16;
+    p.rms_eps = cfg->rms_eps;
+    p.l2_eps = cfg->l2_eps;
+    p.q_scale = cfg->q_scale;
+    p.qkv = qkv; p.b = b; p.z = gate;
+    p.kda_zdec = zdec;
+    p.state = state;
+    p.conv_cache = conv_cache;
+    p.batch = batch;
+    p.y = y;
+    p.conv_w = params->conv_w;
+    p.A_log = params->A_log;
+    p.norm_w = params->norm_w;
+    cudaStream_t s = (cudaStream_t)stream;
+    const ProfileHook hook = take_profile_hook();
+    cudaError_t e = record_if(hook.begin, s);
+    if (e == cudaSuccess)
+        e = launch_kda_decode(p, s);
+    if (e == cudaSuccess)
+        e = record_if(hook.end, s);
+    return cuda_status(e);
+}
+
 } // extern "C"

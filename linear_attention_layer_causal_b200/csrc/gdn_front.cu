@@ -19,13 +19,14 @@
 // q and k rows it has read go back rounded to nearest tf32: the chunk kernel's
 // tensor-core products read them there.
 //
-// tri_kernel, one CTA of 128 threads per (chunk, value head h): the gates of
-// the chunk's tokens (g = -exp(A_log) softplus(a + dt_bias), beta = sigmoid(b),
-// G = prefix sums of g; Gated DeltaNet row), A[r][s] = beta_r exp(G_r - G_s)
-// kk[r][s], T = (I + A)^-1 by block doubling in FP32 (gdn_tri.cuh), and
-// T diag(beta) rounded to nearest tf32 into the workspace as 96 rows of 32
-// floats: the B operand of the chunk kernel's first product, ready for a TMA
-// load with 128-byte swizzle.
+// tri_kernel, 64 threads per (chunk, value head h), two value heads a CTA:
+// the gates of the chunk's tokens (g = -exp(A_log) softplus(a + dt_bias),
+// beta = sigmoid(b), G = prefix sums of g; Gated DeltaNet row),
+// A[r][s] = beta_r exp(G_r - G_s) kk[r][s], T = (I + A)^-1 in FP32 by forward
+// substitution with one column per thread (no barriers; the rows of A are
+// broadcast reads), and T diag(beta) rounded to nearest tf32 into the
+// workspace as 96 rows of 32 floats: the B operand of the chunk kernel's first
+// product, ready for a TMA load with 128-byte swizzle.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
@@ -223,26 +224,62 @@ __device__ __forceinline__ void chunk_of(const int32_t *__restrict__ cu, const i
     nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
 }
 
+// One column of T = (I + A)^-1 by forward substitution, in registers: with
+// x[r] = T[r][c], x[r] = 0 (r < c), x[c] = 1, x[r] = -sum_{s<r} A[r][s] x[s]
+// (r > c).  A is strictly lower triangular in the triangular-tile layout; every
+// thread of a warp reads the same row of A (broadcast).  FIRST = 32 for the
+// warp of columns 32..63: its rows and terms below 32 are zero and skipped.
+template <int FIRST>
+__device__ __forceinline__ void tri_column(const float *__restrict__ A, int c, float (&x)[kC]) {
+#pragma unroll
+    for (int r = 0; r < kC; ++r)
+        x[r] = 0.f;
+#pragma unroll
+    for (int r = FIRST; r < kC; ++r) {
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int s4 = FIRST; s4 < r; s4 += 4) {
+            // A[r][s4 .. s4 + 3]: column block s4 / 32, 16-byte chunk (s4 % 32) / 4
+            const int blk = s4 >> 5, ch = (s4 & 31) >> 2;
+            const float4 a = *reinterpret_cast<const float4 *>(A + 1024 * blk + 32 * r + ((ch ^ (r & 7)) << 2));
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (s4 + e < r)
+                    acc[e] = fmaf(av[e], x[s4 + e], acc[e]);
+        }
+        const float v = -((acc[0] + acc[1]) + (acc[2] + acc[3]));
+        x[r] = r < c ? 0.f : (r == c ? 1.f : v);
+    }
+}
+
+// Two value heads a CTA (64 threads each, named barrier 1 + head): gates, A in
+// shared memory, then T = (I + A)^-1 one column per thread, and T diag(beta)
+// straight to the workspace (a warp writes 128 contiguous bytes per row).
 template <typename T>
-__global__ void __launch_bounds__(128, 8)
+__global__ void __launch_bounds__(128, 4)
 tri_kernel(PrefillArgs p) {
     using namespace sm100;
-    __shared__ __align__(16) float Wk[kTriFloats];
-    __shared__ __align__(16) float Gs[kC], Bs[kC];
-    const int ci = blockIdx.x, h = blockIdx.y, tt = threadIdx.x;
+    __shared__ __align__(16) float As[2][kTriFloats];
+    __shared__ __align__(16) float Gs[2][kC], Bs[2][kC];
+    const int ci = blockIdx.x, gi = threadIdx.x >> 6, tt = threadIdx.x & 63, lane = threadIdx.x & 31;
+    const int h = 2 * blockIdx.y + gi;
     if (ci >= __ldg(p.ws_offs + p.batch))
         return;
     int n, nr;
     int64_t t0;
     chunk_of(p.cu, p.ws_offs, p.batch, p.N, ci, n, t0, nr);
-    const int j = h / p.G;
-    const TriThread tr(tt);
+    const bool live = h < p.Hv;
+    const int j = (live ? h : 0) / p.G;
+    float *A = As[gi];
+    float *G = Gs[gi], *Be = Bs[gi];
+    // the K K^T tile of the chunk: thread tt of the group takes float4s tt + 64 i
     const float *kk = (const float *)p.ws_kk + ((size_t)ci * p.Hk + j) * kTriFloats;
-    float4 x[6];
+    float4 x4[12];
 #pragma unroll
-    for (int jj = 0; jj < 6; ++jj)
-        x[jj] = __ldg(reinterpret_cast<const float4 *>(kk + tr.o(jj)));
-    if (tt < 32) { // gates of rows tt and tt + 32
+    for (int i = 0; i < 12; ++i)
+        x4[i] = live ? __ldg(reinterpret_cast<const float4 *>(kk) + tt + 64 * i) : make_float4(0.f, 0.f, 0.f, 0.f);
+    if (tt < 32 && live) { // gates of rows tt and tt + 32 (first warp of the group)
         const float negA = -expf(__ldg(p.A_log + h)), dtb = __ldg(p.dt_bias + h);
         float g[2], be[2];
 #pragma unroll
@@ -255,44 +292,54 @@ tri_kernel(PrefillArgs p) {
         }
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
-            const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
-            if (tt >= o) {
-                g[0] += x0;
-                g[1] += x1;
+            const float y0 = __shfl_up_sync(0xffffffffu, g[0], o);
+            const float y1 = __shfl_up_sync(0xffffffffu, g[1], o);
+            if (lane >= o) {
+                g[0] += y0;
+                g[1] += y1;
             }
         }
         g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-        Gs[tt] = g[0]; Gs[tt + 32] = g[1];
-        Bs[tt] = be[0]; Bs[tt + 32] = be[1];
+        G[tt] = g[0]; G[tt + 32] = g[1];
+        Be[tt] = be[0]; Be[tt + 32] = be[1];
     }
-    __syncthreads();
+    group_sync(1 + gi, 64);
     // A[r][s] = beta_r e^{G_r - G_s} KK[r][s] (KK is 0 for s >= r; the clamp keeps
-    // the unused upper triangle finite: G_r - G_s > 0 there)
+    // the unused upper triangle finite: G_r - G_s > 0 there).  Float4 f of the
+    // tile: column block f / 512, row (f % 512) / 8, 16-byte chunk f % 8 holding
+    // columns 4 ((f % 8) xor (row % 8)) ..
 #pragma unroll
-    for (int jj = 0; jj < 6; ++jj) {
-        const float Gr = Gs[tr.r(jj)], br = Bs[tr.r(jj)];
-        const float4 Gc = *reinterpret_cast<const float4 *>(&Gs[tr.c(jj)]);
-        x[jj].x *= br * __expf(fminf(Gr - Gc.x, 0.f));
-        x[jj].y *= br * __expf(fminf(Gr - Gc.y, 0.f));
-        x[jj].z *= br * __expf(fminf(Gr - Gc.z, 0.f));
-        x[jj].w *= br * __expf(fminf(Gr - Gc.w, 0.f));
-        *reinterpret_cast<float4 *>(Wk + tr.o(jj)) = x[jj];
+    for (int i = 0; i < 12; ++i) {
+        const int f = tt + 64 * i, blk = f >> 9, r = ((f & 511) >> 3) + (blk ? 32 : 0);
+        const int c0 = 32 * blk + 4 * ((f & 7) ^ (r & 7));
+        const float Gr = G[r], br = Be[r];
+        const float4 Gc = *reinterpret_cast<const float4 *>(&G[c0]);
+        float4 v = x4[i];
+        v.x *= br * __expf(fminf(Gr - Gc.x, 0.f));
+        v.y *= br * __expf(fminf(Gr - Gc.y, 0.f));
+        v.z *= br * __expf(fminf(Gr - Gc.z, 0.f));
+        v.w *= br * __expf(fminf(Gr - Gc.w, 0.f));
+        *reinterpret_cast<float4 *>(A + 4 * f) = v;
     }
-    __syncthreads();
-    tri_invert(Wk, tt, 0); // barrier 0 over the CTA's 128 threads
-    __syncthreads();
-    // T diag(beta), tf32, as 96 rows of 32 floats: row r of column block 0, then row
-    // r of block 1 at row r + 32 (a TMA load with 128-byte swizzle turns them back
-    // into the triangular tile)
+    group_sync(1 + gi, 64);
+    if (!live)
+        return;
+    // column c = tt of T, then T diag(beta) as 96 rows of 32 floats: row r of
+    // column block 0, then row r of block 1 at row r + 32 (a TMA load with
+    // 128-byte swizzle turns them back into the triangular tile)
+    float x[kC];
     float *dst = (float *)p.ws_tb + ((size_t)ci * p.Hv + h) * (96 * 32);
+    const float bc = Be[tt];
+    if (tt < 32) {
+        tri_column<0>(A, tt, x);
 #pragma unroll
-    for (int jj = 0; jj < 6; ++jj) {
-        const float4 t4 = *reinterpret_cast<const float4 *>(Wk + tr.o(jj));
-        const float4 b4 = *reinterpret_cast<const float4 *>(&Bs[tr.c(jj)]);
-        const int row = tr.c(jj) < 32 ? tr.r(jj) : tr.r(jj) + 32;
-        *reinterpret_cast<float4 *>(dst + row * 32 + (tr.c(jj) & 31)) =
-            tf32_rna(make_float4(t4.x * b4.x, t4.y * b4.y, t4.z * b4.z, t4.w * b4.w));
+        for (int r = 0; r < kC; ++r)
+            dst[r * 32 + tt] = tf32_rna(x[r] * bc);
+    } else {
+        tri_column<32>(A, tt, x);
+#pragma unroll
+        for (int r = 32; r < kC; ++r)
+            dst[(r + 32) * 32 + (tt - 32)] = tf32_rna(x[r] * bc);
     }
 }
 
@@ -315,7 +362,7 @@ cudaError_t launch_gram(const PrefillArgs &p, cudaStream_t s) {
 cudaError_t launch_tri(const PrefillArgs &p, cudaStream_t s) {
     if (p.N == 0 || p.batch == 0)
         return cudaSuccess;
-    dim3 grid((unsigned)((p.N + kC - 1) / kC + p.batch), p.Hv);
+    dim3 grid((unsigned)((p.N + kC - 1) / kC + p.batch), (p.Hv + 1) / 2); // two value heads a CTA
     if (p.bf16)
         tri_kernel<__nv_bfloat16><<<grid, 128, 0, s>>>(p);
     else

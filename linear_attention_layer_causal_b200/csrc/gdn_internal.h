@@ -25,6 +25,7 @@ struct PrefillArgs {
     float *o_raw;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
     bool chunked;            // tensor-core chunked path (head_dim 128) or token-serial
+    const void *kda_zdec = nullptr; // KDA: per-channel decay inputs [N, H, d] (a, dt_bias unused)
     long long wait_limit;    // SM cycles a wait between warps may take before the call aborts
     // workspace carve-up
     unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)
@@ -46,6 +47,7 @@ struct DecodeArgs {
     int batch;
     void *y;
     const float *conv_w, *A_log, *dt_bias, *norm_w;
+    const void *kda_zdec = nullptr;    // KDA: per-channel decay inputs [batch, H, d]
     int k = 1;                         // tokens per sequence (multi-token decode)
     const int32_t *accepted = nullptr; // [batch] tokens to take (commit mode)
 };
@@ -112,6 +114,8 @@ size_t tb_workspace_bytes(int Hv, int64_t N, int batch);
 size_t kk_workspace_bytes(int Hk, int64_t N, int batch);
 cudaError_t launch_decode(const DecodeArgs &p, cudaStream_t s);
 cudaError_t launch_decode_multi(const DecodeArgs &p, int mode, cudaStream_t s);
+cudaError_t launch_kda_prefill(const PrefillArgs &p, cudaStream_t s);
+cudaError_t launch_kda_decode(const DecodeArgs &p, cudaStream_t s);
 size_t decode_multi_smem_bytes(int G, int D, int k, int mode);
 
 } // namespace gdn

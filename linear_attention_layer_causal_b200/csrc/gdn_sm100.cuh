@@ -18,20 +18,7 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-    uint32_t ok;
-    // the thread may sleep until the phase completes, for at most 1 ms (the
-    // hint is in nanoseconds), instead of spinning on the barrier
-    asm volatile("{\n\t.reg .pred p;\n\t"
-                 "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-                 "selp.b32 %0, 1, 0, p;\n\t}"
-                 : "=r"(ok)
-                 : "r"(bar), "r"(parity), "r"(1000000u)
-                 : "memory");
-    return ok != 0;
-}
-
-// The same without a suspend hint: the thread polls and reacts at once.
+// One poll of phase `parity` of the barrier (no suspend hint: the thread reacts at once).
 __device__ __forceinline__ bool mbar_try_wait_spin(uint32_t bar, uint32_t parity) {
     uint32_t ok;
     asm volatile("{\n\t.reg .pred p;\n\t"
@@ -56,10 +43,11 @@ __device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of the barrier to complete, giving up after about
-// `limit` SM cycles.  Returns false on time-out.
+// `limit` SM cycles.  Returns false on time-out.  Polls without a suspend hint:
+// a waiter woken late adds its delay to whatever waits on it.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity, long long limit) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(bar, parity)) {
+    while (!mbar_try_wait_spin(bar, parity)) {
         if (clock64() - t0 > limit)
             return false;
     }

@@ -95,7 +95,7 @@ QWEN38_VERY_LONG_MEMORY = Workload("qwen38_very_long_memory", 16, 128, 128, seql
 
 WORKLOADS = {w.name: w for w in (TINY, QWEN38_PREFILL, QWEN38_LONG, QWEN38_DECODE, QWEN36_VARLEN,
                                  QWEN35_PREFILL, QWEN35_DECODE, QWEN38_LONG_MEMORY,
-                                 QWEN38_VERY_LONG_MEMORY)}
+                                 QWEN38_VERY_LONG_MEMORY)}  # (the KDA workload is added below)
 
 
 def _gen(device, seed):
@@ -186,3 +186,53 @@ def make_decode(wl: Workload, device="cpu", batch=None, seed=None, tokens=None):
     out["state"] = _normal((B, H, d, d), wl.state_std if wl.state_std > 0 else 0.02, g, device)
     out["conv_cache"] = _normal((B, wl.conv_kernel - 1, wl.conv_dim), 1.0, g, device, dt)
     return out
+
+
+# Kimi Delta Attention (per-channel decay) at the Kimi K3 layer shape: 96 heads
+# of dimension 128, one q, k and v head each ("Inkling vs Kimi K3", component
+# table, linear-attention row).  Draws, in order: lengths, qkv, the decay
+# inputs zdec ~ N(0, 1), b ~ N(0, 1), the gate inputs ~ N(0, 1), conv_w ~
+# N(0, 0.5^2), A_log = log U(1, 16), norm_w = 1 + 0.1 N(0, 1), states.
+KIMI_K3_KDA = Workload("kimi_k3_kda", 96, 96, 128, seqlens=(1024, 517), state_std=0.02, seed=1009,
+                       notes="Kimi K3 KDA layer prefill, B=2 (1024 + 517 tokens)")
+
+
+def make_kda_prefill(wl: Workload, device="cpu", seqlens=None, seed=None):
+    """Inputs of one KDA prefill call: qkv [N, 3 H d], zdec [N, H, d], b [N, H],
+    gate [N, H, d], cu_seqlens, conv_w [3 H d, K], A_log [H], norm_w [d], and
+    initial_state [B, H, d, d] or None."""
+    g = _gen(device, wl.seed if seed is None else seed)
+    lens = seqlens_of(wl, g, device) if seqlens is None else list(seqlens)
+    N = int(sum(lens))
+    H, d, dt = wl.num_v_heads, wl.head_dim, wl.torch_dtype
+    out = {"seqlens": lens}
+    out["cu_seqlens"] = torch.tensor([0] + list(torch.tensor(lens).cumsum(0).tolist()),
+                                     dtype=torch.int32, device=device)
+    out["qkv"] = _normal((N, wl.conv_dim), 1.0, g, device, dt)
+    out["zdec"] = _normal((N, H, d), 1.0, g, device, dt)
+    out["b"] = _normal((N, H), 1.0, g, device, dt)
+    out["gate"] = _normal((N, H, d), 1.0, g, device, dt)
+    out["conv_w"] = _normal((wl.conv_dim, wl.conv_kernel), 0.5, g, device).contiguous()
+    out["A_log"] = torch.log(torch.rand(H, generator=g, device=device) * 15.0 + 1.0).contiguous()
+    out["norm_w"] = (1.0 + _normal((d,), 0.1, g, device)).contiguous()
+    out["initial_state"] = _normal((len(lens), H, d, d), wl.state_std, g, device) \
+        if wl.state_std > 0 else None
+    return out
+
+
+def make_kda_decode(wl: Workload, device="cpu", batch=8, seed=None):
+    """Inputs of one KDA decode call: one token for each of `batch` sequences."""
+    g = _gen(device, wl.seed if seed is None else seed)
+    H, d, dt = wl.num_v_heads, wl.head_dim, wl.torch_dtype
+    out = {"qkv": _normal((batch, wl.conv_dim), 1.0, g, device, dt),
+           "zdec": _normal((batch, H, d), 1.0, g, device, dt),
+           "b": _normal((batch, H), 1.0, g, device, dt),
+           "gate": _normal((batch, H, d), 1.0, g, device, dt),
+           "conv_w": _normal((wl.conv_dim, wl.conv_kernel), 0.5, g, device).contiguous(),
+           "A_log": torch.log(torch.rand(H, generator=g, device=device) * 15.0 + 1.0).contiguous(),
+           "norm_w": (1.0 + _normal((d,), 0.1, g, device)).contiguous()}
+    out["state"] = _normal((batch, H, d, d), 0.02, g, device)
+    out["conv_cache"] = _normal((batch, wl.conv_kernel - 1, wl.conv_dim), 1.0, g, device, dt)
+    return out
+
+WORKLOADS[KIMI_K3_KDA.name] = KIMI_K3_KDA

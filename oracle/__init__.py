@@ -16,6 +16,12 @@ the layer defines, and composes them into a whole prefill or decode pass:
 (Gated DeltaNet row and output-gate row of the component table on
 "Qwen3.8-2.4T-A95B vs Inkling"; head counts, kernel size, state dtype and
 epsilon from the raw config fields on "Qwen3.8 2.4T A95B".)
+
+The KDA variant (kda_layer, kda_prefill) swaps the gates, the recurrence and
+the output gate for the per-key-channel decay g = -5 sigmoid(exp(A_log) z),
+S_t = S_{t-1} Diag(exp(g_t)) (I - beta k k^T) + beta v k^T, and y = RMSNorm(o)
+w sigmoid(gate) ("Inkling vs Kimi K3", component table, linear-attention and
+output-gate rows); q, k and v go through the same conv, SiLU and L2 norm.
 """
 from __future__ import annotations
 
@@ -62,6 +68,13 @@ def lib():
         L.gdn_oracle_delta_rule.restype = ctypes.c_int
         L.gdn_oracle_gated_rmsnorm.argtypes = [_dp, _dp, _dp, _i64, _i64, ctypes.c_double, _dp]
         L.gdn_oracle_gated_rmsnorm.restype = None
+        L.gdn_oracle_kda_gates.argtypes = [_dp, _dp, _dp, _i64, _i64, _i64, _dp, _dp]
+        L.gdn_oracle_kda_gates.restype = None
+        L.gdn_oracle_kda_rule.argtypes = [_dp, _dp, _dp, _dp, _dp, _i64, _i64, _i64, _i64, _dp,
+                                          _dp, ctypes.c_int]
+        L.gdn_oracle_kda_rule.restype = None
+        L.gdn_oracle_sigmoid_rmsnorm.argtypes = [_dp, _dp, _dp, _i64, _i64, ctypes.c_double, _dp]
+        L.gdn_oracle_sigmoid_rmsnorm.restype = None
         _lib = L
     return _lib
 
@@ -287,3 +300,74 @@ def decode(shape: Shape, qkv, a, b, z, conv_w, A_log, dt_bias, norm_w, state, co
             "o": np.concatenate([r["o"] for r in outs]),
             "state": np.stack([r["state"] for r in outs]),
             "conv_window": np.stack([r["conv_window"] for r in outs])}
+
+
+# ---------------------------------------------------------------- KDA
+
+
+def kda_gates(z, b, A_log):
+    """g = -5 sigmoid(exp(A_log) z) per key channel, beta = sigmoid(b); z: [T, H, d_k], b: [T, H]."""
+    z, b, A_log = _f64(z), _f64(b), _f64(A_log)
+    T, H, dk = z.shape
+    g = np.empty((T, H, dk), np.float64)
+    beta = np.empty((T, H), np.float64)
+    lib().gdn_oracle_kda_gates(_ptr(z), _ptr(b), _ptr(A_log), T, H, dk, _ptr(g), _ptr(beta))
+    return g, beta
+
+
+def kda_rule(q, k, v, g, beta, state=None, threads: int | None = None):
+    """KDA recurrence over one sequence: q, k: [T, H, d_k]; v: [T, H, d_v];
+    g: [T, H, d_k]; beta: [T, H]; state: [H, d_v, d_k] (None = zeros).
+    Returns (o [T, H, d_v], final state)."""
+    q, k, v, g, beta = _f64(q), _f64(k), _f64(v), _f64(g), _f64(beta)
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    S = np.zeros((H, dv, dk)) if state is None else _f64(state).copy()
+    o = np.empty((T, H, dv), np.float64)
+    lib().gdn_oracle_kda_rule(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), T, H, dk, dv, _ptr(S),
+                              _ptr(o), threads or default_threads())
+    return o, S
+
+
+def sigmoid_rmsnorm(o, gate, w, eps: float = 1e-6) -> np.ndarray:
+    """y = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate), over the last axis."""
+    o, gate, w = _f64(o), _f64(gate), _f64(w)
+    d = o.shape[-1]
+    y = np.empty_like(o)
+    lib().gdn_oracle_sigmoid_rmsnorm(_ptr(o), _ptr(gate), _ptr(w), o.size // d, d, eps, _ptr(y))
+    return y
+
+
+def kda_layer(shape: Shape, qkv, zdec, b, gate, conv_w, A_log, norm_w, state=None,
+              conv_window=None, heads=None, threads: int | None = None):
+    """One sequence through the KDA mixer (one q, k and v head per head).
+
+    qkv: [T, 3 H d] pre-conv rows (q heads, k heads, v heads); zdec: [T, H, d]
+    decay inputs; b: [T, H]; gate: [T, H, d]; conv_w: [3 H d, K]; A_log: [H];
+    norm_w: [d]; state: [H, d, d]; conv_window: [K-1, 3 H d].  With `heads`,
+    only those heads are computed (every per-head output holds just them).
+    Returns y, o, state and conv_window (the last K-1 pre-conv rows).
+    """
+    d, H, K = shape.head_dim, shape.num_v_heads, shape.conv_kernel
+    assert shape.num_qk_heads == H
+    T = int(qkv.shape[0])
+    heads = list(range(H)) if heads is None else list(heads)
+    hv = len(heads)
+    cols = np.concatenate([np.arange(h * d, (h + 1) * d) for h in heads] +
+                          [H * d + np.arange(h * d, (h + 1) * d) for h in heads] +
+                          [2 * H * d + np.arange(h * d, (h + 1) * d) for h in heads])
+    x = _take(qkv, cols, 1)
+    w = _take(conv_w, cols, 0)
+    win = None if conv_window is None else _take(conv_window, cols, 1)
+    xc = conv_silu(x, w, win)
+    q = l2norm(xc[:, : hv * d].reshape(T, hv, d), shape.l2_eps, shape.q_scale)
+    k = l2norm(xc[:, hv * d: 2 * hv * d].reshape(T, hv, d), shape.l2_eps, 1.0)
+    v = xc[:, 2 * hv * d:].reshape(T, hv, d)
+    g, beta = kda_gates(_take(zdec, heads, 1), _take(b, heads, 1), _take(A_log, heads, 0))
+    S0 = None if state is None else _take(state, heads, 0)
+    o, S = kda_rule(q, k, v, g, beta, S0, threads)
+    y = sigmoid_rmsnorm(o, _take(gate, heads, 1), norm_w, shape.rms_eps)
+    prev = np.zeros((K - 1, x.shape[1])) if win is None else win
+    hist = np.concatenate([prev, x], axis=0)
+    return {"y": y, "o": o, "state": S, "conv_window": hist[-(K - 1):].copy(), "g": g,
+            "beta": beta, "q": q, "k": k, "v": v}

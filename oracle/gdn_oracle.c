@@ -33,6 +33,17 @@
  *            row: output_gate_type swish after a per-head RMSNorm;
  *            "Qwen3.8 2.4T A95B", raw config fields, rms_norm_eps = 1e-6).
  *
+ * Kimi Delta Attention (KDA), the per-channel-decay variant ("Inkling vs Kimi
+ * K3", component table, linear-attention and output-gate rows), adds
+ *
+ *   kda gates : g = -5 sigmoid(exp(A_log) z), one log-decay per key channel,
+ *               token and head (z is the decay input of the channel), and
+ *               beta = sigmoid(b);
+ *   kda delta : S_t = S_{t-1} Diag(exp(g_t)) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
+ *               o_t = S_t q_t, one state per head (no head sharing);
+ *   kda norm  : per head RMSNorm of o, times a weight, times sigmoid(gate)
+ *               (a full-rank channel-wise sigmoid gate).
+ *
  * All arrays are row-major, contiguous, double precision.
  */
 #include <math.h>
@@ -243,5 +254,144 @@ void gdn_oracle_gated_rmsnorm(const double *o, const double *z, const double *w,
             double zi = z[r * d + i];
             y[r * d + i] = o[r * d + i] * inv * w[i] * (zi / (1.0 + exp(-zi)));
         }
+    }
+}
+
+/* ------------------------------------------------------------------ KDA */
+
+/*
+ * Per token t, head h and key channel c:
+ *   g[t][h][c] = -5 * sigmoid(exp(A_log[h]) * z[t][h][c])
+ *   beta[t][h] = 1 / (1 + exp(-b[t][h]))
+ * z, g are [T, H, d_k]; b, beta are [T, H]; A_log is [H].
+ */
+void gdn_oracle_kda_gates(const double *z, const double *b, const double *A_log, int64_t T,
+                          int64_t H, int64_t d_k, double *g, double *beta)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        for (int64_t h = 0; h < H; ++h) {
+            const double eA = exp(A_log[h]);
+            for (int64_t c = 0; c < d_k; ++c) {
+                const double x = eA * z[(t * H + h) * d_k + c];
+                g[(t * H + h) * d_k + c] = -5.0 / (1.0 + exp(-x));
+            }
+            beta[t * H + h] = 1.0 / (1.0 + exp(-b[t * H + h]));
+        }
+    }
+}
+
+typedef struct {
+    const double *q, *k, *v, *g, *beta;
+    int64_t T, H, d_k, d_v;
+    double *state, *o;
+    int64_t next_head;
+    pthread_mutex_t mu;
+} kda_job;
+
+/*
+ * One head over all T tokens, S = [d_v][d_k].  Per token:
+ *   S[i][c] <- S[i][c] * exp(g[c])   (the decay of key channel c, every row);
+ *   p = S k;  u = beta (v - p);  S <- S + u k^T;  o = S q,
+ * which expands to S_t = S_{t-1} D - beta S_{t-1} D k k^T + beta v k^T with
+ * D = Diag(exp(g_t)): the defining update written above.
+ */
+static void kda_one_head(kda_job *J, int64_t h)
+{
+    const int64_t dk = J->d_k, dv = J->d_v, H = J->H;
+    double *S = J->state + h * dv * dk;
+    double *p = (double *)malloc(sizeof(double) * (size_t)dv);
+    double *alpha = (double *)malloc(sizeof(double) * (size_t)dk);
+    for (int64_t t = 0; t < J->T; ++t) {
+        const double *kt = J->k + (t * H + h) * dk;
+        const double *qt = J->q + (t * H + h) * dk;
+        const double *vt = J->v + (t * H + h) * dv;
+        const double *gt = J->g + (t * H + h) * dk;
+        const double bt = J->beta[t * H + h];
+        for (int64_t c = 0; c < dk; ++c)
+            alpha[c] = exp(gt[c]);
+        for (int64_t i = 0; i < dv; ++i)
+            for (int64_t c = 0; c < dk; ++c)
+                S[i * dk + c] *= alpha[c];
+        for (int64_t i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < dk; ++c)
+                acc += S[i * dk + c] * kt[c];
+            p[i] = acc;
+        }
+        for (int64_t i = 0; i < dv; ++i) {
+            double u = bt * (vt[i] - p[i]);
+            for (int64_t c = 0; c < dk; ++c)
+                S[i * dk + c] += u * kt[c];
+        }
+        double *ot = J->o + (t * H + h) * dv;
+        for (int64_t i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int64_t c = 0; c < dk; ++c)
+                acc += S[i * dk + c] * qt[c];
+            ot[i] = acc;
+        }
+    }
+    free(alpha);
+    free(p);
+}
+
+static void *kda_worker(void *arg)
+{
+    kda_job *J = (kda_job *)arg;
+    for (;;) {
+        pthread_mutex_lock(&J->mu);
+        int64_t h = J->next_head++;
+        pthread_mutex_unlock(&J->mu);
+        if (h >= J->H)
+            break;
+        kda_one_head(J, h);
+    }
+    return NULL;
+}
+
+/*
+ * The KDA recurrence over one sequence of T tokens, all heads.
+ *   q, k  : [T, H, d_k]  (convolved, activated and L2-normalised)
+ *   v     : [T, H, d_v]
+ *   g     : [T, H, d_k] per-channel log-decay;  beta : [T, H]
+ *   state : [H, d_v, d_k] initial state on entry, final state on return
+ *   o     : [T, H, d_v]
+ * Heads are spread over n_threads threads (each runs its tokens in order).
+ */
+void gdn_oracle_kda_rule(const double *q, const double *k, const double *v, const double *g,
+                         const double *beta, int64_t T, int64_t H, int64_t d_k, int64_t d_v,
+                         double *state, double *o, int n_threads)
+{
+    kda_job J = {q, k, v, g, beta, T, H, d_k, d_v, state, o, 0, PTHREAD_MUTEX_INITIALIZER};
+    if (n_threads < 1)
+        n_threads = 1;
+    if (n_threads > H)
+        n_threads = (int)H;
+    if (n_threads == 1) {
+        kda_worker(&J);
+        return;
+    }
+    pthread_t *th = (pthread_t *)malloc(sizeof(pthread_t) * (size_t)n_threads);
+    for (int i = 0; i < n_threads; ++i)
+        pthread_create(&th[i], NULL, kda_worker, &J);
+    for (int i = 0; i < n_threads; ++i)
+        pthread_join(th[i], NULL);
+    free(th);
+}
+
+/*
+ * Per row of length d:  y = o / sqrt(mean(o^2) + eps) * w * sigmoid(gate).
+ *   o, gate, y : [rows, d];  w : [d]
+ */
+void gdn_oracle_sigmoid_rmsnorm(const double *o, const double *gate, const double *w,
+                                int64_t rows, int64_t d, double eps, double *y)
+{
+    for (int64_t r = 0; r < rows; ++r) {
+        double ss = 0.0;
+        for (int64_t i = 0; i < d; ++i)
+            ss += o[r * d + i] * o[r * d + i];
+        double inv = 1.0 / sqrt(ss / (double)d + eps);
+        for (int64_t i = 0; i < d; ++i)
+            y[r * d + i] = o[r * d + i] * inv * w[i] / (1.0 + exp(-gate[r * d + i]));
     }
 }
