@@ -305,6 +305,7 @@ def run_ours(args, rank, world, dev, dist):
     decode = run_decode(args, rank, world, dev, pk, timed, max_over_ranks)
     decode_k = run_decode_k(args, rank, world, dev, pk, timed, max_over_ranks)
     qwen35 = run_prefill_shape(args, rank, world, dev, pk, timed, max_over_ranks, "qwen35_prefill")
+    long_ctx = run_long_context(args, rank, world, dev, pk, timed, max_over_ranks)
 
     # ---- end to end through the public API from pinned host buffers.  Every
     # step uploads its inputs, runs the layer and reads back y and the final
@@ -364,6 +365,7 @@ def run_ours(args, rank, world, dev, dist):
                                 "accumulation, FP32 state and CUDA-core math",
                        "l2": "no flush: inputs of one step (~447 MB) exceed the 126 MB L2"},
             "roofline": roof, "decode": decode, "decode_k": decode_k, "qwen35_prefill": qwen35,
+            "long_context": long_ctx,
             "e2e": e2e,
             # chunked: offsets, conv of q|k and of v (side stream), Gram, inverses, chunk kernel
             "gpu_launches": (6 if kname == "chunk_prefill_kernel" else 2) * args.steps,
@@ -465,6 +467,50 @@ def run_prefill_shape(args, rank, world, dev, pk, timed, max_over_ranks, name):
             "roofline": {"kernel": "chunk_prefill_kernel", "bound": "tensor", "achieved": round(tf, 2),
                          "peak": tf32_peak, "unit": "TFLOP/s", "frac": round(tf / tf32_peak, 4),
                          "kernel_ms": round(kern, 4)}}
+
+
+def run_long_context(args, rank, world, dev, pk, timed, max_over_ranks):
+    """One 262,144-token sequence (the Qwen3.8 context window) at the Qwen3.8 and the
+    Qwen3.5-397B layer shapes: tokens/s with the library's choice of segments per
+    sequence and, where that choice splits the sequence, the single chain beside it."""
+    import torch
+
+    import linear_attention_layer_causal_b200 as gdn
+    from linear_attention_layer_causal_b200 import workloads as W
+    out = {}
+    for name in ("qwen38_262k_prefill", "qwen35_262k_prefill"):
+        wl = W.WORKLOADS[name]
+        inp = W.make_prefill(wl, dev, seed=rank_seed(wl.seed, rank))
+        P = [inp[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
+        N, B = sum(inp["seqlens"]), len(inp["seqlens"])
+        y = torch.empty((N, wl.num_v_heads, wl.head_dim), dtype=torch.bfloat16, device=dev)
+        fs = torch.empty((B, wl.num_v_heads, wl.head_dim, wl.head_dim), device=dev)
+        res = {"config": {"workload": name, "batch": B, "seq_len": N // B,
+                          "num_qk_heads": wl.num_qk_heads, "num_v_heads": wl.num_v_heads}}
+        for label, segs in (("auto", 0), ("single_chain", 1)):
+            cfg = gdn.Config.of(wl, segments=segs)
+            nseg = gdn.prefill_segments(cfg, B, N)
+            if label == "single_chain" and res["auto"]["segments"] == 1:
+                break
+            ws = torch.empty(max(gdn.prefill_workspace_size(cfg, B, N), 1), dtype=torch.uint8,
+                             device=dev)
+
+            def step():
+                gdn.prefill(cfg, inp["qkv"], inp["a"], inp["b"], inp["z"], inp["cu_seqlens"], *P,
+                            y=y, final_state=fs, workspace=ws)
+
+            for _ in range(args.warmup):
+                step()
+            tot, kern = timed(step, args.steps)
+            tot, kern = max_over_ranks(tot), max_over_ranks(kern)
+            res[label] = {"segments": nseg, "value": job_rate(N, world, args.steps, tot),
+                          "unit": "tokens/s", "ms_per_step": tot / args.steps,
+                          "scan_ms": round(kern, 4)}
+            del ws
+        out[name] = res
+        del inp, y, fs
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_decode(args, rank, world, dev, pk, timed, max_over_ranks):

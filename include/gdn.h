@@ -53,7 +53,7 @@
 extern "C" {
 #endif
 
-#define GDN_ABI_VERSION 2
+#define GDN_ABI_VERSION 3
 
 #if defined(__GNUC__)
 #define GDN_API __attribute__((visibility("default")))
@@ -87,7 +87,34 @@ typedef struct gdn_config {
     float q_scale;        /* extra factor on normalised q (1.0 = none) */
     int32_t act_dtype;    /* gdn_dtype of qkv, a, b, z, y and the conv caches */
     int32_t algo;         /* gdn_algo: prefill algorithm (GDN_ALGO_AUTO = 0 is right for most callers) */
+    int32_t segments;     /* chunked prefill: segments per sequence (see below); 0 = the library's choice */
 } gdn_config;
+
+/*
+ * Sequence split of the chunked prefill (gdn_config.segments).
+ *
+ * The state map of a stretch of tokens is affine in the state entering it,
+ * S_end = S_0 M + R, with M the product of the per-token factors
+ * exp(g_t) (I - beta_t k_t k_t^T) and R the state the stretch reaches from
+ * S_0 = 0 (the Gated DeltaNet update of "Qwen3.8-2.4T-A95B vs Inkling",
+ * component table; "Qwen3.8 2.4T A95B", key facts: a 262,144-token context).
+ * With segments = P >= 2 every sequence is cut at chunk boundaries into P
+ * segments of equal chunk count.  A summary pass computes (M, R) of the first
+ * P - 1 segments of every (sequence, value head) in parallel, a short FP32
+ * pass chains them into the state entering each segment, and the output pass
+ * then scans all P segments in parallel.  The results are those of P = 1 up to
+ * rounding.  It pays when batch * H_v is small against the GPU's 148 SMs and
+ * the sequences are long.
+ *   0      the library's choice: 1 unless batch * H_v <= 74, else the P in
+ *          2..16 that a cost model of the two passes favours, with at least
+ *          32 chunks (2,048 tokens) per segment on average
+ *   1      no split: one chain per (sequence, value head)
+ *   2..16  that many segments (a sequence shorter than P chunks leaves some
+ *          segments empty)
+ * The token-serial path and the KDA entry points take 0 or 1 only
+ * (GDN_ERR_UNSUPPORTED otherwise); decode ignores the field.  The workspace
+ * size query counts the split's workspace: 3 (P - 1) batch H_v d^2 floats.
+ */
 
 /* Prefill algorithm.  Both compute the same recurrence; decode ignores it. */
 typedef enum gdn_algo {
@@ -111,6 +138,16 @@ typedef struct gdn_params {
  */
 GDN_API gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
                                       size_t *bytes);
+
+/*
+ * Segments per sequence (see gdn_config.segments) that gdn_prefill runs with
+ * for `total_tokens` packed tokens in `batch` sequences: cfg->segments when
+ * it is nonzero on the chunked path, the library's choice when it is 0, and 1
+ * on the token-serial path or without tokens.  Writes *segments; errors as
+ * gdn_prefill_workspace_size.
+ */
+GDN_API gdn_status gdn_prefill_segments(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
+                                        int32_t *segments);
 
 /*
  * Prefill over a packed varlen batch: sequence n owns token rows

@@ -32,7 +32,7 @@ LIB_PATH = os.path.join(_HERE, "libgdn.so")
  GDN_ERR_TIMEOUT) = range(6)
 GDN_F32, GDN_BF16 = 0, 1
 
-EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode", "gdn_status_string",
+EXPORTED = ("gdn_prefill_workspace_size", "gdn_prefill_segments", "gdn_prefill", "gdn_decode", "gdn_status_string",
             "gdn_abi_version", "gdn_profile_next_call", "gdn_prefill_noalloc",
             "gdn_prefill_status", "gdn_prefill_noalloc_status", "gdn_wait_limit_next_call",
             "gdn_decode_multi", "gdn_decode_verify", "gdn_decode_commit",
@@ -53,7 +53,7 @@ class _Config(ctypes.Structure):
                 ("head_dim", ctypes.c_int32), ("conv_kernel", ctypes.c_int32),
                 ("rms_eps", ctypes.c_float), ("l2_eps", ctypes.c_float),
                 ("q_scale", ctypes.c_float), ("act_dtype", ctypes.c_int32),
-                ("algo", ctypes.c_int32)]
+                ("algo", ctypes.c_int32), ("segments", ctypes.c_int32)]
 
 
 class _KdaParams(ctypes.Structure):
@@ -78,6 +78,7 @@ class Config:
     q_scale: float = 1.0
     act_dtype: str = "bf16"  # "bf16" or "f32"
     algo: str = "auto"       # prefill algorithm: "auto", "serial" or "chunked"
+    segments: int = 0        # chunked prefill: segments per sequence (0 = the library's choice)
 
     @property
     def conv_dim(self) -> int:
@@ -87,13 +88,13 @@ class Config:
         return _Config(self.num_qk_heads, self.num_v_heads, self.head_dim, self.conv_kernel,
                        self.rms_eps, self.l2_eps, self.q_scale,
                        GDN_BF16 if self.act_dtype == "bf16" else GDN_F32,
-                       {"auto": 0, "serial": 1, "chunked": 2}[self.algo])
+                       {"auto": 0, "serial": 1, "chunked": 2}[self.algo], self.segments)
 
     @staticmethod
-    def of(wl, algo: str = "auto") -> "Config":
+    def of(wl, algo: str = "auto", segments: int = 0) -> "Config":
         """The Config of a workloads.Workload."""
         return Config(wl.num_qk_heads, wl.num_v_heads, wl.head_dim, wl.conv_kernel,
-                      act_dtype=wl.dtype, algo=algo)
+                      act_dtype=wl.dtype, algo=algo, segments=segments)
 
 
 _lib = None
@@ -111,6 +112,8 @@ def lib() -> ctypes.CDLL:
         cfgp, parp = ctypes.POINTER(_Config), ctypes.POINTER(_Params)
         L.gdn_prefill_workspace_size.argtypes = [cfgp, i32, i64, ctypes.POINTER(sz)]
         L.gdn_prefill_workspace_size.restype = ctypes.c_int
+        L.gdn_prefill_segments.argtypes = [cfgp, i32, i64, ctypes.POINTER(i32)]
+        L.gdn_prefill_segments.restype = ctypes.c_int
         L.gdn_prefill.argtypes = [cfgp, parp, vp, vp, vp, vp, vp, i32, i64, vp, vp, vp, vp, vp,
                                   vp, vp, sz, vp]
         L.gdn_prefill.restype = ctypes.c_int
@@ -226,6 +229,15 @@ def prefill_workspace_size(cfg: Config, batch: int, total_tokens: int) -> int:
                                           ctypes.byref(n))
     if st != GDN_OK:
         raise GdnError(st, "gdn_prefill_workspace_size")
+    return n.value
+
+
+def prefill_segments(cfg: Config, batch: int, total_tokens: int) -> int:
+    """Segments per sequence a prefill of this size runs with (gdn_prefill_segments)."""
+    n = ctypes.c_int32(0)
+    st = lib().gdn_prefill_segments(ctypes.byref(cfg._c()), batch, total_tokens, ctypes.byref(n))
+    if st != GDN_OK:
+        raise GdnError(st, "gdn_prefill_segments")
     return n.value
 
 

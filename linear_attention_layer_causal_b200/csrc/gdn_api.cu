@@ -37,6 +37,10 @@ gdn_status check_config(const gdn_config *c) {
         return GDN_ERR_INVALID_ARG;
     if (c->algo == GDN_ALGO_CHUNKED && c->head_dim != 128)
         return GDN_ERR_UNSUPPORTED;
+    if (c->segments < 0 || c->segments > kMaxSegments)
+        return GDN_ERR_INVALID_ARG;
+    if (c->segments > 1 && (c->head_dim != 128 || c->algo == GDN_ALGO_SERIAL))
+        return GDN_ERR_UNSUPPORTED; // the split runs on the chunked path only
     // conv_dim * 16-byte channel groups must index in int
     const int64_t conv_dim = (int64_t)(2 * (int64_t)c->num_qk_heads + c->num_v_heads) * c->head_dim;
     if (conv_dim > (int64_t)1 << 26)
@@ -137,9 +141,46 @@ gdn_status validate_prefill(const gdn_config *cfg, const gdn_params *params, con
         !aligned16(o_raw) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
         (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
         return GDN_ERR_INVALID_ARG;
-    *need = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads, cfg->head_dim, bf16,
-                                    total_tokens, batch);
+    *need = prefill_workspace_bytes(cfg, total_tokens, batch);
     return GDN_OK;
+}
+
+// The library's choice of segments per sequence.  Costs are in chunk steps of
+// one chain: unsplit, the average sequence takes L = N / (64 batch) of them;
+// split into P, the summary pass runs 2 (P - 1) CTAs per (sequence, value
+// head) over L / P chunks at about kSummaryCost of an output step (no Q, O or
+// P work, no z or y traffic), in ceil(2 (P - 1) batch H_v / 148) waves of one
+// CTA per SM; the output pass runs P CTAs per unit in ceil(P batch H_v / 148)
+// waves; the combine and the extra launches add about kSplitOverhead steps.
+int prefill_segments(const gdn_config *c, int batch, int64_t N) {
+    if (c->head_dim != 128 || c->algo == GDN_ALGO_SERIAL || batch <= 0 || N <= 0)
+        return 1;
+    if (c->segments > 0)
+        return c->segments;
+    constexpr int64_t kSMs = 148;
+    constexpr double kSummaryCost = 0.6, kSplitOverhead = 8.0, kMinChunksPerSegment = 32.0;
+    const int64_t units = (int64_t)batch * c->num_v_heads;
+    if (2 * units > kSMs)
+        return 1;
+    const double L = (double)N / (64.0 * batch);
+    int best = 1;
+    double best_cost = L;
+    for (int P = 2; P <= kMaxSegments && L / P >= kMinChunksPerSegment; ++P) {
+        const double ws = (double)((2 * units * (P - 1) + kSMs - 1) / kSMs);
+        const double wo = (double)((units * P + kSMs - 1) / kSMs);
+        const double cost = (ws * kSummaryCost + wo) * L / P + kSplitOverhead;
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = P;
+        }
+    }
+    return best;
+}
+
+// R and M of every segment but the last, and the start state of every segment
+// but the first: 3 (P - 1) batch H_v states of 128 x 128 floats.
+size_t seg_workspace_bytes(int Hv, int batch, int segments) {
+    return segments <= 1 ? 0 : (size_t)3 * (segments - 1) * batch * Hv * 128 * 128 * sizeof(float);
 }
 
 gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t stream) {
@@ -156,17 +197,22 @@ gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t 
     return w[0] != 0u ? GDN_ERR_CUDA : GDN_OK;
 }
 
-// Header (status word), float32 normalised q|k, float32 convolved v and, for
-// head_dim 128, the chunked path's Q K^T rows, T diag(beta) tiles and
-// per-sequence chunk offsets.
-size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool /*bf16*/, int64_t N, int batch) {
+// Header (status word), float32 normalised q|k, float32 convolved v (unless
+// the chunk kernel convolves v itself: 16-bit activations) and, on the
+// chunked path, the Q K^T rows, K K^T and T diag(beta) tiles, the
+// per-sequence chunk offsets and the split's states.
+size_t prefill_workspace_bytes(const gdn_config *c, int64_t N, int batch) {
     if (N == 0)
         return 0;
-    size_t b = kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4) +
-               round_up((size_t)N * Hv * D * 4);
-    if (D == 128)
+    const int Hk = c->num_qk_heads, Hv = c->num_v_heads, D = c->head_dim;
+    const bool chunked = D == 128 && c->algo != GDN_ALGO_SERIAL;
+    size_t b = kWorkspaceHeader + round_up((size_t)N * 2 * Hk * D * 4);
+    if (!v_conv_in_chunk(chunked, c->act_dtype == GDN_BF16))
+        b += round_up((size_t)N * Hv * D * 4);
+    if (chunked)
         b += round_up(kq_workspace_bytes(Hk, N)) + round_up(kk_workspace_bytes(Hk, N, batch)) +
-             round_up(tb_workspace_bytes(Hv, N, batch)) + round_up(((size_t)batch + 1) * sizeof(int32_t));
+             round_up(tb_workspace_bytes(Hv, N, batch)) + round_up(((size_t)batch + 1) * sizeof(int32_t)) +
+             seg_workspace_bytes(Hv, batch, prefill_segments(c, batch, N));
     return b;
 }
 
@@ -219,8 +265,18 @@ gdn_status gdn_prefill_workspace_size(const gdn_config *cfg, int32_t batch, int6
         return st;
     if (bytes == nullptr || batch < 0 || total_tokens < 0)
         return GDN_ERR_INVALID_ARG;
-    *bytes = prefill_workspace_bytes(cfg->num_qk_heads, cfg->num_v_heads, cfg->head_dim,
-                                     cfg->act_dtype == GDN_BF16, total_tokens, batch);
+    *bytes = prefill_workspace_bytes(cfg, total_tokens, batch);
+    return GDN_OK;
+}
+
+gdn_status gdn_prefill_segments(const gdn_config *cfg, int32_t batch, int64_t total_tokens,
+                                int32_t *segments) {
+    gdn_status st = check_config(cfg);
+    if (st != GDN_OK)
+        return st;
+    if (segments == nullptr || batch < 0 || total_tokens < 0)
+        return GDN_ERR_INVALID_ARG;
+    *segments = prefill_segments(cfg, batch, total_tokens);
     return GDN_OK;
 }
 
@@ -279,17 +335,25 @@ gdn_status prefill_impl(const gdn_config *cfg, const gdn_params *params, const v
     p.dt_bias = params->dt_bias;
     p.norm_w = params->norm_w;
     p.chunked = p.D == 128 && cfg->algo != GDN_ALGO_SERIAL;
-    if (need > 0) {
+    const bool vconv = v_conv_in_chunk(p.chunked, bf16); // the chunk kernel convolves v
+    if (need > 0) { // the regions of prefill_workspace_bytes, in its order
         char *w = (char *)workspace;
         p.ws_err = (unsigned int *)w;
         p.ws_qk = w + kWorkspaceHeader;
-        p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
-        p.ws_kq = (char *)p.ws_v + round_up((size_t)total_tokens * p.Hv * p.D * 4);
-        if (p.D == 128) {
+        w = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
+        if (!vconv) {
+            p.ws_v = w;
+            w += round_up((size_t)total_tokens * p.Hv * p.D * 4);
+        }
+        if (p.chunked) {
+            p.ws_kq = w;
             p.ws_kk = (char *)p.ws_kq + round_up(kq_workspace_bytes(p.Hk, total_tokens));
             p.ws_tb = (char *)p.ws_kk + round_up(kk_workspace_bytes(p.Hk, total_tokens, batch));
             p.ws_offs = (int32_t *)((char *)p.ws_tb +
                                     round_up(tb_workspace_bytes(p.Hv, total_tokens, batch)));
+            p.segments = prefill_segments(cfg, batch, total_tokens);
+            if (p.segments > 1)
+                p.ws_seg = (float *)((char *)p.ws_offs + round_up(((size_t)batch + 1) * sizeof(int32_t)));
         }
     }
 
@@ -306,10 +370,12 @@ gdn_status prefill_impl(const gdn_config *cfg, const gdn_params *params, const v
     cudaError_t e = cudaSuccess;
     if (!p.chunked) {
         e = launch_conv_prep(p, ConvPart::kAll, s);
-    } else if (!side) { // everything on the caller's stream, in order
+    } else if (vconv || !side) { // everything on the caller's stream, in order
+        // (16-bit activations: the conv of q and k only; the chunk kernel
+        // convolves v from the pre-conv rows)
         e = launch_chunk_offsets(p, s);
         if (e == cudaSuccess)
-            e = launch_conv_prep(p, ConvPart::kAll, s);
+            e = launch_conv_prep(p, vconv ? ConvPart::kQK : ConvPart::kAll, s);
         if (e == cudaSuccess)
             e = launch_gram(p, s);
         if (e == cudaSuccess)
@@ -466,6 +532,8 @@ gdn_status kda_check(const gdn_config *cfg, const gdn_kda_params *params) {
         return st;
     if (cfg->num_qk_heads != cfg->num_v_heads) // one q and one k per head
         return GDN_ERR_INVALID_ARG;
+    if (cfg->segments > 1) // token-serial: no sequence split
+        return GDN_ERR_UNSUPPORTED;
     if (params == nullptr || params->conv_w == nullptr || params->A_log == nullptr ||
         params->norm_w == nullptr || !aligned16(params->conv_w) || !aligned16(params->norm_w) ||
         (reinterpret_cast<uintptr_t>(params->A_log) & 3u))
@@ -482,6 +550,8 @@ gdn_status gdn_kda_prefill_workspace_size(const gdn_config *cfg, int32_t batch, 
         return st;
     if (cfg->num_qk_heads != cfg->num_v_heads)
         return GDN_ERR_INVALID_ARG;
+    if (cfg->segments > 1)
+        return GDN_ERR_UNSUPPORTED;
     if (bytes == nullptr || batch < 0 || total_tokens < 0)
         return GDN_ERR_INVALID_ARG;
     // the token-serial path's regions: header, normalised q|k, convolved v

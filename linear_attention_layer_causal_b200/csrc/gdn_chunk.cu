@@ -242,11 +242,29 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     const int j = h / p.G;
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    // The segment of sequence n this CTA scans: chunks [cb, ce) of its nc, the
+    // sequence cut into p.segments equal runs.  The output pass has one CTA per
+    // segment (blockIdx.z); the summary pass two per segment but the last
+    // (blockIdx.z = 2 seg + which), which run the segment from S0 = 0 (R) and
+    // from S0 = I with the values taken as zero (M), and write no outputs.
+    const bool summary = p.seg_pass != 0;
+    const int seg = summary ? (int)(blockIdx.z >> 1) : (int)blockIdx.z;
+    const bool mpart = summary && (blockIdx.z & 1) != 0;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
-    const int64_t len = end - start;
-    const int nchunks = (int)((len + kC - 1) / kC);
+    const int nc = (int)((end - start + kC - 1) / kC);
+    const int cb = (int)((int64_t)nc * seg / p.segments);
+    const int ce = (int)((int64_t)nc * (seg + 1) / p.segments);
+    start += (int64_t)cb * kC;
+    const int64_t len = (int64_t)(ce - cb) * kC < end - start ? (int64_t)(ce - cb) * kC : end - start;
+    const int nchunks = ce - cb;
     const int64_t HD = (int64_t)p.Hv * kD;
+    // one 128 x 128 state of the split's workspace: region r (0 = R, 1 = M,
+    // 2 = start states, indexed by seg - 1), segment sg
+    const int64_t seg_units = (int64_t)p.batch * (p.segments - 1) * p.Hv;
+    auto seg_state = [&](int r, int sg) {
+        return p.ws_seg + (((int64_t)r * seg_units + ((int64_t)n * (p.segments - 1) + sg) * p.Hv + h) * kD) * kD;
+    };
 
     const uint32_t bar_v = smem_u32(&sm.bar_v), bar_q = smem_u32(&sm.bar_q);
     const uint32_t bar_k = smem_u32(&sm.bar_k), bar_kmaj = smem_u32(&sm.bar_kmaj);
@@ -329,21 +347,30 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         const int lq = warp & 3, hf = warp >> 2; // TMEM lane quarter, column half
         const int vch = lq * 32 + lane;          // this thread's TMEM lane = value channel
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
-        // initial state into TMEM (row vch, this half's 64 columns)
+        // initial state into TMEM (row vch, this half's 64 columns): the call's
+        // (first segment), the chained start state (later segments of the output
+        // pass), zero (R) or the identity (M)
         {
-            const float *src = p.init_state
-                                   ? p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf
-                                   : nullptr;
+            const float *src = nullptr;
+            if (!summary && seg > 0)
+                src = seg_state(2, seg - 1) + (size_t)vch * kD + 64 * hf;
+            else if (!summary && p.init_state != nullptr)
+                src = p.init_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf;
 #pragma unroll
-            for (int cb = 0; cb < 2; ++cb) {
+            for (int bk = 0; bk < 2; ++bk) {
                 float v[32];
 #pragma unroll
                 for (int i = 0; i < 32; i += 4) {
-                    float4 x = src ? *reinterpret_cast<const float4 *>(src + cb * 32 + i)
+                    float4 x = src ? *reinterpret_cast<const float4 *>(src + bk * 32 + i)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
                     v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
                 }
-                tmem_st32(tl + kColS + 64 * hf + 32 * cb, v);
+                if (mpart) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        v[i] = vch == 64 * hf + 32 * bk + i ? 1.f : 0.f;
+                }
+                tmem_st32(tl + kColS + 64 * hf + 32 * bk, v);
             }
             tmem_wait_st();
         }
@@ -382,8 +409,9 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     const float gC = expf(sm.G[sl][kC - 1]); // padded rows carry g = 0
                     // three rounds of two TMEM loads in flight: S columns 0..31 and
                     // 32..63 of this half, then O rows r = 32 hf + 16 q + i
+                    const int nrd = summary ? 2 : 3; // the summary pass forms no O
 #pragma unroll 1
-                    for (int rd = 0; rd < 3; ++rd) {
+                    for (int rd = 0; rd < nrd; ++rd) {
                         float v[2][16];
                         const uint32_t col = rd < 2 ? kColS + 64 * hf + 32 * rd : cO + 32 * hf;
                         tmem_ld16(tl + col, v[0]);
@@ -446,6 +474,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 if (tid == 0)
                     mbar_arrive(bar_u);
             }
+            if (summary)
+                continue; // no outputs
             // ---- epilogue: o[v = vch][r] for this half's rows r = 32 hf + i,
             //      RMSNorm over v, times w[v] SiLU(z), stored
             {
@@ -636,6 +666,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             if (tt == 0)
                 mbar_arrive(bar_pT(c)); // gates and -T diag(beta gamma) of chunk c
+            if (summary)
+                continue; // no O, no P
             // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32 (the Q K^T rows are
             //      0 for s > r; the clamp keeps the unused upper triangle finite)
             good = waitp(bar_qk, phqk);
@@ -723,19 +755,21 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             for (int c = 0; good && c < nchunks; ++c) {
                 const uint32_t dXO = tmem + ((c & 1) ? kColX1 : kColX0);
                 const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0);
-                // ---- MMA 2: [X^T | O^T] = S [K; Q]^T (A = the state in TMEM)
-                good = waitp(bar_q, phq);
+                // ---- MMA 2: [X^T | O^T] = S [K; Q]^T (A = the state in TMEM); the
+                //      summary pass takes X^T alone (N = 64: the K rows of each block)
+                good = summary || waitp(bar_q, phq);
                 good = waitp(bar_kmaj, phkm) && good;
-                if (c >= 2)
+                if (c >= 2 && !summary)
                     good = ((c & 1) ? waitq(bar_of1, ((c >> 1) - 1) & 1)
                                     : waitq(bar_of0, ((c >> 1) - 1) & 1)) && good;
                 if (!all(good))
                     break;
                 tc_fence_after();
+                const uint32_t id2 = summary ? idT64 : id128;
 #pragma unroll 1
                 for (int s = 0; s < kD / 8; ++s) {
                     const uint64_t ks = (uint64_t)((((s >> 2) * 2 * kC * 128) + (s & 3) * 32) >> 4);
-                    mma_tf32_ts_if(dXO, tmem + kColS + 8 * s, dKQ + ks, id128, s > 0, is);
+                    mma_tf32_ts_if(dXO, tmem + kColS + 8 * s, dKQ + ks, id2, s > 0, is);
                 }
                 mma_commit_if(bar_m2, is);
                 // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
@@ -745,10 +779,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     break;
                 tc_fence_after();
                 {
+                    // M of the summary pass has no values: U^T = X^T (-T diag(b gamma))^T
+                    // alone, its first product overwriting U~^T
                     const uint64_t g0 = tg0(c), g1 = tg1(c);
 #pragma unroll 1
                     for (int s = 0; s < 4; ++s)
-                        mma_tf32_ts_if(dU, dXO + 8 * s, g0 + 2 * s, idT64, 1, is);
+                        mma_tf32_ts_if(dU, dXO + 8 * s, g0 + 2 * s, idT64, !mpart || s > 0, is);
 #pragma unroll 1
                     for (int s = 4; s < 8; ++s)
                         mma_tf32_ts_if(dU + 32, dXO + 8 * s, g1 + 2 * (s - 4), idT32, 1, is);
@@ -765,19 +801,21 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K (K MN-major)
                 good = waitp(bar_u, phu);
-                good = waitp(bar_pP, phP) && good;
+                good = (summary || waitp(bar_pP, phP)) && good;
                 good = waitp(bar_k, phk) && good;
                 if (!all(good))
                     break;
                 tc_fence_after();
                 {
                     const uint32_t dO = dXO + 64;
+                    if (!summary) {
 #pragma unroll 1
-                    for (int s = 0; s < 4; ++s)
-                        mma_tf32_ts_if(dO, dU + 8 * s, dP0 + 2 * s, idT64, 1, is);
+                        for (int s = 0; s < 4; ++s)
+                            mma_tf32_ts_if(dO, dU + 8 * s, dP0 + 2 * s, idT64, 1, is);
 #pragma unroll 1
-                    for (int s = 4; s < 8; ++s)
-                        mma_tf32_ts_if(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1, is);
+                        for (int s = 4; s < 8; ++s)
+                            mma_tf32_ts_if(dO + 32, dU + 8 * s, dP1 + 2 * (s - 4), idT32, 1, is);
+                    }
 #pragma unroll 1
                     for (int s = 0; s < kC / 8; ++s)
                         mma_tf32_ts_if(tmem + kColS, dXO + 8 * s, dK + s * 64, idS, 1, is);
@@ -820,13 +858,15 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             // the Q K^T rows of chunk c as a triangular tile: block 0 (64 rows) and the
             // lower half of block 1
             auto qktile = [&](int c) {
+                if (summary)
+                    return;
                 mbar_arrive_expect_tx(bar_qk, (uint32_t)(kTriFloats * sizeof(float)));
                 tma_load_2d(smem_u32(sm.P), &maps.kq, xkk, (int)t_of(c), bar_qk);
                 tma_load_2d(smem_u32(sm.P + 2048), &maps.kq32, xkk + 32, (int)(t_of(c) + 32), bar_qk);
                 ++cnt[6];
             };
             // T diag(beta) of chunk c: one box of 96 rows (the triangular tile)
-            const int chunk0 = __ldg(p.ws_offs + n); // global index of this sequence's first chunk
+            const int chunk0 = __ldg(p.ws_offs + n) + cb; // global index of this segment's first chunk
             auto tbtile = [&](int c) {
                 mbar_arrive_expect_tx(bar_tb(c), (uint32_t)(kTriFloats * sizeof(float)));
                 tma_load_2d(smem_u32(sm.Tb[c & 1]), &maps.tb, 0,
@@ -835,7 +875,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             };
             // the z rows of a chunk: one 128-column box of 64 rows
             auto ztile = [&](int c) {
-                if constexpr (kZTile) {
+                if (kZTile && !summary) {
                     mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
                     tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)t_of(c), bar_z);
                     ++cnt[7];
@@ -845,14 +885,15 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             tbtile(0);
             tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
             tile(3, sm.KQ, &maps.kmaj, xq, t_of(0), 4, kBlkQ);        // rows 0..63 of KQ
-            tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ); // rows 64..127
+            if (!summary)
+                tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ); // rows 64..127
             qktile(0);
             tile(2, sm.K, &maps.k, xq, t_of(0), 4, kBlkV);
             ztile(0);
             if (nchunks > 1)
                 tbtile(1);
             // six event streams, each served in chunk order as it completes
-            int ib = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile ? 0 : nchunks;
+            int ib = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile && !summary ? 0 : nchunks;
             long long t_last = clock64();
             while (ib < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
                 bool prog = false;
@@ -880,7 +921,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 if (i2 < nchunks && mbar_test_wait(bar_m2, i2 & 1)) { // K (K-major) and Q are free
                     if (i2 + 1 < nchunks) {
                         tile(3, sm.KQ, &maps.kmaj, xq, t_of(i2 + 1), 4, kBlkQ);
-                        tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(i2 + 1), 4, kBlkQ);
+                        if (!summary)
+                            tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(i2 + 1), 4, kBlkQ);
                     }
                     ++i2;
                     prog = true;
@@ -918,18 +960,24 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     if (!ok) {
         if (tid == 0 && p.ws_err != nullptr)
             atomicOr(p.ws_err, 1u);
-    } else if (warp < kSG / 32 && p.final_state != nullptr) {
+    } else if (warp < kSG / 32 &&
+               (summary || (seg == p.segments - 1 && p.final_state != nullptr))) {
+        // the final state (last segment of the output pass) or the segment's R or M
         const int lq = warp & 3, hf = warp >> 2, vch = lq * 32 + lane;
         const uint32_t tl = tmem + ((uint32_t)(lq * 32) << 16);
-        float *dst = p.final_state + (((size_t)n * p.Hv + h) * kD + vch) * kD + 64 * hf;
+        float *dst = (summary ? seg_state(mpart ? 1 : 0, seg) + (size_t)vch * kD
+                              : p.final_state + (((size_t)n * p.Hv + h) * kD + vch) * kD) + 64 * hf;
+        // the summary pass has not waited for the last MMA 3 here (the TMA warp has,
+        // before the barrier above)
+        tc_fence_after();
 #pragma unroll
-        for (int cb = 0; cb < 2; ++cb) {
+        for (int bk = 0; bk < 2; ++bk) {
             float v[32];
-            tmem_ld32(tl + kColS + 64 * hf + 32 * cb, v);
+            tmem_ld32(tl + kColS + 64 * hf + 32 * bk, v);
             tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4 *>(dst + cb * 32 + i) =
+                *reinterpret_cast<float4 *>(dst + bk * 32 + i) =
                     make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
         }
     }
@@ -937,6 +985,74 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     __syncthreads();
     if (warp == 0)
         tmem_dealloc(tmem, kTmemCols);
+}
+
+// ------------------------------------------------------------ segment chain
+//
+// The state entering each segment of a split sequence: with S(0) the call's
+// initial state (zero if none), S(s) = S(s - 1) M(s - 1) + R(s - 1) for
+// s = 1 .. P - 1, the affine map of segment s - 1 applied to the state entering
+// it.  FP32 on the CUDA cores: one CTA per (value head, sequence), each of its
+// 256 threads an 8 x 8 block of every 128 x 128 x 128 product; the left factor
+// sits transposed in shared memory so that both operands load as float4.
+constexpr int kCombThreads = 256;
+constexpr size_t kCombSmem = 2 * kD * kD * sizeof(float);
+
+__global__ void __launch_bounds__(kCombThreads)
+seg_combine_kernel(PrefillArgs p) {
+    extern __shared__ __align__(16) float comb_smem[];
+    float *At = comb_smem;           // At[k][i] = S(s - 1)[i][k]
+    float *Ms = comb_smem + kD * kD; // M(s - 1)[k][j]
+    const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
+    const int ty = tid >> 4, tx = tid & 15; // rows 8 ty .. 8 ty + 7, columns 8 tx .. 8 tx + 7
+    const int64_t units = (int64_t)p.batch * (p.segments - 1) * p.Hv;
+    auto st = [&](int r, int sg) {
+        return p.ws_seg + (((int64_t)r * units + ((int64_t)n * (p.segments - 1) + sg) * p.Hv + h) * kD) * kD;
+    };
+    const float *S0 = p.init_state ? p.init_state + ((int64_t)n * p.Hv + h) * kD * kD : nullptr;
+    for (int e = tid; e < kD * kD; e += kCombThreads)
+        At[(e % kD) * kD + e / kD] = S0 ? S0[e] : 0.f;
+    for (int sg = 1; sg < p.segments; ++sg) {
+        const float *M = st(1, sg - 1), *R = st(0, sg - 1);
+        float *out = st(2, sg - 1);
+        for (int e = 4 * tid; e < kD * kD; e += 4 * kCombThreads)
+            *reinterpret_cast<float4 *>(Ms + e) = *reinterpret_cast<const float4 *>(M + e);
+        __syncthreads(); // Ms and At (the previous step's result) are in
+        float acc[8][8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float4 r0 = *reinterpret_cast<const float4 *>(R + (8 * ty + i) * kD + 8 * tx);
+            const float4 r1 = *reinterpret_cast<const float4 *>(R + (8 * ty + i) * kD + 8 * tx + 4);
+            acc[i][0] = r0.x; acc[i][1] = r0.y; acc[i][2] = r0.z; acc[i][3] = r0.w;
+            acc[i][4] = r1.x; acc[i][5] = r1.y; acc[i][6] = r1.z; acc[i][7] = r1.w;
+        }
+#pragma unroll 4
+        for (int k = 0; k < kD; ++k) {
+            const float4 a0 = *reinterpret_cast<const float4 *>(At + k * kD + 8 * ty);
+            const float4 a1 = *reinterpret_cast<const float4 *>(At + k * kD + 8 * ty + 4);
+            const float4 b0 = *reinterpret_cast<const float4 *>(Ms + k * kD + 8 * tx);
+            const float4 b1 = *reinterpret_cast<const float4 *>(Ms + k * kD + 8 * tx + 4);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj)
+                    acc[i][jj] = fmaf(a[i], b[jj], acc[i][jj]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float *o = out + (8 * ty + i) * kD + 8 * tx;
+            *reinterpret_cast<float4 *>(o) = make_float4(acc[i][0], acc[i][1], acc[i][2], acc[i][3]);
+            *reinterpret_cast<float4 *>(o + 4) = make_float4(acc[i][4], acc[i][5], acc[i][6], acc[i][7]);
+        }
+        __syncthreads(); // every thread is done reading At and Ms
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj)
+                At[(8 * tx + jj) * kD + 8 * ty + i] = acc[i][jj];
+    }
 }
 
 template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStream_t s) {
@@ -971,8 +1087,22 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
         if (!okm)
             return cudaErrorInvalidValue;
     }
-    dim3 grid(p.Hv, p.batch);
-    chunk_prefill_kernel<T><<<grid, kThreads, smem, s>>>(p, maps);
+    if (p.segments > 1) {
+        // the split: (M, R) of every segment but the last, then the chained start
+        // states, then the output pass over all segments
+        PrefillArgs ps = p;
+        ps.seg_pass = 1;
+        chunk_prefill_kernel<T><<<dim3(p.Hv, p.batch, 2 * (p.segments - 1)), kThreads, smem, s>>>(ps, maps);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+        if ((e = cudaFuncSetAttribute(seg_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kCombSmem)) != cudaSuccess)
+            return e;
+        seg_combine_kernel<<<dim3(p.Hv, p.batch), kCombThreads, kCombSmem, s>>>(p);
+        if ((e = cudaGetLastError()) != cudaSuccess)
+            return e;
+    }
+    chunk_prefill_kernel<T><<<dim3(p.Hv, p.batch, p.segments), kThreads, smem, s>>>(p, maps);
     return cudaGetLastError();
 }
 

@@ -50,7 +50,8 @@ template <typename T> struct ConvIO {
     int Hk, Hv;
     float l2_eps, q_scale;
     float *qk_out;         // [N, 2 Hk D] normalised q | k
-    float *v_out;          // [N, Hv D] convolved v
+    float *v_out;          // [N, Hv D] convolved v (nullptr: v is not written; the chunk kernel
+                           // of 16-bit activations convolves v itself)
     bool round_v;          // v to its tf32 operand (tensor-core path)
     int block_y0;          // channel block of blockIdx.y = 0 (skips the q/k-only blocks)
 };
@@ -87,7 +88,7 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
     const bool norm_warp = V_ONLY ? false : __any_sync(0xffffffffu, region < 2);
     auto emit = [&](int64_t t, float (&acc)[V]) {
         if (V_ONLY) {
-            if (!active)
+            if (!active || io.v_out == nullptr)
                 return;
             float *dst = io.v_out + t * ((int64_t)io.Hv * D) + (cc - 2 * io.Hk * D);
 #pragma unroll
@@ -110,7 +111,7 @@ __device__ __forceinline__ void conv_emit(const ConvIO<T> &io, int cc, bool acti
         }
         if (norm_warp)
             ss = group_sum<LANES>(ss);
-        if (!active)
+        if (!active || (region == 2 && io.v_out == nullptr))
             return;
         const float f = region == 2 ? 1.0f : rsqrtf(ss + io.l2_eps) * (region == 0 ? io.q_scale : 1.0f);
         if (region == 2 && io.round_v) {

@@ -30,11 +30,15 @@ struct PrefillArgs {
     // workspace carve-up
     unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)
     void *ws_qk;             // [N, 2*Hk*D] float32: normalised q | k
-    void *ws_v;              // [N, Hv*D]   float32: convolved v
+    void *ws_v;              // [N, Hv*D]   float32: convolved v (nullptr where the chunk kernel convolves v)
     void *ws_kq;             // [N, Hk, 64] float32: chunk Q K^T rows (chunked path)
     void *ws_kk;             // [chunks, Hk, 3072] float32: K K^T triangular tiles (chunked path)
     void *ws_tb;             // [chunks, Hv, 96, 32] float32: T diag(beta) tiles (chunked path)
     int32_t *ws_offs;        // [batch + 1] chunk offsets per sequence (chunked path)
+    // sequence split of the chunked path (segments > 1)
+    int segments = 1;        // P: segments per sequence
+    int seg_pass = 0;        // chunk kernel launch: 0 = output pass, 1 = summary pass
+    float *ws_seg = nullptr; // R, M [batch, P-1, Hv, 128, 128] each, then the segment start states
 };
 
 struct DecodeArgs {
@@ -96,7 +100,15 @@ inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
 }
 
 // Workspace bytes for the prefill path (each region 256-byte aligned).
-size_t prefill_workspace_bytes(int Hk, int Hv, int D, bool bf16, int64_t N, int batch);
+size_t prefill_workspace_bytes(const gdn_config *c, int64_t N, int batch);
+// The chunk kernel convolves v itself from the 16-bit pre-conv rows; the
+// front end then writes no convolved v.
+inline bool v_conv_in_chunk(bool chunked, bool bf16) { return false && chunked && bf16; }
+// Segments per sequence a chunked prefill of this config and size runs with
+// (1 for the token-serial path and for calls without tokens).
+int prefill_segments(const gdn_config *c, int batch, int64_t N);
+constexpr int kMaxSegments = 16;
+size_t seg_workspace_bytes(int Hv, int batch, int segments);
 constexpr size_t kWorkspaceHeader = 256; // holds the device status word
 
 // Which channels a conv launch covers: all, the channel blocks holding q or k

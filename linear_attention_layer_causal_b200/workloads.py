@@ -24,12 +24,14 @@ Distributions (all draws from one seeded generator, in the order listed):
   initial states                ~ N(0, 0.02^2) (where the workload has them)
   conv cache (decode)           ~ N(0, 1), activation dtype
 
-Long-memory gates (gates="long_memory:<dt_bias>"): A_log = 0 and dt_bias =
-the given constant instead of the draws above, and b ~ N(2, 0.5^2), so that
-g = -softplus(a + dt_bias) is small (about -0.018 per token at dt_bias = -4,
--3e-4 at -8) and beta = sigmoid(b) is about 0.88: the state keeps its past
-for hundreds to thousands of tokens, where the default draws (exp(A_log) in
-[1, 16]) forget within a few tokens.
+Long-memory gates (gates="long_memory:<dt_bias>[:<b_mean>]"): A_log = 0 and
+dt_bias = the given constant instead of the draws above, and b ~ N(b_mean,
+0.5^2) (b_mean = 2 unless given), so that g = -softplus(a + dt_bias) is small
+(about -0.018 per token at dt_bias = -4, -3e-4 at -8) and beta = sigmoid(b) is
+about 0.88 (0.12 at b_mean = -2): the state keeps its past for hundreds to
+thousands of tokens, where the default draws (exp(A_log) in [1, 16]) forget
+within a few tokens.  A small beta also slows the delta rule's own erasure
+along each new k, so the state carries across thousands of tokens.
 """
 from __future__ import annotations
 
@@ -52,7 +54,7 @@ class Workload:
     state_every: int = 1                 # sequences n with n % state_every == 0 get a state
     seed: int = 0
     conv_kernel: int = 4
-    gates: str = "default"               # or "long_memory:<dt_bias>" (see the module docstring)
+    gates: str = "default"               # or "long_memory:<dt_bias>[:<b_mean>]" (module docstring)
     notes: str = field(default="", compare=False)
 
     @property
@@ -93,9 +95,25 @@ QWEN38_VERY_LONG_MEMORY = Workload("qwen38_very_long_memory", 16, 128, 128, seql
                                    state_std=0.02, seed=1008, gates="long_memory:-8",
                                    notes="Qwen3.8 layer, B=3 T=16384, nearly undecaying state")
 
+# Long context: one sequence of 262,144 tokens, the Qwen3.8 context window
+# ("Qwen3.8 2.4T A95B", key facts and raw config max_position_embeddings), at
+# the Qwen3.8 layer shape and at the Qwen3.5-397B shape, whose 64 value heads
+# leave more than half of the SMs to a split of the sequence.
+QWEN38_262K = Workload("qwen38_262k_prefill", 16, 128, 128, seqlens=(262144,), seed=1010,
+                       notes="Qwen3.8 layer, one 262,144-token sequence")
+QWEN35_262K = Workload("qwen35_262k_prefill", 16, 64, 128, seqlens=(262144,), seed=1011,
+                       notes="Qwen3.5-397B-A17B layer, one 262,144-token sequence")
+# The sequence split under a state that carries across segments: nearly no
+# decay and beta about 0.12; lengths with empty, one-token and ragged
+# sequences beside ones of several segments.
+SPLIT_MEMORY = Workload("qwen35_split_memory", 16, 64, 128, seqlens=(1100, 0, 593, 1, 2048),
+                        state_std=0.02, seed=1012, gates="long_memory:-8:-2",
+                        notes="Qwen3.5 layer, varlen, slowly forgetting state, for the split")
+
 WORKLOADS = {w.name: w for w in (TINY, QWEN38_PREFILL, QWEN38_LONG, QWEN38_DECODE, QWEN36_VARLEN,
                                  QWEN35_PREFILL, QWEN35_DECODE, QWEN38_LONG_MEMORY,
-                                 QWEN38_VERY_LONG_MEMORY)}  # (the KDA workload is added below)
+                                 QWEN38_VERY_LONG_MEMORY, QWEN38_262K, QWEN35_262K,
+                                 SPLIT_MEMORY)}  # (the KDA workload is added below)
 
 
 def _gen(device, seed):
@@ -151,7 +169,9 @@ def make_prefill(wl: Workload, device="cpu", seqlens=None, seed=None):
     out["a"] = _normal((N, H), 1.0, g, device, dt)
     out["b"] = _normal((N, H), 1.0, g, device, dt)
     if wl.gates.startswith("long_memory"):
-        out["b"] = (out["b"].float() * 0.5 + 2.0).to(dt)
+        parts = wl.gates.split(":")
+        b_mean = float(parts[2]) if len(parts) > 2 else 2.0
+        out["b"] = (out["b"].float() * 0.5 + b_mean).to(dt)
     out["z"] = _normal((N, H, d), 1.0, g, device, dt)
     out.update(_params(wl, g, device))
     if wl.state_std > 0:

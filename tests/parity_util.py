@@ -74,7 +74,7 @@ def assert_state_close(got, ref, what="state", rel=STATE_REL_L2):
 
 
 def report(name, rel=None, maxabs=None, state_rel=None):
-    """One line of budget use: each figure as a fraction of its spec bound."""
+    """One line of budget use: each figure as a fraction of its tolerance bound."""
     parts = [name]
     if rel is not None:
         parts.append(f"y_rel={rel:.3e} ({rel / OUT_REL_L2:.1%} of bound)")

@@ -31,7 +31,7 @@ def test_library_exports_every_declared_symbol():
     assert set(gdn.EXPORTED) <= set(declared)
     for name in declared:
         assert hasattr(L, name), f"{name} declared in include/ but not exported"
-    assert L.gdn_abi_version() == 2
+    assert L.gdn_abi_version() == 3
 
 
 def test_status_strings():
@@ -66,6 +66,42 @@ def test_workspace_size_arithmetic():
     assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 1, 3) == 256 + 1536 + 1536
 
 
+def test_segment_workspace_and_choice():
+    """The split's workspace (R, M and start states: 3 (P - 1) batch H_v d^2 floats)
+    and the library's choice of P."""
+    state = 128 * 128 * 4
+    for B, N in ((1, 4096), (3, 20000)):
+        base = gdn.prefill_workspace_size(gdn.Config(16, 128, 128, segments=1), B, N)
+        assert gdn.prefill_workspace_size(QWEN38, B, N) == base  # 128 value heads: no split
+        for P in (2, 5, 16):
+            c = gdn.Config(16, 128, 128, segments=P)
+            assert gdn.prefill_workspace_size(c, B, N) == base + 3 * (P - 1) * B * 128 * state
+    # the token-serial path takes segments 0 and 1
+    for P in (0, 1):
+        assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32, segments=P), 1, 3) == 256 + 1536 + 1536
+    # no tokens: no workspace, whatever P
+    assert gdn.prefill_workspace_size(gdn.Config(16, 128, 128, segments=4), 2, 0) == 0
+    # the library's choice at 64 value heads: one sequence of 262,144 tokens is split
+    # (64 chains would leave 84 of the 148 SMs idle), one of 2,048 is not (too short),
+    # and neither is a batch of 2 x 131,072 (128 chains fill the SMs)
+    q35 = gdn.Config(16, 64, 128)
+    one = gdn.Config(16, 64, 128, segments=1)
+    extra = gdn.prefill_workspace_size(q35, 1, 262144) - gdn.prefill_workspace_size(one, 1, 262144)
+    assert extra > 0 and extra % (3 * 64 * state) == 0
+    assert gdn.prefill_workspace_size(q35, 1, 2048) == gdn.prefill_workspace_size(one, 1, 2048)
+    assert gdn.prefill_workspace_size(q35, 2, 262144) == gdn.prefill_workspace_size(one, 2, 262144)
+    assert gdn.prefill_segments(q35, 1, 262144) == 1 + extra // (3 * 64 * state)
+    assert gdn.prefill_segments(QWEN38, 1, 262144) == 1
+    assert gdn.prefill_segments(gdn.Config(16, 128, 128, segments=7), 1, 100) == 7
+    assert gdn.prefill_segments(gdn.Config(16, 128, 128, segments=7), 1, 0) == 1
+    assert gdn.prefill_segments(gdn.Config(2, 4, 32), 1, 1 << 20) == 1
+    # few heads, a long sequence: several segments
+    small = gdn.Config(2, 8, 128)
+    extra = (gdn.prefill_workspace_size(small, 1, 1 << 20) -
+             gdn.prefill_workspace_size(gdn.Config(2, 8, 128, segments=1), 1, 1 << 20))
+    assert extra // (3 * 8 * state) + 1 >= 4
+
+
 @pytest.mark.parametrize("cfg,code", [
     (gdn.Config(0, 4, 32), gdn.GDN_ERR_INVALID_ARG),
     (gdn.Config(3, 4, 32), gdn.GDN_ERR_INVALID_ARG),        # H_v not a multiple of H_k
@@ -74,6 +110,10 @@ def test_workspace_size_arithmetic():
     (gdn.Config(2, 4, 32, rms_eps=-1.0), gdn.GDN_ERR_INVALID_ARG),
     (gdn.Config(2, 4, 32, l2_eps=float("nan")), gdn.GDN_ERR_INVALID_ARG),
     (gdn.Config(2, 4, 32, algo="chunked"), gdn.GDN_ERR_UNSUPPORTED),  # chunked needs d = 128
+    (gdn.Config(16, 128, 128, segments=-1), gdn.GDN_ERR_INVALID_ARG),
+    (gdn.Config(16, 128, 128, segments=17), gdn.GDN_ERR_INVALID_ARG),
+    (gdn.Config(2, 4, 32, segments=2), gdn.GDN_ERR_UNSUPPORTED),      # the split is chunked-only
+    (gdn.Config(16, 128, 128, algo="serial", segments=2), gdn.GDN_ERR_UNSUPPORTED),
 ])
 def test_bad_config_rejected(cfg, code):
     n = ctypes.c_size_t(0)
