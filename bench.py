@@ -367,8 +367,8 @@ def run_ours(args, rank, world, dev, dist):
             "roofline": roof, "decode": decode, "decode_k": decode_k, "qwen35_prefill": qwen35,
             "long_context": long_ctx,
             "e2e": e2e,
-            # chunked: offsets, conv of q|k and of v (side stream), Gram, inverses, chunk kernel
-            "gpu_launches": (6 if kname == "chunk_prefill_kernel" else 2) * args.steps,
+            # chunked (16-bit activations): offsets, conv of q|k, Gram, inverses, chunk kernel
+            "gpu_launches": (5 if kname == "chunk_prefill_kernel" else 2) * args.steps,
             "clocks": clk}
     return line
 

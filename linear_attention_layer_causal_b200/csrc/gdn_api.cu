@@ -199,8 +199,8 @@ gdn_status read_status_words(const void *header, uint32_t *detail, cudaStream_t 
 
 // Header (status word), float32 normalised q|k, float32 convolved v (unless
 // the chunk kernel convolves v itself: 16-bit activations) and, on the
-// chunked path, the Q K^T rows, K K^T and T diag(beta) tiles, the
-// per-sequence chunk offsets and the split's states.
+// chunked path, the Q K^T rows, K K^T and T diag(beta) tiles, the gate
+// records, the per-sequence chunk offsets and the split's states.
 size_t prefill_workspace_bytes(const gdn_config *c, int64_t N, int batch) {
     if (N == 0)
         return 0;
@@ -211,8 +211,8 @@ size_t prefill_workspace_bytes(const gdn_config *c, int64_t N, int batch) {
         b += round_up((size_t)N * Hv * D * 4);
     if (chunked)
         b += round_up(kq_workspace_bytes(Hk, N)) + round_up(kk_workspace_bytes(Hk, N, batch)) +
-             round_up(tb_workspace_bytes(Hv, N, batch)) + round_up(((size_t)batch + 1) * sizeof(int32_t)) +
-             seg_workspace_bytes(Hv, batch, prefill_segments(c, batch, N));
+             round_up(tb_workspace_bytes(Hv, N, batch)) + round_up(gt_workspace_bytes(Hv, N, batch)) +
+             round_up(((size_t)batch + 1) * sizeof(int32_t)) + seg_workspace_bytes(Hv, batch, prefill_segments(c, batch, N));
     return b;
 }
 
@@ -349,8 +349,9 @@ gdn_status prefill_impl(const gdn_config *cfg, const gdn_params *params, const v
             p.ws_kq = w;
             p.ws_kk = (char *)p.ws_kq + round_up(kq_workspace_bytes(p.Hk, total_tokens));
             p.ws_tb = (char *)p.ws_kk + round_up(kk_workspace_bytes(p.Hk, total_tokens, batch));
-            p.ws_offs = (int32_t *)((char *)p.ws_tb +
-                                    round_up(tb_workspace_bytes(p.Hv, total_tokens, batch)));
+            p.ws_gt = (float *)((char *)p.ws_tb + round_up(tb_workspace_bytes(p.Hv, total_tokens, batch)));
+            p.ws_offs = (int32_t *)((char *)p.ws_gt +
+                                    round_up(gt_workspace_bytes(p.Hv, total_tokens, batch)));
             p.segments = prefill_segments(cfg, batch, total_tokens);
             if (p.segments > 1)
                 p.ws_seg = (float *)((char *)p.ws_offs + round_up(((size_t)batch + 1) * sizeof(int32_t)));

@@ -148,7 +148,9 @@ constexpr uint32_t kTmemCols = 512;
 struct __align__(1024) ChunkSmem {
     // B of MMA 2 (K-major, N = 128 rows): rows 0..63 = K, rows 64..127 = Q
     float KQ[2 * kC * kD];
-    float V[kC * kD];          // A of MMA 1 (MN-major)
+    // A of MMA 1: V by TMA, MN-major (fp32 activations), or V^T (rows = value
+    // channels) written by the prep team, K-major (16-bit activations)
+    float V[kC * kD];
     float K[kC * kD];          // B of MMA 3 (MN-major): lands as K, becomes diag(gamma_C/gamma) K
     float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta) (from the front kernel, by TMA), by chunk parity
     float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma), by chunk parity
@@ -156,6 +158,9 @@ struct __align__(1024) ChunkSmem {
     // z rows of the chunk (16-bit activations).  Once the state group has formed
     // the gate from it, it stages the chunk's y rows for one TMA store.
     __nv_bfloat16 Z[kC * kD];
+    // pre-conv v rows t0 - 3 .. t0 + 63 of the head (16-bit activations), from
+    // which the prep team convolves V
+    __nv_bfloat16 Vx[(kC + 3) * kD];
     float red[4][kC];          // epilogue: partial sums of o^2 per TMEM lane quarter
     float rstd[kC];            // epilogue: reciprocal RMS of each row
     float G[4][kC], kd[4][kC]; // log-decay prefix and gamma_C / gamma by chunk index mod 4
@@ -167,15 +172,18 @@ struct __align__(1024) ChunkSmem {
     unsigned long long bar_zf;                                  // state group -> TMA: z tile free
     unsigned long long bar_pT[4], bar_pP;                       // prep team -> MMA, TMA, state group
     unsigned long long bar_fin;                                 // MMA drain on abort
+    unsigned long long bar_vx, bar_vxf;                         // TMA landing of Vx; prep team -> TMA: Vx read
     uint32_t tmem;
     int abort;
 };
+static_assert(sizeof(ChunkSmem) <= 227 * 1024, "the chunk kernel's shared memory exceeds a CTA's 227 KB");
 
 
 // The tensor maps of one call: 64-row boxes (32-row for the lower half of
 // the Gram tiles' second column block) of the workspace.
 struct ChunkMaps {
-    CUtensorMap v;    // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle
+    CUtensorMap v;    // convolved v, [N, Hv*128] fp32, 32-column boxes, MN-major tf32 swizzle (fp32 activations)
+    CUtensorMap vx;   // pre-conv qkv rows, [N, conv_dim] bf16, 128 x 67 boxes, no swizzle (bf16 activations)
     CUtensorMap k;    // normalised k, [N, Hk*128] of the q|k rows, MN-major tf32 swizzle
     CUtensorMap q;    // normalised q, [N, Hk*128], 128-byte swizzle (K-major)
     CUtensorMap kmaj; // normalised k, [N, Hk*128], 128-byte swizzle (K-major)
@@ -273,6 +281,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     auto bar_tb = [&](int c) { return smem_u32(&sm.bar_tb[c & 1]); };
     const uint32_t bar_z = smem_u32(&sm.bar_z);
     constexpr bool kZTile = sizeof(T) == 2; // z comes by TMA (16-bit) or from global (fp32)
+    constexpr bool kVConv = sizeof(T) == 2; // the prep team convolves v from the pre-conv rows (16-bit)
     const uint32_t bar_m1 = smem_u32(&sm.bar_m1), bar_m2 = smem_u32(&sm.bar_m2);
     const uint32_t bar_m3 = smem_u32(&sm.bar_m3);
     // MMA 2b done, by chunk parity (its waiters are a chunk apart)
@@ -288,7 +297,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     if (tid == 0) {
         const uint32_t one[] = {bar_v,  bar_q,  bar_k,   bar_kmaj, bar_qk,  bar_z,  bar_m1,
                                 bar_m2, bar_m3, bar_u,   bar_of0,  bar_of1, bar_pP, bar_zf,
-                                smem_u32(&sm.bar_fin)};
+                                smem_u32(&sm.bar_fin), smem_u32(&sm.bar_vx), smem_u32(&sm.bar_vxf)};
 #pragma unroll
         for (int b = 0; b < (int)(sizeof(one) / sizeof(one[0])); ++b)
             mbar_init(one[b], 1);
@@ -578,67 +587,104 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             *abort_flag = 1;
     } else if (warp < (kSG + kTeam) / 32) {
         // ==================================================== prep team
-        // Per chunk: the gates; -T diag(beta gamma) from the T diag(beta) tile that
+        // Per chunk: the gate record; -T diag(beta gamma) from the T diag(beta) tile that
         // the front kernel formed (the B operands of MMA 2b and MMA 1); P from the
         // Q K^T rows.  All tf32, in the triangular-tile layout.
-        const int tt = tid - kSG, tw = tt >> 5;
+        const int tt = tid - kSG;
         const TriThread tr(tt);
-        // raw gate inputs of chunk c, rows lane and lane + 32 (first warp of the team)
-        auto load_ab = [&](int c, T (&ra)[2], T (&rb)[2]) {
-            if (tw == 0) {
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int r = lane + 32 * q;
-                    ra[q] = from_f<T>(0.f);
-                    rb[q] = from_f<T>(0.f);
-                    if (c < nchunks && r < rows_of(c)) {
-                        const int64_t t = start + (int64_t)c * kC + r;
-                        ra[q] = ((const T *)p.a)[t * p.Hv + h];
-                        rb[q] = ((const T *)p.b)[t * p.Hv + h];
-                    }
-                }
+        // The gate record of chunk c, formed by the inverse kernel: G, gamma_C /
+        // gamma and gamma of its 64 rows (padded rows carry g = 0), 48 float4s
+        // that threads tt < 48 load one chunk ahead and store into slot c mod 4.
+        // (a call without tokens has no workspace: nothing is read then)
+        const float *grec =
+            nchunks > 0 ? p.ws_gt + ((size_t)(__ldg(p.ws_offs + n) + cb) * p.Hv + h) * kGateRec : nullptr;
+        auto load_gt = [&](int c) {
+            return tt < kGateRec / 4 && c < nchunks
+                       ? __ldg(reinterpret_cast<const float4 *>(grec + (size_t)c * p.Hv * kGateRec) + tt)
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+        };
+        auto put_gt = [&](const float4 &v, int sl) {
+            if (tt < kGateRec / 4) {
+                const int arr = tt >> 4, e = 4 * (tt & 15);
+                float *d = (arr == 0 ? sm.G[sl] : (arr == 1 ? sm.kd[sl] : sm.gam[sl])) + e;
+                *reinterpret_cast<float4 *>(d) = v;
             }
         };
-        const float negA = -expf(__ldg(p.A_log + h));
-        const float dtb = __ldg(p.dt_bias + h);
-        // g, the inclusive prefix G, gamma_C / gamma and gamma of a chunk into slot
-        // `sl` (first warp; rows lane and lane + 32).  The same arithmetic as the
-        // front kernel's, so that both see the same G.
-        auto gates = [&](int c, const T (&ra)[2], int sl) {
-            if (tw == 0) {
-                float g[2];
+        // ---- (16-bit activations) V of chunk c: thread tt convolves value channel tt
+        //      of the head over the chunk's rows (kernel 4, SiLU, tf32 rounding, the
+        //      front end's arithmetic for q and k) from the staged pre-conv rows and, in
+        //      the first chunk of a sequence, the initial conv window.  Written as V^T
+        //      (rows = value channels, columns = tokens) in the K-major 128-byte-swizzled
+        //      layout, four tokens per float4; rows past the chunk's end are zero.
+        //      M of the summary pass ignores V and skips the arithmetic.
+        const int Cd = (2 * p.Hk + p.Hv) * kD;
+        const int cv = 2 * p.Hk * kD + h * kD + tt; // this thread's qkv channel
+        float4 cw = make_float4(0.f, 0.f, 0.f, 0.f);
+        if constexpr (kVConv)
+            cw = __ldg(reinterpret_cast<const float4 *>(p.conv_w) + cv);
+        uint32_t phvx = 0;
+        auto vconv = [&](int c) {
+            bool good = waitp(smem_u32(&sm.bar_vx), phvx);       // the pre-conv rows of chunk c
+            good = (c < 1 || waitq(bar_m1, (c - 1) & 1)) && good; // MMA 1 of chunk c - 1 has read V
+            if (good && !mpart) {
+                // four quarters of 16 tokens: the quarter's 19 staged rows are loaded
+                // before any arithmetic and its 16 outputs are independent; then four
+                // float4 stores
+                const __nv_bfloat16 *x = sm.Vx + tt;
+                const int rows = rows_of(c);
+                const T *iw = (const T *)p.init_conv + (int64_t)n * 3 * Cd + cv;
+                float *vt = sm.V + 32 * tt;
+#pragma unroll 1
+                for (int qt = 0; qt < kC / 16; ++qt) {
+                    float xr[19]; // rows t - 3 .. t + 15 of the quarter's tokens t
 #pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const bool in = lane + 32 * q < rows_of(c);
-                    g[q] = in ? negA * softplusf_(to_f(ra[q]) + dtb) : 0.f;
-                }
+                    for (int i = 0; i < 19; ++i)
+                        xr[i] = to_f(x[(16 * qt + i) * kD]);
+                    if (qt == 0 && cb + c == 0) { // taps before the sequence: the initial window
 #pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    const float x0 = __shfl_up_sync(0xffffffffu, g[0], o);
-                    const float x1 = __shfl_up_sync(0xffffffffu, g[1], o);
-                    if (lane >= o) {
-                        g[0] += x0;
-                        g[1] += x1;
+                        for (int i = 0; i < 3; ++i)
+                            xr[i] = p.init_conv ? to_f(iw[i * Cd]) : 0.f;
+                    }
+                    float o[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        float acc = cw.x * xr[i];
+                        acc = fmaf(cw.y, xr[i + 1], acc);
+                        acc = fmaf(cw.z, xr[i + 2], acc);
+                        acc = fmaf(cw.w, xr[i + 3], acc);
+                        o[i] = tf32_rna(siluf_(acc));
+                        // rows past the end of a partial chunk: zero (a branch uniform
+                        // over the CTA; a select around the SiLU measured far slower)
+                        if (rows < kC && 16 * qt + i >= rows)
+                            o[i] = 0.f;
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) { // tokens 16 qt + 4 q4 .. + 3
+                        const int t4 = 16 * qt + 4 * q4;
+                        *reinterpret_cast<float4 *>(vt + (t4 >> 5) * (kD * 32) + 4 * (((t4 & 31) >> 2) ^ (tt & 7))) =
+                            make_float4(o[4 * q4], o[4 * q4 + 1], o[4 * q4 + 2], o[4 * q4 + 3]);
                     }
                 }
-                g[1] += __shfl_sync(0xffffffffu, g[0], 31);
-                const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    const int r = lane + 32 * q;
-                    sm.G[sl][r] = g[q];
-                    sm.kd[sl][r] = expf(Glast - g[q]);
-                    sm.gam[sl][r] = __expf(g[q]);
-                }
             }
+            fence_proxy_async_smem();
+            if (group_sync_or(kBarT, kTeam, !good || *abort_flag))
+                return false;
+            if (tt == 0) {
+                mbar_arrive(bar_v);                  // V of chunk c, for MMA 1
+                mbar_arrive(smem_u32(&sm.bar_vxf)); // the staged rows may take chunk c + 1
+            }
+            return true;
         };
         uint32_t phqk = 0;
-        T av[2], bv[2];
-        load_ab(0, av, bv);
-        for (int c = 0; c < nchunks; ++c) {
+        float4 gv = load_gt(0);
+        if constexpr (kVConv) {
+            if (nchunks > 0 && !vconv(0))
+                ok = false;
+        }
+        for (int c = 0; ok && c < nchunks; ++c) {
             const int sl = c & 3;
-            gates(c, av, sl);
-            load_ab(c + 1, av, bv);
+            put_gt(gv, sl);
+            gv = load_gt(c + 1);
             group_sync(kBarT, kTeam); // the gates are in
             // ---- -T diag(beta gamma) = -(T diag beta) diag(gamma) into this chunk's
             //      parity slot once MMA 2b of chunk c - 2 has read it
@@ -666,12 +712,11 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             if (tt == 0)
                 mbar_arrive(bar_pT(c)); // gates and -T diag(beta gamma) of chunk c
-            if (summary)
-                continue; // no O, no P
             // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32 (the Q K^T rows are
-            //      0 for s > r; the clamp keeps the unused upper triangle finite)
-            good = waitp(bar_qk, phqk);
-            if (good) {
+            //      0 for s > r; the clamp keeps the unused upper triangle finite); the
+            //      summary pass has no O and no P
+            good = summary || waitp(bar_qk, phqk);
+            if (good && !summary) {
                 float4 x[6];
 #pragma unroll
                 for (int jj = 0; jj < 6; ++jj)
@@ -692,8 +737,14 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 ok = false;
                 break;
             }
-            if (tt == 0)
+            if (tt == 0 && !summary)
                 mbar_arrive(bar_pP); // P of chunk c
+            if constexpr (kVConv) { // V of the next chunk
+                if (c + 1 < nchunks && !vconv(c + 1)) {
+                    ok = false;
+                    break;
+                }
+            }
         }
         if (!ok)
             *abort_flag = 1;
@@ -705,7 +756,12 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         if (nchunks > 0) {
             const uint32_t is = elect_one();
             auto all = [&](bool g) { return __all_sync(0xffffffffu, g) != 0; };
-            const uint64_t dV = sdesc_sw128_b32(smem_u32(sm.V), kC * 128, 512);
+            // V: MN-major from TMA, or V^T K-major from the prep team (128 rows a block)
+            const uint64_t dV = kVConv ? sdesc_sw128(smem_u32(sm.V), 16, 1024)
+                                       : sdesc_sw128_b32(smem_u32(sm.V), kC * 128, 512);
+            auto aV = [&](int s) -> uint64_t {
+                return kVConv ? dV + (uint64_t)((((s >> 2) * kD * 128) + (s & 3) * 32) >> 4) : dV + s * 64;
+            };
             const uint64_t dK = sdesc_sw128_b32(smem_u32(sm.K), kC * 128, 512);
             const uint64_t dKQ = sdesc_sw128(smem_u32(sm.KQ), 16, 1024);
             const uint64_t dP0 = sdesc_sw128(smem_u32(sm.P), 16, 1024);
@@ -720,6 +776,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             constexpr uint32_t idT64 = idesc_tf32(128, 64, false, false);  // MMA 2b, MMA 3 O
             constexpr uint32_t idT32 = idesc_tf32(128, 32, false, false);
             constexpr uint32_t idS = idesc_tf32(128, 128, false, true);    // MMA 3 S (B MN-major)
+            constexpr uint32_t idV64 = kVConv ? idT64 : id64, idV32 = kVConv ? idT32 : id32; // MMA 1
             uint32_t phv = 0, phkm = 0, phq = 0, phu = 0, phP = 0, ph2 = 0, phk = 0;
             // MMA 1 of chunk c: U~^T into U_(c%2).  K steps 0..3 run over column
             // block 0 of the T tile (N = 64), 4..7 over block 1 (rows 32..63)
@@ -728,10 +785,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 const uint64_t b0 = tb0(c), b1 = tb1(c);
 #pragma unroll 1
                 for (int s = 0; s < 4; ++s)
-                    mma_tf32_ss_if(dU, dV + s * 64, b0 + 2 * s, id64, s > 0, is);
+                    mma_tf32_ss_if(dU, aV(s), b0 + 2 * s, idV64, s > 0, is);
 #pragma unroll 1
                 for (int s = 4; s < 8; ++s)
-                    mma_tf32_ss_if(dU + 32, dV + s * 64, b1 + 2 * (s - 4), id32, 1, is);
+                    mma_tf32_ss_if(dU + 32, aV(s), b1 + 2 * (s - 4), idV32, 1, is);
                 mma_commit_if(bar_m1, is);
             };
             // the inputs of MMA 1 of chunk c: its T diag(beta) tile and V (both by TMA);
@@ -746,12 +803,23 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 g = g && waitq(bar_v, phv);
                 return all(g);
             };
-            bool good = m1_ready(0, true);
-            good = all(waitp(bar_u, phu) && good); // phase 0 of U: the initial state
-            phv ^= 1u;
-            tc_fence_after();
+            // MMA 1 of chunk c runs any time between MMA 3 of chunk c - 2 (the last
+            // reader of its U buffer) and MMA 2b of chunk c (its first consumer): it is
+            // issued as soon as its T diag(beta) tile and V are in, at the latest
+            // (waiting for them) just before MMA 2b, so that neither the V loads nor
+            // the prep team's v conv hold up MMA 2
+            int m1_next = 0; // the chunk whose MMA 1 is issued next
+            auto issue_m1 = [&](bool block) {
+                if (!m1_ready(m1_next, block))
+                    return false;
+                phv ^= 1u;
+                tc_fence_after();
+                mma1(m1_next++);
+                return true;
+            };
+            bool good = all(waitp(bar_u, phu)); // phase 0 of U: the initial state
             if (good)
-                mma1(0);
+                issue_m1(false);
             for (int c = 0; good && c < nchunks; ++c) {
                 const uint32_t dXO = tmem + ((c & 1) ? kColX1 : kColX0);
                 const uint32_t dU = tmem + ((c & 1) ? kColU1 : kColU0);
@@ -772,6 +840,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     mma_tf32_ts_if(dXO, tmem + kColS + 8 * s, dKQ + ks, id2, s > 0, is);
                 }
                 mma_commit_if(bar_m2, is);
+                if (m1_next == c && !issue_m1(true)) {
+                    good = false;
+                    break;
+                }
                 // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
                 good = waitp(bar_m2, ph2);
                 good = waitq(bar_pT(c), (c >> 2) & 1) && good; // -T diag(b gamma) of chunk c
@@ -792,13 +864,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 mma_commit_if(bar_m2b(c), is);
                 // ---- MMA 1 of the next chunk beside the U pass, if its inputs are in
                 //      (its U buffer was last read by MMA 3 of chunk c - 1)
-                bool m1_issued = false;
-                if (c + 1 < nchunks && m1_ready(c + 1, false)) {
-                    phv ^= 1u;
-                    tc_fence_after();
-                    mma1(c + 1);
-                    m1_issued = true;
-                }
+                if (m1_next == c + 1 && c + 1 < nchunks)
+                    issue_m1(false);
                 // ---- MMA 3: O^T += U^T P^T, S += (U diag(gamma_C/gamma))^T K (K MN-major)
                 good = waitp(bar_u, phu);
                 good = (summary || waitp(bar_pP, phP)) && good;
@@ -821,14 +888,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                         mma_tf32_ts_if(tmem + kColS, dXO + 8 * s, dK + s * 64, idS, 1, is);
                 }
                 mma_commit_if(bar_m3, is);
-                if (c + 1 < nchunks && !m1_issued) {
-                    good = m1_ready(c + 1, true);
-                    phv ^= 1u;
-                    if (!good)
-                        break;
-                    tc_fence_after();
-                    mma1(c + 1);
-                }
+                if (m1_next == c + 1 && c + 1 < nchunks)
+                    issue_m1(false);
             }
             ok = good;
             // let every MMA issued so far finish before the CTA releases TMEM
@@ -843,15 +904,22 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
     } else {
         // ==================================================== TMA issue
         if (lane == 0 && nchunks > 0) {
-            // loads armed on v, q, k, kmaj, tb (parity 0, 1), qk, z
-            uint32_t cnt[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-            const uint32_t lbar[8] = {bar_v, bar_q, bar_k, bar_kmaj, bar_tb(0), bar_tb(1), bar_qk, bar_z};
+            // loads armed on v, q, k, kmaj, tb (parity 0, 1), qk, z, vx
+            uint32_t cnt[9] = {0, 0, 0, 0, 0, 0, 0, 0, 0};
+            const uint32_t bar_vx = smem_u32(&sm.bar_vx), bar_vxf = smem_u32(&sm.bar_vxf);
+            const uint32_t lbar[9] = {bar_v,  bar_q,  bar_k, bar_kmaj, bar_tb(0),
+                                      bar_tb(1), bar_qk, bar_z, bar_vx};
             // nb 32-column boxes of 64 rows at x0 + 32 b, row t0, block b landing at dst + b * bstride
+            // (each load also asks L2 for the next chunk's boxes of the same stream, so
+            // that a long sequence's loads, which miss L2, do not wait on DRAM)
             auto tile = [&](int which, float *dst, const CUtensorMap *m, int x0, int64_t t0, int nb,
                             int bstride) {
                 mbar_arrive_expect_tx(lbar[which], (uint32_t)(nb * kC * 32 * sizeof(float)));
                 for (int b = 0; b < nb; ++b)
                     tma_load_2d(smem_u32(dst + b * bstride), m, x0 + 32 * b, (int)t0, lbar[which]);
+                if (t0 + kC < end)
+                    for (int b = 0; b < nb; ++b)
+                        tma_prefetch_2d(m, x0 + 32 * b, (int)(t0 + kC));
                 ++cnt[which];
             };
             auto t_of = [&](int c) { return start + (int64_t)c * kC; };
@@ -863,6 +931,10 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 mbar_arrive_expect_tx(bar_qk, (uint32_t)(kTriFloats * sizeof(float)));
                 tma_load_2d(smem_u32(sm.P), &maps.kq, xkk, (int)t_of(c), bar_qk);
                 tma_load_2d(smem_u32(sm.P + 2048), &maps.kq32, xkk + 32, (int)(t_of(c) + 32), bar_qk);
+                if (c + 1 < nchunks) {
+                    tma_prefetch_2d(&maps.kq, xkk, (int)t_of(c + 1));
+                    tma_prefetch_2d(&maps.kq32, xkk + 32, (int)(t_of(c + 1) + 32));
+                }
                 ++cnt[6];
             };
             // T diag(beta) of chunk c: one box of 96 rows (the triangular tile)
@@ -878,12 +950,26 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 if (kZTile && !summary) {
                     mbar_arrive_expect_tx(bar_z, (uint32_t)(kC * kD * sizeof(T)));
                     tma_load_2d(smem_u32(sm.Z), &maps.z, h * kD, (int)t_of(c), bar_z);
+                    if (c + 1 < nchunks)
+                        tma_prefetch_2d(&maps.z, h * kD, (int)t_of(c + 1));
                     ++cnt[7];
                 }
             };
+            // the pre-conv v rows t0 - 3 .. t0 + 63 of a chunk (16-bit activations;
+            // rows before the first token read as zero and are not used)
+            auto vxtile = [&](int c) {
+                mbar_arrive_expect_tx(bar_vx, (uint32_t)((kC + 3) * kD * sizeof(T)));
+                tma_load_2d(smem_u32(sm.Vx), &maps.vx, 2 * p.Hk * kD + h * kD, (int)(t_of(c) - 3), bar_vx);
+                if (c + 1 < nchunks)
+                    tma_prefetch_2d(&maps.vx, 2 * p.Hk * kD + h * kD, (int)(t_of(c + 1) - 3));
+                ++cnt[8];
+            };
             constexpr int kBlkV = kC * 32, kBlkQ = 2 * kC * 32;
             tbtile(0);
-            tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
+            if (kVConv)
+                vxtile(0);
+            else
+                tile(0, sm.V, &maps.v, xv, t_of(0), 4, kBlkV);
             tile(3, sm.KQ, &maps.kmaj, xq, t_of(0), 4, kBlkQ);        // rows 0..63 of KQ
             if (!summary)
                 tile(1, sm.KQ + kC * 32, &maps.q, xq, t_of(0), 4, kBlkQ); // rows 64..127
@@ -893,10 +979,23 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             if (nchunks > 1)
                 tbtile(1);
             // six event streams, each served in chunk order as it completes
-            int ib = 0, i1 = 0, i2 = 0, i3 = 0, iz = kZTile && !summary ? 0 : nchunks;
+            // Every stream polls a barrier whose next phase cannot complete before
+            // the reload it triggers: a parity test cannot then miss a phase.  (MMA 1
+            // completions are polled only where the TMA warp feeds V; with the v conv
+            // on the prep team two MMA 1 phases can complete between two polls.)
+            int ib = 0, i1 = kVConv ? nchunks : 0, i2 = 0, i3 = 0, iz = kZTile && !summary ? 0 : nchunks;
+            int ix = kVConv ? 0 : nchunks;
             long long t_last = clock64();
-            while (ib < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks) {
+            while (ib < nchunks || i1 < nchunks || i2 < nchunks || i3 < nchunks || iz < nchunks ||
+                   ix < nchunks) {
                 bool prog = false;
+                // the prep team has convolved chunk ix from the staged rows
+                if (ix < nchunks && mbar_test_wait(bar_vxf, ix & 1)) {
+                    if (ix + 1 < nchunks)
+                        vxtile(ix + 1);
+                    ++ix;
+                    prog = true;
+                }
                 // the epilogue of chunk iz has released the z tile
                 if (iz < nchunks && mbar_test_wait(bar_zf, iz & 1)) {
                     if (iz + 1 < nchunks)
@@ -904,16 +1003,17 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     ++iz;
                     prog = true;
                 }
-                // MMA 1 (seen below, i1 > ib) and the prep team (its gates-and-Tg
-                // arrival) have read T diag(beta) of chunk ib: its slot takes chunk ib + 2
-                if (ib < nchunks && i1 > ib && mbar_test_wait(bar_pT(ib), (ib >> 2) & 1)) {
+                // MMA 2b of chunk ib is done, so MMA 1 (issued before it) and the prep
+                // team (whose -T diag(beta gamma) MMA 2b waited for) have read T diag(beta)
+                // of chunk ib: its slot takes chunk ib + 2
+                if (ib < nchunks && mbar_test_wait(bar_m2b(ib), (ib >> 1) & 1)) {
                     if (ib + 2 < nchunks)
                         tbtile(ib + 2);
                     ++ib;
                     prog = true;
                 }
                 if (i1 < nchunks && mbar_test_wait(bar_m1, i1 & 1)) { // V is free
-                    if (i1 + 1 < nchunks)
+                    if (i1 + 1 < nchunks && !kVConv)
                         tile(0, sm.V, &maps.v, xv, t_of(i1 + 1), 4, kBlkV);
                     ++i1;
                     prog = true;
@@ -946,7 +1046,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             // every armed load lands before the CTA exits
 #pragma unroll
-            for (int b = 0; b < 8; ++b)
+            for (int b = 0; b < 9; ++b)
                 if (cnt[b] > 0)
                     mbar_wait_bounded(lbar[b], (cnt[b] - 1) & 1, kWaitLimit);
             if (!ok)
@@ -1067,9 +1167,13 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
         const uint64_t N = (uint64_t)p.N, F = sizeof(float);
         const uint64_t qkw = 2ull * p.Hk * kD, kqw = (uint64_t)p.Hk * kC;
         const uint64_t tb_rows = (uint64_t)((p.N + kC - 1) / kC + p.batch) * p.Hv * 96;
+        const uint64_t Cd = (uint64_t)(2 * p.Hk + p.Hv) * kD;
         const bool okm =
-            encode_2d(&maps.v, p.ws_v, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * F, 32, kC,
-                      CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
+            (sizeof(T) == 2
+                 ? encode_2d(&maps.vx, p.qkv, Cd, N, Cd * sizeof(T), kD, kC + 3, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_DATA_TYPE_BFLOAT16)
+                 : encode_2d(&maps.v, p.ws_v, (uint64_t)p.Hv * kD, N, (uint64_t)p.Hv * kD * F, 32, kC,
+                             CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B)) &&
             encode_2d(&maps.k, (const float *)p.ws_qk + (size_t)p.Hk * kD, (uint64_t)p.Hk * kD, N,
                       qkw * F, 32, kC, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B) &&
             encode_2d(&maps.q, p.ws_qk, (uint64_t)p.Hk * kD, N, qkw * F, 32, kC,
@@ -1114,6 +1218,11 @@ size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * kC * size
 // sequence adds at most one partial chunk to the N / 64 full ones.
 size_t tb_workspace_bytes(int Hv, int64_t N, int batch) {
     return (size_t)((N + kC - 1) / kC + batch) * Hv * 96 * 32 * sizeof(float);
+}
+
+// Gate records: one per (chunk, value head).
+size_t gt_workspace_bytes(int Hv, int64_t N, int batch) {
+    return (size_t)((N + kC - 1) / kC + batch) * Hv * kGateRec * sizeof(float);
 }
 
 // K K^T triangular tiles: one per (chunk, q/k head).

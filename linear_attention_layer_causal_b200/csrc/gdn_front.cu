@@ -302,6 +302,16 @@ tri_kernel(PrefillArgs p) {
         g[1] += __shfl_sync(0xffffffffu, g[0], 31);
         G[tt] = g[0]; G[tt + 32] = g[1];
         Be[tt] = be[0]; Be[tt + 32] = be[1];
+        // the chunk's gate record for the chunk kernel: G, gamma_C / gamma =
+        // e^{G_C - G} and gamma = e^G (fast exponential) of every row
+        const float Glast = __shfl_sync(0xffffffffu, g[1], 31);
+        float *rec = p.ws_gt + ((size_t)ci * p.Hv + h) * kGateRec;
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            rec[tt + 32 * q] = g[q];
+            rec[kC + tt + 32 * q] = expf(Glast - g[q]);
+            rec[2 * kC + tt + 32 * q] = __expf(g[q]);
+        }
     }
     group_sync(1 + gi, 64);
     // A[r][s] = beta_r e^{G_r - G_s} KK[r][s] (KK is 0 for s >= r; the clamp keeps

@@ -34,6 +34,7 @@ struct PrefillArgs {
     void *ws_kq;             // [N, Hk, 64] float32: chunk Q K^T rows (chunked path)
     void *ws_kk;             // [chunks, Hk, 3072] float32: K K^T triangular tiles (chunked path)
     void *ws_tb;             // [chunks, Hv, 96, 32] float32: T diag(beta) tiles (chunked path)
+    float *ws_gt;            // [chunks, Hv, 3, 64] float32: per chunk G, gamma_C / gamma, gamma (chunked path)
     int32_t *ws_offs;        // [batch + 1] chunk offsets per sequence (chunked path)
     // sequence split of the chunked path (segments > 1)
     int segments = 1;        // P: segments per sequence
@@ -103,7 +104,7 @@ inline cudaError_t record_if(cudaEvent_t ev, cudaStream_t s) {
 size_t prefill_workspace_bytes(const gdn_config *c, int64_t N, int batch);
 // The chunk kernel convolves v itself from the 16-bit pre-conv rows; the
 // front end then writes no convolved v.
-inline bool v_conv_in_chunk(bool chunked, bool bf16) { return false && chunked && bf16; }
+inline bool v_conv_in_chunk(bool chunked, bool bf16) { return chunked && bf16; }
 // Segments per sequence a chunked prefill of this config and size runs with
 // (1 for the token-serial path and for calls without tokens).
 int prefill_segments(const gdn_config *c, int batch, int64_t N);
@@ -124,6 +125,8 @@ cudaError_t launch_chunk_prefill(const PrefillArgs &p, cudaStream_t s);
 size_t kq_workspace_bytes(int Hk, int64_t N);
 size_t tb_workspace_bytes(int Hv, int64_t N, int batch);
 size_t kk_workspace_bytes(int Hk, int64_t N, int batch);
+size_t gt_workspace_bytes(int Hv, int64_t N, int batch);
+constexpr int kGateRec = 192; // floats of one (chunk, value head) gate record: G, gamma_C / gamma, gamma
 cudaError_t launch_decode(const DecodeArgs &p, cudaStream_t s);
 cudaError_t launch_decode_multi(const DecodeArgs &p, int mode, cudaStream_t s);
 cudaError_t launch_kda_prefill(const PrefillArgs &p, cudaStream_t s);

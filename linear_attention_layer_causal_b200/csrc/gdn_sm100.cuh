@@ -71,6 +71,14 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int 
                  : "memory");
 }
 
+// L2 prefetch of the box at (x, y) of `tmap`: no shared memory, no completion;
+// a later load of the same box then reads L2.  x times the element size a
+// multiple of 16 bytes; parts of the box outside the tensor are skipped.
+__device__ __forceinline__ void tma_prefetch_2d(const void *tmap, int x, int y) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(tmap), "r"(x), "r"(y)
+                 : "memory");
+}
+
 // 2-D tiled TMA store of the shared-memory tile at `src` to the box at (x, y)
 // of `tmap` (bulk-group completion).  x, y >= 0; x times the element size a
 // multiple of 16 bytes.  Elements outside the tensor are not written.

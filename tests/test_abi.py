@@ -46,13 +46,20 @@ QWEN38 = gdn.Config(16, 128, 128)
 
 def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
-    # 256-byte header (status word), float32 normalised q|k and convolved v, and
-    # for head_dim 128 the chunks' Q K^T rows [N, H_k, 64], K K^T tiles
-    # [N / 64 + batch chunks, H_k, 3072], T diag(beta) tiles [chunks, H_v, 96, 32]
-    # and the chunk offsets [batch + 1]; regions rounded to 256 B
-    tile = 128 * 96 * 32 * 4 + 16 * 3072 * 4  # one chunk's tiles, all heads
-    assert n == (256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4 + 4096 * 16 * 64 * 4 +
-                 (64 + 1) * tile + 256)
+    # 256-byte header (status word), float32 normalised q|k and, on the chunked
+    # path, the chunks' Q K^T rows [N, H_k, 64], K K^T tiles [N / 64 + batch
+    # chunks, H_k, 3072], T diag(beta) tiles [chunks, H_v, 96, 32], gate records
+    # [chunks, H_v, 3, 64] and the chunk offsets [batch + 1]; regions rounded to
+    # 256 B.  With 16-bit activations the chunk kernel convolves v itself: no
+    # float32 v
+    tile = 128 * 96 * 32 * 4 + 16 * 3072 * 4 + 128 * 192 * 4  # one chunk's tiles, all heads
+    assert n == (256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 16 * 64 * 4 + (64 + 1) * tile + 256)
+    # float32 activations add the convolved v [N, H_v * 128]
+    assert gdn.prefill_workspace_size(gdn.Config(16, 128, 128, act_dtype="f32"), 1, 4096) == \
+        n + 4096 * 128 * 128 * 4
+    # the token-serial path: header, q|k and v only
+    assert gdn.prefill_workspace_size(gdn.Config(16, 128, 128, algo="serial"), 1, 4096) == \
+        256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 128 * 128 * 4
     # 99 more sequences: at most 99 more (partial) chunks, and 512 bytes of offsets
     assert gdn.prefill_workspace_size(QWEN38, 100, 4096) == n + 99 * tile + 256
     assert gdn.prefill_workspace_size(QWEN38, 0, 0) == 0
@@ -224,7 +231,9 @@ def test_noalloc_rejects_oversized_calls_on_the_host():
     cfg = gdn.Config(16, 128, 128)
     P = 1 << 20
     par = gdn._Params(P, P + 256, P + 512, P + 768)
-    args = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, 745, None, None, P * 7, None, None, None, None]
+    n_big = 2000
+    assert gdn.prefill_workspace_size(cfg, 1, n_big) > gdn.NOALLOC_SCRATCH_BYTES
+    args = [P * 2, P * 3, P * 4, P * 5, P * 6, 1, n_big, None, None, P * 7, None, None, None, None]
     assert L.gdn_prefill_noalloc(ctypes.byref(cfg._c()), ctypes.byref(par), *args) == \
         gdn.GDN_ERR_WORKSPACE
     bad = gdn.Config(3, 4, 32)
