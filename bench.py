@@ -230,6 +230,9 @@ def run_ours(args, rank, world, dev, dist):
 
     pk = peaks()
     wl = W.QWEN38_PREFILL
+    if args.seq_len != 4096:
+        import dataclasses
+        wl = dataclasses.replace(wl, seqlens=(args.seq_len,))
     cfg = gdn.Config.of(wl, args.algo)
     inp = W.make_prefill(wl, dev, seed=rank_seed(wl.seed, rank))
     P = [inp[k] for k in ("conv_w", "A_log", "dt_bias", "norm_w")]
@@ -555,11 +558,15 @@ def main():
     ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
                     help="run only one part (for profiling small cases)")
     ap.add_argument("--decode-batch", type=int, default=256)
+    ap.add_argument("--seq-len", type=int, default=4096,
+                    help="with --only prefill: the prefill sequence length (profiling cases)")
     ap.add_argument("--algo", default="auto", choices=["auto", "chunked", "serial"],
                     help="prefill algorithm (auto = tensor-core chunks at head dim 128)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.seq_len != 4096 and args.only != "prefill":
+        ap.error("--seq-len applies to --only prefill")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

@@ -677,17 +677,14 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         };
         uint32_t phqk = 0;
         float4 gv = load_gt(0);
-        if constexpr (kVConv) {
-            if (nchunks > 0 && !vconv(0))
-                ok = false;
-        }
-        for (int c = 0; ok && c < nchunks; ++c) {
+        // ---- the gate record of chunk c into slot c mod 4, then -T diag(beta gamma)
+        //      = -(T diag beta) diag(gamma) into the chunk's parity slot once MMA 2b of
+        //      chunk c - 2 has read it
+        auto gates_tg = [&](int c) {
             const int sl = c & 3;
             put_gt(gv, sl);
             gv = load_gt(c + 1);
             group_sync(kBarT, kTeam); // the gates are in
-            // ---- -T diag(beta gamma) = -(T diag beta) diag(gamma) into this chunk's
-            //      parity slot once MMA 2b of chunk c - 2 has read it
             bool good = waitq(bar_tb(c), (c >> 1) & 1); // T diag(beta) of chunk c landed
             good = (c < 2 || waitq(bar_m2b(c), ((c - 2) >> 1) & 1)) && good;
             if (good) {
@@ -706,16 +703,27 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
             }
             fence_proxy_async_smem();
-            if (group_sync_or(kBarT, kTeam, !good || *abort_flag)) {
-                ok = false;
-                break;
-            }
+            if (group_sync_or(kBarT, kTeam, !good || *abort_flag))
+                return false;
             if (tt == 0)
                 mbar_arrive(bar_pT(c)); // gates and -T diag(beta gamma) of chunk c
+            return true;
+        };
+        // Order: gates and -T diag(beta gamma) of chunk c + 1, then its V, as soon as
+        // P of chunk c is out.  The state group's S *= gamma_C of a chunk needs only
+        // its gates, so the v conv never delays it; MMA 1 of chunk c + 1 waits for V
+        // only at MMA 2b, a whole MMA 2 later.
+        if (nchunks > 0) {
+            ok = gates_tg(0);
+            if constexpr (kVConv)
+                ok = ok && vconv(0);
+        }
+        for (int c = 0; ok && c < nchunks; ++c) {
+            const int sl = c & 3;
             // ---- P[r][s] = e^{G_r - G_s} QK[r][s] in place, tf32 (the Q K^T rows are
             //      0 for s > r; the clamp keeps the unused upper triangle finite); the
             //      summary pass has no O and no P
-            good = summary || waitp(bar_qk, phqk);
+            bool good = summary || waitp(bar_qk, phqk);
             if (good && !summary) {
                 float4 x[6];
 #pragma unroll
@@ -739,10 +747,16 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             }
             if (tt == 0 && !summary)
                 mbar_arrive(bar_pP); // P of chunk c
-            if constexpr (kVConv) { // V of the next chunk
-                if (c + 1 < nchunks && !vconv(c + 1)) {
+            if (c + 1 < nchunks) {
+                if (!gates_tg(c + 1)) {
                     ok = false;
                     break;
+                }
+                if constexpr (kVConv) {
+                    if (!vconv(c + 1)) {
+                        ok = false;
+                        break;
+                    }
                 }
             }
         }
