@@ -141,6 +141,11 @@ gdn_status validate_prefill(const gdn_config *cfg, const gdn_params *params, con
         !aligned16(o_raw) || !elem_aligned(a, bf16) || !elem_aligned(b, bf16) ||
         (reinterpret_cast<uintptr_t>(cu_seqlens) & 3u))
         return GDN_ERR_INVALID_ARG;
+    // the chunked path addresses its per-(chunk, value head) tiles by 32-bit TMA
+    // row coordinates: 192 rows per (chunk, value head)
+    const bool chunked = cfg->head_dim == 128 && cfg->algo != GDN_ALGO_SERIAL;
+    if (chunked && ((total_tokens + 63) / 64 + (int64_t)batch) * cfg->num_v_heads * 192 > INT32_MAX)
+        return GDN_ERR_UNSUPPORTED;
     *need = prefill_workspace_bytes(cfg, total_tokens, batch);
     return GDN_OK;
 }

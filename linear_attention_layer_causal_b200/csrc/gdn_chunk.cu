@@ -152,8 +152,8 @@ struct __align__(1024) ChunkSmem {
     // channels) written by the prep team, K-major (16-bit activations)
     float V[kC * kD];
     float K[kC * kD];          // B of MMA 3 (MN-major): lands as K, becomes diag(gamma_C/gamma) K
-    float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta) (from the front kernel, by TMA), by chunk parity
-    float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma), by chunk parity
+    float Tb[2][kTriFloats];   // B of MMA 1: T diag(beta) (from the inverse kernel, by TMA), by chunk parity
+    float Tg[2][kTriFloats];   // B of MMA 2b: -T diag(beta gamma) (the same), by chunk parity
     float P[kTriFloats];       // B of MMA 3: lands as Q K^T rows, becomes P
     // z rows of the chunk (16-bit activations).  Once the state group has formed
     // the gate from it, it stages the chunk's y rows for one TMA store.
@@ -587,9 +587,8 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             *abort_flag = 1;
     } else if (warp < (kSG + kTeam) / 32) {
         // ==================================================== prep team
-        // Per chunk: the gate record; -T diag(beta gamma) from the T diag(beta) tile that
-        // the front kernel formed (the B operands of MMA 2b and MMA 1); P from the
-        // Q K^T rows.  All tf32, in the triangular-tile layout.
+        // Per chunk: the gate record; P from the Q K^T rows (tf32, in the
+        // triangular-tile layout); with 16-bit activations the v conv.
         const int tt = tid - kSG;
         const TriThread tr(tt);
         // The gate record of chunk c, formed by the inverse kernel: G, gamma_C /
@@ -677,46 +676,26 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
         };
         uint32_t phqk = 0;
         float4 gv = load_gt(0);
-        // ---- the gate record of chunk c into slot c mod 4, then -T diag(beta gamma)
-        //      = -(T diag beta) diag(gamma) into the chunk's parity slot once MMA 2b of
-        //      chunk c - 2 has read it
-        auto gates_tg = [&](int c) {
-            const int sl = c & 3;
-            put_gt(gv, sl);
+        // ---- the gate record of chunk c into slot c mod 4 (the state group's
+        //      S *= gamma_C, O *= gamma and U pass and P read it).  Slot c mod 4 last
+        //      held chunk c - 4, whose readers are all done: this runs after P of
+        //      chunk c - 1, which waited for MMA 3 of chunk c - 2 and so for the
+        //      state group's U pass of that chunk.
+        auto gates = [&](int c) {
+            put_gt(gv, c & 3);
             gv = load_gt(c + 1);
             group_sync(kBarT, kTeam); // the gates are in
-            bool good = waitq(bar_tb(c), (c >> 1) & 1); // T diag(beta) of chunk c landed
-            good = (c < 2 || waitq(bar_m2b(c), ((c - 2) >> 1) & 1)) && good;
-            if (good) {
-                const float *tb = sm.Tb[c & 1];
-                float *tg = sm.Tg[c & 1];
-                float4 t4[6];
-#pragma unroll
-                for (int jj = 0; jj < 6; ++jj)
-                    t4[jj] = *reinterpret_cast<const float4 *>(tb + tr.o(jj));
-#pragma unroll
-                for (int jj = 0; jj < 6; ++jj) {
-                    const float4 g4 = *reinterpret_cast<const float4 *>(&sm.gam[sl][tr.c(jj)]);
-                    *reinterpret_cast<float4 *>(tg + tr.o(jj)) =
-                        tf32_rna(make_float4(-t4[jj].x * g4.x, -t4[jj].y * g4.y, -t4[jj].z * g4.z,
-                                             -t4[jj].w * g4.w));
-                }
-            }
-            fence_proxy_async_smem();
-            if (group_sync_or(kBarT, kTeam, !good || *abort_flag))
-                return false;
             if (tt == 0)
-                mbar_arrive(bar_pT(c)); // gates and -T diag(beta gamma) of chunk c
-            return true;
+                mbar_arrive(bar_pT(c)); // gates of chunk c
         };
-        // Order: gates and -T diag(beta gamma) of chunk c + 1, then its V, as soon as
-        // P of chunk c is out.  The state group's S *= gamma_C of a chunk needs only
-        // its gates, so the v conv never delays it; MMA 1 of chunk c + 1 waits for V
-        // only at MMA 2b, a whole MMA 2 later.
+        // Order: the gates of chunk c + 1, then its V, as soon as P of chunk c is
+        // out.  The state group's S *= gamma_C of a chunk needs only its gates, so
+        // the v conv never delays it; MMA 1 of chunk c + 1 waits for V only at
+        // MMA 2b, a whole MMA 2 later.
         if (nchunks > 0) {
-            ok = gates_tg(0);
+            gates(0);
             if constexpr (kVConv)
-                ok = ok && vconv(0);
+                ok = vconv(0);
         }
         for (int c = 0; ok && c < nchunks; ++c) {
             const int sl = c & 3;
@@ -748,10 +727,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
             if (tt == 0 && !summary)
                 mbar_arrive(bar_pP); // P of chunk c
             if (c + 1 < nchunks) {
-                if (!gates_tg(c + 1)) {
-                    ok = false;
-                    break;
-                }
+                gates(c + 1);
                 if constexpr (kVConv) {
                     if (!vconv(c + 1)) {
                         ok = false;
@@ -858,9 +834,9 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     good = false;
                     break;
                 }
-                // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM)
+                // ---- MMA 2b: U^T = U~^T + X^T (-T diag(b gamma))^T (A = X^T in TMEM);
+                //      its B tile landed with T diag(beta), which MMA 1 waited for
                 good = waitp(bar_m2, ph2);
-                good = waitq(bar_pT(c), (c >> 2) & 1) && good; // -T diag(b gamma) of chunk c
                 if (!all(good))
                     break;
                 tc_fence_after();
@@ -951,12 +927,14 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                 }
                 ++cnt[6];
             };
-            // T diag(beta) of chunk c: one box of 96 rows (the triangular tile)
+            // T diag(beta) and -T diag(beta gamma) of chunk c: one box of 96 rows each
+            // (triangular tiles), one barrier
             const int chunk0 = __ldg(p.ws_offs + n) + cb; // global index of this segment's first chunk
             auto tbtile = [&](int c) {
-                mbar_arrive_expect_tx(bar_tb(c), (uint32_t)(kTriFloats * sizeof(float)));
-                tma_load_2d(smem_u32(sm.Tb[c & 1]), &maps.tb, 0,
-                            (int)(((int64_t)(chunk0 + c) * p.Hv + h) * 96), bar_tb(c));
+                mbar_arrive_expect_tx(bar_tb(c), (uint32_t)(2 * kTriFloats * sizeof(float)));
+                const int row = (int)(((int64_t)(chunk0 + c) * p.Hv + h) * 2 * 96);
+                tma_load_2d(smem_u32(sm.Tb[c & 1]), &maps.tb, 0, row, bar_tb(c));
+                tma_load_2d(smem_u32(sm.Tg[c & 1]), &maps.tb, 0, row + 96, bar_tb(c));
                 ++cnt[4 + (c & 1)];
             };
             // the z rows of a chunk: one 128-column box of 64 rows
@@ -1180,7 +1158,7 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
     if (p.N > 0) {
         const uint64_t N = (uint64_t)p.N, F = sizeof(float);
         const uint64_t qkw = 2ull * p.Hk * kD, kqw = (uint64_t)p.Hk * kC;
-        const uint64_t tb_rows = (uint64_t)((p.N + kC - 1) / kC + p.batch) * p.Hv * 96;
+        const uint64_t tb_rows = (uint64_t)((p.N + kC - 1) / kC + p.batch) * p.Hv * 2 * 96;
         const uint64_t Cd = (uint64_t)(2 * p.Hk + p.Hv) * kD;
         const bool okm =
             (sizeof(T) == 2
@@ -1228,10 +1206,11 @@ template <typename T> cudaError_t launch_chunk_t(const PrefillArgs &p, cudaStrea
 
 size_t kq_workspace_bytes(int Hk, int64_t N) { return (size_t)N * Hk * kC * sizeof(float); }
 
-// T diag(beta) tiles: one per (chunk, value head), 96 rows of 32 floats; every
-// sequence adds at most one partial chunk to the N / 64 full ones.
+// T diag(beta) and -T diag(beta gamma) tiles: two per (chunk, value head), 96
+// rows of 32 floats each; every sequence adds at most one partial chunk to the
+// N / 64 full ones.
 size_t tb_workspace_bytes(int Hv, int64_t N, int batch) {
-    return (size_t)((N + kC - 1) / kC + batch) * Hv * 96 * 32 * sizeof(float);
+    return (size_t)((N + kC - 1) / kC + batch) * Hv * 2 * 96 * 32 * sizeof(float);
 }
 
 // Gate records: one per (chunk, value head).

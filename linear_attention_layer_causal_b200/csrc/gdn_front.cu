@@ -334,22 +334,31 @@ tri_kernel(PrefillArgs p) {
     group_sync(1 + gi, 64);
     if (!live)
         return;
-    // column c = tt of T, then T diag(beta) as 96 rows of 32 floats: row r of
-    // column block 0, then row r of block 1 at row r + 32 (a TMA load with
-    // 128-byte swizzle turns them back into the triangular tile)
+    // column c = tt of T, then T diag(beta) and -T diag(beta gamma) (the B tiles
+    // of the chunk kernel's MMA 1 and MMA 2b), each as 96 rows of 32 floats: row r
+    // of column block 0, then row r of block 1 at row r + 32 (a TMA load with
+    // 128-byte swizzle turns them back into the triangular tile).  gamma = e^G
+    // by the same fast exponential as the gate record's.
     float x[kC];
-    float *dst = (float *)p.ws_tb + ((size_t)ci * p.Hv + h) * (96 * 32);
-    const float bc = Be[tt];
+    float *dst = (float *)p.ws_tb + ((size_t)ci * p.Hv + h) * (2 * 96 * 32);
+    float *dsg = dst + 96 * 32;
+    const float bc = Be[tt], gc = __expf(G[tt]);
     if (tt < 32) {
         tri_column<0>(A, tt, x);
 #pragma unroll
-        for (int r = 0; r < kC; ++r)
-            dst[r * 32 + tt] = tf32_rna(x[r] * bc);
+        for (int r = 0; r < kC; ++r) {
+            const float tb = tf32_rna(x[r] * bc);
+            dst[r * 32 + tt] = tb;
+            dsg[r * 32 + tt] = tf32_rna(-tb * gc);
+        }
     } else {
         tri_column<32>(A, tt, x);
 #pragma unroll
-        for (int r = 32; r < kC; ++r)
-            dst[(r + 32) * 32 + (tt - 32)] = tf32_rna(x[r] * bc);
+        for (int r = 32; r < kC; ++r) {
+            const float tb = tf32_rna(x[r] * bc);
+            dst[(r + 32) * 32 + (tt - 32)] = tb;
+            dsg[(r + 32) * 32 + (tt - 32)] = tf32_rna(-tb * gc);
+        }
     }
 }
 

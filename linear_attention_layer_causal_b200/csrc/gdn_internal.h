@@ -33,7 +33,7 @@ struct PrefillArgs {
     void *ws_v;              // [N, Hv*D]   float32: convolved v (nullptr where the chunk kernel convolves v)
     void *ws_kq;             // [N, Hk, 64] float32: chunk Q K^T rows (chunked path)
     void *ws_kk;             // [chunks, Hk, 3072] float32: K K^T triangular tiles (chunked path)
-    void *ws_tb;             // [chunks, Hv, 96, 32] float32: T diag(beta) tiles (chunked path)
+    void *ws_tb;             // [chunks, Hv, 2, 96, 32] float32: T diag(beta), -T diag(beta gamma) tiles (chunked path)
     float *ws_gt;            // [chunks, Hv, 3, 64] float32: per chunk G, gamma_C / gamma, gamma (chunked path)
     int32_t *ws_offs;        // [batch + 1] chunk offsets per sequence (chunked path)
     // sequence split of the chunked path (segments > 1)

@@ -48,11 +48,11 @@ def test_workspace_size_arithmetic():
     n = gdn.prefill_workspace_size(QWEN38, 1, 4096)
     # 256-byte header (status word), float32 normalised q|k and, on the chunked
     # path, the chunks' Q K^T rows [N, H_k, 64], K K^T tiles [N / 64 + batch
-    # chunks, H_k, 3072], T diag(beta) tiles [chunks, H_v, 96, 32], gate records
-    # [chunks, H_v, 3, 64] and the chunk offsets [batch + 1]; regions rounded to
-    # 256 B.  With 16-bit activations the chunk kernel convolves v itself: no
-    # float32 v
-    tile = 128 * 96 * 32 * 4 + 16 * 3072 * 4 + 128 * 192 * 4  # one chunk's tiles, all heads
+    # chunks, H_k, 3072], T diag(beta) and -T diag(beta gamma) tiles [chunks, H_v,
+    # 2, 96, 32], gate records [chunks, H_v, 3, 64] and the chunk offsets [batch +
+    # 1]; regions rounded to 256 B.  With 16-bit activations the chunk kernel
+    # convolves v itself: no float32 v
+    tile = 2 * 128 * 96 * 32 * 4 + 16 * 3072 * 4 + 128 * 192 * 4  # one chunk's tiles, all heads
     assert n == (256 + 4096 * 2 * 16 * 128 * 4 + 4096 * 16 * 64 * 4 + (64 + 1) * tile + 256)
     # float32 activations add the convolved v [N, H_v * 128]
     assert gdn.prefill_workspace_size(gdn.Config(16, 128, 128, act_dtype="f32"), 1, 4096) == \
@@ -172,6 +172,10 @@ no_gpu = pytest.mark.skipif(
     (dict(params=gdn._Params(None, 256, 512, 768)), gdn.GDN_ERR_INVALID_ARG),
     (dict(params=gdn._Params(8, 256, 512, 768)), gdn.GDN_ERR_INVALID_ARG),
     (dict(cfg=gdn.Config(2, 4, 48)), gdn.GDN_ERR_UNSUPPORTED),
+    # the chunked path's tile rows (192 per chunk and value head) exceed 32-bit
+    # TMA coordinates; the token-serial path has no such tiles
+    (dict(cfg=gdn.Config(16, 128, 128), N=6_000_000), gdn.GDN_ERR_UNSUPPORTED),
+    (dict(cfg=gdn.Config(16, 128, 128, algo="serial"), N=6_000_000), gdn.GDN_ERR_WORKSPACE),
 ])
 def test_prefill_argument_errors(over, code):
     assert _fake_call(**over) == code
