@@ -1033,7 +1033,7 @@ chunk_prefill_kernel(PrefillArgs p, const __grid_constant__ ChunkMaps maps) {
                     ok = false;
                     break;
                 } else {
-                    __nanosleep(64); // leave the issue slots to the working warps
+                    __nanosleep(16); // leave the issue slots to the working warps
                 }
             }
             // every armed load lands before the CTA exits

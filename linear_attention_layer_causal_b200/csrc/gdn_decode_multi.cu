@@ -30,7 +30,7 @@ namespace gdn {
 
 namespace {
 
-constexpr int kMtThreads = 512;
+constexpr int kMtThreads = 256; // two CTAs per SM: one streams the state while the other convolves
 constexpr int kMtWarps = kMtThreads / 32;
 constexpr int kRowUnroll = 2; // rows in flight per lane group
 
@@ -164,8 +164,11 @@ decode_multi_kernel(DecodeArgs p) {
     __syncthreads();
 
     // ---- phase 2: every row of the group's G states through the Kc tokens
-    const int lr = lane / LR;         // row within the warp step
-    const int c0 = (lane % LR) * 16;  // first column of this lane
+    // a row's LR lanes interleave its float4s: lane l8 holds float4s l8, l8 + LR,
+    // l8 + 2 LR, l8 + 3 LR, so that the lanes read k and q from shared memory
+    // without bank conflicts and each load of the state is contiguous
+    const int lr = lane / LR;  // row within the warp step
+    const int l8 = lane % LR;  // lane within the row
     const int R = G * D;
     float *Sg = p.state + ((size_t)n * p.Hv + (size_t)j * G) * D * D;
     for (int base = warp * RPW; base < R; base += kMtWarps * RPW * kRowUnroll) {
@@ -177,7 +180,7 @@ decode_multi_kernel(DecodeArgs p) {
             for (int i = 0; i < 4; ++i) {
                 float4 x4 = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (r < R) {
-                    const float4 *src = reinterpret_cast<const float4 *>(Sg + (size_t)r * D + c0) + i;
+                    const float4 *src = reinterpret_cast<const float4 *>(Sg + (size_t)r * D) + l8 + LR * i;
                     x4 = MODE == kDecodeVerify ? __ldg(src) : __ldcs(src);
                 }
                 s[uu][4 * i] = x4.x; s[uu][4 * i + 1] = x4.y;
@@ -186,8 +189,8 @@ decode_multi_kernel(DecodeArgs p) {
         }
 #pragma unroll 1
         for (int t = 0; t < Kc; ++t) {
-            const float4 *k4 = reinterpret_cast<const float4 *>(ks + t * D + c0);
-            const float4 *q4 = reinterpret_cast<const float4 *>(qs + t * D + c0);
+            const float4 *k4 = reinterpret_cast<const float4 *>(ks + t * D) + l8;
+            const float4 *q4 = reinterpret_cast<const float4 *>(qs + t * D) + l8;
             const float kq = nrm[3 * t + 2];
 #pragma unroll
             for (int uu = 0; uu < kRowUnroll; ++uu) {
@@ -195,13 +198,13 @@ decode_multi_kernel(DecodeArgs p) {
                 float pk = 0.f, pq = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float4 kv = k4[i];
+                    const float4 kv = k4[LR * i];
                     pk = fmaf(s[uu][4 * i], kv.x, pk);
                     pk = fmaf(s[uu][4 * i + 1], kv.y, pk);
                     pk = fmaf(s[uu][4 * i + 2], kv.z, pk);
                     pk = fmaf(s[uu][4 * i + 3], kv.w, pk);
                     if (MODE != kDecodeCommit) {
-                        const float4 qv = q4[i];
+                        const float4 qv = q4[LR * i];
                         pq = fmaf(s[uu][4 * i], qv.x, pq);
                         pq = fmaf(s[uu][4 * i + 1], qv.y, pq);
                         pq = fmaf(s[uu][4 * i + 2], qv.z, pq);
@@ -219,7 +222,7 @@ decode_multi_kernel(DecodeArgs p) {
                 const float u = be * ((r < R ? vs[t * R + r] : 0.f) - al * pk);
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float4 kv = k4[i];
+                    const float4 kv = k4[LR * i];
                     s[uu][4 * i] = fmaf(u, kv.x, al * s[uu][4 * i]);
                     s[uu][4 * i + 1] = fmaf(u, kv.y, al * s[uu][4 * i + 1]);
                     s[uu][4 * i + 2] = fmaf(u, kv.z, al * s[uu][4 * i + 2]);
@@ -236,7 +239,7 @@ decode_multi_kernel(DecodeArgs p) {
                 if (r < R) {
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        __stcs(reinterpret_cast<float4 *>(Sg + (size_t)r * D + c0) + i,
+                        __stcs(reinterpret_cast<float4 *>(Sg + (size_t)r * D) + l8 + LR * i,
                                make_float4(s[uu][4 * i], s[uu][4 * i + 1], s[uu][4 * i + 2],
                                            s[uu][4 * i + 3]));
                 }
