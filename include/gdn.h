@@ -359,7 +359,7 @@ GDN_API gdn_status gdn_kda_decode(const gdn_config *cfg, const gdn_kda_params *p
  *   - Limit: a call whose gdn_prefill_workspace_size exceeds
  *     GDN_NOALLOC_SCRATCH_BYTES returns GDN_ERR_WORKSPACE before any CUDA
  *     call (at the Qwen3.8 layer shape with 16-bit activations, about
- *     47 KiB per token plus 1.7 MiB per sequence: up to 1,344 tokens of one
+ *     72.5 KiB per token plus 3.3 MiB per sequence: up to 832 tokens of one
  *     sequence).
  *   - Set-up: the first call on a device, with that device current, looks up
  *     the array's device address (cudaGetSymbolAddress) and caches it; make
