@@ -309,6 +309,7 @@ def run_ours(args, rank, world, dev, dist):
     decode_k = run_decode_k(args, rank, world, dev, pk, timed, max_over_ranks)
     qwen35 = run_prefill_shape(args, rank, world, dev, pk, timed, max_over_ranks, "qwen35_prefill")
     long_ctx = run_long_context(args, rank, world, dev, pk, timed, max_over_ranks)
+    kda = run_kda(args, rank, world, dev, pk, timed, max_over_ranks)
 
     # ---- end to end through the public API from pinned host buffers.  Every
     # step uploads its inputs, runs the layer and reads back y and the final
@@ -368,7 +369,7 @@ def run_ours(args, rank, world, dev, dist):
                                 "accumulation, FP32 state and CUDA-core math",
                        "l2": "no flush: inputs of one step (~447 MB) exceed the 126 MB L2"},
             "roofline": roof, "decode": decode, "decode_k": decode_k, "qwen35_prefill": qwen35,
-            "long_context": long_ctx,
+            "long_context": long_ctx, "kda": kda,
             "e2e": e2e,
             # chunked (16-bit activations): offsets, conv of q|k, Gram, inverses, chunk kernel
             "gpu_launches": (5 if kname == "chunk_prefill_kernel" else 2) * args.steps,
@@ -513,6 +514,80 @@ def run_long_context(args, rank, world, dev, pk, timed, max_over_ranks):
         out[name] = res
         del inp, y, fs
         torch.cuda.empty_cache()
+    return out
+
+
+def kda_decode_bytes(H, d, B, act_bytes=2, K=4):
+    """HBM bytes of one KDA decode call: state read + write, the token's q|k|v,
+    zdec, gate and b read, y written, conv cache read and written (K-1 rows)."""
+    conv_dim = 3 * H * d
+    per_seq = 2 * 4 * H * d * d + act_bytes * (conv_dim + 3 * H * d + H) + 2 * act_bytes * (K - 1) * conv_dim
+    return per_seq * B
+
+
+# FP32 FMA peak of the CUDA cores (148 SMs x 128 FMA lanes x 2 FLOP x 1.965 GHz),
+# the bound of the token-serial recurrences
+FP32_CUDA_CORE_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_kda(args, rank, world, dev, pk, timed, max_over_ranks):
+    """Kimi Delta Attention at the Kimi K3 layer shape (96 heads of dim 128): a
+    prefill of one 4,096-token sequence (token-serial FP32 recurrence on the CUDA
+    cores) and a decode of 256 sequences (state streamed through registers)."""
+    import torch
+
+    import linear_attention_layer_causal_b200 as gdn
+    from linear_attention_layer_causal_b200 import workloads as W
+    wl = W.KIMI_K3_KDA
+    cfg = gdn.Config.of(wl)
+    H, D = wl.num_v_heads, wl.head_dim
+    inp = W.make_kda_prefill(wl, dev, seqlens=(4096,), seed=rank_seed(wl.seed, rank))
+    P = [inp[k] for k in ("conv_w", "A_log", "norm_w")]
+    N = 4096
+    y = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
+    fs = torch.empty((1, H, D, D), device=dev)
+    ws = torch.empty(max(gdn.kda_prefill_workspace_size(cfg, 1, N), 1), dtype=torch.uint8, device=dev)
+
+    def pstep():
+        gdn.kda_prefill(cfg, inp["qkv"], inp["zdec"], inp["b"], inp["gate"], inp["cu_seqlens"], *P,
+                        y=y, final_state=fs, workspace=ws)
+
+    for _ in range(args.warmup):
+        pstep()
+    tot, kern = timed(pstep, args.steps)
+    tot, kern = max_over_ranks(tot), max_over_ranks(kern)
+    # per token and head: decay, k-projection, rank-1 update and q-projection of
+    # the d x d state, one FMA (2 FLOP) each per element
+    flops = 4 * 2 * H * D * D * N
+    tf = flops / (kern / 1e3) / 1e12
+    out = {"metric": "KDA prefill tokens/s and decode tokens/s, Kimi K3 layer shape", "unit": "tokens/s",
+           "config": {"workload": wl.name, "num_heads": H, "head_dim": D},
+           "prefill": {"value": job_rate(N, world, args.steps, tot), "ms_per_step": tot / args.steps,
+                       "batch": 1, "seq_len": N,
+                       "roofline": {"kernel": "kda_prefill_kernel", "bound": "alu", "achieved": round(tf, 2),
+                                    "peak": round(FP32_CUDA_CORE_TFLOPS, 1), "unit": "TFLOP/s",
+                                    "frac": round(tf / FP32_CUDA_CORE_TFLOPS, 4), "kernel_ms": round(kern, 4),
+                                    "peak_source": "FP32 FMA lanes x clock (148 x 128 x 2 x 1.965 GHz)"}}}
+    del inp, y, fs, ws
+    B = args.decode_batch
+    d = W.make_kda_decode(wl, dev, batch=B, seed=rank_seed(wl.seed, rank) + 1)
+    Pd = [d[k] for k in ("conv_w", "A_log", "norm_w")]
+    yd = torch.empty((B, H, D), dtype=torch.bfloat16, device=dev)
+
+    def dstep():
+        gdn.kda_decode(cfg, d["qkv"], d["zdec"], d["b"], d["gate"], d["state"], d["conv_cache"], *Pd, y=yd)
+
+    for _ in range(args.warmup):
+        dstep()
+    tot, _ = timed(dstep, args.steps)
+    tot = max_over_ranks(tot)
+    ms = tot / args.steps
+    nbytes = kda_decode_bytes(H, D, B)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    out["decode"] = {"value": job_rate(B, world, args.steps, tot), "ms_per_step": ms, "batch": B,
+                     "roofline": {"kernel": "kda_decode_kernel", "bound": "hbm", "achieved": round(gbs, 1),
+                                  "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": round(gbs / pk["hbm_gbs"], 4),
+                                  "algorithmic_bytes": nbytes}}
     return out
 
 

@@ -126,3 +126,27 @@ def test_262k_single_sequence(cuda_device, wl):
     for t0 in range(0, N, 32768):
         assert torch.isfinite(out["y"][t0:t0 + 32768].float()).all()
     np.testing.assert_array_equal(to64(out["final_conv"][0]), to64(inp["qkv"][N - 3:N]))
+
+
+@pytest.mark.parametrize("segments", [3, 7])
+def test_split_float32_activations(cuda_device, segments):
+    """fp32 activations: the passes read the front end's convolved v by TMA
+    instead of convolving it; all heads of a small layer against the oracle."""
+    wl = W.Workload("split_f32", 2, 4, 128, dtype="f32", seqlens=(700, 0, 300), state_std=0.02,
+                    seed=13, gates="long_memory:-8:-2")
+    cfg = gdn.Config.of(wl, "chunked", segments)
+    inp = W.make_prefill(wl, cuda_device)
+    out = _prefill(cfg, inp, return_final_state=True, return_o_raw=True)
+    torch.cuda.synchronize()
+    cu = inp["cu_seqlens"].tolist()
+    for n in range(len(cu) - 1):
+        s, e = cu[n], cu[n + 1]
+        ref = oracle.prefill(_shape(wl), inp["qkv"][s:e], inp["a"][s:e], inp["b"][s:e], inp["z"][s:e],
+                             [0, e - s], *[inp[k] for k in PARAMS],
+                             initial_state=inp["initial_state"][n:n + 1])
+        r = m = None
+        if e > s:
+            r, m = assert_output_close(out["y"][s:e], ref["y"], f"y seq {n}")
+            assert_output_close(out["o_raw"][s:e], ref["o"], f"o seq {n}")
+        rs = assert_state_close(out["final_state"][n], ref["state"][0], f"state seq {n}")
+        report(f"split fp32 P={segments} seq {n} len {e - s}", r, m, rs)
