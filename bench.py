@@ -275,6 +275,8 @@ def run_ours(args, rank, world, dev, dist):
 
     if args.only == "decode":
         return run_decode(args, rank, world, dev, pk, timed, max_over_ranks)
+    if args.only == "kda":
+        return run_kda(args, rank, world, dev, pk, timed, max_over_ranks)
     clocks = ClockSampler(dev.index)
     for _ in range(args.warmup):
         step()
@@ -541,9 +543,9 @@ def run_kda(args, rank, world, dev, pk, timed, max_over_ranks):
     wl = W.KIMI_K3_KDA
     cfg = gdn.Config.of(wl)
     H, D = wl.num_v_heads, wl.head_dim
-    inp = W.make_kda_prefill(wl, dev, seqlens=(4096,), seed=rank_seed(wl.seed, rank))
+    N = args.seq_len
+    inp = W.make_kda_prefill(wl, dev, seqlens=(N,), seed=rank_seed(wl.seed, rank))
     P = [inp[k] for k in ("conv_w", "A_log", "norm_w")]
-    N = 4096
     y = torch.empty((N, H, D), dtype=torch.bfloat16, device=dev)
     fs = torch.empty((1, H, D, D), device=dev)
     ws = torch.empty(max(gdn.kda_prefill_workspace_size(cfg, 1, N), 1), dtype=torch.uint8, device=dev)
@@ -630,18 +632,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode"],
+    ap.add_argument("--only", default="all", choices=["all", "prefill", "decode", "kda"],
                     help="run only one part (for profiling small cases)")
     ap.add_argument("--decode-batch", type=int, default=256)
     ap.add_argument("--seq-len", type=int, default=4096,
-                    help="with --only prefill: the prefill sequence length (profiling cases)")
+                    help="with --only prefill or kda: the prefill sequence length (profiling cases)")
     ap.add_argument("--algo", default="auto", choices=["auto", "chunked", "serial"],
                     help="prefill algorithm (auto = tensor-core chunks at head dim 128)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
-    if args.seq_len != 4096 and args.only != "prefill":
-        ap.error("--seq-len applies to --only prefill")
+    if args.seq_len != 4096 and args.only not in ("prefill", "kda"):
+        ap.error("--seq-len applies to --only prefill or kda")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

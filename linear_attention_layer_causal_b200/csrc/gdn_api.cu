@@ -560,10 +560,11 @@ gdn_status gdn_kda_prefill_workspace_size(const gdn_config *cfg, int32_t batch, 
         return GDN_ERR_UNSUPPORTED;
     if (bytes == nullptr || batch < 0 || total_tokens < 0)
         return GDN_ERR_INVALID_ARG;
-    // the token-serial path's regions: header, normalised q|k, convolved v
+    // header, normalised q|k, convolved v, and the raw output before the gated norm
+    const size_t hd = (size_t)total_tokens * cfg->num_v_heads * cfg->head_dim * 4;
     *bytes = total_tokens == 0 ? 0
                                : kWorkspaceHeader + round_up((size_t)total_tokens * 2 * cfg->num_qk_heads * cfg->head_dim * 4) +
-                                     round_up((size_t)total_tokens * cfg->num_v_heads * cfg->head_dim * 4);
+                                     round_up(hd) + round_up(hd);
     return GDN_OK;
 }
 
@@ -624,6 +625,7 @@ gdn_status gdn_kda_prefill(const gdn_config *cfg, const gdn_kda_params *params, 
         p.ws_err = (unsigned int *)w;
         p.ws_qk = w + kWorkspaceHeader;
         p.ws_v = (char *)p.ws_qk + round_up((size_t)total_tokens * 2 * p.Hk * p.D * 4);
+        p.ws_o = (float *)((char *)p.ws_v + round_up((size_t)total_tokens * p.Hv * p.D * 4));
     }
     cudaStream_t s = (cudaStream_t)stream;
     const ProfileHook hook = take_profile_hook();

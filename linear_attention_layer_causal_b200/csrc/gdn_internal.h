@@ -26,6 +26,7 @@ struct PrefillArgs {
     const float *conv_w, *A_log, *dt_bias, *norm_w;
     bool chunked;            // tensor-core chunked path (head_dim 128) or token-serial
     const void *kda_zdec = nullptr; // KDA: per-channel decay inputs [N, H, d] (a, dt_bias unused)
+    float *ws_o = nullptr;          // KDA: [N, H, d] float32 raw output before the gated norm
     long long wait_limit;    // SM cycles a wait between warps may take before the call aborts
     // workspace carve-up
     unsigned int *ws_err;    // device status word (0 = ok; bit 0: a bounded wait timed out)

@@ -9,10 +9,12 @@
 //     S_t = S_{t-1} D (I - beta k k^T) + beta v k^T,   o_t = S_t q_t,
 //     y_t = o_t / rms(o_t) * w * sigmoid(gate_t),
 // which, one state row s (value channel) at a time, is
-//     s <- s * alpha;  u = beta (v - s . k);  s <- s + u k;  o = s . q.
+//     s <- s * alpha;  u = beta (v - s . k);  s <- s + u k;  o = s . q
+// (the last equal to (s * alpha) . q + u (k . q)).
 // Each head has its own q and k (no sharing).  Both kernels run the update on
-// CUDA cores in FP32: the token-serial prefill (one CTA per (head, sequence);
-// the conv, SiLU and L2 norm come from the shared front kernel) and the
+// CUDA cores in FP32: the token-serial prefill (D / 32 CTAs of 32 state rows per
+// (head, sequence); the conv, SiLU and L2 norm come from the shared front
+// kernel; the gated RMSNorm is a separate pass over the raw output) and the
 // one-token decode (one CTA per (sequence, head), conv from the cache).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
@@ -21,139 +23,291 @@ namespace gdn {
 
 namespace {
 
-constexpr int kTB = 32; // tokens staged per batch
+constexpr int kTB = 16;  // tokens staged per batch
+constexpr int kRows = 32; // state rows (value channels) per CTA
 
-template <int D> struct KdaSmem {
-    float k[kTB][D];
-    float q[kTB][D];
-    float v[kTB][D];
-    float al[kTB][D]; // per-channel decay factors
-    float o[kTB][D];
-    float beta[kTB];
+// Double-buffered token batches: q, k, z and this CTA's v rows arrive by
+// cp.async while the previous batch runs.  Per pair of tokens (t0, t1) of the
+// current batch, with a0, a1 their decay vectors, the vectors the pair step
+// reads are formed once:
+//     pv[0] = a0 k0,  pv[1] = a0 q0,  pv[2] = a0 a1 k1,  pv[3] = a0 a1 q1,
+//     pv[4] = a0 a1,  pv[5] = a1 k0,
+// and the scalars pc = (k0 . a1 k1, k0 . a1 q1, k0 . q0, k1 . q1).
+template <typename T, int D> struct KdaSmem {
+    float q[2][kTB][D];
+    float k[2][kTB][D];
+    T z[2][kTB][D];
+    float v[2][kTB][kRows];
+    float beta[2][kTB];
+    float pv[kTB / 2][6][D];
+    float4 pc[kTB / 2];
 };
 
-// -5 sigmoid(e^A z): the bounded per-channel log-decay
+// -5 sigmoid(e^A z): the bounded per-channel log-decay, and its exponential
 __device__ __forceinline__ float kda_log_decay(float eA, float z) { return -5.0f * sigmoidf_(eA * z); }
+__device__ __forceinline__ float kda_decay(float eA, float z) {
+    return __expf(-5.0f * __fdividef(1.0f, 1.0f + __expf(-eA * z)));
+}
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, bool valid) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
-// Thread (row v, part p) keeps D/4 entries of row v of the FP32 state (columns
-// 16 i + 4 p + e).
+// Columns held by lane cg (of 16) of a row group: C = D / 16 of them, taken as
+// float4s at 4 cg + 64 j (D = 64, 128) or as one float2 at 2 cg (D = 32), so
+// that the 16 lanes of a load phase read consecutive shared-memory words.
+template <int D> struct KdaCols {
+    static constexpr int C = D / 16;
+    static_assert(C == 2 || C % 4 == 0, "head dim 32, 64 or 128");
+    __device__ static __forceinline__ void load(const float *row, int cg, float (&x)[C]) {
+        if constexpr (C == 2) {
+            const float2 t = reinterpret_cast<const float2 *>(row)[cg];
+            x[0] = t.x; x[1] = t.y;
+        } else {
+#pragma unroll
+            for (int j = 0; j < C / 4; ++j) {
+                const float4 t = reinterpret_cast<const float4 *>(row + 64 * j)[cg];
+                x[4 * j] = t.x; x[4 * j + 1] = t.y; x[4 * j + 2] = t.z; x[4 * j + 3] = t.w;
+            }
+        }
+    }
+    __device__ static __forceinline__ void store(float *row, int cg, const float (&x)[C]) {
+        if constexpr (C == 2) {
+            reinterpret_cast<float2 *>(row)[cg] = make_float2(x[0], x[1]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < C / 4; ++j)
+                reinterpret_cast<float4 *>(row + 64 * j)[cg] =
+                    make_float4(x[4 * j], x[4 * j + 1], x[4 * j + 2], x[4 * j + 3]);
+        }
+    }
+};
+
+// The rows of a head's state evolve independently given each token's k, decay
+// and beta, so a head is split over D / 32 CTAs of 32 rows (blockIdx.z), which
+// fills the SMs and runs several token chains per SM.  A warp holds 8 rows as
+// two groups of 16 lanes; each lane keeps 4 rows x D/16 columns of the FP32
+// state, so the shared vectors are read once per 4 rows.
+//
+// Tokens go two at a time.  From the row s entering the pair, with
+// s0' = a0 s and s1' = a1 (s0' + u0 k0):
+//     s0' . k0 = s . pv[0],   s0' . q0 = s . pv[1],
+//     s1' . k1 = s . pv[2] + u0 (k0 . a1 k1),
+//     s1' . q1 = s . pv[3] + u0 (k0 . a1 q1),
+// so the four projections of the pair come from one pass over s, and
+//     u0 = beta0 (v0 - s0' . k0),        o0 = s0' . q0 + u0 (k0 . q0),
+//     u1 = beta1 (v1 - s1' . k1),        o1 = s1' . q1 + u1 (k1 . q1),
+//     s <- (a0 a1) s + u0 (a1 k0) + u1 k1.
+// The 16 partial sums of a lane (4 rows x 4 projections) are reduced over its
+// 16 lanes by a butterfly that halves the values it carries at each exchange,
+// so that lane 4 d + r of a group ends with projection d of row r; u0 and u1
+// then go back to the group by shuffles.  An odd last token is paired with a
+// neutral one (decay 1, beta 0, zero q, k, v) whose output is not written.
+// Each CTA writes its 32 channels of the raw output o (FP32) to `ob` (the
+// call's o_raw, or the workspace); kda_norm_kernel then applies the gated
+// RMSNorm, which needs all D channels of a token.
 template <typename T, int D>
-__global__ void __launch_bounds__(4 * D)
-kda_prefill_kernel(PrefillArgs p) {
-    constexpr int NT = 4 * D;
-    constexpr int NI = D / 16;
+__global__ void __launch_bounds__(4 * kRows)
+kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
+    constexpr int NT = 4 * kRows;
+    constexpr int R = 4;              // rows per lane
+    constexpr int C = KdaCols<D>::C;  // columns per lane
+    constexpr int ZV = 16 / (int)sizeof(T); // z elements per 16-byte copy
+    constexpr unsigned FULL = 0xffffffffu;
     extern __shared__ __align__(16) unsigned char kda_smem_raw[];
-    KdaSmem<D> &sm = *reinterpret_cast<KdaSmem<D> *>(kda_smem_raw);
+    KdaSmem<T, D> &sm = *reinterpret_cast<KdaSmem<T, D> *>(kda_smem_raw);
     const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
-    const int row = tid >> 2, part = tid & 3;
+    const int warp = tid >> 5, lane = tid & 31, cg = lane & 15, gl = lane & 16;
+    const int lrow0 = warp * 8 + (lane >> 4) * R; // first of this lane's rows within the CTA's 32
+    const int row0 = (int)blockIdx.z * kRows + lrow0;
+    // after the butterfly: projection d of row r of the group
+    const bool b3 = (lane & 8) != 0, b2 = (lane & 4) != 0, b1 = (lane & 2) != 0, b0 = (lane & 1) != 0;
+    const int r = cg & 3, d = cg >> 2;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
     const float *qk = (const float *)p.ws_qk;
     const float *vv = (const float *)p.ws_v;
+    const T *zd = (const T *)p.kda_zdec;
     const int QK = 2 * p.Hk * D;
     const int64_t HD = (int64_t)p.Hv * D;
-    float s[NI][4];
-    const size_t sbase = (((size_t)n * p.Hv + h) * D + row) * D;
-#pragma unroll
-    for (int i = 0; i < NI; ++i) {
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (p.init_state != nullptr)
-            x = *reinterpret_cast<const float4 *>(p.init_state + sbase + 16 * i + 4 * part);
-        s[i][0] = x.x; s[i][1] = x.y; s[i][2] = x.z; s[i][3] = x.w;
-    }
-    const float eA = expf(__ldg(p.A_log + h));
-    for (int64_t b0 = 0; b0 < len; b0 += kTB) {
-        const int nb = (len - b0) < kTB ? (int)(len - b0) : kTB;
+
+    // batch [b0, b0 + kTB) into buffer `buf`; rows past the sequence are zero-filled
+    auto stage = [&](int buf, int64_t t0) {
+        const int nb = (len - t0) < kTB ? (int)(len - t0) : kTB;
         for (int e = tid; e < kTB * (D / 4); e += NT) {
             const int tk = e / (D / 4), c = (e % (D / 4)) * 4;
-            if (tk < nb) {
-                const int64_t t = start + b0 + tk;
-                *reinterpret_cast<float4 *>(&sm.q[tk][c]) =
-                    __ldg(reinterpret_cast<const float4 *>(qk + t * QK + h * D + c));
-                *reinterpret_cast<float4 *>(&sm.k[tk][c]) =
-                    __ldg(reinterpret_cast<const float4 *>(qk + t * QK + p.Hk * D + h * D + c));
-                *reinterpret_cast<float4 *>(&sm.v[tk][c]) =
-                    __ldg(reinterpret_cast<const float4 *>(vv + t * HD + (int64_t)h * D + c));
-                const T *zp = (const T *)p.kda_zdec + t * HD + (int64_t)h * D + c;
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    sm.al[tk][c + i] = expf(kda_log_decay(eA, to_f(zp[i])));
-            }
+            const int64_t t = start + t0 + (tk < nb ? tk : 0);
+            cp_async16(&sm.q[buf][tk][c], qk + t * QK + h * D + c, tk < nb);
+            cp_async16(&sm.k[buf][tk][c], qk + t * QK + p.Hk * D + h * D + c, tk < nb);
         }
-        if (tid < nb)
-            sm.beta[tid] = sigmoidf_(to_f(((const T *)p.b)[(start + b0 + tid) * p.Hv + h]));
-        __syncthreads();
-        for (int tk = 0; tk < nb; ++tk) {
-            const float beta = sm.beta[tk];
-            const float4 *k4 = reinterpret_cast<const float4 *>(sm.k[tk]);
-            const float4 *q4 = reinterpret_cast<const float4 *>(sm.q[tk]);
-            const float4 *a4 = reinterpret_cast<const float4 *>(sm.al[tk]);
-            float kr[NI][4];
-            float pk0 = 0.f, pk1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                const float4 kk = k4[4 * i + part], aa = a4[4 * i + part];
-                kr[i][0] = kk.x; kr[i][1] = kk.y; kr[i][2] = kk.z; kr[i][3] = kk.w;
-                s[i][0] *= aa.x; s[i][1] *= aa.y; s[i][2] *= aa.z; s[i][3] *= aa.w;
-                pk0 = fmaf(s[i][0], kk.x, pk0);
-                pk1 = fmaf(s[i][1], kk.y, pk1);
-                pk0 = fmaf(s[i][2], kk.z, pk0);
-                pk1 = fmaf(s[i][3], kk.w, pk1);
-            }
-            float pk = pk0 + pk1;
-            pk += __shfl_xor_sync(0xffffffffu, pk, 1);
-            pk += __shfl_xor_sync(0xffffffffu, pk, 2);
-            const float u = beta * (sm.v[tk][row] - pk);
-            float po0 = 0.f, po1 = 0.f;
-#pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                const float4 qq = q4[4 * i + part];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    s[i][e] = fmaf(u, kr[i][e], s[i][e]);
-                po0 = fmaf(s[i][0], qq.x, po0);
-                po1 = fmaf(s[i][1], qq.y, po1);
-                po0 = fmaf(s[i][2], qq.z, po0);
-                po1 = fmaf(s[i][3], qq.w, po1);
-            }
-            float po = po0 + po1;
-            po += __shfl_xor_sync(0xffffffffu, po, 1);
-            po += __shfl_xor_sync(0xffffffffu, po, 2);
-            if (part == 0)
-                sm.o[tk][row] = po;
+        for (int e = tid; e < kTB * (D / ZV); e += NT) {
+            const int tk = e / (D / ZV), c = (e % (D / ZV)) * ZV;
+            const int64_t t = start + t0 + (tk < nb ? tk : 0);
+            cp_async16(&sm.z[buf][tk][c], zd + t * HD + (int64_t)h * D + c, tk < nb);
         }
-        __syncthreads();
-        // RMSNorm of each token's output times w sigmoid(gate), one warp per token
-        const int warp = tid >> 5, lane = tid & 31;
-        constexpr int PER = D / 32;
-        for (int tk = warp; tk < nb; tk += NT / 32) {
-            const int64_t t = start + b0 + tk;
-            float ov[PER];
-            float ss = 0.f;
-#pragma unroll
-            for (int e = 0; e < PER; ++e) {
-                ov[e] = sm.o[tk][lane * PER + e];
-                ss = fmaf(ov[e], ov[e], ss);
-            }
-            ss = group_sum<32>(ss);
-            const float r = rsqrtf(ss / (float)D + p.rms_eps);
-            const int64_t base = t * HD + (int64_t)h * D + lane * PER;
-#pragma unroll
-            for (int e = 0; e < PER; ++e) {
-                const float gt = to_f(((const T *)p.z)[base + e]);
-                ((T *)p.y)[base + e] = from_f<T>(ov[e] * r * __ldg(p.norm_w + lane * PER + e) * sigmoidf_(gt));
-                if (p.o_raw != nullptr)
-                    p.o_raw[base + e] = ov[e];
-            }
+        for (int e = tid; e < kTB * (kRows / 4); e += NT) {
+            const int tk = e / (kRows / 4), c = (e % (kRows / 4)) * 4;
+            const int64_t t = start + t0 + (tk < nb ? tk : 0);
+            cp_async16(&sm.v[buf][tk][c], vv + t * HD + (int64_t)h * D + (int)blockIdx.z * kRows + c, tk < nb);
         }
-        __syncthreads();
+        cp_async_commit();
+        if (tid < kTB)
+            sm.beta[buf][tid] = tid < nb ? sigmoidf_(to_f(((const T *)p.b)[(start + t0 + tid) * p.Hv + h])) : 0.f;
+    };
+
+    float s[R][C];
+    float *const srow = p.final_state == nullptr ? nullptr
+                                                 : p.final_state + (((size_t)n * p.Hv + h) * D + row0) * D;
+    {
+        const float *irow = p.init_state == nullptr ? nullptr
+                                                    : p.init_state + (((size_t)n * p.Hv + h) * D + row0) * D;
+#pragma unroll
+        for (int i = 0; i < R; ++i) {
+            if (irow != nullptr)
+                KdaCols<D>::load(irow + (size_t)i * D, cg, s[i]);
+            else
+#pragma unroll
+                for (int c = 0; c < C; ++c)
+                    s[i][c] = 0.f;
+        }
     }
-    if (p.final_state != nullptr) {
+    const float eA = expf(__ldg(p.A_log + h));
+    if (len > 0)
+        stage(0, 0);
+    int buf = 0;
+    for (int64_t tb = 0; tb < len; tb += kTB, buf ^= 1) {
+        const int nb = (len - tb) < kTB ? (int)(len - tb) : kTB;
+        const int np = (nb + 1) / 2;
+        cp_async_wait_all();
+        __syncthreads(); // batch tb has landed; the previous batch's tokens are done
+        if (tb + kTB < len)
+            stage(buf ^ 1, tb + kTB);
+        for (int pp = warp; pp < np; pp += NT / 32) {
+            const int t0 = 2 * pp, t1 = t0 + 1;
+            const bool has1 = t1 < nb;
+            float ckk = 0.f, ckq = 0.f, kq0 = 0.f, kq1 = 0.f;
+            for (int c = lane; c < D; c += 32) {
+                const float a0 = kda_decay(eA, to_f(sm.z[buf][t0][c]));
+                const float a1 = has1 ? kda_decay(eA, to_f(sm.z[buf][t1][c])) : 1.0f;
+                const float k0 = sm.k[buf][t0][c], q0 = sm.q[buf][t0][c];
+                const float k1 = sm.k[buf][t1][c], q1 = sm.q[buf][t1][c];
+                const float a01 = a0 * a1, a1k0 = a1 * k0;
+                sm.pv[pp][0][c] = a0 * k0;
+                sm.pv[pp][1][c] = a0 * q0;
+                sm.pv[pp][2][c] = a01 * k1;
+                sm.pv[pp][3][c] = a01 * q1;
+                sm.pv[pp][4][c] = a01;
+                sm.pv[pp][5][c] = a1k0;
+                ckk = fmaf(a1k0, k1, ckk);
+                ckq = fmaf(a1k0, q1, ckq);
+                kq0 = fmaf(k0, q0, kq0);
+                kq1 = fmaf(k1, q1, kq1);
+            }
+            ckk = group_sum<32>(ckk);
+            ckq = group_sum<32>(ckq);
+            kq0 = group_sum<32>(kq0);
+            kq1 = group_sum<32>(kq1);
+            if (lane == 0)
+                sm.pc[pp] = make_float4(ckk, ckq, kq0, kq1);
+        }
+        __syncthreads();
+        for (int pp = 0; pp < np; ++pp) {
+            const int t0 = 2 * pp;
+            float a[4 * R];
+            {
+                float x0[C], x1[C], x2[C], x3[C];
+                KdaCols<D>::load(sm.pv[pp][0], cg, x0);
+                KdaCols<D>::load(sm.pv[pp][1], cg, x1);
+                KdaCols<D>::load(sm.pv[pp][2], cg, x2);
+                KdaCols<D>::load(sm.pv[pp][3], cg, x3);
 #pragma unroll
-        for (int i = 0; i < NI; ++i)
-            *reinterpret_cast<float4 *>(p.final_state + sbase + 16 * i + 4 * part) =
-                make_float4(s[i][0], s[i][1], s[i][2], s[i][3]);
+                for (int i = 0; i < R; ++i) {
+                    float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+                    for (int c = 0; c < C; ++c) {
+                        y0 = fmaf(s[i][c], x0[c], y0);
+                        y1 = fmaf(s[i][c], x1[c], y1);
+                        y2 = fmaf(s[i][c], x2[c], y2);
+                        y3 = fmaf(s[i][c], x3[c], y3);
+                    }
+                    a[i] = y0;
+                    a[R + i] = y1;
+                    a[2 * R + i] = y2;
+                    a[3 * R + i] = y3;
+                }
+            }
+            // butterfly over the 16 lanes: 16 values -> 8 -> 4 -> 2 -> 1
+            float r8[8], r4[4], r2[2];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                r8[j] = (b3 ? a[j + 8] : a[j]) + __shfl_xor_sync(FULL, b3 ? a[j] : a[j + 8], 8);
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                r4[j] = (b2 ? r8[j + 4] : r8[j]) + __shfl_xor_sync(FULL, b2 ? r8[j] : r8[j + 4], 4);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+                r2[j] = (b1 ? r4[j + 2] : r4[j]) + __shfl_xor_sync(FULL, b1 ? r4[j] : r4[j + 2], 2);
+            const float pr = (b0 ? r2[1] : r2[0]) + __shfl_xor_sync(FULL, b0 ? r2[0] : r2[1], 1);
+            // every lane of row r: the two u of the pair
+            const float pk0 = __shfl_sync(FULL, pr, gl | r);
+            const float xk1 = __shfl_sync(FULL, pr, gl | 8 | r);
+            const float4 sc = sm.pc[pp];
+            const float u0 = sm.beta[buf][t0] * (sm.v[buf][t0][lrow0 + r] - pk0);
+            const float u1 = sm.beta[buf][t0 + 1] * (sm.v[buf][t0 + 1][lrow0 + r] - fmaf(u0, sc.x, xk1));
+            const int64_t ot = (start + tb + t0) * HD + (int64_t)h * D + row0 + r;
+            if (d == 1)
+                ob[ot] = fmaf(u0, sc.z, pr);
+            else if (d == 3 && t0 + 1 < nb)
+                ob[ot + HD] = fmaf(u1, sc.w, fmaf(u0, sc.y, pr));
+            float w2[C], w1[C], w0[C];
+            KdaCols<D>::load(sm.pv[pp][4], cg, w2);
+            KdaCols<D>::load(sm.pv[pp][5], cg, w1);
+            KdaCols<D>::load(sm.k[buf][t0 + 1], cg, w0);
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                const float u0i = __shfl_sync(FULL, u0, gl | i);
+                const float u1i = __shfl_sync(FULL, u1, gl | i);
+#pragma unroll
+                for (int c = 0; c < C; ++c)
+                    s[i][c] = fmaf(u1i, w0[c], fmaf(u0i, w1[c], s[i][c] * w2[c]));
+            }
+        }
+    }
+    if (srow != nullptr) {
+#pragma unroll
+        for (int i = 0; i < R; ++i)
+            KdaCols<D>::store(srow + (size_t)i * D, cg, s[i]);
+    }
+}
+
+// y = o / rms(o) * w * sigmoid(gate) for each (token, head): one warp each,
+// D / 32 channels a lane
+template <typename T, int D>
+__global__ void __launch_bounds__(256)
+kda_norm_kernel(PrefillArgs p, const float *__restrict__ ob) {
+    constexpr int PER = D / 32;
+    const int64_t unit = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (unit >= p.N * p.Hv)
+        return;
+    const int64_t base = unit * D + lane * PER; // [N, H, D] row-major: unit = t * H + h
+    float ov[PER];
+    float ss = 0.f;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        ov[e] = ob[base + e];
+        ss = fmaf(ov[e], ov[e], ss);
+    }
+    ss = group_sum<32>(ss);
+    const float r = rsqrtf(ss / (float)D + p.rms_eps);
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+        const float gt = to_f(((const T *)p.z)[base + e]);
+        ((T *)p.y)[base + e] = from_f<T>(ov[e] * r * __ldg(p.norm_w + lane * PER + e) * sigmoidf_(gt));
     }
 }
 
@@ -221,24 +375,38 @@ kda_decode_kernel(DecodeArgs p) {
         qa[e] = qs[c4 + e] * sq * al[e]; // (S D) q
     }
     float *Sg = p.state + ((size_t)n * H + h) * D * D;
-    for (int r = warp * RPI + lr; r < D; r += NW * RPI) {
-        const float4 sv = __ldcs(reinterpret_cast<const float4 *>(Sg + (size_t)r * D + c4));
-        float pk = sv.x * ka[0] + sv.y * ka[1] + sv.z * ka[2] + sv.w * ka[3];
-        float pq = sv.x * qa[0] + sv.y * qa[1] + sv.z * qa[2] + sv.w * qa[3];
+    // four rows per warp in flight: their loads are issued before any of them is used
+    constexpr int KU = 4;
+    for (int r0 = warp * RPI + lr; r0 < D; r0 += NW * RPI * KU) {
+        float4 sv[KU];
 #pragma unroll
-        for (int o = L / 2; o > 0; o >>= 1) {
-            pk += __shfl_xor_sync(0xffffffffu, pk, o);
-            pq += __shfl_xor_sync(0xffffffffu, pq, o);
+        for (int uu = 0; uu < KU; ++uu) {
+            const int r = r0 + uu * NW * RPI;
+            sv[uu] = r < D ? __ldcs(reinterpret_cast<const float4 *>(Sg + (size_t)r * D + c4))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        const float u = beta * (vs[r] - pk);
-        float4 nv;
-        nv.x = fmaf(u, kr[0], al[0] * sv.x);
-        nv.y = fmaf(u, kr[1], al[1] * sv.y);
-        nv.z = fmaf(u, kr[2], al[2] * sv.z);
-        nv.w = fmaf(u, kr[3], al[3] * sv.w);
-        __stcs(reinterpret_cast<float4 *>(Sg + (size_t)r * D + c4), nv);
-        if ((lane % L) == 0)
-            os[r] = pq + u * kq; // o = (S D) q + u (k . q)
+#pragma unroll
+        for (int uu = 0; uu < KU; ++uu) {
+            const int r = r0 + uu * NW * RPI;
+            float pk = sv[uu].x * ka[0] + sv[uu].y * ka[1] + sv[uu].z * ka[2] + sv[uu].w * ka[3];
+            float pq = sv[uu].x * qa[0] + sv[uu].y * qa[1] + sv[uu].z * qa[2] + sv[uu].w * qa[3];
+#pragma unroll
+            for (int o = L / 2; o > 0; o >>= 1) {
+                pk += __shfl_xor_sync(0xffffffffu, pk, o);
+                pq += __shfl_xor_sync(0xffffffffu, pq, o);
+            }
+            if (r < D) {
+                const float u = beta * (vs[r] - pk);
+                float4 nv;
+                nv.x = fmaf(u, kr[0], al[0] * sv[uu].x);
+                nv.y = fmaf(u, kr[1], al[1] * sv[uu].y);
+                nv.z = fmaf(u, kr[2], al[2] * sv[uu].z);
+                nv.w = fmaf(u, kr[3], al[3] * sv[uu].w);
+                __stcs(reinterpret_cast<float4 *>(Sg + (size_t)r * D + c4), nv);
+                if ((lane % L) == 0)
+                    os[r] = pq + u * kq; // o = (S D) q + u (k . q)
+            }
+        }
     }
     __syncthreads();
     if (warp == 0) {
@@ -261,13 +429,17 @@ kda_decode_kernel(DecodeArgs p) {
 }
 
 template <typename T, int D> cudaError_t launch_prefill_t(const PrefillArgs &p, cudaStream_t s) {
-    const size_t smem = sizeof(KdaSmem<D>);
+    const size_t smem = sizeof(KdaSmem<T, D>);
     cudaError_t e = cudaFuncSetAttribute(kda_prefill_kernel<T, D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess)
         return e;
-    dim3 grid(p.Hv, p.batch);
-    kda_prefill_kernel<T, D><<<grid, 4 * D, smem, s>>>(p);
+    float *ob = p.o_raw != nullptr ? p.o_raw : p.ws_o;
+    kda_prefill_kernel<T, D><<<dim3(p.Hv, p.batch, D / kRows), 4 * kRows, smem, s>>>(p, ob);
+    if ((e = cudaGetLastError()) != cudaSuccess || p.N == 0)
+        return e;
+    const int64_t units = p.N * p.Hv;
+    kda_norm_kernel<T, D><<<(unsigned)((units + 7) / 8), 256, 0, s>>>(p, ob);
     return cudaGetLastError();
 }
 
