@@ -104,7 +104,10 @@ template <int D> struct KdaCols {
 // The 16 partial sums of a lane (4 rows x 4 projections) are reduced over its
 // 16 lanes by a butterfly that halves the values it carries at each exchange,
 // so that lane 4 d + r of a group ends with projection d of row r; u0 and u1
-// then go back to the group by shuffles.  An odd last token is paired with a
+// then go back to the group by shuffles.  Lane 4 d + r holds its rows and
+// projections in the order i ^ r and e ^ d (register slot i holds row
+// lrow0 + (i ^ r); slot group e holds projection e ^ d), so that at every
+// exchange it keeps the lower half of its values and sends the upper half.  An odd last token is paired with a
 // neutral one (decay 1, beta 0, zero q, k, v) whose output is not written.
 // Each CTA writes its 32 channels of the raw output o (FP32) to `ob` (the
 // call's o_raw, or the workspace); kda_norm_kernel then applies the gated
@@ -124,7 +127,6 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
     const int lrow0 = warp * 8 + (lane >> 4) * R; // first of this lane's rows within the CTA's 32
     const int row0 = (int)blockIdx.z * kRows + lrow0;
     // after the butterfly: projection d of row r of the group
-    const bool b3 = (lane & 8) != 0, b2 = (lane & 4) != 0, b1 = (lane & 2) != 0, b0 = (lane & 1) != 0;
     const int r = cg & 3, d = cg >> 2;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
@@ -168,7 +170,7 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
 #pragma unroll
         for (int i = 0; i < R; ++i) {
             if (irow != nullptr)
-                KdaCols<D>::load(irow + (size_t)i * D, cg, s[i]);
+                KdaCols<D>::load(irow + (size_t)(i ^ r) * D, cg, s[i]);
             else
 #pragma unroll
                 for (int c = 0; c < C; ++c)
@@ -220,10 +222,10 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
             float a[4 * R];
             {
                 float x0[C], x1[C], x2[C], x3[C];
-                KdaCols<D>::load(sm.pv[pp][0], cg, x0);
-                KdaCols<D>::load(sm.pv[pp][1], cg, x1);
-                KdaCols<D>::load(sm.pv[pp][2], cg, x2);
-                KdaCols<D>::load(sm.pv[pp][3], cg, x3);
+                KdaCols<D>::load(sm.pv[pp][d], cg, x0);
+                KdaCols<D>::load(sm.pv[pp][1 ^ d], cg, x1);
+                KdaCols<D>::load(sm.pv[pp][2 ^ d], cg, x2);
+                KdaCols<D>::load(sm.pv[pp][3 ^ d], cg, x3);
 #pragma unroll
                 for (int i = 0; i < R; ++i) {
                     float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
@@ -244,14 +246,14 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
             float r8[8], r4[4], r2[2];
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                r8[j] = (b3 ? a[j + 8] : a[j]) + __shfl_xor_sync(FULL, b3 ? a[j] : a[j + 8], 8);
+                r8[j] = a[j] + __shfl_xor_sync(FULL, a[j + 8], 8);
 #pragma unroll
             for (int j = 0; j < 4; ++j)
-                r4[j] = (b2 ? r8[j + 4] : r8[j]) + __shfl_xor_sync(FULL, b2 ? r8[j] : r8[j + 4], 4);
+                r4[j] = r8[j] + __shfl_xor_sync(FULL, r8[j + 4], 4);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
-                r2[j] = (b1 ? r4[j + 2] : r4[j]) + __shfl_xor_sync(FULL, b1 ? r4[j] : r4[j + 2], 2);
-            const float pr = (b0 ? r2[1] : r2[0]) + __shfl_xor_sync(FULL, b0 ? r2[0] : r2[1], 1);
+                r2[j] = r4[j] + __shfl_xor_sync(FULL, r4[j + 2], 2);
+            const float pr = r2[0] + __shfl_xor_sync(FULL, r2[1], 1);
             // every lane of row r: the two u of the pair
             const float pk0 = __shfl_sync(FULL, pr, gl | r);
             const float xk1 = __shfl_sync(FULL, pr, gl | 8 | r);
@@ -269,8 +271,8 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
             KdaCols<D>::load(sm.k[buf][t0 + 1], cg, w0);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float u0i = __shfl_sync(FULL, u0, gl | i);
-                const float u1i = __shfl_sync(FULL, u1, gl | i);
+                const float u0i = __shfl_sync(FULL, u0, gl | (i ^ r));
+                const float u1i = __shfl_sync(FULL, u1, gl | (i ^ r));
 #pragma unroll
                 for (int c = 0; c < C; ++c)
                     s[i][c] = fmaf(u1i, w0[c], fmaf(u0i, w1[c], s[i][c] * w2[c]));
@@ -280,7 +282,7 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
     if (srow != nullptr) {
 #pragma unroll
         for (int i = 0; i < R; ++i)
-            KdaCols<D>::store(srow + (size_t)i * D, cg, s[i]);
+            KdaCols<D>::store(srow + (size_t)(i ^ r) * D, cg, s[i]);
     }
 }
 
