@@ -25,6 +25,9 @@ namespace {
 
 constexpr int kTB = 16;  // tokens staged per batch
 constexpr int kRows = 32; // state rows (value channels) per CTA
+constexpr int kLaneRows = 4; // state rows per lane (2 or 4; 2 measured slower)
+// 16 lanes share a row group, two groups per warp
+constexpr int kPfThreads = 32 * kRows / (2 * kLaneRows);
 
 // Double-buffered token batches: q, k, z and this CTA's v rows arrive by
 // cp.async while the previous batch runs.  Per pair of tokens (t0, t1) of the
@@ -88,9 +91,9 @@ template <int D> struct KdaCols {
 
 // The rows of a head's state evolve independently given each token's k, decay
 // and beta, so a head is split over D / 32 CTAs of 32 rows (blockIdx.z), which
-// fills the SMs and runs several token chains per SM.  A warp holds 8 rows as
-// two groups of 16 lanes; each lane keeps 4 rows x D/16 columns of the FP32
-// state, so the shared vectors are read once per 4 rows.
+// fills the SMs and runs several token chains per SM.  A warp holds 2 R rows
+// (R = kLaneRows) as two groups of 16 lanes; each lane keeps R rows x D/16
+// columns of the FP32 state, so the shared vectors are read once per R rows.
 //
 // Tokens go two at a time.  From the row s entering the pair, with
 // s0' = a0 s and s1' = a1 (s0' + u0 k0):
@@ -101,22 +104,25 @@ template <int D> struct KdaCols {
 //     u0 = beta0 (v0 - s0' . k0),        o0 = s0' . q0 + u0 (k0 . q0),
 //     u1 = beta1 (v1 - s1' . k1),        o1 = s1' . q1 + u1 (k1 . q1),
 //     s <- (a0 a1) s + u0 (a1 k0) + u1 k1.
-// The 16 partial sums of a lane (4 rows x 4 projections) are reduced over its
-// 16 lanes by a butterfly that halves the values it carries at each exchange,
-// so that lane 4 d + r of a group ends with projection d of row r; u0 and u1
-// then go back to the group by shuffles.  Lane 4 d + r holds its rows and
-// projections in the order i ^ r and e ^ d (register slot i holds row
-// lrow0 + (i ^ r); slot group e holds projection e ^ d), so that at every
-// exchange it keeps the lower half of its values and sends the upper half.  An odd last token is paired with a
+// The 4 R partial sums of a lane (R rows x 4 projections) are reduced over its
+// 16 lanes by a butterfly that halves the values it carries at each exchange
+// (a plain add once one is left), so that group lane cg ends with projection
+// d = cg >> 2 of row r, r the next log2(R) bits of cg; u0 and u1 then go back
+// to the group by shuffles.  A lane holds its rows and projections in the
+// order i ^ r and e ^ d (register slot i holds row lrow0 + (i ^ r); slot group
+// e holds projection e ^ d), so that at every exchange it keeps the lower half
+// of its values and sends the upper half.  An odd last token is paired with a
 // neutral one (decay 1, beta 0, zero q, k, v) whose output is not written.
 // Each CTA writes its 32 channels of the raw output o (FP32) to `ob` (the
 // call's o_raw, or the workspace); kda_norm_kernel then applies the gated
 // RMSNorm, which needs all D channels of a token.
 template <typename T, int D>
-__global__ void __launch_bounds__(4 * kRows)
+__global__ void __launch_bounds__(kPfThreads)
 kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
-    constexpr int NT = 4 * kRows;
-    constexpr int R = 4;              // rows per lane
+    constexpr int NT = kPfThreads;
+    constexpr int R = kLaneRows;
+    static_assert(R == 2 || R == 4, "2 or 4 rows per lane");
+    constexpr int RS = R == 4 ? 0 : 1; // row r = (cg >> RS) & (R - 1)
     constexpr int C = KdaCols<D>::C;  // columns per lane
     constexpr int ZV = 16 / (int)sizeof(T); // z elements per 16-byte copy
     constexpr unsigned FULL = 0xffffffffu;
@@ -124,10 +130,10 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
     KdaSmem<T, D> &sm = *reinterpret_cast<KdaSmem<T, D> *>(kda_smem_raw);
     const int h = blockIdx.x, n = blockIdx.y, tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31, cg = lane & 15, gl = lane & 16;
-    const int lrow0 = warp * 8 + (lane >> 4) * R; // first of this lane's rows within the CTA's 32
+    const int lrow0 = warp * 2 * R + (lane >> 4) * R; // first of this lane's rows within the CTA's 32
     const int row0 = (int)blockIdx.z * kRows + lrow0;
     // after the butterfly: projection d of row r of the group
-    const int r = cg & 3, d = cg >> 2;
+    const int r = (cg >> RS) & (R - 1), d = cg >> 2;
     int64_t start, end;
     seq_bounds(p.cu, n, p.N, start, end);
     const int64_t len = end - start;
@@ -242,28 +248,30 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
                     a[3 * R + i] = y3;
                 }
             }
-            // butterfly over the 16 lanes: 16 values -> 8 -> 4 -> 2 -> 1
-            float r8[8], r4[4], r2[2];
+            // butterfly over the 16 lanes: 4 R values halved at each exchange
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-                r8[j] = a[j] + __shfl_xor_sync(FULL, a[j + 8], 8);
+            for (int m = 8, nv = 4 * R; m >= 1; m >>= 1) {
+                if (nv > 1) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-                r4[j] = r8[j] + __shfl_xor_sync(FULL, r8[j + 4], 4);
-#pragma unroll
-            for (int j = 0; j < 2; ++j)
-                r2[j] = r4[j] + __shfl_xor_sync(FULL, r4[j + 2], 2);
-            const float pr = r2[0] + __shfl_xor_sync(FULL, r2[1], 1);
+                    for (int j = 0; j < nv / 2; ++j)
+                        a[j] += __shfl_xor_sync(FULL, a[j + nv / 2], m);
+                    nv /= 2;
+                } else {
+                    a[0] += __shfl_xor_sync(FULL, a[0], m);
+                }
+            }
+            const float pr = a[0];
             // every lane of row r: the two u of the pair
-            const float pk0 = __shfl_sync(FULL, pr, gl | r);
-            const float xk1 = __shfl_sync(FULL, pr, gl | 8 | r);
+            const float pk0 = __shfl_sync(FULL, pr, gl | (r << RS));
+            const float xk1 = __shfl_sync(FULL, pr, gl | 8 | (r << RS));
             const float4 sc = sm.pc[pp];
             const float u0 = sm.beta[buf][t0] * (sm.v[buf][t0][lrow0 + r] - pk0);
             const float u1 = sm.beta[buf][t0 + 1] * (sm.v[buf][t0 + 1][lrow0 + r] - fmaf(u0, sc.x, xk1));
             const int64_t ot = (start + tb + t0) * HD + (int64_t)h * D + row0 + r;
-            if (d == 1)
+            const bool lead = (cg & ((1 << RS) - 1)) == 0; // one lane per (d, r)
+            if (d == 1 && lead)
                 ob[ot] = fmaf(u0, sc.z, pr);
-            else if (d == 3 && t0 + 1 < nb)
+            else if (d == 3 && lead && t0 + 1 < nb)
                 ob[ot + HD] = fmaf(u1, sc.w, fmaf(u0, sc.y, pr));
             float w2[C], w1[C], w0[C];
             KdaCols<D>::load(sm.pv[pp][4], cg, w2);
@@ -271,8 +279,8 @@ kda_prefill_kernel(PrefillArgs p, float *__restrict__ ob) {
             KdaCols<D>::load(sm.k[buf][t0 + 1], cg, w0);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                const float u0i = __shfl_sync(FULL, u0, gl | (i ^ r));
-                const float u1i = __shfl_sync(FULL, u1, gl | (i ^ r));
+                const float u0i = __shfl_sync(FULL, u0, gl | ((i ^ r) << RS));
+                const float u1i = __shfl_sync(FULL, u1, gl | ((i ^ r) << RS));
 #pragma unroll
                 for (int c = 0; c < C; ++c)
                     s[i][c] = fmaf(u1i, w0[c], fmaf(u0i, w1[c], s[i][c] * w2[c]));
@@ -437,7 +445,7 @@ template <typename T, int D> cudaError_t launch_prefill_t(const PrefillArgs &p, 
     if (e != cudaSuccess)
         return e;
     float *ob = p.o_raw != nullptr ? p.o_raw : p.ws_o;
-    kda_prefill_kernel<T, D><<<dim3(p.Hv, p.batch, D / kRows), 4 * kRows, smem, s>>>(p, ob);
+    kda_prefill_kernel<T, D><<<dim3(p.Hv, p.batch, D / kRows), kPfThreads, smem, s>>>(p, ob);
     if ((e = cudaGetLastError()) != cudaSuccess || p.N == 0)
         return e;
     const int64_t units = p.N * p.Hv;
