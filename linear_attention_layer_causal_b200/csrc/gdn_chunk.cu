@@ -100,25 +100,25 @@ chunk_offsets_kernel(const int32_t *__restrict__ cu, int batch, int64_t N, int32
 
 // ------------------------------------------------------------ chunk kernel
 //
-// One CTA per (value head, sequence), five roles that run consecutive chunks
-// at once and hand over through mbarriers:
+// One CTA per (value head, sequence) (or per segment of a split sequence),
+// four roles that run consecutive chunks at once and hand over through
+// mbarriers:
 //   state group (warps 0..7): once MMA 2 is done, S *= gamma_C and O^T *=
-//     diag(gamma); once MMA 2b is done, U rounded to tf32 in place; then the
-//     gated-RMSNorm epilogue.  Warps w and w + 4 share TMEM lanes 32 (w % 4) ..
-//     + 31 (lane = value channel) and split the columns.  X/O and U are
+//     diag(gamma); once MMA 2b is done, U rounded to tf32 in place and
+//     U diag(gamma_C / gamma) into the X columns; then the gated-RMSNorm
+//     epilogue.  Warps w and w + 4 share TMEM lanes 32 (w % 4) .. + 31
+//     (lane = value channel) and split the columns.  X/O and U are
 //     double-buffered in TMEM, so the epilogue of chunk c overlaps MMA 2 of
 //     chunk c + 1;
-//   T team (warps 8..11): gates (G, beta, gamma_C / gamma, gamma), A,
-//     T = (I + A)^-1 in a working tile of its own, then T diag(beta) and
-//     -T diag(beta gamma) into the tiles of the chunk's parity once MMA 1 and
-//     2b of chunk c - 2 have read them;
-//   P team (warps 12..13): diag(gamma_C / gamma) K in place on the MN-major K
-//     tile and P from the Q K^T tile (MMA 3 waits for both);
-//   MMA warp (warp 14): the whole warp runs the issue loop, one elected lane
-//     issues; TMA warp (warp 15): one lane.
-// Sixteen warps, four per scheduler, leave 128 registers a thread.  The
-// per-chunk critical path is MMA 2 -> MMA 2b -> U rounding -> MMA 3 -> MMA 2;
-// MMA 1 of the next chunk runs beside the U rounding.  The roles' loops are
+//   prep team (warps 8..11): P of chunk c from the Q K^T rows, then for chunk
+//     c + 1 the gate record (written by the inverse kernel) and, with 16-bit
+//     activations, the v conv into V^T;
+//   MMA warp (warp 12): the whole warp runs the issue loop, one elected lane
+//     issues;
+//   TMA warp (warp 13): one lane reloads each buffer once its last reader is
+//     done.
+// The per-chunk critical path is MMA 2 -> MMA 2b -> U pass -> MMA 3 -> MMA 2;
+// MMA 1 of the next chunk runs beside the U pass.  The roles' loops are
 // rolled where that measured faster: the SMs fetch the kernel's code from L2,
 // and smaller hot code runs faster.
 
