@@ -22,11 +22,13 @@
 // tri_kernel, 64 threads per (chunk, value head h), two value heads a CTA:
 // the gates of the chunk's tokens (g = -exp(A_log) softplus(a + dt_bias),
 // beta = sigmoid(b), G = prefix sums of g; Gated DeltaNet row),
-// A[r][s] = beta_r exp(G_r - G_s) kk[r][s], T = (I + A)^-1 in FP32 by forward
-// substitution with one column per thread (no barriers; the rows of A are
-// broadcast reads), and T diag(beta) rounded to nearest tf32 into the
-// workspace as 96 rows of 32 floats: the B operand of the chunk kernel's first
-// product, ready for a TMA load with 128-byte swizzle.
+// A[r][s] = beta_r exp(G_r - G_s) kk[r][s], T = (I + A)^-1 as 2 x 2 blocks of
+// 32 (each warp solves a diagonal block by forward substitution, one column a
+// lane; T21 = -T22 A21 T11 on the tensor core with three tf32 products a tile,
+// about FP32 accuracy), and T diag(beta) and -T diag(beta gamma) rounded to
+// nearest tf32 into the workspace as 96 rows of 32 floats: the B operands of
+// the chunk kernel's MMA 1 and MMA 2b, ready for a TMA load with 128-byte
+// swizzle.
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 #include "gdn_sm100.cuh"
@@ -224,24 +226,22 @@ __device__ __forceinline__ void chunk_of(const int32_t *__restrict__ cu, const i
     nr = (int)((e0 - t0) < kC ? (e0 - t0) : kC);
 }
 
-// One column of T = (I + A)^-1 by forward substitution, in registers: with
-// x[r] = T[r][c], x[r] = 0 (r < c), x[c] = 1, x[r] = -sum_{s<r} A[r][s] x[s]
-// (r > c).  A is strictly lower triangular in the triangular-tile layout; every
-// thread of a warp reads the same row of A (broadcast).  FIRST = 32 for the
-// warp of columns 32..63: its rows and terms below 32 are zero and skipped.
-template <int FIRST>
-__device__ __forceinline__ void tri_column(const float *__restrict__ A, int c, float (&x)[kC]) {
+// One column of a 32 x 32 diagonal block T_bb = (I + A_bb)^-1 by forward
+// substitution, in registers: with x[r] = T_bb[r][c], x[r] = 0 (r < c),
+// x[c] = 1, x[r] = -sum_{s<r} A_bb[r][s] x[s] (r > c).  Ab points at row 32 b
+// of column block b of the triangular tile (A + 2048 b), so element (r, s) of
+// the block sits at Ab + 32 r + 4 ((s / 4) xor (r mod 8)) + s mod 4; every lane
+// of the warp reads the same row (broadcast).
+__device__ __forceinline__ void tri_diag32(const float *__restrict__ Ab, int c, float (&x)[32]) {
 #pragma unroll
-    for (int r = 0; r < kC; ++r)
+    for (int r = 0; r < 32; ++r)
         x[r] = 0.f;
 #pragma unroll
-    for (int r = FIRST; r < kC; ++r) {
+    for (int r = 0; r < 32; ++r) {
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int s4 = FIRST; s4 < r; s4 += 4) {
-            // A[r][s4 .. s4 + 3]: column block s4 / 32, 16-byte chunk (s4 % 32) / 4
-            const int blk = s4 >> 5, ch = (s4 & 31) >> 2;
-            const float4 a = *reinterpret_cast<const float4 *>(A + 1024 * blk + 32 * r + ((ch ^ (r & 7)) << 2));
+        for (int s4 = 0; s4 < r; s4 += 4) {
+            const float4 a = *reinterpret_cast<const float4 *>(Ab + 32 * r + (((s4 >> 2) ^ (r & 7)) << 2));
             const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e)
@@ -253,15 +253,80 @@ __device__ __forceinline__ void tri_column(const float *__restrict__ A, int c, f
     }
 }
 
+// D += A B for one m16n8k8 tile on the tensor core (tf32 operands, FP32
+// accumulation; A row-major, B column-major).  Lane (g, t) = (lane / 4,
+// lane % 4) holds A[g][t], A[g + 8][t], A[g][t + 4], A[g + 8][t + 4],
+// B[t][g], B[t + 4][g] and D[g][2t], D[g][2t + 1], D[g + 8][2t], D[g + 8][2t + 1].
+__device__ __forceinline__ void mma_16x8x8_tf32(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile("mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+                 "{%0,%1,%2,%3};"
+                 : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// x = hi + lo with both parts tf32 (round to nearest): the split that lets
+// three tf32 products, hi hi + hi lo + lo hi, carry about FP32 accuracy
+__device__ __forceinline__ void split_tf32(float x, uint32_t &hi, uint32_t &lo) {
+    const float h = sm100::tf32_rna(x);
+    hi = __float_as_uint(h);
+    lo = __float_as_uint(sm100::tf32_rna(x - h));
+}
+
+// Columns j0 .. j0 + 15 of a 32 x 32 product D = X Y on the tensor core with
+// about FP32 accuracy (three tf32 products a tile).  xa(i, k) and yb(k, j)
+// read the operands; D comes back as two 16-row tiles x two 8-column tiles of
+// m16n8 accumulators.
+template <typename XA, typename YB>
+__device__ __forceinline__ void mm32x16_3xtf32(XA xa, YB yb, int j0, int lane, float (&d)[2][2][4]) {
+    const int g = lane >> 2, t = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                d[mt][nt][e] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < 32; k0 += 8) {
+        uint32_t ah[2][4], al[2][4], bh[2][2], bl[2][2];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+            const int i = 16 * mt + g;
+            split_tf32(xa(i, k0 + t), ah[mt][0], al[mt][0]);
+            split_tf32(xa(i + 8, k0 + t), ah[mt][1], al[mt][1]);
+            split_tf32(xa(i, k0 + t + 4), ah[mt][2], al[mt][2]);
+            split_tf32(xa(i + 8, k0 + t + 4), ah[mt][3], al[mt][3]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int j = j0 + 8 * nt + g;
+            split_tf32(yb(k0 + t, j), bh[nt][0], bl[nt][0]);
+            split_tf32(yb(k0 + t + 4, j), bh[nt][1], bl[nt][1]);
+        }
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                mma_16x8x8_tf32(d[mt][nt], al[mt], bh[nt]);
+                mma_16x8x8_tf32(d[mt][nt], ah[mt], bl[nt]);
+                mma_16x8x8_tf32(d[mt][nt], ah[mt], bh[nt]);
+            }
+    }
+}
+
 // Two value heads a CTA (64 threads each, named barrier 1 + head): gates, A in
-// shared memory, then T = (I + A)^-1 one column per thread, and T diag(beta)
-// straight to the workspace (a warp writes 128 contiguous bytes per row).
+// shared memory, then T = (I + A)^-1 by 32 x 32 blocks, and the two B tiles
+// straight to the workspace.
 template <typename T>
 __global__ void __launch_bounds__(128, 4)
 tri_kernel(PrefillArgs p) {
     using namespace sm100;
     __shared__ __align__(16) float As[2][kTriFloats];
     __shared__ __align__(16) float Gs[2][kC], Bs[2][kC];
+    // the diagonal blocks T11 (row stride 40: read as B fragments without bank
+    // conflicts; later the product W = A21 T11 in the same columns) and T22
+    // (row stride 36: read as A fragments)
+    __shared__ __align__(16) float T1s[2][32 * 40], T2s[2][32 * 36];
     const int ci = blockIdx.x, gi = threadIdx.x >> 6, tt = threadIdx.x & 63, lane = threadIdx.x & 31;
     const int h = 2 * blockIdx.y + gi;
     if (ci >= __ldg(p.ws_offs + p.batch))
@@ -334,31 +399,68 @@ tri_kernel(PrefillArgs p) {
     group_sync(1 + gi, 64);
     if (!live)
         return;
-    // column c = tt of T, then T diag(beta) and -T diag(beta gamma) (the B tiles
-    // of the chunk kernel's MMA 1 and MMA 2b), each as 96 rows of 32 floats: row r
-    // of column block 0, then row r of block 1 at row r + 32 (a TMA load with
-    // 128-byte swizzle turns them back into the triangular tile).  gamma = e^G
-    // by the same fast exponential as the gate record's.
-    float x[kC];
+    // T = (I + A)^-1 as 2 x 2 blocks of 32: each warp solves its diagonal block
+    // T_ww = (I + A_ww)^-1 (lane = column); then T21 = -T22 (A21 T11), the two
+    // warps taking 16 columns each, on the tensor core.  T diag(beta) and
+    // -T diag(beta gamma) (the B tiles of the chunk kernel's MMA 1 and MMA 2b)
+    // go out as 96 rows of 32 floats: row r of column block 0, then row r of
+    // block 1 at row r + 32 (a TMA load with 128-byte swizzle turns them back
+    // into the triangular tile).  gamma = e^G by the same fast exponential as the
+    // gate record's.
     float *dst = (float *)p.ws_tb + ((size_t)ci * p.Hv + h) * (2 * 96 * 32);
     float *dsg = dst + 96 * 32;
-    const float bc = Be[tt], gc = __expf(G[tt]);
-    if (tt < 32) {
-        tri_column<0>(A, tt, x);
+    const int w = tt >> 5;
+    float *T1 = T1s[gi], *T2 = T2s[gi];
+    {
+        float x[32];
+        tri_diag32(A + 2048 * w, lane, x);
+        const float bc = Be[tt], gc = __expf(G[tt]);
+        float *tw = w ? T2 : T1;
+        const int ts = w ? 36 : 40;
+        float *db = w ? dst + 64 * 32 + lane : dst + lane; // block 1 rows 32.. / block 0 rows 0..
+        float *dg = db + 96 * 32;
 #pragma unroll
-        for (int r = 0; r < kC; ++r) {
+        for (int r = 0; r < 32; ++r) {
+            tw[r * ts + lane] = x[r];
             const float tb = tf32_rna(x[r] * bc);
-            dst[r * 32 + tt] = tb;
-            dsg[r * 32 + tt] = tf32_rna(-tb * gc);
+            db[r * 32] = tb;
+            dg[r * 32] = tf32_rna(-tb * gc);
         }
-    } else {
-        tri_column<32>(A, tt, x);
+    }
+    group_sync(1 + gi, 64);
+    const int j0 = 16 * w; // this warp's columns of W and T21
+    float d[2][2][4];
+    // W = A21 T11: A21 = rows 32..63, columns 0..31 of A (column block 0)
+    mm32x16_3xtf32([&](int i, int k) { return A[32 * (32 + i) + (((k >> 2) ^ (i & 7)) << 2) + (k & 3)]; },
+                   [&](int k, int j) { return T1[k * 40 + j]; }, j0, lane, d);
+    __syncwarp();
+    // W takes the place of T11's columns j0 .. j0 + 15, which only this warp reads
+    const int g = lane >> 2, t = lane & 3;
 #pragma unroll
-        for (int r = 32; r < kC; ++r) {
-            const float tb = tf32_rna(x[r] * bc);
-            dst[(r + 32) * 32 + (tt - 32)] = tb;
-            dsg[(r + 32) * 32 + (tt - 32)] = tf32_rna(-tb * gc);
+    for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int i = 16 * mt + g, j = j0 + 8 * nt + 2 * t;
+            *reinterpret_cast<float2 *>(T1 + i * 40 + j) = make_float2(d[mt][nt][0], d[mt][nt][1]);
+            *reinterpret_cast<float2 *>(T1 + (i + 8) * 40 + j) = make_float2(d[mt][nt][2], d[mt][nt][3]);
         }
+    __syncwarp();
+    // T21 = -T22 W, rows 32..63 of column block 0
+    mm32x16_3xtf32([&](int i, int k) { return T2[i * 36 + k]; }, [&](int k, int j) { return T1[k * 40 + j]; },
+                   j0, lane, d);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        const int j = j0 + 8 * nt + 2 * t;
+        const float b0 = Be[j], b1 = Be[j + 1], e0 = __expf(G[j]), e1 = __expf(G[j + 1]);
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+            for (int hr = 0; hr < 2; ++hr) {
+                const int r = 32 + 16 * mt + g + 8 * hr;
+                const float t0 = tf32_rna(-d[mt][nt][2 * hr] * b0), t1 = tf32_rna(-d[mt][nt][2 * hr + 1] * b1);
+                *reinterpret_cast<float2 *>(dst + r * 32 + j) = make_float2(t0, t1);
+                *reinterpret_cast<float2 *>(dsg + r * 32 + j) = make_float2(tf32_rna(-t0 * e0), tf32_rna(-t1 * e1));
+            }
     }
 }
 
