@@ -299,7 +299,8 @@ GDN_API gdn_status gdn_decode_commit(const gdn_config *cfg, const gdn_params *pa
  *     S_t = S_{t-1} Diag(alpha_t) (I - beta_t k_t k_t^T) + beta_t v_t k_t^T,
  *     o_t = S_t q_t,   beta_t = sigmoid(b_t),
  *     y_t = o_t / sqrt(mean(o_t^2) + rms_eps) * norm_w * sigmoid(gate_t).
- * Arithmetic is FP32 on CUDA cores (token-serial prefill, one-token decode).
+ * Arithmetic is FP32 on CUDA cores: the prefill takes two tokens per step (an
+ * exact refactoring of the recurrence above), the decode one token.
  */
 typedef struct gdn_kda_params {
     const float *conv_w; /* [3 H d, conv_kernel] (q heads, k heads, v heads) */
@@ -307,7 +308,14 @@ typedef struct gdn_kda_params {
     const float *norm_w; /* [d], shared by all heads */
 } gdn_kda_params;
 
-/* Workspace bytes of gdn_kda_prefill (as gdn_prefill_workspace_size). */
+/*
+ * Workspace bytes of gdn_kda_prefill (as gdn_prefill_workspace_size): a
+ * 256-byte header, float32 normalised q|k [N, 2 H d], float32 convolved v
+ * [N, H d] and the float32 raw output [N, H, d] before the gated norm, each
+ * region rounded up to 256 bytes; 0 when total_tokens is 0.  Requires
+ * num_qk_heads == num_v_heads (GDN_ERR_INVALID_ARG otherwise) and segments
+ * 0 or 1 (GDN_ERR_UNSUPPORTED otherwise).
+ */
 GDN_API gdn_status gdn_kda_prefill_workspace_size(const gdn_config *cfg, int32_t batch,
                                                   int64_t total_tokens, size_t *bytes);
 

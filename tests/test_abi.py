@@ -73,6 +73,27 @@ def test_workspace_size_arithmetic():
     assert gdn.prefill_workspace_size(gdn.Config(2, 4, 32), 1, 3) == 256 + 1536 + 1536
 
 
+def test_kda_workspace_size_arithmetic():
+    """KDA prefill: a 256-byte header, float32 normalised q|k [N, 2 H d], float32
+    convolved v [N, H d] and the float32 raw output [N, H, d] that the recurrence
+    writes and the gated-norm pass reads; regions rounded to 256 B."""
+    kimi = gdn.Config(96, 96, 128)
+    N = 4096
+    assert gdn.kda_prefill_workspace_size(kimi, 1, N) == 256 + N * 2 * 96 * 128 * 4 + 2 * N * 96 * 128 * 4
+    # the size does not depend on the sequence count, and no tokens need none
+    assert gdn.kda_prefill_workspace_size(kimi, 7, N) == gdn.kda_prefill_workspace_size(kimi, 1, N)
+    assert gdn.kda_prefill_workspace_size(kimi, 3, 0) == 0
+    small = gdn.Config(4, 4, 32, act_dtype="f32")
+    # 3 tokens: q|k 3 * 2 * 4 * 32 * 4 = 3072 B, v and o 1536 B each
+    assert gdn.kda_prefill_workspace_size(small, 2, 3) == 256 + 3072 + 1536 + 1536
+    # 1 token: 1024 B, then 512 B each
+    assert gdn.kda_prefill_workspace_size(small, 1, 1) == 256 + 1024 + 512 + 512
+    # KDA has one q/k head per value head and no sequence split
+    for bad in (gdn.Config(2, 4, 32), gdn.Config(4, 4, 32, segments=2)):
+        with pytest.raises(gdn.GdnError):
+            gdn.kda_prefill_workspace_size(bad, 1, 8)
+
+
 def test_segment_workspace_and_choice():
     """The split's workspace (R, M and start states: 3 (P - 1) batch H_v d^2 floats)
     and the library's choice of P."""
