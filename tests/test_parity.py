@@ -182,6 +182,28 @@ def test_edge_lengths_full(cuda_device, with_conv, algo):
         assert torch.equal(out["final_state"][n], inp["initial_state"][n])
 
 
+@ALGOS
+@pytest.mark.parametrize("shape", [(1, 3), (3, 9)], ids=["1x3", "3x9"])
+def test_odd_value_head_count(cuda_device, shape, algo):
+    """An odd number of value heads (G = 3): the inverse kernel's CTAs take two
+    value heads each, so the last one has an idle half.  Every head of two
+    ragged sequences against the oracle."""
+    Hk, Hv = shape
+    wl = W.Workload(f"odd_heads_{Hk}x{Hv}", Hk, Hv, 128, seqlens=(70, 129), state_std=0.02, seed=23)
+    cfg = gdn.Config.of(wl, algo)
+    inp = W.make_prefill(wl, cuda_device)
+    out = _gpu_prefill(cfg, inp, return_final_state=True, return_o_raw=True)
+    torch.cuda.synchronize()
+    cu = inp["cu_seqlens"].tolist()
+    for n in range(len(wl.seqlens)):
+        ref = _oracle_seq(wl, inp, n)
+        s, e = cu[n], cu[n + 1]
+        r, m = assert_output_close(out["y"][s:e], ref["y"], f"y seq {n}")
+        assert_output_close(out["o_raw"][s:e], ref["o"], f"o seq {n}")
+        rs = assert_state_close(out["final_state"][n], ref["state"], f"state seq {n}")
+        report(f"{wl.name} {algo} seq {n}", r, m, rs)
+
+
 EDGE_F32 = W.Workload("edge_f32", 2, 4, 128, dtype="f32", seqlens=(0, 5, 64, 100, 31),
                       state_std=0.02, seed=78)
 
