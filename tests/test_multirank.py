@@ -35,7 +35,9 @@ def _rank_main(rank, world, port, out):
 
 def test_two_gloo_ranks_agree_on_max_and_rate():
     world, port = 2, 29500 + os.getpid() % 2000
-    with mp.Manager() as m:
+    # the manager's server process is spawned too: forking a process that
+    # already runs threads (torch's) can deadlock the child
+    with mp.get_context("spawn").Manager() as m:
         out = m.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, start_method="spawn")
         res = dict(out)
