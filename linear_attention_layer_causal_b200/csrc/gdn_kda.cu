@@ -12,10 +12,11 @@
 //     s <- s * alpha;  u = beta (v - s . k);  s <- s + u k;  o = s . q
 // (the last equal to (s * alpha) . q + u (k . q)).
 // Each head has its own q and k (no sharing).  Both kernels run the update on
-// CUDA cores in FP32: the token-serial prefill (D / 32 CTAs of 32 state rows per
-// (head, sequence); the conv, SiLU and L2 norm come from the shared front
-// kernel; the gated RMSNorm is a separate pass over the raw output) and the
-// one-token decode (one CTA per (sequence, head), conv from the cache).
+// CUDA cores in FP32: the prefill (D / 32 CTAs of 32 state rows per (head,
+// sequence), two tokens per step; the conv, SiLU and L2 norm come from the
+// shared front kernel; the gated RMSNorm is a separate pass over the raw
+// output) and the one-token decode (one CTA per (sequence, head), conv from
+// the cache).
 #include "gdn_common.cuh"
 #include "gdn_internal.h"
 
